@@ -1,0 +1,400 @@
+"""Pins of the fp64 oracle to things other than itself: closed forms, library routines,
+invariants, hand-derived worked examples (tests/golden/) and brute force on tiny inputs.
+
+Each group names the oracle function it pins.  tests/test_oracle_mutants.py plants plausible
+mistakes into copies of the oracle and checks that these pins catch every one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------------------------
+# attend: softmax attention of G heads over n tokens
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("G,D,n", [(1, 8, 1), (4, 8, 16), (3, 16, 37), (8, 64, 5)])
+def test_attend_matches_torch_sdpa(G, D, n):
+    q, k, v = _rand((G, D), 1), _rand((n, D), 2), _rand((n, D), 3)
+    out, lse = oracle.attend(q, k, v)
+    tq, tk, tv = (torch.from_numpy(a) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq[None], tk[None], tv[None])[0]
+    ref_lse = torch.logsumexp(tq @ tk.T / math.sqrt(D), dim=-1)
+    assert np.allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
+
+
+def test_attend_identical_keys_gives_mean_of_v():
+    # every logit equals z = q.k/sqrt(D): weights 1/n, out = mean(v), lse = z + ln n
+    G, D, n = 4, 16, 23
+    q, v = _rand((G, D), 4), _rand((n, D), 5)
+    k1 = _rand((1, D), 6)
+    out, lse = oracle.attend(q, np.repeat(k1, n, axis=0), v)
+    assert np.allclose(out, np.broadcast_to(v.mean(axis=0), (G, D)), atol=1e-13)
+    z = (q @ k1[0]) / math.sqrt(D)
+    assert np.allclose(lse, z + math.log(n), atol=1e-13)
+
+
+def test_attend_one_token_returns_its_value():
+    G, D = 4, 32
+    q, k, v = _rand((G, D), 7), _rand((1, D), 8), _rand((1, D), 9)
+    out, lse = oracle.attend(q, k, v)
+    assert np.array_equal(out, np.broadcast_to(v[0], (G, D)))
+    assert np.allclose(lse, q @ k[0] / math.sqrt(D), atol=1e-14)
+
+
+def test_attend_two_tokens_closed_form():
+    # two tokens: weight of token 0 is the logistic function of the logit difference
+    D = 4
+    q = np.array([[1.0, 0.0, 0.0, 0.0]])
+    k = np.array([[2.0, 0, 0, 0], [0.0, 0, 0, 0]])  # logits 1 and 0
+    v = np.array([[1.0, 0, 0, 0], [0.0, 1, 0, 0]])
+    out, lse = oracle.attend(q, k, v)
+    w0 = math.e / (math.e + 1.0)
+    assert np.allclose(out[0], [w0, 1 - w0, 0, 0], atol=1e-15)
+    assert abs(lse[0] - math.log(math.e + 1.0)) < 1e-15
+
+
+def test_attend_permutation_invariance_and_v_linearity():
+    G, D, n = 2, 8, 19
+    q, k, v = _rand((G, D), 10), _rand((n, D), 11), _rand((n, D), 12)
+    out, lse = oracle.attend(q, k, v)
+    p = np.random.default_rng(13).permutation(n)
+    out_p, lse_p = oracle.attend(q, k[p], v[p])
+    assert np.allclose(out, out_p, atol=1e-13) and np.allclose(lse, lse_p, atol=1e-13)
+    out2, lse2 = oracle.attend(q, k, 3.0 * v)
+    assert np.allclose(out2, 3.0 * out, atol=1e-13) and np.array_equal(lse, lse2)
+
+
+def test_attend_rejects_empty():
+    with pytest.raises(ValueError):
+        oracle.attend(np.ones((1, 4)), np.ones((0, 4)), np.ones((0, 4)))
+
+
+# ---------------------------------------------------------------------------------------------
+# decode: GQA head mapping (query head h -> KV head h // G), G = 1 is MHA
+# ---------------------------------------------------------------------------------------------
+def _tiny_batch(G, D=16, lengths=(7, 30, 1), Hkv=2, seed=0, dtype="f32"):
+    wl = workloads.Workload("tiny", B=len(lengths), Hkv=Hkv, G=G, D=D, kv_dtype=dtype,
+                            dist="normal", lengths=tuple(lengths))
+    return workloads.generate(wl, seed)
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_decode_matches_sdpa_with_repeat_interleave(G):
+    bt = _tiny_batch(G)
+    out, lse = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G)
+    cu = bt.cu_seqlens.numpy()
+    for b in range(bt.wl.B):
+        s, e = int(cu[b]), int(cu[b + 1])
+        kk = bt.k[:, s:e].double().repeat_interleave(G, dim=0)  # [Hq, L, D], [AO] GQA example
+        vv = bt.v[:, s:e].double().repeat_interleave(G, dim=0)
+        qq = bt.q[b].double()[:, None, :]  # [Hq, 1, D]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv)[:, 0]
+        assert np.allclose(out[b], ref.numpy(), atol=1e-12)
+        ref_lse = torch.logsumexp((qq @ kk.transpose(1, 2))[:, 0] / math.sqrt(bt.wl.D), dim=-1)
+        assert np.allclose(lse[b], ref_lse.numpy(), atol=1e-12)
+
+
+def test_gqa_example_numbers(golden_dir):
+    g = _load(golden_dir, "gqa_example.json")
+    H, Hkv, D, L = g["num_heads"], g["num_kv_heads"], g["head_dim"], g["seq_len"]
+    assert 2 * H * D * L == g["mha_cache_entries"]
+    assert 2 * Hkv * D * L == g["gqa_cache_entries"]
+    assert round(100 * (1 - g["gqa_cache_entries"] / g["mha_cache_entries"])) == g["saving_percent"]
+    # our layout: k, v [Hkv, T, D] hold exactly the GQA cache entries
+    bt = _tiny_batch(G=H // Hkv, D=D, lengths=(L,), Hkv=Hkv)
+    assert bt.k.numel() + bt.v.numel() == g["gqa_cache_entries"]
+    # and head h reads KV head h // G, as repeat_interleave does
+    G = g["heads_per_group"]
+    mapping = torch.arange(Hkv).repeat_interleave(G).tolist()
+    assert mapping == g["kv_head_of_query_head"] == [h // G for h in range(H)]
+
+
+# ---------------------------------------------------------------------------------------------
+# merge: split = unsplit for every chunking
+# ---------------------------------------------------------------------------------------------
+def test_merge_single_chunk_is_identity():
+    o, l = _rand((1, 3, 5), 20), _rand((1, 3), 21)
+    out, lse = oracle.merge(o, l)
+    assert np.allclose(out, o[0], atol=1e-15) and np.allclose(lse, l[0], atol=1e-15)
+
+
+@pytest.mark.parametrize("n", [1, 2, 7, 13])
+def test_merge_of_every_chunking_equals_unsplit(n):
+    G, D = 3, 8
+    q, k, v = _rand((G, D), 30 + n), _rand((n, D), 31 + n, 2.0), _rand((n, D), 32 + n)
+    ref_out, ref_lse = oracle.attend(q, k, v)
+    # every composition of n into contiguous chunks (2^(n-1) of them) for small n
+    cuts_all = range(1, n)
+    for r in range(0, n):
+        for cuts in itertools.combinations(cuts_all, r):
+            bounds = [0, *cuts, n]
+            parts = [oracle.attend(q, k[a:b], v[a:b]) for a, b in zip(bounds[:-1], bounds[1:])]
+            out, lse = oracle.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+            assert np.allclose(out, ref_out, atol=1e-12) and np.allclose(lse, ref_lse, atol=1e-12)
+
+
+def test_merge_random_chunkings_long_row():
+    G, D, n = 4, 16, 500
+    q, k, v = _rand((G, D), 40), _rand((n, D), 41, 3.0), _rand((n, D), 42)
+    ref_out, ref_lse = oracle.attend(q, k, v)
+    rng = np.random.default_rng(43)
+    for trial in range(20):
+        cuts = np.sort(rng.choice(np.arange(1, n), size=rng.integers(1, 30), replace=False))
+        bounds = [0, *cuts.tolist(), n]
+        parts = [oracle.attend(q, k[a:b], v[a:b]) for a, b in zip(bounds[:-1], bounds[1:])]
+        out, lse = oracle.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+        assert np.allclose(out, ref_out, atol=1e-12) and np.allclose(lse, ref_lse, atol=1e-12)
+
+
+def test_printed_merge_update_without_chunk_factor_is_not_exact():
+    """The page's printed out-update lacks exp(m_chunk - m_new) on the chunk term; written out
+    literally it disagrees with unsplit attention, which is why the oracle merges in LSE form."""
+    G, D, n = 1, 8, 40
+    q, k, v = _rand((G, D), 50), _rand((n, D), 51, 2.0), _rand((n, D), 52)
+    ref_out, _ = oracle.attend(q, k, v)
+    (o1, l1), (o2, l2) = oracle.attend(q, k[:20], v[:20]), oracle.attend(q, k[20:], v[20:])
+    # per chunk: m = chunk max logit, exp_sum = sum exp(z - m) = exp(lse - m)
+    z1 = (q @ k[:20].T)[0] / math.sqrt(D)
+    z2 = (q @ k[20:].T)[0] / math.sqrt(D)
+    m1, m2 = z1.max(), z2.max()
+    s1, s2 = math.exp(l1[0] - m1), math.exp(l2[0] - m2)
+    m_new = max(m1, m2)
+    exp_sum = math.exp(m1 - m_new) * s1 + math.exp(m2 - m_new) * s2
+    printed = (math.exp(m1 - m_new) * o1[0] * s1 + o2[0] * s2) / exp_sum
+    restored = (math.exp(m1 - m_new) * o1[0] * s1 + math.exp(m2 - m_new) * o2[0] * s2) / exp_sum
+    assert np.allclose(restored, ref_out[0], atol=1e-12)
+    assert not np.allclose(printed, ref_out[0], atol=1e-6)
+
+
+# ---------------------------------------------------------------------------------------------
+# quantisation
+# ---------------------------------------------------------------------------------------------
+def test_quantize_worked_cases(golden_dir):
+    for grp in _load(golden_dir, "quantize_worked_cases.json")["groups"]:
+        x = np.array(grp["values"], np.float32)
+        s = oracle.scale_from_amax(oracle.amax(x))
+        assert s == np.float32(grp["scale"])
+        assert oracle.quantize(x, s).tolist() == grp["codes"]
+
+
+def test_quantize_clamps_to_127(golden_dir):
+    c = _load(golden_dir, "quantize_worked_cases.json")["clamp"]
+    assert oracle.quantize(np.array(c["values"], np.float32), c["scale"]).tolist() == c["codes"]
+
+
+def test_quantize_matches_numpy_float32_route():
+    # independent route: numpy's IEEE float32 division and round-half-even
+    rng = np.random.default_rng(60)
+    for trial in range(20):
+        x = (rng.standard_normal(4096) * rng.lognormal(0, 2)).astype(np.float32)
+        s = oracle.scale_from_amax(oracle.amax(x))
+        assert s == np.float32(np.abs(x).max()) / np.float32(127.0)
+        ref = np.clip(np.rint(x / s), -127, 127).astype(np.int8)
+        assert np.array_equal(oracle.quantize(x, s), ref)
+
+
+def test_quantize_amax_element_maps_to_127_and_bounds():
+    rng = np.random.default_rng(61)
+    for trial in range(50):
+        x = (rng.standard_normal(257) * 10 ** rng.uniform(-30, 30)).astype(np.float32)
+        s = oracle.scale_from_amax(oracle.amax(x))
+        c = oracle.quantize(x, s)
+        i = int(np.argmax(np.abs(x)))
+        assert c[i] == (127 if x[i] > 0 else -127)
+        assert c.min() >= -127 and c.max() <= 127
+        err = np.abs(x.astype(np.float64) - c.astype(np.float64) * np.float64(s))
+        assert (err <= np.float64(s) * 0.5 * (1 + 1e-5)).all()
+
+
+def test_quantize_integers_reproduce_and_ties_go_to_even():
+    x = np.arange(-127, 128, dtype=np.float32)
+    s = oracle.scale_from_amax(oracle.amax(x))
+    assert s == 1.0
+    assert np.array_equal(oracle.quantize(x, s), x.astype(np.int8))
+    halves = np.arange(-126.5, 127.0, 1.0, dtype=np.float32)
+    halves = np.concatenate([halves, [127.0]]).astype(np.float32)
+    c = oracle.quantize(halves, oracle.scale_from_amax(oracle.amax(halves)))
+    assert (c[:-1] % 2 == 0).all()  # every .5 case rounds to the even neighbour
+
+
+def test_quantize_zero_group_gives_zero_scale_and_codes():
+    x = np.zeros(64, np.float32)
+    s = oracle.scale_from_amax(oracle.amax(x))
+    assert s == 0.0 and not oracle.quantize(x, s).any()
+
+
+def test_scheme_a_partitions_start_at_each_sequence():
+    bt = _tiny_batch(G=2, D=8, lengths=(70, 64, 3, 129), Hkv=2, dtype="bf16")
+    kc, vc, ks, vs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    cu = bt.cu_seqlens.numpy()
+    assert ks.shape == (2, 2 + 1 + 1 + 3)
+    col = 0
+    for b in range(4):
+        s0, e0 = int(cu[b]), int(cu[b + 1])
+        for p in range(0, e0 - s0, 64):
+            for h in range(2):
+                block = bt.k[h, s0 + p:min(s0 + p + 64, e0)].float().numpy()
+                assert ks[h, col] == np.float32(np.abs(block).max()) / np.float32(127)
+                ref = np.clip(np.rint(block / ks[h, col]), -127, 127)
+                assert np.array_equal(kc[h, s0 + p:min(s0 + p + 64, e0)], ref.astype(np.int8))
+            col += 1
+    assert vs[0] == np.float32(bt.v.float().abs().max().item()) / np.float32(127)
+
+
+def test_scheme_b_equals_scheme_a_with_one_partition():
+    bt = _tiny_batch(G=2, D=8, lengths=(100,), Hkv=1, dtype="bf16")
+    kc_b, vc_b, ks_b, vs_b = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "B")
+    kc_a, vc_a, ks_a, vs_a = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A", part=100)
+    assert np.array_equal(kc_a, kc_b) and np.array_equal(vc_a, vc_b)
+    assert ks_a.ravel()[0] == ks_b[0] and vs_a[0] == vs_b[0]
+
+
+# ---------------------------------------------------------------------------------------------
+# OAM scores and top-K
+# ---------------------------------------------------------------------------------------------
+def test_oam_hand_example(golden_dir):
+    g = _load(golden_dir, "oam_hand_example.json")
+    s = oracle.oam_scores(np.array(g["q"], float), np.array(g["k"], float), np.array(g["v"], float),
+                          g["beta"], g["eps"])
+    assert np.allclose(s, g["scores"], rtol=0, atol=1e-15)
+
+
+def test_oam_scores_match_torch_route():
+    G, D, n = 8, 64, 300
+    q, k, v = _rand((G, D), 70), _rand((n, D), 71), _rand((n, D), 72)
+    s = oracle.oam_scores(q, k, v, 0.7, 1e-6)
+    tq, tk, tv = (torch.from_numpy(a) for a in (q, k, v))
+    ref = (tk @ tq.T / math.sqrt(D)).max(dim=1).values + 0.7 * torch.log(torch.linalg.vector_norm(tv, dim=1) + 1e-6)
+    assert np.allclose(s, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_topk_matches_brute_force_sort():
+    rng = np.random.default_rng(80)
+    for trial in range(30):
+        n = int(rng.integers(1, 200))
+        s = np.round(rng.standard_normal(n), 1)  # many exact ties
+        K = int(rng.integers(1, n + 1))
+        ref = sorted(sorted(range(n), key=lambda t: (-s[t], t))[:K])
+        assert oracle.topk(s, K).tolist() == ref
+
+
+def test_topk_all_equal_keeps_lowest_indices_and_keep_all():
+    assert oracle.topk(np.zeros(50), 7).tolist() == list(range(7))
+    s = _rand(33, 81)
+    assert oracle.topk(s, 33).tolist() == list(range(33))
+
+
+def test_kept_count():
+    assert [oracle.kept_count(L, 1, 8) for L in (1, 7, 8, 9, 16, 17, 131072)] == [1, 1, 1, 2, 2, 3, 16384]
+    assert oracle.kept_count(10, 1, 1) == 10 and oracle.kept_count(5, 0, 8) == 1
+
+
+def test_beta_zero_is_classic_qk_ranking_and_q_zero_is_norm_ranking():
+    G, D, n = 4, 16, 120
+    q, k, v = _rand((G, D), 90), _rand((n, D), 91), _rand((n, D), 92)
+    s0 = oracle.oam_scores(q, k, v, 0.0, 1e-6)
+    qk = (k @ q.T).max(axis=1)  # classic Q x K score, group max
+    assert np.array_equal(oracle.topk(s0, 15), np.sort(np.argsort(-qk, kind="stable")[:15]))
+    sz = oracle.oam_scores(np.zeros((G, D)), k, v, 1.0, 1e-6)
+    norms = np.linalg.norm(v, axis=1)
+    assert np.array_equal(oracle.topk(sz, 15), np.sort(np.argsort(-norms, kind="stable")[:15]))
+    # equal |v| for every token: OAM ranks exactly like Q x K
+    vu = v / np.linalg.norm(v, axis=1, keepdims=True) * 2.0
+    su = oracle.oam_scores(q, k, vu, 1.0, 1e-6)
+    assert np.array_equal(oracle.topk(su, 15), np.sort(np.argsort(-qk, kind="stable")[:15]))
+
+
+def test_keep_all_selection_equals_dense_decode():
+    bt = _tiny_batch(G=4, D=16, lengths=(9, 40), Hkv=2, dtype="bf16")
+    idx, cu_kept, _ = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 4, 1.0, 1e-6, 1, 1)
+    assert cu_kept.tolist() == [0, 9, 49]
+    assert idx[:, :9].tolist() == [list(range(9))] * 2
+    dense = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 4)
+    sel = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 4, idx=idx, cu_kept=cu_kept)
+    assert np.allclose(dense[0], sel[0], atol=1e-13) and np.allclose(dense[1], sel[1], atol=1e-13)
+
+
+def test_indexed_decode_equals_attention_over_the_subset():
+    bt = _tiny_batch(G=2, D=8, lengths=(50,), Hkv=1)
+    idx, cu_kept, _ = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, 1.0, 1e-6, 1, 8)
+    out, lse = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, idx=idx, cu_kept=cu_kept)
+    sel = idx[0]
+    assert sel.size == 7 and (np.diff(sel) > 0).all()
+    q = bt.q[0].double()
+    kk, vv = bt.k[0, sel].double(), bt.v[0, sel].double()
+    ref = torch.nn.functional.scaled_dot_product_attention(q[:, None], kk[None].expand(2, -1, -1),
+                                                           vv[None].expand(2, -1, -1))[:, 0]
+    assert np.allclose(out[0], ref.numpy(), atol=1e-12)
+
+
+def test_int8_decode_is_attention_over_dequantised_cache():
+    bt = _tiny_batch(G=2, D=8, lengths=(70, 5), Hkv=2, dtype="bf16")
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    kc, vc, ks, vs = quant
+    out, lse = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, quant=(*quant, "A"))
+    # independent dequantisation: partition p of sequence 0 head 1 holds tokens 64p .. 64p+63
+    k_hat = torch.from_numpy(kc[1, :70].astype(np.float64))
+    k_hat[:64] *= float(ks[1, 0])
+    k_hat[64:] *= float(ks[1, 1])
+    v_hat = torch.from_numpy(vc[1, :70].astype(np.float64)) * float(vs[0])
+    q = bt.q[0, 2:4].double()
+    ref = torch.nn.functional.scaled_dot_product_attention(q[:, None], k_hat[None].expand(2, -1, -1),
+                                                           v_hat[None].expand(2, -1, -1))[:, 0]
+    assert np.allclose(out[0, 2:4], ref.numpy(), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# partition
+# ---------------------------------------------------------------------------------------------
+def test_plan_hand_example(golden_dir):
+    g = _load(golden_dir, "plan_hand_example.json")
+    p = oracle.plan(g["row_lengths"], g["n_req"], g["granule"], g["min_chunk"], 0)
+    segs = [list(map(int, t)) for t in zip(p["cta"], p["row"], p["start"], p["len"])]
+    assert segs == g["segments"] and p["n_cta"] == g["n_cta"]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_plan_covers_every_token_once_with_equal_work(seed):
+    rng = np.random.default_rng(seed)
+    R = int(rng.integers(1, 40))
+    lens = np.rint(np.exp(rng.uniform(0, 10, R))).astype(np.int64)
+    n_req = int(rng.integers(1, 300))
+    gran = 16
+    p = oracle.plan(lens, n_req, gran, gran, 0)
+    assert p["n_cta"] <= n_req
+    covered = [np.zeros(L, np.int32) for L in lens]
+    for c, r, s, l in zip(p["cta"], p["row"], p["start"], p["len"]):
+        assert l >= 1 and s % gran == 0
+        covered[r][s:s + l] += 1
+    assert all((cv == 1).all() for cv in covered)
+    # segments come in stream order; a CTA's padded work is at most S
+    order = list(zip(p["cta"], p["row"]))
+    assert order == sorted(order)
+    W = int(sum((L + gran - 1) // gran * gran for L in lens))
+    S = max(gran, -(-(-(-W // n_req)) // gran) * gran)
+    work = np.zeros(p["n_cta"], np.int64)
+    for c, l in zip(p["cta"], p["len"]):
+        work[c] += (l + gran - 1) // gran * gran
+    assert work.max() <= S
+    one = oracle.plan(lens, 0, gran, gran, 1)
+    assert one["n_cta"] == R and one["len"].tolist() == lens.tolist()
