@@ -1,0 +1,207 @@
+/*
+ * sgd.h -- C ABI of libsgd.so: single-token GQA decode attention over a long,
+ * ragged KV cache on NVIDIA B200 (sm_100a), with output-aware token dropping
+ * (OAM), an INT8 KV cache and split-KV flash-decoding with an exact
+ * log-sum-exp merge.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [TD] "优化稀疏注意力中的令牌丢弃机制" (Optimizing token dropping in sparse
+ *        attention), lzwjava.github.io -- section 3 (OAM score and token
+ *        dropping), section 5 (split-KV load balancing and the cross-chunk
+ *        online-softmax merge), section 6 (INT8 KV cache, schemes A and B),
+ *        section 7 (the three stack: OAM -> INT8 -> split-KV).
+ *   [AO] "注意力优化（Attention Optimization）", learnagent.wiki -- scaled
+ *        dot-product attention; GQA (query head h uses KV head h / G).
+ *   [CD] "共同设计 AI 模型注意力，实现快速的交互式长上下文推理" (Co-designing AI
+ *        model attention for fast interactive long-context inference), NVIDIA
+ *        developer blog -- decode equations 5-7 (decode streams the KV cache
+ *        and is HBM-bound; arithmetic intensity about 2G).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  A packed ragged cache of B sequences and Hkv KV heads:
+ *     k, v        [Hkv, T, D] row-major, T = cu_seqlens[B]; sequence b is tokens
+ *                 cu_seqlens[b] .. cu_seqlens[b+1]-1 of every head.
+ *     q           [B, Hq, D], Hq = Hkv * G; query head h = kvh * G + g reads KV
+ *                 head kvh ([AO], GQA example).
+ *     out         [B, Hq, D] float32; lse [B, Hq] float32, the natural log of
+ *                 sum_t exp(q.k_t / sqrt(D)) over the tokens attended.
+ * Pointers.  Every array argument is a DEVICE pointer of the current device
+ * unless its comment says "host".  Arrays must start on a 16-byte boundary.
+ * Ownership.  The caller allocates and frees every buffer, including the
+ * workspace; the library never allocates, frees or synchronises, and never
+ * changes the current device.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  All work is enqueued on it; results are ready when it completes.
+ * Errors.  Every int-returning call returns SGD_OK (0) or a negative SGD_ERR_*
+ * code; invalid arguments are rejected on the host before anything is
+ * launched.  Conditions only the device can see (a sequence of length 0 in a
+ * device array, a bounded wait that ran out) set bits in the 32-bit status word
+ * at the start of the workspace (SGD_WS_STATUS_OFFSET), read it with
+ * sgd_workspace_status after the stream completes.  No call aborts, traps or
+ * throws.
+ * Limits.  1 <= G <= 16; D in {64, 128}; Hkv * T < 2^31; B >= 1, Hkv >= 1.
+ */
+#ifndef SGD_H_
+#define SGD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types of q and of the cache */
+typedef enum { SGD_F32 = 0, SGD_BF16 = 1, SGD_I8 = 2 } sgd_dtype;
+
+/* INT8 scale granularity ([TD] section 6):
+ *   A: one K scale per (KV head, sequence, 64-token partition counted from
+ *      the sequence's first token; the last partition takes the remainder),
+ *      one V scale for the whole tensor;
+ *   B: one K scale and one V scale, each for the whole tensor. */
+typedef enum { SGD_SCHEME_A = 0, SGD_SCHEME_B = 1 } sgd_scheme;
+
+#define SGD_PARTITION 64 /* scheme-A partition length in tokens */
+
+/* status codes */
+#define SGD_OK 0
+#define SGD_ERR_NULL -1          /* a required pointer is NULL */
+#define SGD_ERR_SHAPE -2         /* B, Hkv, T, D, G or a size out of range */
+#define SGD_ERR_DTYPE -3         /* unsupported dtype / scheme combination */
+#define SGD_ERR_ALIGN -4         /* an array is not 16-byte aligned */
+#define SGD_ERR_WORKSPACE -5     /* workspace smaller than sgd_workspace_size */
+#define SGD_ERR_CUDA -6          /* a CUDA runtime call or launch failed */
+#define SGD_ERR_DEVICE -7        /* current device is not sm_100 */
+#define SGD_ERR_ARG -8           /* any other invalid argument */
+
+/* device status bits (status word at the start of the workspace) */
+#define SGD_STATUS_EMPTY_SEQUENCE 0x1 /* a sequence has length < 1 */
+#define SGD_STATUS_WAIT_TIMEOUT 0x2   /* a bounded pipeline wait gave up */
+#define SGD_STATUS_SIZE_MISMATCH 0x4  /* device lengths disagree with host sizes */
+#define SGD_STATUS_BAD_INDEX 0x8      /* a kept index was outside its sequence */
+
+#define SGD_WS_STATUS_OFFSET 0
+
+/* A packed ragged KV cache (all pointers device pointers). */
+typedef struct {
+    sgd_dtype dtype;            /* of k and v: F32, BF16 or I8 (codes) */
+    int32_t B;                  /* sequences */
+    int32_t Hkv;                /* KV heads */
+    int32_t D;                  /* head dim, 64 or 128 */
+    int64_t T;                  /* total tokens = cu_seqlens[B] (host value) */
+    const int32_t *cu_seqlens;  /* [B+1] prefix sums of the sequence lengths */
+    const void *k;              /* [Hkv, T, D] */
+    const void *v;              /* [Hkv, T, D] */
+    /* I8 only */
+    sgd_scheme scheme;
+    const float *k_scale;       /* A: [Hkv, n_parts], sequence b's partitions start at
+                                   sum_{b'<b} ceil(L_b'/64); B: [1] */
+    const float *v_scale;       /* [1] */
+    int64_t n_parts;            /* A: sum_b ceil(L_b / 64) (host value); B: ignored */
+} sgd_kv;
+
+/* operations, for sgd_workspace_size */
+#define SGD_OP_QUANTIZE 0
+#define SGD_OP_OAM_SELECT 1
+#define SGD_OP_DECODE 2
+
+/*
+ * sgd_quantize_kv -- INT8 KV cache ([TD] section 6).
+ *   scale = max|x| / 127 over the group sharing it (float32, IEEE division);
+ *   code  = clamp(round_half_even(x / scale), -127, 127), with x / scale the
+ *           correctly rounded float32 quotient; a zero scale gives zero codes.
+ *   Scheme A: K groups are (KV head, sequence, 64-token partition); V is one
+ *   group.  Scheme B: K is one group and V is one group.
+ * in       cache to quantise: dtype BF16 or F32 (k_scale/v_scale/scheme ignored)
+ * k_codes, v_codes   [Hkv, T, D] int8 outputs
+ * k_scale  A: [Hkv, n_parts] (n_parts = sum_b ceil(L_b/64), passed below), B: [1]
+ * v_scale  [1]
+ * Codes and scales are bit-exact functions of the input.
+ */
+int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts,
+                    int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_oam_select -- output-aware token dropping ([TD] section 3).
+ *   For every token t of sequence b and KV head kvh:
+ *     s_t = max_g (q[b, kvh*G+g] . k_t) / sqrt(D) + beta * ln(||v_t||_2 + eps)
+ *   (one index set per KV head, shared by its G query heads); keep the
+ *   K_b = clamp(ceil(L_b * keep_num / keep_den), 1, L_b) highest-scoring
+ *   tokens, ties broken by the lower token index.
+ * q        [B, Hq, D], BF16 or F32 (q_dtype)
+ * kv       the cache as the caller holds it before quantisation: BF16 or F32
+ * idx      [Hkv, kept_total] int32 output: row (b, kvh) is
+ *          idx[kvh, cu_kept[b] .. cu_kept[b+1]-1], kept token positions local
+ *          to sequence b, ascending
+ * cu_kept  [B+1] int32 output, prefix sums of K_b
+ * kept_total  sum_b K_b (host value; the library checks it on the device)
+ */
+int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                   float beta, float eps, int keep_num, int keep_den,
+                   int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_decode_attn -- split-KV flash-decoding ([TD] section 5, [CD] eq. 5-7).
+ *   out[b, h] = sum_t softmax_t(z_t) vhat_t, z_t = q[b, h] . khat_t / sqrt(D),
+ *   over every token of sequence b (idx == NULL) or over the kept tokens
+ *   idx[kvh, cu_kept[b] ..] (softmax renormalised over that set); khat, vhat
+ *   are the cache values (I8: code * scale).  The work of all (sequence, KV
+ *   head) rows is cut into equal token ranges, one per CTA (schedule 0: as many
+ *   CTAs as fill the GPU, or n_splits when > 0; schedule 1: one CTA per row);
+ *   each range emits partial (o_c, lse_c) per row it touches and a merge
+ *   kernel combines them exactly: lse = ln sum_c exp(lse_c),
+ *   out = sum_c exp(lse_c - lse) o_c.
+ * q        [B, Hq, D], BF16 (F32 only with an F32 cache)
+ * idx, cu_kept, kept_total   as produced by sgd_oam_select, or NULL/NULL/0
+ * out      [B, Hq, D] float32;  lse [B, Hq] float32
+ */
+int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                    const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
+                    int schedule, int n_splits, float *out, float *lse,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes an operation needs for this cache shape (>= 256). For
+ * SGD_OP_DECODE, `schedule` and `n_splits` as in sgd_decode_attn; for the
+ * other ops they are ignored.  Returns 0 on invalid arguments. */
+size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_splits);
+
+/* Number of CTAs sgd_decode_attn launches for these arguments (the partition's
+ * n_req), or a negative SGD_ERR_* code. */
+int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedule,
+                        int n_splits);
+
+/*
+ * sgd_plan_segments -- the split-KV partition used by sgd_decode_attn, for
+ * inspection.  Rows are (KV head, sequence) pairs in memory order
+ * (row = kvh * B + b) with lengths cu[b+1] - cu[b]; each row is padded to a
+ * multiple of 16 tokens and the rows are laid end to end; mode 0 cuts this
+ * stream into CTA ranges of S = max(min_chunk, round_up(ceil(W / n_req), 16))
+ * tokens, mode 1 gives each row its own CTA.  A segment is the intersection of
+ * one CTA range with the real tokens of one row.
+ * cu        [B+1] device int32 (cu_seqlens, or cu_kept for a kept set)
+ * segs      [max_segs, 4] device int32 output: (cta, row, row-local start, length)
+ *           in stream order
+ * n_segs    [2] device int32 output: number of segments, number of CTAs used
+ */
+int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode,
+                      int32_t *segs, int64_t max_segs, int32_t *n_segs,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Copies the device status word of `workspace` to *status (host) after
+ * synchronising `stream`.  The only call that synchronises. */
+int sgd_workspace_status(const void *workspace, int32_t *status, void *stream);
+
+/* Static text for a status code. */
+const char *sgd_error_string(int code);
+
+/* Library version, (major << 16) | minor. */
+int sgd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGD_H_ */

@@ -1,0 +1,220 @@
+"""Single-token GQA decode attention for B200 (sm_100a): output-aware token dropping (OAM),
+an INT8 KV cache and split-KV flash-decoding with an exact log-sum-exp merge.
+
+This module is a thin binding over the C ABI of ``libsgd.so`` (``include/sgd.h``): it turns
+torch tensors into device pointers, allocates outputs and the workspace with torch, and
+passes the current CUDA stream.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and importing fails loudly when the library
+has not been built (``python -m sparse_gqa_decode_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "lib", "quantize_kv", "oam_select", "decode_attn", "plan_segments", "workspace_status",
+    "workspace_size", "decode_num_ctas", "kept_total", "n_parts", "SGD_F32", "SGD_BF16", "SGD_I8",
+    "SCHEME_A", "SCHEME_B", "STATUS_BITS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsgd.so")
+
+SGD_F32, SGD_BF16, SGD_I8 = 0, 1, 2
+SCHEME_A, SCHEME_B = 0, 1
+OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE = 0, 1, 2
+PARTITION = 64
+STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_gqa_decode_b200.build` "
+                      "(there is no fallback implementation)")
+
+
+class SgdKv(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("B", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("T", ctypes.c_int64),
+        ("cu_seqlens", ctypes.c_void_p),
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("scheme", ctypes.c_int),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("n_parts", ctypes.c_int64),
+    ]
+
+
+_vp, _sz, _i64, _i32, _f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+_kvp = ctypes.POINTER(SgdKv)
+
+lib = ctypes.CDLL(LIB_PATH)
+lib.sgd_version.restype = ctypes.c_int
+lib.sgd_error_string.argtypes = [ctypes.c_int]
+lib.sgd_error_string.restype = ctypes.c_char_p
+lib.sgd_workspace_size.argtypes = [_i32, _kvp, _i32, _i32, _i32]
+lib.sgd_workspace_size.restype = _sz
+lib.sgd_decode_num_ctas.argtypes = [_kvp, _i32, _vp, _i32, _i32]
+lib.sgd_quantize_kv.argtypes = [_kvp, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _vp, _i64, _vp, _sz, _vp]
+lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
+lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
+
+_DT = {torch.float32: SGD_F32, torch.bfloat16: SGD_BF16, torch.int8: SGD_I8}
+
+
+class SgdError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise SgdError(f"{what}: {lib.sgd_error_string(rc).decode()} ({rc})")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def n_parts(lengths: Sequence[int]) -> int:
+    """Scheme-A K partitions over all sequences: sum_b ceil(L_b / 64) (a buffer size)."""
+    return int(sum((int(L) + PARTITION - 1) // PARTITION for L in lengths))
+
+
+def kept_total(lengths: Sequence[int], keep_num: int, keep_den: int) -> int:
+    """Size of the kept-index buffer per KV head: sum_b clamp(ceil(L_b*num/den), 1, L_b)."""
+    return int(sum(max(1, min(int(L), -(-int(L) * keep_num // keep_den))) for L in lengths))
+
+
+def _kv(k, v, cu_seqlens, k_scale=None, v_scale=None, scheme=SCHEME_A, parts=0) -> SgdKv:
+    if k.dim() != 3 or k.shape != v.shape or k.dtype != v.dtype:
+        raise ValueError("k and v must both be [Hkv, T, D] of one dtype")
+    if k.dtype not in _DT:
+        raise ValueError(f"unsupported cache dtype {k.dtype}")
+    if not (k.is_contiguous() and v.is_contiguous() and cu_seqlens.is_contiguous()):
+        raise ValueError("k, v and cu_seqlens must be contiguous")
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    Hkv, T, D = k.shape
+    return SgdKv(_DT[k.dtype], cu_seqlens.numel() - 1, Hkv, D, T, cu_seqlens.data_ptr(), k.data_ptr(),
+                 v.data_ptr(), scheme, None if k_scale is None else k_scale.data_ptr(),
+                 None if v_scale is None else v_scale.data_ptr(), int(parts))
+
+
+def workspace_size(op: int, kv: SgdKv, G: int = 1, schedule: int = 0, n_splits: int = 0) -> int:
+    n = lib.sgd_workspace_size(op, ctypes.byref(kv), G, schedule, n_splits)
+    if n == 0:
+        raise SgdError("sgd_workspace_size rejected the arguments")
+    return int(n)
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise SgdError("workspace too small")
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Device status bits recorded by the last call that used ``workspace`` (synchronises)."""
+    st = ctypes.c_int32(0)
+    _check(lib.sgd_workspace_status(_ptr(workspace), ctypes.byref(st), _stream(stream)), "sgd_workspace_status")
+    return int(st.value)
+
+
+def quantize_kv(k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, scheme: str,
+                lengths: Sequence[int], out=None, workspace=None, stream=None):
+    """INT8 codes and scales of a bf16/f32 cache.  Returns (k_codes, v_codes, k_scale, v_scale, ws).
+
+    ``lengths`` are the host copies of the sequence lengths (buffer sizes only).
+    """
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    Hkv, T, D = k.shape
+    parts = n_parts(lengths) if sch == SCHEME_A else 0
+    kv = _kv(k, v, cu_seqlens)
+    if out is None:
+        kc = torch.empty((Hkv, T, D), dtype=torch.int8, device=k.device)
+        vc = torch.empty_like(kc)
+        ks = torch.empty((Hkv, parts) if sch == SCHEME_A else (1,), dtype=torch.float32, device=k.device)
+        vs = torch.empty(1, dtype=torch.float32, device=k.device)
+    else:
+        kc, vc, ks, vs = out
+    ws = _workspace(workspace_size(OP_QUANTIZE, kv), k.device, workspace)
+    _check(lib.sgd_quantize_kv(ctypes.byref(kv), sch, parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(ws),
+                               ws.numel(), _stream(stream)), "sgd_quantize_kv")
+    return kc, vc, ks, vs, ws
+
+
+def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+               beta: float, eps: float, keep_num: int, keep_den: int, lengths: Sequence[int],
+               out=None, workspace=None, stream=None):
+    """Kept token positions per (sequence, KV head).  Returns (idx [Hkv, Kt], cu_kept [B+1], ws)."""
+    Hkv = k.shape[0]
+    Kt = kept_total(lengths, keep_num, keep_den)
+    kv = _kv(k, v, cu_seqlens)
+    if out is None:
+        idx = torch.empty((Hkv, Kt), dtype=torch.int32, device=k.device)
+        cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
+    else:
+        idx, cu_kept = out
+    ws = _workspace(workspace_size(OP_OAM_SELECT, kv, G), k.device, workspace)
+    _check(lib.sgd_oam_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, _ptr(idx),
+                              _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)), "sgd_oam_select")
+    return idx, cu_kept, ws
+
+
+def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                k_scale=None, v_scale=None, scheme: str = "A", n_parts_: int = 0,
+                idx=None, cu_kept=None, kept_total_: int = 0, schedule: int = 0, n_splits: int = 0,
+                out=None, workspace=None, stream=None):
+    """Attention output and log-sum-exp per query head.  Returns (out [B,Hq,D] f32, lse [B,Hq] f32, ws)."""
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, sch, n_parts_)
+    B = cu_seqlens.numel() - 1
+    Hq = k.shape[0] * G
+    D = k.shape[2]
+    if out is None:
+        o = torch.empty((B, Hq, D), dtype=torch.float32, device=k.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=k.device)
+    else:
+        o, lse = out
+    ws = _workspace(workspace_size(OP_DECODE, kv, G, schedule, n_splits), k.device, workspace)
+    _check(lib.sgd_decode_attn(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
+                               int(kept_total_), schedule, n_splits, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                               _stream(stream)), "sgd_decode_attn")
+    return o, lse, ws
+
+
+def decode_num_ctas(k, v, cu_seqlens, G: int, indexed: bool = False, schedule: int = 0, n_splits: int = 0) -> int:
+    kv = _kv(k, v, cu_seqlens)
+    n = lib.sgd_decode_num_ctas(ctypes.byref(kv), G, ctypes.c_void_p(1) if indexed else None, schedule, n_splits)
+    _check(min(n, 0), "sgd_decode_num_ctas")
+    return int(n)
+
+
+def plan_segments(cu: torch.Tensor, B: int, Hkv: int, n_req: int, min_chunk: int, mode: int, stream=None):
+    """The split-KV partition: int32 [n_segs, 4] rows (cta, row, start, length), and the CTA count."""
+    R = B * Hkv
+    cap = n_req + R + 8
+    segs = torch.full((cap, 4), -1, dtype=torch.int32, device=cu.device)
+    nseg = torch.zeros(2, dtype=torch.int32, device=cu.device)
+    nbytes = 256 + 4 * 256 + 8 * (R + n_req + B + 8) + 4096
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=cu.device)
+    _check(lib.sgd_plan_segments(_ptr(cu), B, Hkv, n_req, min_chunk, mode, _ptr(segs), cap, _ptr(nseg), _ptr(ws),
+                                 ws.numel(), _stream(stream)), "sgd_plan_segments")
+    n, ncta = (int(x) for x in nseg.tolist())
+    return segs[:n].cpu(), ncta

@@ -1,0 +1,347 @@
+// api.cu -- the C ABI of libsgd.so (declared and documented in include/sgd.h).
+//
+// Each entry point validates its arguments on the host, lays out the caller's
+// workspace, and enqueues its kernels on the caller's stream.  Nothing here
+// allocates, frees or synchronises (except sgd_workspace_status, which reads the
+// device status word).
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+
+namespace sgd {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kAutoMinChunk = 256;  // smallest CTA range when the split is automatic
+
+struct DevInfo {
+    int ok = -1;  // -1 unknown, 0 not sm_100, 1 ok
+    int sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+int current_device(DevInfo **info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SGD_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo &d = g_dev[dev];
+    if (d.ok < 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return SGD_ERR_CUDA;
+        d.ok = (major == 10 && minor == 0) ? 1 : 0;
+        d.sms = sms;
+    }
+    *info = &d;
+    return d.ok ? SGD_OK : SGD_ERR_DEVICE;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_kv(const sgd_kv *kv) {
+    if (!kv || !kv->cu_seqlens || !kv->k || !kv->v) return SGD_ERR_NULL;
+    if (kv->B < 1 || kv->Hkv < 1 || kv->T < 1) return SGD_ERR_SHAPE;
+    if (kv->D != 64 && kv->D != 128) return SGD_ERR_SHAPE;
+    if ((int64_t)kv->Hkv * kv->T >= (int64_t(1) << 31)) return SGD_ERR_SHAPE;
+    if ((int64_t)kv->B * kv->Hkv >= (int64_t(1) << 24)) return SGD_ERR_SHAPE;
+    if (kv->dtype != SGD_F32 && kv->dtype != SGD_BF16 && kv->dtype != SGD_I8) return SGD_ERR_DTYPE;
+    if (!aligned16(kv->k) || !aligned16(kv->v)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(kv->cu_seqlens) & 3u) != 0) return SGD_ERR_ALIGN;
+    return SGD_OK;
+}
+
+// workspace layout
+struct Layout {
+    size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, seq_part0 = 0;
+    size_t o_part = 0, lse_part = 0, scores = 0, total = 0;
+};
+
+size_t take(size_t &off, size_t bytes) {
+    const size_t at = off;
+    off += (bytes + 255) / 256 * 256;
+    return at;
+}
+
+Layout layout(int op, int B, int Hkv, int G, int D, int64_t T, int n_req) {
+    Layout L;
+    size_t off = sizeof(WsHeader);
+    const int64_t R = (int64_t)B * Hkv;
+    L.seq_part0 = take(off, (size_t)(B + 1) * 4);
+    if (op != SGD_OP_QUANTIZE) {
+        L.row_pos = take(off, (size_t)(R + 1) * 4);
+        L.row_slot0 = take(off, (size_t)(R + 1) * 4);
+        L.cta_begin = take(off, (size_t)(n_req + 1) * 4);
+        L.cta_slot0 = take(off, (size_t)(n_req + 1) * 4);
+    }
+    if (op == SGD_OP_DECODE) {
+        const int64_t slots = (int64_t)n_req + R;
+        L.o_part = take(off, (size_t)slots * G * D * 4);
+        L.lse_part = take(off, (size_t)slots * G * 4);
+    }
+    if (op == SGD_OP_OAM_SELECT) L.scores = take(off, (size_t)Hkv * T * 4);
+    L.total = off;
+    return L;
+}
+
+PlanView plan_view(uint8_t *ws, const Layout &L) {
+    PlanView pv;
+    pv.row_pos = reinterpret_cast<int32_t *>(ws + L.row_pos);
+    pv.row_slot0 = reinterpret_cast<int32_t *>(ws + L.row_slot0);
+    pv.cta_begin = reinterpret_cast<int32_t *>(ws + L.cta_begin);
+    pv.cta_slot0 = reinterpret_cast<int32_t *>(ws + L.cta_slot0);
+    pv.seq_part0 = reinterpret_cast<int32_t *>(ws + L.seq_part0);
+    return pv;
+}
+
+// CTAs requested from the partition for a decode / score launch.
+int decode_n_req(const DevInfo &dev, const sgd_kv *kv, sgd_dtype q_dtype, int G, bool indexed, bool score,
+                 int schedule, int n_splits, int *n_req) {
+    if (schedule == 1 && !score) {
+        *n_req = kv->B * kv->Hkv;
+        return SGD_OK;
+    }
+    if (schedule != 0) return SGD_ERR_ARG;
+    if (n_splits > 0 && !score) {
+        *n_req = n_splits;
+        return SGD_OK;
+    }
+    if (n_splits < 0) return SGD_ERR_ARG;
+    const int per = decode_ctas_per_sm(kv->dtype, q_dtype, kv->D, G, indexed, score);
+    if (per < 1) return SGD_ERR_CUDA;
+    *n_req = dev.sms * per;
+    return SGD_OK;
+}
+
+cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+}  // namespace sgd
+
+using namespace sgd;
+
+extern "C" {
+
+int sgd_version(void) { return (1 << 16) | 0; }
+
+const char *sgd_error_string(int code) {
+    switch (code) {
+        case SGD_OK: return "ok";
+        case SGD_ERR_NULL: return "a required pointer is NULL";
+        case SGD_ERR_SHAPE: return "a size is out of range (B, Hkv, T, D in {64,128}, G in [1,16], Hkv*T < 2^31)";
+        case SGD_ERR_DTYPE: return "unsupported dtype or scheme";
+        case SGD_ERR_ALIGN: return "an array is not 16-byte aligned";
+        case SGD_ERR_WORKSPACE: return "workspace smaller than sgd_workspace_size";
+        case SGD_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+        case SGD_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+        case SGD_ERR_ARG: return "invalid argument";
+        default: return "unknown status";
+    }
+}
+
+size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_splits) {
+    if (check_kv(kv) != SGD_OK) return 0;
+    if (op == SGD_OP_QUANTIZE) return layout(op, kv->B, kv->Hkv, 0, kv->D, kv->T, 0).total;
+    if (G < 1 || G > 16) return 0;
+    DevInfo *dev;
+    if (current_device(&dev) != SGD_OK) return 0;
+    int n_req = 0;
+    const bool score = op == SGD_OP_OAM_SELECT;
+    if (op != SGD_OP_DECODE && !score) return 0;
+    // indexed or not does not change the count
+    if (decode_n_req(*dev, kv, SGD_BF16, G, false, score, score ? 0 : schedule, score ? 0 : n_splits, &n_req) !=
+        SGD_OK)
+        return 0;
+    int n_req_f32 = 0;  // an F32 query may pick another kernel family
+    if (decode_n_req(*dev, kv, SGD_F32, G, false, score, score ? 0 : schedule, score ? 0 : n_splits, &n_req_f32) ==
+        SGD_OK)
+        n_req = std::max(n_req, n_req_f32);
+    return layout(op, kv->B, kv->Hkv, G, kv->D, kv->T, n_req).total;
+}
+
+int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedule, int n_splits) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    rc = decode_n_req(*dev, kv, SGD_BF16, G, idx != nullptr, false, schedule, n_splits, &n_req);
+    return rc == SGD_OK ? n_req : rc;
+}
+
+int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes, int8_t *v_codes,
+                    float *k_scale, float *v_scale, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_kv(in);
+    if (rc != SGD_OK) return rc;
+    if (!k_codes || !v_codes || !k_scale || !v_scale || !workspace) return SGD_ERR_NULL;
+    if (in->dtype != SGD_BF16 && in->dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (scheme != SGD_SCHEME_A && scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+    if (scheme == SGD_SCHEME_A && (n_parts < in->B || n_parts > in->T / SGD_PARTITION + in->B)) return SGD_ERR_SHAPE;
+    if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u)) return SGD_ERR_ALIGN;
+    const Layout L = layout(SGD_OP_QUANTIZE, in->B, in->Hkv, 0, in->D, in->T, 0);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int e = launch_quantize(in->k, in->v, in->dtype, in->cu_seqlens, in->B, in->Hkv, in->D, in->T, scheme,
+                                  n_parts, k_codes, v_codes, k_scale, v_scale, reinterpret_cast<WsHeader *>(ws),
+                                  reinterpret_cast<int32_t *>(ws + L.seq_part0), dev->sms, as_stream(stream));
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps, int keep_num,
+                   int keep_den, int32_t *idx, int32_t *cu_kept, int64_t kept_total, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    if (!q || !idx || !cu_kept || !workspace) return SGD_ERR_NULL;
+    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
+    if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
+    if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
+    if (!aligned16(q) || !aligned16(workspace)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u)) return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    launch_plan(kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, kAutoMinChunk, 0, pv, hdr, s);
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.q_f32 = q_dtype == SGD_F32;
+    a.cu_seq = kv->cu_seqlens;
+    a.k = kv->k;
+    a.v = kv->v;
+    a.B = kv->B;
+    a.Hkv = kv->Hkv;
+    a.G = G;
+    a.D = kv->D;
+    a.T = kv->T;
+    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
+    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
+    a.beta = beta;
+    a.eps = eps;
+    a.scores = reinterpret_cast<float *>(ws + L.scores);
+    a.plan = pv;
+    a.status = &hdr->status;
+    int e = launch_decode(a, kv->dtype, q_dtype, false, true, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
+                    &hdr->status, s);
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, const int32_t *idx,
+                    const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, float *out, float *lse,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
+    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (q_dtype == SGD_F32 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
+    const bool indexed = idx != nullptr;
+    if (indexed != (cu_kept != nullptr)) return SGD_ERR_NULL;
+    if (indexed && (kept_total < kv->B || kept_total > kv->T)) return SGD_ERR_SHAPE;
+    if (kv->dtype == SGD_I8) {
+        if (!kv->k_scale || !kv->v_scale) return SGD_ERR_NULL;
+        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
+            return SGD_ERR_SHAPE;
+    }
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (indexed && (reinterpret_cast<uintptr_t>(idx) & 3u)))
+        return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    if ((rc = decode_n_req(*dev, kv, q_dtype, G, indexed, false, schedule, n_splits, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_DECODE, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    const int min_chunk = (n_splits > 0 || schedule == 1) ? kGranule : kAutoMinChunk;
+    launch_plan(indexed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
+                hdr, s);
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.q_f32 = q_dtype == SGD_F32;
+    a.cu_seq = kv->cu_seqlens;
+    a.cu_kept = cu_kept;
+    a.idx = idx;
+    a.k = kv->k;
+    a.v = kv->v;
+    a.k_scale = kv->k_scale;
+    a.v_scale = kv->v_scale;
+    a.scheme = kv->scheme;
+    a.B = kv->B;
+    a.Hkv = kv->Hkv;
+    a.G = G;
+    a.D = kv->D;
+    a.T = kv->T;
+    a.Kt = indexed ? kept_total : 0;
+    a.n_parts = kv->dtype == SGD_I8 && kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
+    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
+    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
+    a.plan = pv;
+    a.o_part = reinterpret_cast<float *>(ws + L.o_part);
+    a.lse_part = reinterpret_cast<float *>(ws + L.lse_part);
+    a.status = &hdr->status;
+    int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    e = launch_merge(a, out, lse, s);
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode, int32_t *segs,
+                      int64_t max_segs, int32_t *n_segs, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!cu || !segs || !n_segs || !workspace) return SGD_ERR_NULL;
+    if (B < 1 || Hkv < 1 || (int64_t)B * Hkv >= (int64_t(1) << 24)) return SGD_ERR_SHAPE;
+    if (mode != 0 && mode != 1) return SGD_ERR_ARG;
+    if (mode == 1) n_req = B * Hkv;
+    if (n_req < 1 || min_chunk < kGranule || min_chunk % kGranule != 0 || max_segs < 0) return SGD_ERR_ARG;
+    if (!aligned16(workspace)) return SGD_ERR_ALIGN;
+    const Layout L = layout(SGD_OP_DECODE, B, Hkv, 1, 64, 1, n_req);
+    if (workspace_bytes < L.o_part) return SGD_ERR_WORKSPACE;
+    DevInfo *dev;
+    int rc = current_device(&dev);
+    if (rc != SGD_OK) return rc;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    launch_plan(cu, cu, B, Hkv, n_req, min_chunk, mode, pv, hdr, s);
+    launch_plan_dump(pv, cu, B, Hkv, n_req, segs, max_segs, n_segs, hdr, s);
+    return cudaGetLastError() == cudaSuccess ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_workspace_status(const void *workspace, int32_t *status, void *stream) {
+    if (!workspace || !status) return SGD_ERR_NULL;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(status, static_cast<const uint8_t *>(workspace) + SGD_WS_STATUS_OFFSET, sizeof(int32_t),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SGD_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? SGD_OK : SGD_ERR_CUDA;
+}
+
+}  // extern "C"

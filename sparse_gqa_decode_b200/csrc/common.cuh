@@ -1,0 +1,214 @@
+// common.cuh -- device helpers shared by the sm_100a kernels of libsgd.so:
+// inline-PTX wrappers for mbarriers, TMA (cp.async.bulk.tensor), cp.async,
+// warp-level MMA fragments, and the internal launch interface.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sgd.h"
+
+namespace sgd {
+
+// ------------------------------------------------------------------------------------------
+// workspace header (first 256 bytes of every workspace)
+// ------------------------------------------------------------------------------------------
+struct WsHeader {
+    int32_t status;       // SGD_STATUS_* bits, offset SGD_WS_STATUS_OFFSET
+    int32_t pad0;
+    uint32_t amax_bits[2];  // quantize: running max |K|, max |V| as float bits
+    int64_t plan_W;       // plan: padded stream length
+    int64_t plan_S;       // plan: CTA range length
+    int32_t plan_ncta;    // plan: CTAs with work
+    int32_t plan_nslots;  // plan: segments (partial results)
+    int32_t n_parts;      // quantize/decode: partitions counted on the device
+    int32_t pad1[53];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr int kGranule = 16;      // plan granularity (tokens)
+constexpr int kPart = SGD_PARTITION;
+constexpr long long kWaitLimit = 1 << 22;  // bounded mbarrier polls before giving up
+
+__host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity.  Every wait is bounded: after kWaitLimit polls
+// the wait records SGD_STATUS_WAIT_TIMEOUT, raises the CTA's abort flag and returns false.
+// Once the flag is up every later wait of the CTA returns false at once, so all warps still
+// run through the same (named) barriers and the kernel ends promptly instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
+                                          volatile int32_t *abort_flag) {
+    if (*abort_flag) return false;
+    for (long long i = 0; i < kWaitLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023) == 1023 && *abort_flag) return false;
+    }
+    *abort_flag = 1;
+    atomicOr(status, SGD_STATUS_WAIT_TIMEOUT);
+    return false;
+}
+
+// 2-D tiled TMA load of one box into shared memory, completing on `bar` (tx bytes).
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only), and its completion signal.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+// D += A(16x16, row) * B(16x8, col), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Four signed bytes -> two f16x2 (exact).  Each byte b is biased to u = b ^ 0x80 = b + 128,
+// placed under the f16 exponent of 1024 (bits 0x64uu = 1024 + u, exact because f16 has a
+// 10-bit mantissa), and 1152 = 1024 + 128 is subtracted.
+__device__ __forceinline__ void s8x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    lo = __byte_perm(u, 0x64646464u, 0x4140);  // bytes [u0, 0x64, u1, 0x64]
+    hi = __byte_perm(u, 0x64646464u, 0x4342);  // bytes [u2, 0x64, u3, 0x64]
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    __half2 l = __hsub2(*reinterpret_cast<__half2 *>(&lo), bias);
+    __half2 h = __hsub2(*reinterpret_cast<__half2 *>(&hi), bias);
+    lo = *reinterpret_cast<uint32_t *>(&l);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Two already-biased bytes (u = b ^ 0x80) sitting in byte lanes `sel` of (a, b) -> f16x2.
+__device__ __forceinline__ uint32_t biased_pair_to_f16x2(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t x = __byte_perm(a, b, sel);                 // bytes [ua, ub, *, *] in lanes 0, 1
+    x = __byte_perm(x, 0x64646464u, 0x4140);             // [ua, 0x64, ub, 0x64]
+    const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+    __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&x), bias);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ------------------------------------------------------------------------------------------
+// internal launch interface (host side)
+// ------------------------------------------------------------------------------------------
+struct PlanView {  // device arrays of a plan inside a workspace
+    int32_t *row_pos;    // [R+1] padded stream position of each row
+    int32_t *row_slot0;  // [R+1] first partial slot of each row
+    int32_t *cta_begin;  // [N+1] stream position where each CTA starts
+    int32_t *cta_slot0;  // [N+1] first partial slot of each CTA
+    int32_t *seq_part0;  // [B+1] scheme-A partition offset of each sequence
+};
+
+}  // namespace sgd

@@ -1,0 +1,862 @@
+// decode.cu -- split-KV flash-decoding kernels, the OAM score kernel that shares their
+// pipeline, and the exact log-sum-exp merge.
+//
+// Sources: "优化稀疏注意力中的令牌丢弃机制" (Optimizing token dropping in sparse
+// attention) section 5 (split the KV of a row across CTAs; each chunk reports a
+// partial result that an online-softmax reduction combines) and section 3 (OAM
+// score); "注意力优化（Attention Optimization）" core principle (running max m and
+// sum l with a rescaled accumulator, the FlashAttention recurrence); "共同设计 AI
+// 模型注意力..." (Co-designing AI model attention), decode equations 5-7: decode
+// reads every KV byte once at about 2G flops per byte, far below the tensor-core
+// ridge, so the kernel is built around streaming HBM at full rate.
+//
+// Tensor-core decode kernel (kv BF16 with D in {64,128}, or INT8 codes with D = 128):
+//   * one producer warp streams the CTA's token range through a 3-stage ring of
+//     shared-memory tiles (K and V, ROWS tokens each).  Dense rows are fetched with
+//     2-D TMA boxes (cp.async.bulk.tensor, 128-byte swizzle, L2 evict-first);
+//     kept-index rows are gathered with 16-byte cp.async into the same swizzled
+//     layout.  Full/empty mbarriers hand stages between producer and consumers; every
+//     wait is bounded.
+//   * four consumer warps each own 16-token sub-tiles.  QK: S^T[token, g] with
+//     m16n8k16 MMAs (tokens as M, the G heads of the group as N, D as K); the fp32
+//     logits get the dequantisation scales and 1/sqrt(D); online softmax in the log2
+//     domain; P is transposed in registers (movmatrix) into the B operand of the
+//     PV MMA O^T[d, g] += V^T[d, token] P^T[token, g].  INT8 codes are widened to f16
+//     in registers (exact), Q is pre-scaled by a power of two into f16 range.
+//   * rows of a 16-token MMA tile are permuted (0,5,2,7,4,1,6,3) so that the
+//     swizzled shared-memory reads of both K and V are bank-conflict free.
+//   * at the end of each (row, token range) segment the four warps' (m, l, O) are
+//     combined through shared memory into one partial (o_c, lse_c).
+// CUDA-core kernel: every other dtype/shape (F32 cache, INT8 with D = 64, ...).
+#include <math.h>
+
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "plan.cuh"
+
+namespace sgd {
+
+constexpr float kLn2 = 0.69314718055994530942f;
+
+__device__ __forceinline__ int mma_row_perm(int i) { return (i & 1) ? (i ^ 4) : i; }
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D_, int GT_, bool I8_, bool IDX_, int MODE_>
+struct MmaCfg {
+    static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
+    static constexpr bool I8 = I8_, IDX = IDX_;
+    static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score
+    static constexpr int NW = 4;        // consumer warps
+    static constexpr int SUB = I8 ? 2 : 1;  // 16-token sub-tiles per consumer warp per stage
+    static constexpr int ROWS = NW * 16 * SUB;
+    static constexpr int EB = I8 ? 1 : 2;
+    static constexpr int ROWB = D * EB;
+    static constexpr int BOXES = ROWB / 128;
+    static constexpr int BOX_ELEMS = 128 / EB;
+    static constexpr int TILE = ROWS * ROWB;  // bytes of one tensor per stage
+    static constexpr int STAGES = 3;
+    static constexpr int KB = D / 16;
+    static constexpr int THREADS = (NW + 1) * 32;
+    static constexpr int SMEM_STAGES = STAGES * 2 * TILE;
+    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16;
+    static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
+    static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
+    static_assert(!(I8 && MODE == 1), "scores read the unquantised cache");
+};
+
+// ------------------------------------------------------------------------------------------
+// producer warp
+// ------------------------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUtensorMap *tmV, const DecodeArgs &a,
+                                             uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                             volatile int32_t *abort_flag, const int32_t *cu_rows, int cta,
+                                             int lane) {
+    if (!C::IDX && lane != 0) return;
+    uint64_t pol = 0;
+    if constexpr (!C::IDX) {
+        prefetch_tensormap(tmK);
+        prefetch_tensormap(tmV);
+        pol = l2_evict_first_policy();
+    }
+    SegCursor cur;
+    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    int stage = 0;
+    uint32_t phase = 0;
+    int row, slot;
+    int32_t t0, t1;
+    while (cur.next(row, t0, t1, slot)) {
+        const int b = row % a.B, kvh = row / a.B;
+        const int64_t seq0 = (int64_t)kvh * a.T + a.cu_seq[b];
+        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
+        const int32_t *ip = nullptr;
+        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
+        for (int32_t t = t0; t < t1; t += C::ROWS) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
+            uint8_t *sk = smem + stage * 2 * C::TILE;
+            uint8_t *sv = sk + C::TILE;
+            if constexpr (!C::IDX) {
+                mbar_arrive_expect_tx(&full[stage], 2 * C::TILE);
+                const int y = (int)(seq0 + t);
+#pragma unroll
+                for (int bx = 0; bx < C::BOXES; ++bx) {
+                    tma_load_2d(sk + bx * C::ROWS * 128, tmK, &full[stage], bx * C::BOX_ELEMS, y, pol);
+                    tma_load_2d(sv + bx * C::ROWS * 128, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
+                }
+            } else if (Lb >= 1) {
+                for (int rr = lane; rr < C::ROWS; rr += 32) {
+                    const int32_t j = min(t + rr, t1 - 1);  // rows past the segment repeat its last token
+                    int32_t tok = __ldg(ip + j);
+                    if (tok < 0 || tok >= Lb) {
+                        atomicOr(a.status, SGD_STATUS_BAD_INDEX);
+                        tok = min(max(tok, 0), Lb - 1);
+                    }
+                    const uint8_t *gk = static_cast<const uint8_t *>(a.k) + (seq0 + tok) * C::ROWB;
+                    const uint8_t *gv = static_cast<const uint8_t *>(a.v) + (seq0 + tok) * C::ROWB;
+#pragma unroll
+                    for (int bx = 0; bx < C::BOXES; ++bx)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int off = bx * C::ROWS * 128 + rr * 128 + ((c ^ (rr & 7)) << 4);
+                            cp_async_16(sk + off, gk + bx * 128 + c * 16);
+                            cp_async_16(sv + off, gv + bx * 128 + c * 16);
+                        }
+                }
+                cp_async_mbar_arrive_noinc(&full[stage]);
+            } else {
+                // rows of an empty sequence (inconsistent kept counts): nothing to fetch
+                if (lane == 0) atomicOr(a.status, SGD_STATUS_SIZE_MISMATCH);
+                mbar_arrive(&full[stage]);
+            }
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// consumer helpers
+// ------------------------------------------------------------------------------------------
+// Q of one KV group as MMA B fragments (k <-> d order matching the K fragments) and the
+// per-column logit factor (log2 units; INT8 also undoes the power-of-two Q pre-scale).
+template <class C>
+__device__ __forceinline__ void load_q_frags(const DecodeArgs &a, int b, int kvh, int g4, int t4,
+                                             uint32_t (&qf)[C::GT][C::KB][2], float (&colf)[C::GT][2]) {
+    const int Hq = a.Hkv * a.G;
+#pragma unroll
+    for (int gt = 0; gt < C::GT; ++gt) {
+        const int g = 8 * gt + g4;
+        const bool live = g < a.G;
+        const __nv_bfloat16 *qrow =
+            static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)b * Hq + kvh * a.G + (live ? g : 0)) * C::D;
+        if constexpr (!C::I8) {
+#pragma unroll
+            for (int h = 0; h < C::KB / 2; ++h) {
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (live) v = __ldg(reinterpret_cast<const uint4 *>(qrow) + (t4 + 4 * h));
+                qf[gt][2 * h][0] = v.x;
+                qf[gt][2 * h][1] = v.y;
+                qf[gt][2 * h + 1][0] = v.z;
+                qf[gt][2 * h + 1][1] = v.w;
+            }
+            colf[gt][0] = colf[gt][1] = a.sm_scale_log2;
+        } else {
+            float x[C::KB / 4][16];
+            float mx = 0.f;
+#pragma unroll
+            for (int h = 0; h < C::KB / 4; ++h) {
+                uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+                if (live) {
+                    const uint4 *p = reinterpret_cast<const uint4 *>(qrow + 16 * (t4 + 4 * h));
+                    v0 = __ldg(p);
+                    v1 = __ldg(p + 1);
+                }
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    x[h][2 * i] = __uint_as_float(w[i] << 16);
+                    x[h][2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+                    mx = fmaxf(mx, fmaxf(fabsf(x[h][2 * i]), fabsf(x[h][2 * i + 1])));
+                }
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            int ex = 0;
+            if (mx > 0.f) frexpf(mx, &ex);
+            const int sh = 14 - ex;  // max |q| * 2^sh < 2^14: inside f16 range
+#pragma unroll
+            for (int h = 0; h < C::KB / 4; ++h)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    qf[gt][4 * h + j][0] = pack_f16(ldexpf(x[h][4 * j], sh), ldexpf(x[h][4 * j + 1], sh));
+                    qf[gt][4 * h + j][1] = pack_f16(ldexpf(x[h][4 * j + 2], sh), ldexpf(x[h][4 * j + 3], sh));
+                }
+            // column factor of this thread's columns g0 = 8gt + 2t4 and g0 + 1: their rows live on
+            // lanes 4 * (2t4) and 4 * (2t4 + 1)
+            const float inv = ldexpf(1.f, -sh);
+            const float i0 = __shfl_sync(0xffffffffu, inv, 4 * (2 * t4));
+            const float i1 = __shfl_sync(0xffffffffu, inv, 4 * (2 * t4 + 1));
+            float f = a.sm_scale_log2;
+            if (a.scheme == SGD_SCHEME_B) f *= __ldg(a.k_scale);
+            colf[gt][0] = f * i0;
+            colf[gt][1] = f * i1;
+        }
+    }
+}
+
+// S^T = K_tile(16 x D) * Q^T(D x NG) for this warp's sub-tile.
+template <class C>
+__device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t4,
+                                           const uint32_t (&qf)[C::GT][C::KB][2], float (&sacc)[C::GT][4]) {
+#pragma unroll
+    for (int gt = 0; gt < C::GT; ++gt) sacc[gt][0] = sacc[gt][1] = sacc[gt][2] = sacc[gt][3] = 0.f;
+    const int rA = rb + pA, rB = rA + 8;
+    if constexpr (!C::I8) {
+#pragma unroll
+        for (int h = 0; h < C::KB / 2; ++h) {
+            const int c = t4 + 4 * h, bx = c >> 3, cc = c & 7;
+            const uint32_t base = kbase + bx * C::ROWS * 128 + ((cc ^ pA) << 4);
+            const uint4 ka = lds128(base + rA * 128), kb = lds128(base + rB * 128);
+#pragma unroll
+            for (int gt = 0; gt < C::GT; ++gt) {
+                mma_bf16(sacc[gt], ka.x, kb.x, ka.y, kb.y, qf[gt][2 * h][0], qf[gt][2 * h][1]);
+                mma_bf16(sacc[gt], ka.z, kb.z, ka.w, kb.w, qf[gt][2 * h + 1][0], qf[gt][2 * h + 1][1]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < C::KB / 4; ++h) {
+            const int c = t4 + 4 * h;
+            const uint32_t base = kbase + ((c ^ pA) << 4);
+            const uint4 ka = lds128(base + rA * 128), kb = lds128(base + rB * 128);
+            const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t a0, a1, a2, a3;
+                s8x4_to_f16x2x2(wa[j], a0, a2);
+                s8x4_to_f16x2x2(wb[j], a1, a3);
+#pragma unroll
+                for (int gt = 0; gt < C::GT; ++gt)
+                    mma_f16(sacc[gt], a0, a1, a2, a3, qf[gt][4 * h + j][0], qf[gt][4 * h + j][1]);
+            }
+        }
+    }
+}
+
+// O^T(D x NG) += V_tile^T(D x 16) * P^T(16 x NG)
+template <class C>
+__device__ __forceinline__ void pv_subtile(uint32_t vbase, int rb, int lane, const uint32_t (&pb)[C::GT][2],
+                                           float (&o)[C::GT][C::KB][4]) {
+    if constexpr (!C::I8) {
+        const int lrow = rb + mma_row_perm(lane & 7) + ((lane >> 4) << 3);
+        const int lhalf = (lane >> 3) & 1;
+        const int sw = lrow & 7;
+#pragma unroll
+        for (int mt = 0; mt < C::KB; ++mt) {
+            const int c = 2 * mt + lhalf, bx = c >> 3, cc = c & 7;
+            uint32_t va[4];
+            ldmatrix_x4_trans(va, vbase + bx * C::ROWS * 128 + lrow * 128 + ((cc ^ sw) << 4));
+#pragma unroll
+            for (int gt = 0; gt < C::GT; ++gt) mma_bf16(o[gt][mt], va[0], va[1], va[2], va[3], pb[gt][0], pb[gt][1]);
+        }
+    } else {
+        const int g4 = lane >> 2, t4 = lane & 3;
+        const int tA = rb + 2 * t4, tB = rb + ((2 * t4 + 1) ^ 4);
+        const uint32_t off = (uint32_t)(g4 ^ (tA & 7)) << 4, offB = (uint32_t)(g4 ^ (tB & 7)) << 4;
+        uint4 wA = lds128(vbase + tA * 128 + off), wA8 = lds128(vbase + (tA + 8) * 128 + off);
+        uint4 wB = lds128(vbase + tB * 128 + offB), wB8 = lds128(vbase + (tB + 8) * 128 + offB);
+        const uint32_t A[4] = {wA.x ^ 0x80808080u, wA.y ^ 0x80808080u, wA.z ^ 0x80808080u, wA.w ^ 0x80808080u};
+        const uint32_t Bv[4] = {wB.x ^ 0x80808080u, wB.y ^ 0x80808080u, wB.z ^ 0x80808080u, wB.w ^ 0x80808080u};
+        const uint32_t A8[4] = {wA8.x ^ 0x80808080u, wA8.y ^ 0x80808080u, wA8.z ^ 0x80808080u,
+                                wA8.w ^ 0x80808080u};
+        const uint32_t B8[4] = {wB8.x ^ 0x80808080u, wB8.y ^ 0x80808080u, wB8.z ^ 0x80808080u,
+                                wB8.w ^ 0x80808080u};
+#pragma unroll
+        for (int mt = 0; mt < C::KB; ++mt) {
+            const int w = mt >> 1;
+            const uint32_t slo = (mt & 1) ? 0x0062u : 0x0040u, shi = (mt & 1) ? 0x0073u : 0x0051u;
+            const uint32_t a0 = biased_pair_to_f16x2(A[w], Bv[w], slo);
+            const uint32_t a1 = biased_pair_to_f16x2(A[w], Bv[w], shi);
+            const uint32_t a2 = biased_pair_to_f16x2(A8[w], B8[w], slo);
+            const uint32_t a3 = biased_pair_to_f16x2(A8[w], B8[w], shi);
+#pragma unroll
+            for (int gt = 0; gt < C::GT; ++gt) mma_f16(o[gt][mt], a0, a1, a2, a3, pb[gt][0], pb[gt][1]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// the kernel
+// ------------------------------------------------------------------------------------------
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 2)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const DecodeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::SMEM_STAGES);
+    uint64_t *empty = full + C::STAGES;
+    float *ml = reinterpret_cast<float *>(empty + C::STAGES);  // [NW][NG][2]: m, l
+    volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(ml + C::NW * C::NG * 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], C::IDX ? 32u : 1u);
+            mbar_init(&empty[s], (uint32_t)C::NW);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int cta = blockIdx.x;
+    if (a.plan.cta_begin[cta] >= a.plan.cta_begin[cta + 1]) return;
+    const int32_t *cu_rows = C::IDX ? a.cu_kept : a.cu_seq;
+
+    if (warp == C::NW) {
+        mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, cu_rows, cta, lane);
+        return;
+    }
+
+    const int g4 = lane >> 2, t4 = lane & 3;
+    const int pA = mma_row_perm(g4);
+    SegCursor cur;
+    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    int stage = 0;
+    uint32_t phase = 0;
+    int row, slot;
+    int32_t t0, t1;
+    while (cur.next(row, t0, t1, slot)) {
+        const int b = row % a.B, kvh = row / a.B;
+        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
+        uint32_t qf[C::GT][C::KB][2];
+        float colf[C::GT][2];
+        load_q_frags<C>(a, b, kvh, g4, t4, qf, colf);
+        float m[C::GT][2], l[C::GT][2], o[C::GT][C::KB][4];
+#pragma unroll
+        for (int gt = 0; gt < C::GT; ++gt) {
+            m[gt][0] = m[gt][1] = -INFINITY;
+            l[gt][0] = l[gt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < C::KB; ++mt) o[gt][mt][0] = o[gt][mt][1] = o[gt][mt][2] = o[gt][mt][3] = 0.f;
+        }
+        const float *ksc = nullptr;
+        const int32_t *ip = nullptr;
+        if constexpr (C::I8) ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
+        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
+
+        for (int32_t t = t0; t < t1; t += C::ROWS) {
+            const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
+            uint8_t *sk = smem + stage * 2 * C::TILE;
+            uint8_t *sv = sk + C::TILE;
+            const uint32_t kbase = smem_u32(sk), vbase = smem_u32(sv);
+#pragma unroll
+            for (int s = 0; s < C::SUB; ++s) {
+                const int rb = 16 * (s * C::NW + warp);
+                const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
+                if (j0 >= t1 || !ready) continue;
+                float sacc[C::GT][4];
+                qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
+                const bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
+                if constexpr (C::MODE == 1) {
+                    // OAM score: max over the group's heads of the logit, plus beta * ln(|v| + eps)
+                    float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+                    for (int gt = 0; gt < C::GT; ++gt) {
+                        const int g0 = 8 * gt + 2 * t4;
+                        if (g0 < a.G) {
+                            mA = fmaxf(mA, sacc[gt][0]);
+                            mB = fmaxf(mB, sacc[gt][2]);
+                        }
+                        if (g0 + 1 < a.G) {
+                            mA = fmaxf(mA, sacc[gt][1]);
+                            mB = fmaxf(mB, sacc[gt][3]);
+                        }
+                    }
+                    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+                    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+                    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+                    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+                    const int rho = lane >> 1, half = lane & 1;
+                    const int vr = rb + rho;
+                    float ss = 0.f;
+                    constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
+#pragma unroll
+                    for (int i = 0; i < CPR / 2; ++i) {
+                        const int c = half * (CPR / 2) + i, bx = c >> 3, cc = c & 7;
+                        const uint4 w = lds128(vbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
+                            ss = fmaf(lo, lo, ss);
+                            ss = fmaf(hi, hi, ss);
+                        }
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    const int src = 4 * mma_row_perm(rho & 7);
+                    const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
+                    const float rmax = (rho < 8) ? rA : rB;
+                    const int32_t j = j0 + rho;
+                    if (half == 0 && j < t1) {
+                        float sc = rmax * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
+                        if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
+                        a.scores[(int64_t)kvh * a.T + a.cu_seq[b] + j] = sc;
+                    }
+                } else {
+                    // row (token) factors: scheme-A K scale of the token's 64-token partition
+                    float rfA = 1.f, rfB = 1.f;
+                    if constexpr (C::I8) {
+                        if (a.scheme == SGD_SCHEME_A) {
+                            if constexpr (!C::IDX) {
+                                rfA = rfB = __ldg(ksc + min(j0, Lb - 1) / kPart);
+                            } else {
+                                const int32_t tA = __ldg(ip + min(j0 + pA, t1 - 1));
+                                const int32_t tB = __ldg(ip + min(j0 + pA + 8, t1 - 1));
+                                rfA = __ldg(ksc + min(max(tA, 0), Lb - 1) / kPart);
+                                rfB = __ldg(ksc + min(max(tB, 0), Lb - 1) / kPart);
+                            }
+                        }
+                    }
+                    uint32_t pb[C::GT][2];
+#pragma unroll
+                    for (int gt = 0; gt < C::GT; ++gt) {
+                        const float z0 = vA ? sacc[gt][0] * rfA * colf[gt][0] : -INFINITY;
+                        const float z1 = vA ? sacc[gt][1] * rfA * colf[gt][1] : -INFINITY;
+                        const float z2 = vB ? sacc[gt][2] * rfB * colf[gt][0] : -INFINITY;
+                        const float z3 = vB ? sacc[gt][3] * rfB * colf[gt][1] : -INFINITY;
+                        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                        }
+                        if (mx0 > m[gt][0]) {
+                            const float al = exp2f(m[gt][0] - mx0);
+                            m[gt][0] = mx0;
+                            l[gt][0] *= al;
+#pragma unroll
+                            for (int mt = 0; mt < C::KB; ++mt) {
+                                o[gt][mt][0] *= al;
+                                o[gt][mt][2] *= al;
+                            }
+                        }
+                        if (mx1 > m[gt][1]) {
+                            const float al = exp2f(m[gt][1] - mx1);
+                            m[gt][1] = mx1;
+                            l[gt][1] *= al;
+#pragma unroll
+                            for (int mt = 0; mt < C::KB; ++mt) {
+                                o[gt][mt][1] *= al;
+                                o[gt][mt][3] *= al;
+                            }
+                        }
+                        const float mu0 = (m[gt][0] == -INFINITY) ? 0.f : m[gt][0];
+                        const float mu1 = (m[gt][1] == -INFINITY) ? 0.f : m[gt][1];
+                        const float p0 = exp2f(z0 - mu0), p2 = exp2f(z2 - mu0);
+                        const float p1 = exp2f(z1 - mu1), p3 = exp2f(z3 - mu1);
+                        l[gt][0] += p0 + p2;
+                        l[gt][1] += p1 + p3;
+                        const uint32_t r0 = C::I8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
+                        const uint32_t r1 = C::I8 ? pack_f16(p2, p3) : pack_bf16(p2, p3);
+                        pb[gt][0] = movmatrix_trans(r0);
+                        pb[gt][1] = movmatrix_trans(r1);
+                    }
+                    pv_subtile<C>(vbase, rb, lane, pb, o);
+                }
+            }
+            const bool last = (t + C::ROWS >= t1);
+            if (C::MODE == 0 && last) {
+                // ---- segment epilogue: combine the four warps' (m, l, O) in this stage's memory ----
+                named_barrier_sync(1, C::NW * 32);  // every warp is done reading the stage
+                float *eo = reinterpret_cast<float *>(sk);  // [NW][NG][D]
+#pragma unroll
+                for (int gt = 0; gt < C::GT; ++gt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) l[gt][j] += __shfl_xor_sync(0xffffffffu, l[gt][j], off);
+#pragma unroll
+                for (int gt = 0; gt < C::GT; ++gt) {
+                    const int g0 = 8 * gt + 2 * t4;
+                    float *e0 = eo + (warp * C::NG + g0) * C::D, *e1 = e0 + C::D;
+#pragma unroll
+                    for (int mt = 0; mt < C::KB; ++mt) {
+                        const int da = C::I8 ? 16 * g4 + 2 * mt : 16 * mt + g4;
+                        const int db = C::I8 ? da + 1 : da + 8;
+                        e0[da] = o[gt][mt][0];
+                        e1[da] = o[gt][mt][1];
+                        e0[db] = o[gt][mt][2];
+                        e1[db] = o[gt][mt][3];
+                    }
+                    if (g4 == 0) {
+                        ml[(warp * C::NG + g0) * 2 + 0] = m[gt][0];
+                        ml[(warp * C::NG + g0) * 2 + 1] = l[gt][0];
+                        ml[(warp * C::NG + g0 + 1) * 2 + 0] = m[gt][1];
+                        ml[(warp * C::NG + g0 + 1) * 2 + 1] = l[gt][1];
+                    }
+                }
+                named_barrier_sync(1, C::NW * 32);
+                const float vfac = C::I8 ? __ldg(a.v_scale) : 1.f;
+                for (int e = threadIdx.x; e < a.G * C::D; e += C::NW * 32) {
+                    const int g = e / C::D, d = e - g * C::D;
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int w = 0; w < C::NW; ++w) M = fmaxf(M, ml[(w * C::NG + g) * 2]);
+                    float L = 0.f, O = 0.f;
+                    if (M != -INFINITY) {
+#pragma unroll
+                        for (int w = 0; w < C::NW; ++w) {
+                            const float f = exp2f(ml[(w * C::NG + g) * 2] - M);
+                            L += f * ml[(w * C::NG + g) * 2 + 1];
+                            O += f * eo[(w * C::NG + g) * C::D + d];
+                        }
+                    }
+                    a.o_part[((int64_t)slot * a.G + g) * C::D + d] = (L > 0.f) ? O / L * vfac : 0.f;
+                    if (d == 0) a.lse_part[(int64_t)slot * a.G + g] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+                }
+                fence_proxy_async_shared();
+                named_barrier_sync(1, C::NW * 32);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// CUDA-core kernel: any dtype, D in {64, 128}, G <= 16
+// ------------------------------------------------------------------------------------------
+template <typename KT>
+__device__ __forceinline__ float load_elem(const void *p, int64_t i) {
+    if constexpr (sizeof(KT) == 4) return __ldg(static_cast<const float *>(p) + i);
+    else if constexpr (sizeof(KT) == 2)
+        return __bfloat162float(__ldg(static_cast<const __nv_bfloat16 *>(p) + i));
+    else return (float)__ldg(static_cast<const int8_t *>(p) + i);
+}
+
+template <int D, typename KT, bool IDX, int MODE>
+__global__ void __launch_bounds__(128) decode_generic_kernel(const DecodeArgs a) {
+    constexpr int NW = 4, PER = D / 32, MG = 16;
+    constexpr bool I8 = sizeof(KT) == 1;
+    __shared__ float eo[NW][MG][D];
+    __shared__ float eml[NW][MG][2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    if (a.plan.cta_begin[cta] >= a.plan.cta_begin[cta + 1]) return;
+    const int32_t *cu_rows = IDX ? a.cu_kept : a.cu_seq;
+    const int Hq = a.Hkv * a.G;
+    SegCursor cur;
+    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    int row, slot;
+    int32_t t0, t1;
+    while (cur.next(row, t0, t1, slot)) {
+        const int b = row % a.B, kvh = row / a.B;
+        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
+        const int64_t seq0 = (int64_t)kvh * a.T + a.cu_seq[b];
+        float q[MG][PER];
+#pragma unroll
+        for (int g = 0; g < MG; ++g)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                float x = 0.f;
+                if (g < a.G) {
+                    const int64_t qi = ((int64_t)b * Hq + kvh * a.G + g) * D + lane + 32 * i;
+                    x = a.q_f32 ? __ldg(static_cast<const float *>(a.q) + qi)
+                                : __bfloat162float(__ldg(static_cast<const __nv_bfloat16 *>(a.q) + qi));
+                }
+                q[g][i] = x;
+            }
+        float m[MG], l[MG], acc[MG][PER];
+#pragma unroll
+        for (int g = 0; g < MG; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) acc[g][i] = 0.f;
+        }
+        float kfac = 1.f, vfac = 1.f;
+        const float *ksc = nullptr;
+        if constexpr (I8) {
+            vfac = __ldg(a.v_scale);
+            if (a.scheme == SGD_SCHEME_B) kfac = __ldg(a.k_scale);
+            else ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
+        }
+        const int32_t *ip = IDX ? a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b] : nullptr;
+        for (int32_t j = t0 + warp; j < t1; j += NW) {
+            int32_t tok = j;
+            if constexpr (IDX) {
+                tok = __ldg(ip + j);
+                if (tok < 0 || tok >= Lb) {
+                    if (lane == 0) atomicOr(a.status, SGD_STATUS_BAD_INDEX);
+                    tok = min(max(tok, 0), Lb - 1);
+                }
+            }
+            const int64_t base = (seq0 + tok) * D;
+            float kf = kfac;
+            if (I8 && ksc) kf = __ldg(ksc + tok / kPart);
+            float kk[PER], vv[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                kk[i] = load_elem<KT>(a.k, base + lane + 32 * i) * kf;
+                vv[i] = load_elem<KT>(a.v, base + lane + 32 * i) * vfac;
+            }
+            if constexpr (MODE == 1) {
+                float best = -INFINITY, ss = 0.f;
+#pragma unroll
+                for (int g = 0; g < MG; ++g) {
+                    if (g < a.G) {
+                        float dot = 0.f;
+#pragma unroll
+                        for (int i = 0; i < PER; ++i) dot = fmaf(q[g][i], kk[i], dot);
+                        best = fmaxf(best, warp_sum(dot));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < PER; ++i) ss = fmaf(vv[i], vv[i], ss);
+                ss = warp_sum(ss);
+                if (lane == 0) {
+                    float sc = best * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
+                    if (sc == 0.f) sc = 0.f;
+                    a.scores[seq0 + j] = sc;
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < MG; ++g) {
+                    if (g < a.G) {
+                        float dot = 0.f;
+#pragma unroll
+                        for (int i = 0; i < PER; ++i) dot = fmaf(q[g][i], kk[i], dot);
+                        const float z = warp_sum(dot) * a.sm_scale_log2;
+                        if (z > m[g]) {
+                            const float al = exp2f(m[g] - z);
+                            m[g] = z;
+                            l[g] *= al;
+#pragma unroll
+                            for (int i = 0; i < PER; ++i) acc[g][i] *= al;
+                        }
+                        const float p = exp2f(z - m[g]);
+                        l[g] += p;
+#pragma unroll
+                        for (int i = 0; i < PER; ++i) acc[g][i] = fmaf(p, vv[i], acc[g][i]);
+                    }
+                }
+            }
+        }
+        if constexpr (MODE == 0) {
+#pragma unroll
+            for (int g = 0; g < MG; ++g) {
+#pragma unroll
+                for (int i = 0; i < PER; ++i) eo[warp][g][lane + 32 * i] = acc[g][i];
+                if (lane == 0) {
+                    eml[warp][g][0] = m[g];
+                    eml[warp][g][1] = l[g];
+                }
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < a.G * D; e += NW * 32) {
+                const int g = e / D, d = e - g * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) M = fmaxf(M, eml[w][g][0]);
+                float L = 0.f, O = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < NW; ++w) {
+                        const float f = exp2f(eml[w][g][0] - M);
+                        L += f * eml[w][g][1];
+                        O += f * eo[w][g][d];
+                    }
+                }
+                a.o_part[((int64_t)slot * a.G + g) * D + d] = (L > 0.f) ? O / L : 0.f;
+                if (d == 0) a.lse_part[(int64_t)slot * a.G + g] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// exact LSE merge: per (sequence, query head), lse = ln sum_c exp(lse_c),
+// out = sum_c exp(lse_c - lse) o_c
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, float *__restrict__ out,
+                                                    float *__restrict__ lse) {
+    const int r = blockIdx.x;
+    const int b = r % a.B, kvh = r / a.B;
+    const int s0 = a.plan.row_slot0[r], n = a.plan.row_slot0[r + 1] - s0;
+    const int Hq = a.Hkv * a.G;
+    for (int e = threadIdx.x; e < a.G * a.D; e += blockDim.x) {
+        const int g = e / a.D, d = e - g * a.D;
+        const int64_t oi = ((int64_t)b * Hq + kvh * a.G + g) * a.D + d;
+        float L, O;
+        if (n <= 0) {
+            L = -INFINITY;
+            O = 0.f;
+        } else if (n == 1) {
+            L = a.lse_part[(int64_t)s0 * a.G + g];
+            O = a.o_part[((int64_t)s0 * a.G + g) * a.D + d];
+        } else {
+            float M = -INFINITY;
+            for (int c = 0; c < n; ++c) M = fmaxf(M, a.lse_part[(int64_t)(s0 + c) * a.G + g]);
+            float S = 0.f;
+            for (int c = 0; c < n; ++c) S += expf(a.lse_part[(int64_t)(s0 + c) * a.G + g] - M);
+            L = M + logf(S);
+            O = 0.f;
+            for (int c = 0; c < n; ++c)
+                O += expf(a.lse_part[(int64_t)(s0 + c) * a.G + g] - L) * a.o_part[((int64_t)(s0 + c) * a.G + g) * a.D + d];
+        }
+        out[oi] = O;
+        if (d == 0) lse[(int64_t)b * Hq + kvh * a.G + g] = L;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D map over a [rows, D] row-major tensor with boxes of (box_elems x box_rows), 128B swizzle.
+static bool make_map(CUtensorMap *map, const void *base, bool i8, int D, int64_t rows, int box_elems, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int eb = i8 ? 1 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * eb};
+    cuuint32_t box[2] = {(cuuint32_t)box_elems, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <class C>
+static int ctas_per_sm_mma() {
+    auto k = decode_mma_kernel<C>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::THREADS, C::SMEM) != cudaSuccess) return 0;
+    return n;
+}
+
+template <class C>
+static int launch_mma(const DecodeArgs &a, int n_cta, cudaStream_t s) {
+    CUtensorMap mk, mv;
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    if constexpr (!C::IDX) {
+        const int64_t rows = (int64_t)a.Hkv * a.T;
+        if (!make_map(&mk, a.k, C::I8, C::D, rows, C::BOX_ELEMS, C::ROWS) ||
+            !make_map(&mv, a.v, C::I8, C::D, rows, C::BOX_ELEMS, C::ROWS))
+            return (int)cudaErrorInvalidValue;
+    }
+    auto k = decode_mma_kernel<C>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return (int)e;
+    k<<<n_cta, C::THREADS, C::SMEM, s>>>(mk, mv, a);
+    return (int)cudaGetLastError();
+}
+
+template <int D, int GT, bool I8, int MODE>
+static int launch_mma_idx(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
+    if constexpr (MODE == 1) {
+        return launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
+    } else {
+        return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE>>(a, n_cta, s)
+                       : launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
+    }
+}
+
+template <int D, typename KT, int MODE>
+static int launch_generic(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
+    if (indexed && MODE == 0)
+        decode_generic_kernel<D, KT, true, MODE><<<n_cta, 128, 0, s>>>(a);
+    else
+        decode_generic_kernel<D, KT, false, MODE><<<n_cta, 128, 0, s>>>(a);
+    return (int)cudaGetLastError();
+}
+
+Family decode_family(sgd_dtype kv, sgd_dtype q, int D, bool score) {
+    if (q != SGD_BF16) return kFamilyGeneric;
+    if (kv == SGD_BF16 && (D == 64 || D == 128)) return kFamilyMma;
+    if (kv == SGD_I8 && D == 128 && !score) return kFamilyMma;
+    return kFamilyGeneric;
+}
+
+int decode_ctas_per_sm(sgd_dtype kv, sgd_dtype q, int D, int G, bool indexed, bool score) {
+    if (decode_family(kv, q, D, score) == kFamilyGeneric) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_generic_kernel<128, float, false, 0>, 128, 0) !=
+            cudaSuccess)
+            return 0;
+        return n;
+    }
+    const bool g2 = G > 8;
+    // the shared-memory footprint decides residency; all variants of one dtype/D share it
+    if (kv == SGD_I8) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, false, 0>>();
+    if (D == 128) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, false, false, 0>>();
+    (void)indexed;
+    return g2 ? ctas_per_sm_mma<MmaCfg<64, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<64, 1, false, false, 0>>();
+}
+
+int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, bool score, int n_cta,
+                  cudaStream_t s) {
+    if (n_cta <= 0) return 0;
+    const bool g2 = a.G > 8;
+    if (decode_family(kv, q, a.D, score) == kFamilyMma) {
+        if (score) {
+            if (a.D == 128) return g2 ? launch_mma_idx<128, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, false, 1>(a, false, n_cta, s);
+            return g2 ? launch_mma_idx<64, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<64, 1, false, 1>(a, false, n_cta, s);
+        }
+        if (kv == SGD_I8)
+            return g2 ? launch_mma_idx<128, 2, true, 0>(a, indexed, n_cta, s) : launch_mma_idx<128, 1, true, 0>(a, indexed, n_cta, s);
+        if (a.D == 128)
+            return g2 ? launch_mma_idx<128, 2, false, 0>(a, indexed, n_cta, s) : launch_mma_idx<128, 1, false, 0>(a, indexed, n_cta, s);
+        return g2 ? launch_mma_idx<64, 2, false, 0>(a, indexed, n_cta, s) : launch_mma_idx<64, 1, false, 0>(a, indexed, n_cta, s);
+    }
+    if (score) {
+        if (kv == SGD_F32) return a.D == 128 ? launch_generic<128, float, 1>(a, false, n_cta, s) : launch_generic<64, float, 1>(a, false, n_cta, s);
+        return a.D == 128 ? launch_generic<128, __nv_bfloat16, 1>(a, false, n_cta, s) : launch_generic<64, __nv_bfloat16, 1>(a, false, n_cta, s);
+    }
+    switch (kv) {
+        case SGD_F32:
+            return a.D == 128 ? launch_generic<128, float, 0>(a, indexed, n_cta, s) : launch_generic<64, float, 0>(a, indexed, n_cta, s);
+        case SGD_BF16:
+            return a.D == 128 ? launch_generic<128, __nv_bfloat16, 0>(a, indexed, n_cta, s) : launch_generic<64, __nv_bfloat16, 0>(a, indexed, n_cta, s);
+        default:
+            return a.D == 128 ? launch_generic<128, int8_t, 0>(a, indexed, n_cta, s) : launch_generic<64, int8_t, 0>(a, indexed, n_cta, s);
+    }
+}
+
+int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s) {
+    merge_kernel<<<a.B * a.Hkv, 256, 0, s>>>(a, out, lse);
+    return (int)cudaGetLastError();
+}
+
+}  // namespace sgd

@@ -1,0 +1,59 @@
+// internal.h -- host-side interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace sgd {
+
+// Arguments of the decode / score kernels (device pointers unless noted).
+struct DecodeArgs {
+    const void *q;           // [B, Hq, D]
+    const int32_t *cu_seq;   // cu_seqlens [B+1]
+    const int32_t *cu_kept;  // kept-set prefix sums [B+1] (indexed mode)
+    const int32_t *idx;      // [Hkv, Kt] kept positions (indexed mode)
+    const void *k, *v;       // [Hkv, T, D]
+    const float *k_scale;    // I8
+    const float *v_scale;    // I8
+    int scheme;              // I8: SGD_SCHEME_A / SGD_SCHEME_B
+    int B, Hkv, G, D;
+    int64_t T, Kt, n_parts;
+    int q_f32;               // q is float32 (otherwise bf16)
+    float sm_scale_log2;     // log2(e) / sqrt(D)
+    float sm_scale;          // 1 / sqrt(D)
+    float beta, eps;         // score mode
+    float *scores;           // score mode output [Hkv, T]
+    PlanView plan;
+    float *o_part;           // [slots, G, D]
+    float *lse_part;         // [slots, G]
+    int32_t *status;
+};
+
+// kernel families
+enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
+
+// plan.cu
+void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s);
+void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
+                      int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
+
+// decode.cu
+// Family the decode/score of these arguments runs on.
+Family decode_family(sgd_dtype kv_dtype, sgd_dtype q_dtype, int D, bool score);
+// CTAs resident per SM for that kernel (0 on error).
+int decode_ctas_per_sm(sgd_dtype kv_dtype, sgd_dtype q_dtype, int D, int G, bool indexed, bool score);
+// Launches the split decode (or score) kernel over n_cta CTAs; returns a cudaError_t.
+int launch_decode(const DecodeArgs &a, sgd_dtype kv_dtype, sgd_dtype q_dtype, bool indexed, bool score,
+                  int n_cta, cudaStream_t s);
+int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s);
+
+// quantize.cu
+int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
+                    int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
+                    float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s);
+
+// oam.cu
+int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t T, int keep_num, int keep_den,
+                int32_t *idx, int32_t *cu_kept, int64_t kept_total, int32_t *status, cudaStream_t s);
+
+}  // namespace sgd

@@ -1,0 +1,157 @@
+// plan.cu -- the split-KV partition kernel (one CTA) and its inspection kernel.
+// The rule is stated in plan.cuh.
+#include "internal.h"
+#include "plan.cuh"
+#include "scan.cuh"
+
+namespace sgd {
+
+// cu_len: lengths of the attended rows (cu_seqlens, or cu_kept for a kept set);
+// cu_seq: cu_seqlens (for the scheme-A partition offsets of each sequence).
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu_len,
+                                                    const int32_t *__restrict__ cu_seq, int B, int Hkv,
+                                                    int n_req, int min_chunk, int mode, PlanView pv,
+                                                    WsHeader *hdr) {
+    __shared__ int32_t sm[33];
+    const int tid = threadIdx.x;
+    const int R = B * Hkv;
+    if (tid == 0) hdr->status = 0;
+
+    // 1. padded stream position of every row
+    int32_t carry = 0;
+    for (int base = 0; base < R; base += blockDim.x) {
+        const int r = base + tid;
+        int32_t v = 0;
+        if (r < R) {
+            const int b = r % B;
+            const int32_t L = cu_len[b + 1] - cu_len[b];
+            if (L < 1) atomicOr(&hdr->status, SGD_STATUS_EMPTY_SEQUENCE);
+            v = (int32_t)align_up(max(L, 0), kGranule);
+        }
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (r < R) pv.row_pos[r] = carry + ex;
+        carry += total;
+    }
+    const int32_t W = carry;
+    if (tid == 0) pv.row_pos[R] = W;
+
+    int64_t S = 0;
+    int ncta;
+    if (mode == 0) {
+        S = align_up((W + (int64_t)n_req - 1) / n_req, kGranule);
+        if (S < min_chunk) S = min_chunk;
+        ncta = (int)((W + S - 1) / S);
+    } else {
+        ncta = R;
+    }
+    __syncthreads();
+
+    // 2. CTA ranges
+    for (int i = tid; i <= n_req; i += blockDim.x) {
+        int32_t a;
+        if (mode == 0)
+            a = (int32_t)(((int64_t)i * S < (int64_t)W) ? (int64_t)i * S : (int64_t)W);
+        else
+            a = pv.row_pos[min(i, R)];
+        pv.cta_begin[i] = a;
+    }
+    __syncthreads();
+
+    // 3. segments per CTA -> first slot of each CTA
+    carry = 0;
+    for (int base = 0; base < n_req; base += blockDim.x) {
+        const int i = base + tid;
+        int32_t v = 0;
+        if (i < n_req) {
+            const int32_t a = pv.cta_begin[i], e = pv.cta_begin[i + 1];
+            if (a < e) {
+                for (int r = upper_bound_i32(pv.row_pos, R + 1, a) - 1; r < R && pv.row_pos[r] < e; ++r)
+                    v += (pv.row_pos[r + 1] > pv.row_pos[r]) ? 1 : 0;
+            }
+        }
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (i < n_req) pv.cta_slot0[i] = carry + ex;
+        carry += total;
+    }
+    const int32_t nslots_cta = carry;
+    if (tid == 0) pv.cta_slot0[n_req] = nslots_cta;
+
+    // 4. segments per row -> first slot of each row (same stream order)
+    carry = 0;
+    for (int base = 0; base < R; base += blockDim.x) {
+        const int r = base + tid;
+        int32_t v = 0;
+        if (r < R) {
+            const int32_t p0 = pv.row_pos[r];
+            const int b = r % B;
+            const int32_t L = max(cu_len[b + 1] - cu_len[b], 0);
+            if (L > 0) v = (mode == 0) ? (int32_t)((p0 + L - 1) / S - p0 / S + 1) : 1;
+        }
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (r < R) pv.row_slot0[r] = carry + ex;
+        carry += total;
+    }
+    if (tid == 0) {
+        pv.row_slot0[R] = carry;
+        if (carry != nslots_cta) atomicOr(&hdr->status, SGD_STATUS_SIZE_MISMATCH);
+    }
+
+    // 5. scheme-A partition offset of every sequence: sum_{b'<b} ceil(L_b' / 64)
+    carry = 0;
+    for (int base = 0; base < B; base += blockDim.x) {
+        const int b = base + tid;
+        int32_t v = 0;
+        if (b < B) v = (int32_t)((max(cu_seq[b + 1] - cu_seq[b], 0) + kPart - 1) / kPart);
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (b < B) pv.seq_part0[b] = carry + ex;
+        carry += total;
+    }
+    if (tid == 0) {
+        pv.seq_part0[B] = carry;
+        hdr->plan_W = W;
+        hdr->plan_S = S;
+        hdr->plan_ncta = ncta;
+        hdr->plan_nslots = nslots_cta;
+        hdr->n_parts = carry;
+    }
+}
+
+// One thread per CTA: writes (cta, row, start, length) of its segments at their slots.
+__global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
+                                 int64_t max_segs, int32_t *n_segs, const WsHeader *hdr) {
+    const int cta = blockIdx.x * blockDim.x + threadIdx.x;
+    if (cta == 0) {
+        n_segs[0] = pv.cta_slot0[n_req];
+        n_segs[1] = hdr->plan_ncta;
+    }
+    if (cta >= n_req) return;
+    SegCursor cur;
+    cur.init(pv, cu, B, Hkv, cta);
+    int row, slot;
+    int32_t t0, t1;
+    while (cur.next(row, t0, t1, slot)) {
+        if (slot < max_segs) {
+            int32_t *o = segs + (int64_t)slot * 4;
+            o[0] = cta;
+            o[1] = row;
+            o[2] = t0;
+            o[3] = t1 - t0;
+        }
+    }
+}
+
+void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s) {
+    plan_kernel<<<1, 1024, 0, s>>>(cu_len, cu_seq, B, Hkv, n_req, min_chunk, mode, pv, hdr);
+}
+
+void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
+                      int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s) {
+    plan_dump_kernel<<<(n_req + 127) / 128, 128, 0, s>>>(pv, cu, B, Hkv, n_req, segs, max_segs, n_segs, hdr);
+}
+
+}  // namespace sgd

@@ -1,0 +1,77 @@
+// plan.cuh -- equal-work split-KV partition of a ragged batch over CTAs.
+//
+// "Optimizing token dropping in sparse attention" (优化稀疏注意力中的令牌丢弃机制),
+// section 5: sequences of very different lengths (128K next to 512) leave CTAs
+// idle when each CTA owns a whole sequence; splitting the KV of every row
+// across CTAs and reducing afterwards balances the work.  The reading used here:
+//   rows = (KV head, sequence) pairs in memory order, row = kvh * B + b;
+//   each row is padded to a multiple of kGranule tokens and the rows are laid
+//   end to end into one stream of W tokens;
+//   mode 0 cuts the stream into CTA ranges of S = max(min_chunk,
+//   round_up(ceil(W / n_req), kGranule)) tokens, mode 1 gives each row a CTA;
+//   a segment = one CTA range intersected with the real tokens of one row;
+//   segments are numbered in stream order and each yields one partial result.
+// Because CTA boundaries are multiples of kGranule and a row's padding is
+// shorter than kGranule, no CTA starts inside padding and every segment holds
+// at least one real token.
+#pragma once
+
+#include "common.cuh"
+
+namespace sgd {
+
+__device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int32_t x) {
+    int lo = 0, hi = n;  // first i with a[i] > x
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a[mid] <= x)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Walks the segments of one CTA in stream order.
+struct SegCursor {
+    const int32_t *row_pos;
+    const int32_t *cu;  // lengths of row r are cu[b+1] - cu[b], b = r % B
+    int R, B;
+    int32_t end;  // CTA range end (stream position)
+    int32_t pos;  // next stream position to cover
+    int r;        // current row candidate
+    int slot;     // slot of the next segment
+
+    __device__ void init(const PlanView &pv, const int32_t *cu_, int B_, int Hkv, int cta) {
+        row_pos = pv.row_pos;
+        cu = cu_;
+        B = B_;
+        R = B_ * Hkv;
+        pos = pv.cta_begin[cta];
+        end = pv.cta_begin[cta + 1];
+        slot = pv.cta_slot0[cta];
+        r = (pos < end) ? upper_bound_i32(row_pos, R + 1, pos) - 1 : R;
+    }
+
+    // Next segment: row, row-local token range [t0, t1), slot.  False when done.
+    __device__ bool next(int &row, int32_t &t0, int32_t &t1, int &s) {
+        while (r < R && row_pos[r] < end) {
+            const int b = r % B;
+            const int32_t L = cu[b + 1] - cu[b];
+            const int32_t rp = row_pos[r];
+            const int32_t lo = max(pos, rp), hi = min(end, rp + max(L, 0));
+            ++r;
+            if (hi > lo) {
+                row = r - 1;
+                t0 = lo - rp;
+                t1 = hi - rp;
+                s = slot++;
+                pos = hi;
+                return true;
+            }
+        }
+        return false;
+    }
+};
+
+}  // namespace sgd

@@ -1,0 +1,286 @@
+// quantize.cu -- INT8 KV cache, schemes A and B.
+//
+// "优化稀疏注意力中的令牌丢弃机制" (Optimizing token dropping in sparse attention),
+// section 6: q_val = round(val / scale) with scale = max|x| / 127 over the group
+// that shares it.  Scheme A ("fine-grained QK"): K has one scale per partition of
+// 64 consecutive tokens (counted from each sequence's first token, per KV head),
+// V one scale for the whole tensor.  Scheme B ("coarser KV"): one scale each for K
+// and for V.  Readings: scale = float32 nearest to amax/127; the quotient is the
+// correctly rounded float32 x/scale; rounding is half-to-even; codes clamp to
+// [-127, 127]; a zero scale gives zero codes.
+//
+// Passes.  A per-tensor scale needs the tensor's max before any code, so V (and K
+// for scheme B) is read twice:
+//   scheme A: pass 1 quantises each K partition from registers (one read of K) and
+//             accumulates max|V|; pass 2 quantises V.
+//   scheme B: pass 1 accumulates max|K| and max|V|; pass 2 quantises both.
+//
+// Exact codes without a divide per element: q' = x * RN(1/s) differs from the
+// correctly rounded quotient Q = RN(x/s) by at most |x/s| * 2^-23 + ulp(Q)/2 <= 2.3e-5
+// (|x/s| <= 127 * (1 + 2^-23) because s is the group's own scale), so
+// round_half_even(q') == round_half_even(Q) unless q' lies within 2.3e-5 of a
+// half-integer.  Whenever q' is within 1e-4 of one (or is not finite) the IEEE
+// division __fdiv_rn(x, s) is taken instead.
+#include "internal.h"
+#include "scan.cuh"
+
+namespace sgd {
+
+__device__ __forceinline__ int code_of(float x, float s, float r) {
+    float q = x * r;
+    float n = rintf(q);
+    if (!(fabsf(q - n) < 0.4999f)) {
+        q = __fdiv_rn(x, s);
+        n = rintf(q);
+    }
+    n = fminf(fmaxf(n, -127.f), 127.f);
+    return (int)n;
+}
+
+template <typename T>
+struct Vec;  // 16 bytes of input -> VE elements -> VE code bytes
+template <>
+struct Vec<__nv_bfloat16> {
+    static constexpr int VE = 8;
+    __device__ static void unpack(const uint4 &w, float (&x)[8]) {
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(ww[i] << 16);
+            x[2 * i + 1] = __uint_as_float(ww[i] & 0xffff0000u);
+        }
+    }
+};
+template <>
+struct Vec<float> {
+    static constexpr int VE = 4;
+    __device__ static void unpack(const uint4 &w, float (&x)[4]) {
+        x[0] = __uint_as_float(w.x);
+        x[1] = __uint_as_float(w.y);
+        x[2] = __uint_as_float(w.z);
+        x[3] = __uint_as_float(w.w);
+    }
+};
+
+template <int VE>
+__device__ __forceinline__ void store_codes(int8_t *dst, const float (&x)[VE], float s, float r) {
+    uint32_t w[VE / 4];
+#pragma unroll
+    for (int i = 0; i < VE / 4; ++i) {
+        uint32_t b = 0;
+        if (s != 0.f) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b |= (uint32_t)(code_of(x[4 * i + j], s, r) & 0xff) << (8 * j);
+        }
+        w[i] = b;
+    }
+    if constexpr (VE == 8)
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+    else
+        *reinterpret_cast<uint32_t *>(dst) = w[0];
+}
+
+__device__ __forceinline__ float block_max(float v, float *sm) {
+    v = warp_max(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    __syncthreads();
+    if (lane == 0) sm[warp] = v;
+    __syncthreads();
+    float r = 0.f;
+    for (int w = 0; w < nw; ++w) r = fmaxf(r, sm[w]);
+    return r;
+}
+
+// Zero the max accumulators, partition offsets of every sequence, consistency checks.
+__global__ void __launch_bounds__(1024) quant_prep_kernel(const int32_t *cu, int B, int64_t n_parts_host,
+                                                          int check_parts, int32_t *seq_part0, WsHeader *hdr) {
+    __shared__ int32_t sm[33];
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        hdr->status = 0;
+        hdr->amax_bits[0] = hdr->amax_bits[1] = 0u;
+    }
+    int32_t carry = 0;
+    for (int base = 0; base < B; base += blockDim.x) {
+        const int b = base + tid;
+        int32_t v = 0;
+        if (b < B) {
+            const int32_t L = cu[b + 1] - cu[b];
+            if (L < 1) atomicOr(&hdr->status, SGD_STATUS_EMPTY_SEQUENCE);
+            v = (max(L, 0) + kPart - 1) / kPart;
+        }
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (b < B) seq_part0[b] = carry + ex;
+        carry += total;
+    }
+    if (tid == 0) {
+        seq_part0[B] = carry;
+        hdr->n_parts = carry;
+        if (check_parts && carry != n_parts_host) atomicOr(&hdr->status, SGD_STATUS_SIZE_MISMATCH);
+    }
+}
+
+// Scheme A pass 1: one CTA per (KV head, partition): K codes and scale from registers, max|V|.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) quant_k_partition_kernel(const T *__restrict__ k, const T *__restrict__ v,
+                                                                const int32_t *__restrict__ cu,
+                                                                const int32_t *__restrict__ seq_part0, int B,
+                                                                int Hkv, int64_t Ttot, int64_t n_parts,
+                                                                int8_t *__restrict__ kc,
+                                                                float *__restrict__ k_scale, WsHeader *hdr) {
+    constexpr int VE = Vec<T>::VE;
+    constexpr int NV = (kPart * D / VE + 255) / 256;  // vectors per thread
+    __shared__ float sm[32];
+    if (hdr->n_parts != n_parts) return;  // sizes disagree: flagged by the prep kernel
+    const int64_t total = (int64_t)Hkv * n_parts;
+    float vmax = 0.f;
+    for (int64_t p = blockIdx.x; p < total; p += gridDim.x) {
+        const int kvh = (int)(p / n_parts);
+        const int32_t lp = (int32_t)(p - (int64_t)kvh * n_parts);
+        int lo = 0, hi = B;  // sequence b with seq_part0[b] <= lp < seq_part0[b+1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (seq_part0[mid] <= lp) lo = mid;
+            else hi = mid;
+        }
+        const int b = lo;
+        const int32_t tok0 = cu[b] + (lp - seq_part0[b]) * kPart;
+        const int32_t ntok = min(kPart, cu[b + 1] - tok0);
+        const int64_t e0 = ((int64_t)kvh * Ttot + tok0) * D;
+        const int nvec = ntok * D / VE;
+        const uint4 *kp = reinterpret_cast<const uint4 *>(k + e0);
+        const uint4 *vp = reinterpret_cast<const uint4 *>(v + e0);
+        float x[NV][VE];
+        float kmax = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = threadIdx.x + 256 * i;
+            uint4 kw = make_uint4(0, 0, 0, 0), vw = kw;
+            if (vi < nvec) {
+                kw = __ldcs(kp + vi);
+                vw = __ldcs(vp + vi);
+            }
+            Vec<T>::unpack(kw, x[i]);
+            float y[VE];
+            Vec<T>::unpack(vw, y);
+#pragma unroll
+            for (int j = 0; j < VE; ++j) {
+                kmax = fmaxf(kmax, fabsf(x[i][j]));
+                vmax = fmaxf(vmax, fabsf(y[j]));
+            }
+        }
+        kmax = block_max(kmax, sm);
+        const float s = __fdiv_rn(kmax, 127.f);
+        const float r = (s != 0.f) ? __frcp_rn(s) : 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int vi = threadIdx.x + 256 * i;
+            if (vi < nvec) store_codes<VE>(kc + e0 + (int64_t)vi * VE, x[i], s, r);
+        }
+        if (threadIdx.x == 0) k_scale[p] = s;
+    }
+    vmax = block_max(vmax, sm);
+    if (threadIdx.x == 0) atomicMax(&hdr->amax_bits[1], __float_as_uint(vmax));
+}
+
+// Scheme B pass 1: max|K| and max|V| over the whole tensors.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_amax_kernel(const T *__restrict__ k, const T *__restrict__ v,
+                                                         int64_t nvec, WsHeader *hdr) {
+    constexpr int VE = Vec<T>::VE;
+    __shared__ float sm[32];
+    const uint4 *kp = reinterpret_cast<const uint4 *>(k);
+    const uint4 *vp = reinterpret_cast<const uint4 *>(v);
+    float km = 0.f, vm = 0.f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * blockDim.x) {
+        float x[VE], y[VE];
+        Vec<T>::unpack(__ldcs(kp + i), x);
+        Vec<T>::unpack(__ldcs(vp + i), y);
+#pragma unroll
+        for (int j = 0; j < VE; ++j) {
+            km = fmaxf(km, fabsf(x[j]));
+            vm = fmaxf(vm, fabsf(y[j]));
+        }
+    }
+    km = block_max(km, sm);
+    vm = block_max(vm, sm);
+    if (threadIdx.x == 0) {
+        atomicMax(&hdr->amax_bits[0], __float_as_uint(km));
+        atomicMax(&hdr->amax_bits[1], __float_as_uint(vm));
+    }
+}
+
+// Pass 2: codes of one or two whole tensors with their global scales.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__ x0, int8_t *__restrict__ c0,
+                                                           float *scale0, int which0, const T *__restrict__ x1,
+                                                           int8_t *__restrict__ c1, float *scale1, int which1,
+                                                           int64_t nvec, const WsHeader *hdr) {
+    constexpr int VE = Vec<T>::VE;
+    const float s0 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which0]), 127.f);
+    const float r0 = (s0 != 0.f) ? __frcp_rn(s0) : 0.f;
+    float s1 = 0.f, r1 = 0.f;
+    if (x1) {
+        s1 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which1]), 127.f);
+        r1 = (s1 != 0.f) ? __frcp_rn(s1) : 0.f;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *scale0 = s0;
+        if (x1) *scale1 = s1;
+    }
+    const uint4 *p0 = reinterpret_cast<const uint4 *>(x0);
+    const uint4 *p1 = reinterpret_cast<const uint4 *>(x1);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += stride) {
+        float x[VE];
+        Vec<T>::unpack(__ldcs(p0 + i), x);
+        store_codes<VE>(c0 + i * VE, x, s0, r0);
+        if (x1) {
+            Vec<T>::unpack(__ldcs(p1 + i), x);
+            store_codes<VE>(c1 + i * VE, x, s1, r1);
+        }
+    }
+}
+
+template <typename T, int D>
+static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int Hkv, int64_t Ttot,
+                         sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
+                         float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
+    constexpr int VE = Vec<T>::VE;
+    const int64_t nvec = (int64_t)Hkv * Ttot * D / VE;
+    quant_prep_kernel<<<1, 1024, 0, s>>>(cu, B, n_parts, scheme == SGD_SCHEME_A, seq_part0, hdr);
+    const int grid_stream = sm_count * 8;
+    if (scheme == SGD_SCHEME_A) {
+        const int64_t total = (int64_t)Hkv * n_parts;
+        const int grid = (int)std::min<int64_t>(total, (int64_t)sm_count * 8);
+        if (grid > 0)
+            quant_k_partition_kernel<T, D><<<grid, 256, 0, s>>>(k, v, cu, seq_part0, B, Hkv, Ttot, n_parts, kc,
+                                                                k_scale, hdr);
+        quant_global_kernel<T><<<grid_stream, 256, 0, s>>>(v, vc, v_scale, 1, nullptr, nullptr, nullptr, 0, nvec,
+                                                           hdr);
+    } else {
+        quant_amax_kernel<T><<<grid_stream, 256, 0, s>>>(k, v, nvec, hdr);
+        quant_global_kernel<T><<<grid_stream, 256, 0, s>>>(k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
+    }
+    return (int)cudaGetLastError();
+}
+
+int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
+                    int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
+                    float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
+    if (dt == SGD_BF16) {
+        auto kk = static_cast<const __nv_bfloat16 *>(k), vv = static_cast<const __nv_bfloat16 *>(v);
+        return D == 128 ? quantize_impl<__nv_bfloat16, 128>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale,
+                                                            v_scale, hdr, seq_part0, sm_count, s)
+                        : quantize_impl<__nv_bfloat16, 64>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale,
+                                                           v_scale, hdr, seq_part0, sm_count, s);
+    }
+    auto kk = static_cast<const float *>(k), vv = static_cast<const float *>(v);
+    return D == 128 ? quantize_impl<float, 128>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale, v_scale,
+                                                hdr, seq_part0, sm_count, s)
+                    : quantize_impl<float, 64>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale, v_scale, hdr,
+                                               seq_part0, sm_count, s);
+}
+
+}  // namespace sgd

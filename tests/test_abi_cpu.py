@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: the library loads, exports every function include/sgd.h declares,
+and rejects invalid arguments on the host before anything touches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sgd.h")
+
+
+@pytest.fixture(scope="module")
+def sgd():
+    from sparse_gqa_decode_b200 import build
+    build.build()
+    import sparse_gqa_decode_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sgd_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sgd_oam_select", "sgd_quantize_kv", "sgd_decode_attn", "sgd_workspace_size",
+                     "sgd_error_string", "sgd_plan_segments", "sgd_workspace_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(sgd):
+    for name in declared_functions():
+        assert hasattr(sgd.lib, name), f"{name} not exported"
+
+
+def test_error_strings_and_version(sgd):
+    assert sgd.lib.sgd_version() == (1 << 16)
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert sgd.lib.sgd_error_string(code)
+    assert sgd.lib.sgd_error_string(-99) == b"unknown status"
+
+
+def test_struct_layout_matches_header(sgd):
+    # dtype, B, Hkv, D (4 x 4 bytes), T (8), 3 pointers, scheme (+pad), 2 pointers, n_parts
+    assert ctypes.sizeof(sgd.SgdKv) == 4 * 4 + 8 + 3 * 8 + 8 + 2 * 8 + 8
+    assert sgd.SgdKv.T.offset == 16 and sgd.SgdKv.k_scale.offset == 56 and sgd.SgdKv.n_parts.offset == 72
+
+
+def _kv(sgd, **kw):
+    base = dict(dtype=sgd.SGD_BF16, B=2, Hkv=2, D=128, T=100, cu_seqlens=0x1000, k=0x10000, v=0x20000,
+                scheme=0, k_scale=None, v_scale=None, n_parts=0)
+    base.update(kw)
+    return sgd.SgdKv(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), -1), (dict(cu_seqlens=None), -1), (dict(B=0), -2), (dict(D=96), -2),
+    (dict(T=2**31), -2), (dict(dtype=7), -3), (dict(k=0x10008), -4),
+])
+def test_decode_rejects_bad_cache_on_host(sgd, kw, code):
+    kv = _kv(sgd, **kw)
+    rc = sgd.lib.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv), None, None, 0, 0, 0,
+                                 ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000), 1 << 20,
+                                 None)
+    assert rc == code
+
+
+def test_decode_rejects_bad_args_on_host(sgd):
+    kv = _kv(sgd)
+    L = sgd.lib
+
+    def call(q=0x3000, qdt=sgd.SGD_BF16, G=8, idx=None, cu_kept=None, kt=0, out=0x4000, lse=0x5000, ws=0x6000):
+        return L.sgd_decode_attn(ctypes.c_void_p(q) if q else None, qdt, G, ctypes.byref(kv),
+                                 ctypes.c_void_p(idx) if idx else None, ctypes.c_void_p(cu_kept) if cu_kept else None,
+                                 kt, 0, 0, ctypes.c_void_p(out) if out else None,
+                                 ctypes.c_void_p(lse) if lse else None, ctypes.c_void_p(ws) if ws else None,
+                                 1 << 20, None)
+
+    assert call(q=0) == -1
+    assert call(out=0) == -1
+    assert call(G=0) == -2 and call(G=17) == -2
+    assert call(qdt=sgd.SGD_F32) == -3  # an f32 query needs an f32 cache
+    assert call(idx=0x7000) == -1  # idx without cu_kept
+    assert call(idx=0x7000, cu_kept=0x8000, kt=1) == -2  # fewer kept tokens than sequences
+    assert call(q=0x3004) == -4
+    kv8 = _kv(sgd, dtype=sgd.SGD_I8)
+    assert L.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv8), None, None, 0, 0, 0,
+                             ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000), 1 << 20,
+                             None) == -1  # int8 cache without scales
+
+
+def test_quantize_and_select_reject_bad_args_on_host(sgd):
+    L = sgd.lib
+    kv = _kv(sgd)
+    p = ctypes.c_void_p
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, None, p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+                             None) == -1
+    assert L.sgd_quantize_kv(ctypes.byref(_kv(sgd, dtype=sgd.SGD_I8)), 0, 3, p(0x1000), p(0x1000), p(0x2000),
+                             p(0x3000), p(0x4000), 4096, None) == -3
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 5, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+                             None) == -3
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 1, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+                             None) == -2  # fewer partitions than sequences
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 16,
+                             None) == -5  # workspace too small
+    sel = lambda **kw: L.sgd_oam_select(p(0x3000), kw.get("qdt", sgd.SGD_BF16), kw.get("G", 8), ctypes.byref(kv),
+                                        kw.get("beta", 1.0), 1e-6, kw.get("num", 1), kw.get("den", 8), p(0x1000),
+                                        p(0x2000), kw.get("kt", 20), p(0x4000), 1 << 20, None)
+    assert sel(num=9, den=8) == -8
+    assert sel(den=0) == -8
+    assert sel(kt=1) == -2
+    assert sel(beta=float("nan")) == -8
+    assert sel(G=20) == -2

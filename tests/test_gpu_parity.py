@@ -1,0 +1,290 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs, through the C ABI.
+
+Tolerances (the stated acceptance bar): outputs max-abs error <= 1e-2 * max|out| for bf16 (and
+INT8) inputs, <= 1e-3 * max|out| for fp32 inputs; lse <= 1e-3 absolute; INT8 codes and scales
+bit-exact; the work partition bit-exact; kept index sets exact except tokens whose oracle score is
+within 1e-4 of the K-th score.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = {"f32": 1e-3, "bf16": 1e-2}
+LSE_TOL = 1e-3
+TIE_WINDOW = 1e-4
+
+
+@pytest.fixture(scope="module")
+def sgd():
+    from sparse_gqa_decode_b200 import build
+    build.build()
+    import sparse_gqa_decode_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def dev(bt):
+    return (bt.q.cuda(), bt.k.cuda(), bt.v.cuda(), bt.cu_seqlens.cuda())
+
+
+def make(lengths, G=8, D=128, Hkv=2, dtype="bf16", dist="normal", seed=0):
+    wl = workloads.Workload("t", B=len(lengths), Hkv=Hkv, G=G, D=D, kv_dtype=dtype, dist=dist,
+                            lengths=tuple(lengths))
+    return workloads.generate(wl, seed)
+
+
+def assert_close(out, lse, ref_out, ref_lse, tol, rows=None):
+    out = out.double().cpu().numpy()
+    lse = lse.double().cpu().numpy()
+    if rows is not None:  # compare only the computed (b, kvh) rows
+        mask = ~np.isnan(ref_lse)
+        out, lse, ref_out, ref_lse = out[mask], lse[mask], ref_out[mask], ref_lse[mask]
+    scale = np.abs(ref_out).max()
+    err = np.abs(out - ref_out).max()
+    lerr = np.abs(lse - ref_lse).max()
+    assert err <= tol * scale, f"out error {err:.3e} > {tol} * {scale:.3e}"
+    assert lerr <= LSE_TOL, f"lse error {lerr:.3e}"
+    return err / scale, lerr
+
+
+def check_status(sgd, ws):
+    assert sgd.workspace_status(ws) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# dense decode
+# ---------------------------------------------------------------------------------------------
+def test_config1_fp32_four_chunks(sgd):
+    bt = workloads.generate(workloads.config(1))
+    q, k, v, cu = dev(bt)
+    out, lse, ws = sgd.decode_attn(q, 4, k, v, cu, n_splits=4)
+    segs, ncta = sgd.plan_segments(cu, 1, 1, 4, 16, 0)
+    assert ncta == 4 and segs[:, 3].tolist() == [64, 64, 64, 64]
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 4)
+    assert_close(out, lse, *ref, OUT_TOL["f32"])
+    check_status(sgd, ws)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_dense_decode_shapes(sgd, dtype, D, G):
+    bt = make((1, 63, 64, 65, 1000, 2053), G=G, D=D, Hkv=2, dtype=dtype, seed=G * 7 + D)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G)
+    for n_splits in (0, 3, 37):
+        out, lse, ws = sgd.decode_attn(q, G, k, v, cu, n_splits=n_splits)
+        assert_close(out, lse, *ref, OUT_TOL[dtype])
+        check_status(sgd, ws)
+
+
+def test_bf16_multi_tile_several_ctas(sgd):
+    # config-2 shapes with shorter rows: many 64-token tiles per CTA and CTA ranges crossing rows
+    bt = workloads.generate(workloads.config(2, lengths=(4096 + 37,) * 3, B=3), seed=2)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8)
+    out, lse, ws = sgd.decode_attn(q, 8, k, v, cu)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
+
+
+def test_ragged_equal_work_equals_one_cta_per_row(sgd):
+    wl = workloads.config(3, length_range=(17, 6000))
+    bt = workloads.generate(wl, seed=3)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8)
+    o0, l0, ws0 = sgd.decode_attn(q, 8, k, v, cu, schedule=0)
+    o1, l1, ws1 = sgd.decode_attn(q, 8, k, v, cu, schedule=1)
+    assert_close(o0, l0, *ref, OUT_TOL["bf16"])
+    assert_close(o1, l1, *ref, OUT_TOL["bf16"])
+    assert (o0 - o1).abs().max().item() <= 1e-2 * np.abs(ref[0]).max()
+    check_status(sgd, ws0)
+    check_status(sgd, ws1)
+
+
+def test_identical_keys_give_mean_of_v(sgd):
+    bt = make((300,), G=4, D=128, Hkv=1)
+    bt.k[:] = bt.k[:, :1]  # every key equal
+    q, k, v, cu = dev(bt)
+    out, lse, _ = sgd.decode_attn(q, 4, k, v, cu, n_splits=5)
+    mean = bt.v[0].double().mean(dim=0)
+    assert (out[0].double().cpu() - mean).abs().max().item() <= 1e-2 * mean.abs().max().item()
+
+
+# ---------------------------------------------------------------------------------------------
+# partition
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("mode", [0, 1])
+def test_plan_matches_oracle_bit_exact(sgd, seed, mode):
+    rng = np.random.default_rng(seed)
+    B, Hkv = int(rng.integers(1, 20)), int(rng.integers(1, 9))
+    lens = np.rint(np.exp(rng.uniform(0, 11, B))).astype(np.int64)
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).cuda()
+    n_req = int(rng.integers(1, 400))
+    min_chunk = 16 * int(rng.integers(1, 20))
+    segs, ncta = sgd.plan_segments(cu, B, Hkv, n_req, min_chunk, mode)
+    row_len = np.tile(lens, Hkv)  # row = kvh * B + b
+    ref = oracle.plan(row_len, n_req, 16, min_chunk, mode)
+    got = segs.numpy()
+    assert ncta == ref["n_cta"]
+    assert got[:, 0].tolist() == ref["cta"].tolist()
+    assert got[:, 1].tolist() == ref["row"].tolist()
+    assert got[:, 2].tolist() == ref["start"].tolist()
+    assert got[:, 3].tolist() == ref["len"].tolist()
+
+
+# ---------------------------------------------------------------------------------------------
+# INT8 cache
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_quantize_bit_exact(sgd, scheme, dtype):
+    bt = make((1, 63, 64, 65, 700, 4099), G=8, D=128, Hkv=3, dtype=dtype, dist="outlier", seed=11)
+    # plant exact rounding ties in partition 1 of sequence 5 (tokens 64..127) of head 1
+    s0 = int(bt.cu_seqlens[5])
+    bt.k[1, s0 + 64:s0 + 128] = 0
+    if dtype == "f32":  # max |x| = 889 -> scale 7: quotients 6.5, 12.5, 14.5, -22.5
+        ties, want = [45.5, 87.5, 101.5, -157.5, 889.0], [6, 12, 14, -22, 127]
+    else:  # bf16 holds these exactly; max |x| = 127 -> scale 1
+        ties, want = [2.5, 3.5, -2.5, 126.5, 127.0, -0.5], [2, 4, -2, 126, 127, 0]
+    bt.k[1, s0 + 64, :len(ties)] = torch.tensor(ties).to(bt.k.dtype)
+    q, k, v, cu = dev(bt)
+    kc, vc, ks, vs, ws = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    assert np.array_equal(ks.cpu().numpy().reshape(rks.shape), rks)
+    assert np.array_equal(vs.cpu().numpy(), rvs)
+    assert np.array_equal(kc.cpu().numpy(), rkc)
+    assert np.array_equal(vc.cpu().numpy(), rvc)
+    if scheme == "A":
+        assert kc[1, s0 + 64, :len(want)].tolist() == want
+    check_status(sgd, ws)
+
+
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("G", [4, 8, 16])
+def test_int8_decode(sgd, scheme, G):
+    bt = make((1, 65, 700, 3000), G=G, D=128, Hkv=2, dist="outlier", seed=21 + G)
+    q, k, v, cu = dev(bt)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G, quant=(rkc, rvc, rks, rvs, scheme))
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+    parts = sgd.n_parts(bt.lengths)
+    for n_splits in (0, 7):
+        out, lse, ws = sgd.decode_attn(q, G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=scheme, n_parts_=parts,
+                                       n_splits=n_splits)
+        assert_close(out, lse, *ref, OUT_TOL["bf16"])
+        check_status(sgd, ws)
+
+
+def test_int8_d64_uses_cuda_core_path(sgd):
+    bt = make((5, 300), G=8, D=64, Hkv=2, dist="outlier", seed=5)
+    q, k, v, cu = dev(bt)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, quant=(rkc, rvc, rks, rvs, "A"))
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    assert np.array_equal(kc.cpu().numpy(), rkc)
+    out, lse, _ = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                  n_parts_=sgd.n_parts(bt.lengths))
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------------------------
+# OAM selection
+# ---------------------------------------------------------------------------------------------
+def check_selection(idx, cu_kept, ref_idx, ref_cu, scores, B, Hkv):
+    assert cu_kept.tolist() == ref_cu.tolist()
+    idx = idx.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            a, e = int(ref_cu[b]), int(ref_cu[b + 1])
+            got, want = set(idx[h, a:e].tolist()), set(ref_idx[h, a:e].tolist())
+            assert (np.diff(idx[h, a:e]) > 0).all(), "kept positions must ascend"
+            s = scores[(b, h)]
+            kth = np.sort(s)[::-1][e - a - 1]
+            for t in got ^ want:
+                assert abs(s[t] - kth) <= TIE_WINDOW, f"token {t} differs and is not a near-tie"
+
+
+@pytest.mark.parametrize("G,D", [(8, 128), (4, 64), (16, 128), (1, 128)])
+def test_oam_select_matches_oracle(sgd, G, D):
+    bt = make((1, 7, 64, 500, 5000), G=G, D=D, Hkv=2, dist="outlier", seed=31 + G)
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, ws = sgd.oam_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, bt.lengths)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, bt.wl.B, 2)
+    check_status(sgd, ws)
+
+
+def test_oam_select_f32_cache(sgd):
+    bt = make((40, 333), G=4, D=64, Hkv=1, dtype="f32", seed=41)
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, 4, 0.5, 1e-6, 3, 10, bt.lengths)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 4, 0.5, 1e-6, 3, 10)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, 2, 1)
+
+
+def test_oam_ties_keep_lowest_indices(sgd):
+    # q = 0 and every value row of the same norm: all scores equal -> tokens 0 .. K-1
+    bt = make((100, 9, 1000), G=8, D=128, Hkv=2, seed=51)
+    bt.q.zero_()
+    bt.v[:] = 0
+    bt.v[..., 0] = 2.0
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, bt.lengths)
+    assert cu_kept.tolist() == [0, 13, 15, 140]
+    for h in range(2):
+        assert idx[h, :13].tolist() == list(range(13))
+        assert idx[h, 13:15].tolist() == [0, 1]
+        assert idx[h, 15:].tolist() == list(range(125))
+
+
+def test_oam_keep_all_then_decode_equals_dense(sgd):
+    bt = make((33, 700), G=8, D=128, Hkv=2, seed=61)
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 1, bt.lengths)
+    assert idx[0, :33].tolist() == list(range(33))
+    dense = sgd.decode_attn(q, 8, k, v, cu)
+    sel = sgd.decode_attn(q, 8, k, v, cu, idx=idx, cu_kept=cu_kept, kept_total_=idx.shape[1])
+    assert (dense[0] - sel[0]).abs().max().item() <= 1e-5
+    assert (dense[1] - sel[1]).abs().max().item() <= 1e-5
+
+
+@pytest.mark.parametrize("kvdt", ["bf16", "int8A", "int8B"])
+def test_oam_then_decode_over_kept(sgd, kvdt):
+    bt = make((1, 90, 2000, 4500), G=8, D=128, Hkv=2, dist="outlier", seed=71)
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, bt.lengths)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 1.0, 1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, 4, 2)
+    Kt = idx.shape[1]
+    if kvdt == "bf16":
+        ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=ref_idx, cu_kept=ref_cu)
+        out, lse, ws = sgd.decode_attn(q, 8, k, v, cu, idx=idx, cu_kept=cu_kept, kept_total_=Kt)
+    else:
+        scheme = kvdt[-1]
+        quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+        ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=ref_idx, cu_kept=ref_cu, quant=(*quant, scheme))
+        kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+        out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=scheme,
+                                       n_parts_=sgd.n_parts(bt.lengths), idx=idx, cu_kept=cu_kept, kept_total_=Kt)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
+
+
+# ---------------------------------------------------------------------------------------------
+# device status reporting
+# ---------------------------------------------------------------------------------------------
+def test_empty_sequence_is_reported(sgd):
+    bt = make((5, 40), G=8, D=128, Hkv=1, seed=81)
+    q, k, v, _ = dev(bt)
+    cu = torch.tensor([0, 5, 5, 45], dtype=torch.int32, device="cuda")  # sequence 1 is empty
+    q3 = torch.cat([q[:1], q[:1], q[1:]])
+    out, lse, ws = sgd.decode_attn(q3, 8, k, v, cu)
+    assert sgd.workspace_status(ws) & 0x1
+    assert torch.isinf(lse[1]).all() and (out[1] == 0).all()
