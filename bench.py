@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the decode hot path: INT8 scheme-A quantisation -> OAM token selection ->
+split-KV decode over the kept tokens (-> LSE merge), on seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5] [--impl reference]
+
+One step = one pass of the whole path over one batch (the default workload: 4 sequences of
+32K-128K tokens, 8 KV heads, G = 8, D = 128, beta = 1, eps = 1e-6, keep 1/8).  Prints one JSON
+line.  `value` is algorithmic KV bytes moved per second by the whole job (GB/s); stage times,
+sequences*heads/s, a roofline entry for the dominant stage and the fp64 oracle's CPU rate on a
+bounded sample are included.  With N > 1 (torchrun), every rank runs its own copy of the
+workload on its own GPU (independent rows: weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic bytes
+# ------------------------------------------------------------------------------------------------
+def kept_of(L, num, den):
+    return max(1, min(int(L), -(-int(L) * num // den)))
+
+
+def algorithmic_bytes(wl, lengths):
+    """Bytes each stage must move at minimum (inputs read once, outputs written once)."""
+    Hkv, D, G, B = wl.Hkv, wl.D, wl.G, wl.B
+    T = int(sum(lengths))
+    P = int(sum((int(L) + 63) // 64 for L in lengths))
+    kv_bf16 = 2 * Hkv * T * D * 2
+    q = B * Hkv * G * D * 2
+    out = B * Hkv * G * (D + 1) * 4
+    st = {}
+    if wl.scheme:
+        st["quantize"] = kv_bf16 + 2 * Hkv * T * D + (Hkv * P * 4 if wl.scheme == "A" else 4) + 4
+    if wl.oam:
+        Kt = sum(kept_of(L, wl.keep_num, wl.keep_den) for L in lengths)
+        st["select"] = kv_bf16 + q + Hkv * Kt * 4 + (B + 1) * 4
+        n_att = Kt
+        idx_bytes = Hkv * Kt * 4
+    else:
+        n_att = T
+        idx_bytes = 0
+    eb = 1 if wl.scheme else 2
+    scales = (Hkv * P * 4 if wl.scheme == "A" else 8) if wl.scheme else 0
+    st["decode"] = 2 * Hkv * n_att * D * eb + idx_bytes + scales + q + out
+    return st
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sgd_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+class Pipeline:
+    """Device buffers and the three C-ABI calls of one step (outputs and workspaces reused)."""
+
+    def __init__(self, sgd, wl, bt, dev):
+        self.sgd, self.wl, self.bt, self.dev = sgd, wl, bt, dev
+        self.lengths = [int(x) for x in bt.lengths]
+        self.q = bt.q.to(dev)
+        self.k = bt.k.to(dev)
+        self.v = bt.v.to(dev)
+        self.cu = bt.cu_seqlens.to(dev)
+        self.parts = sgd.n_parts(self.lengths)
+        self.qout = self.kept = None
+        self.ws_q = self.ws_s = self.ws_d = None
+        self.sel_out = None
+        self.dec_out = None
+        self.stage_events = {}
+
+    def run(self, record=None):
+        """One step.  record: dict stage -> (start_event, end_event) to time each stage."""
+        sgd, wl = self.sgd, self.wl
+
+        def ev(name, i):
+            if record is not None:
+                record[name][i].record()
+
+        kc, vc, ks, vs = self.k, self.v, None, None
+        if wl.scheme:
+            ev("quantize", 0)
+            kc, vc, ks, vs, self.ws_q = sgd.quantize_kv(self.k, self.v, self.cu, wl.scheme, self.lengths,
+                                                        out=self.qout, workspace=self.ws_q)
+            self.qout = (kc, vc, ks, vs)
+            ev("quantize", 1)
+        idx = cu_kept = None
+        Kt = 0
+        if wl.oam:
+            ev("select", 0)
+            idx, cu_kept, self.ws_s = sgd.oam_select(self.q, self.k, self.v, self.cu, wl.G, wl.beta, wl.eps,
+                                                     wl.keep_num, wl.keep_den, self.lengths, out=self.sel_out,
+                                                     workspace=self.ws_s)
+            self.sel_out = (idx, cu_kept)
+            Kt = idx.shape[1]
+            ev("select", 1)
+        ev("decode", 0)
+        o, lse, self.ws_d = sgd.decode_attn(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
+                                            scheme=wl.scheme or "A", n_parts_=self.parts, idx=idx,
+                                            cu_kept=cu_kept, kept_total_=Kt, out=self.dec_out,
+                                            workspace=self.ws_d)
+        self.dec_out = (o, lse)
+        ev("decode", 1)
+        return o, lse
+
+    def launches_per_step(self):
+        return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 3
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, torch copy)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)"
+
+
+def load_traffic(stage, wl_name):
+    """DRAM bytes of the stage from a committed ncu summary, if its kernels are unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        d = json.load(open(path))
+    except (OSError, ValueError):
+        return None
+    ent = d.get(wl_name, {}).get(stage)
+    if not ent:
+        return None
+    srcs = [os.path.join(ROOT, p) for p in ent["sources"]]
+    if source_hash(srcs) != ent["source_hash"]:
+        return None
+    return ent["bytes_per_launch"]
+
+
+def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
+    """The fp64 oracle on a bounded sample of the workload's rows; returns (GB/s, sample text)."""
+    import oracle
+    cu = bt.cu_seqlens.numpy().astype(np.int64)
+    order = rows or [(b, h) for h in range(wl.Hkv) for b in range(wl.B)]
+    order = sorted(order, key=lambda r: int(cu[r[0] + 1] - cu[r[0]]))  # shortest rows first
+    done, nbytes, t0 = [], 0, time.perf_counter()
+    for b, h in order:
+        if max_rows is not None and len(done) >= max_rows:
+            break
+        s, e = int(cu[b]), int(cu[b + 1])
+        L = e - s
+        kk = bt.k[h:h + 1, s:e]
+        vv = bt.v[h:h + 1, s:e]
+        one = np.array([0, L], np.int64)
+        qrow = bt.q[b:b + 1, h * wl.G:(h + 1) * wl.G]
+        quant = None
+        if wl.scheme:
+            quant = oracle.quantize_kv(kk, vv, one, wl.scheme)
+        idx = cu_kept = None
+        if wl.oam:
+            idx, cu_kept, _ = oracle.oam_select(qrow, kk, vv, one, wl.G, wl.beta, wl.eps, wl.keep_num,
+                                                wl.keep_den)
+        oracle.decode(qrow, kk, vv, one, wl.G, idx=idx, cu_kept=cu_kept,
+                      quant=None if quant is None else (*quant, wl.scheme))
+        done.append((b, h, L))
+        rowwl = wl.with_(B=1, Hkv=1, lengths=(L,), length_range=None)
+        nbytes += sum(algorithmic_bytes(rowwl, [L]).values())
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sample = (f"{len(done)} (sequence, KV head) rows of the workload, {sum(r[2] for r in done)} tokens, "
+              f"full pipeline per row in the fp64 oracle; {dt:.1f} s")
+    return nbytes / dt / 1e9, sample, dt
+
+
+def run_ours(args, rank, world, local_rank):
+    import sparse_gqa_decode_b200 as sgd
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workloads.config(args.workload)
+    bt = workloads.generate(wl, seed=args.workload)  # the same batch on every rank
+    pipe = Pipeline(sgd, wl, bt, dev)
+    stages = algorithmic_bytes(wl, pipe.lengths)
+    step_bytes = sum(stages.values())
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(max(args.warmup, 3)):
+        pipe.run()
+    torch.cuda.synchronize()
+    st = sgd.workspace_status(pipe.ws_d)
+    if st:
+        raise RuntimeError(f"device status {st:#x} after warm-up")
+
+    names = [n for n in ("quantize", "select", "decode") if n in stages]
+    K = args.steps
+    rec = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
+           for _ in range(K)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(K):
+        flush.fill_(i & 0xff)  # evict the previous step's lines from L2 (untimed)
+        step_ev[i][0].record()
+        pipe.run(rec[i])
+        step_ev[i][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    stage_ms = {n: [r[n][0].elapsed_time(r[n][1]) for r in rec] for n in names}
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * step_bytes * K / (total_ms / 1e3) / 1e9
+
+    # e2e: host buffers through the same calls, copies inside the timed region
+    pin_q, pin_k, pin_v, pin_cu = (x.pin_memory() for x in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    B, Hq, D = bt.q.shape
+    h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    h_lse = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (pin_q, pin_k, pin_v, pin_cu))
+    d2h = h_out.numel() * 4 + h_lse.numel() * 4
+    e2e_steps = max(2, min(K, 5))
+    for _ in range(2):
+        pipe.q.copy_(pin_q, non_blocking=True)
+        pipe.k.copy_(pin_k, non_blocking=True)
+        pipe.v.copy_(pin_v, non_blocking=True)
+        pipe.cu.copy_(pin_cu, non_blocking=True)
+        o, lse = pipe.run()
+        h_out.copy_(o, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        pipe.q.copy_(pin_q, non_blocking=True)
+        pipe.k.copy_(pin_k, non_blocking=True)
+        pipe.v.copy_(pin_v, non_blocking=True)
+        pipe.cu.copy_(pin_cu, non_blocking=True)
+        o, lse = pipe.run()
+        h_out.copy_(o, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    et = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(et.item())
+
+    if rank != 0:
+        return None
+    peak, peak_src = load_peaks()
+    med = {n: statistics.median(v) for n, v in stage_ms.items()}
+    dom = max(med, key=lambda n: med[n])
+    achieved = stages[dom] / (med[dom] / 1e3) / 1e9
+    kernels = {"quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
+               "select": "sgd_oam_select (plan + OAM score + top-K kernels)",
+               "decode": "sgd_decode_attn (plan + split decode + merge kernels)"}
+    srcs = {"quantize": ["sparse_gqa_decode_b200/csrc/quantize.cu"],
+            "select": ["sparse_gqa_decode_b200/csrc/decode.cu", "sparse_gqa_decode_b200/csrc/oam.cu"],
+            "decode": ["sparse_gqa_decode_b200/csrc/decode.cu"]}
+    traffic = load_traffic(dom, wl.name)
+    stage_report = {}
+    for n in names:
+        gbs = stages[n] / (med[n] / 1e3) / 1e9
+        stage_report[n] = {"ms": round(med[n], 4), "algorithmic_bytes": stages[n], "GB_s": round(gbs, 1),
+                           "frac_of_hbm": round(gbs / peak, 4)}
+    line = {
+        "metric": "decode-attn KV GB/s & % of B200 HBM peak at 128K; seq·heads/s, INT8+OAM",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8" if wl.scheme else "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D, "lengths": pipe.lengths,
+            "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
+            "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": args.workload,
+            "step": "quantize_kv -> oam_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn",
+            "l2": "flushed between steps (256 MiB write, untimed); inputs > L2",
+            "parallelism": f"dp{world} (independent copies, no collective)",
+        },
+        "pct_hbm_peak": round(100 * value / world / peak, 2),
+        "seq_heads_per_s": round(world * wl.B * wl.Hq / (ms_per_step / 1e3), 1),
+        "stages": stage_report,
+        "roofline": {"bound": "hbm", "kernel": kernels[dom], "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes": stages[dom]},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": pipe.launches_per_step() * K,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = cpu_baseline_sample(bt, wl, budget_s=20.0)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores, one bounded sample of the workload per step
+# ------------------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = workloads.config(args.workload)
+    bt = workloads.generate(wl, seed=args.workload)
+    cu = bt.cu_seqlens.numpy()
+    rows = [(b, h) for h in range(wl.Hkv) for b in range(wl.B)]
+    shortest = min(rows, key=lambda r: int(cu[r[0] + 1] - cu[r[0]]))
+    for _ in range(args.warmup):
+        cpu_baseline_sample(bt, wl, budget_s=1e9, max_rows=1, rows=[shortest])
+    total_b, total_t = 0.0, 0.0
+    for _ in range(args.steps):
+        gbs, sample, dt = cpu_baseline_sample(bt, wl, budget_s=1e9, max_rows=1, rows=[shortest])
+        total_b += gbs * dt
+        total_t += dt
+    v = total_b / total_t
+    line = {
+        "impl": "reference",
+        "metric": "decode-attn KV GB/s & % of B200 HBM peak at 128K; seq·heads/s, INT8+OAM",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total_t / args.steps, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D,
+                   "lengths": [int(x) for x in bt.lengths], "parallelism": "host cores (1 thread)"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"per step: the shortest (sequence, KV head) row, {sample}"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit without work
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
