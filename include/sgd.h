@@ -74,6 +74,7 @@ typedef enum { SGD_SCHEME_A = 0, SGD_SCHEME_B = 1 } sgd_scheme;
 #define SGD_ERR_CUDA -6          /* a CUDA runtime call or launch failed */
 #define SGD_ERR_DEVICE -7        /* current device is not sm_100 */
 #define SGD_ERR_ARG -8           /* any other invalid argument */
+#define SGD_ERR_SCRATCH_LIMIT -9 /* needs more scratch than SGD_NOALLOC_SCRATCH_BYTES */
 
 /* device status bits (status word at the start of the workspace) */
 #define SGD_STATUS_EMPTY_SEQUENCE 0x1 /* a sequence has length < 1 */
@@ -189,6 +190,31 @@ int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedul
 int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode,
                       int32_t *segs, int64_t max_segs, int32_t *n_segs,
                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_decode_attn_noalloc -- sgd_decode_attn for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it serves callers, not the method.
+ *   Some callers cannot provide a workspace: a plugin inside a framework that owns all device
+ *   memory and offers its plugins no allocator, or a latency-critical loop that may not call
+ *   cudaMalloc (it can synchronise the whole device and its latency is unbounded).  This call
+ *   takes the same arguments as sgd_decode_attn minus the workspace and computes the same out
+ *   and lse with the same kernels.  Their scratch lives in one device array inside the
+ *   library, SGD_NOALLOC_SCRATCH_BYTES long, that every GPU which loads the library holds
+ *   until the process exits.  Nothing is allocated or freed.
+ * status   optional [1] int32 device output: the SGD_STATUS_* bits of this call (or NULL)
+ * Returns SGD_ERR_SCRATCH_LIMIT, before launching anything, when the problem needs more scratch
+ * than the array holds (sgd_workspace_size(SGD_OP_DECODE, ...) > SGD_NOALLOC_SCRATCH_BYTES).
+ * The first call on a device looks up the array's device address (once per device, with that
+ * device current); make that first call before any stream capture.  All calls on a device
+ * share the array and each starts from the previous call's contents (the call clears the
+ * status word itself), so calls whose GPU work overlaps, e.g. on two streams, race: serialise
+ * them.
+ */
+#define SGD_NOALLOC_SCRATCH_BYTES (4u << 20)
+int sgd_decode_attn_noalloc(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                            const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
+                            int schedule, int n_splits, float *out, float *lse, int32_t *status,
+                            void *stream);
 
 /* Copies the device status word of `workspace` to *status (host) after
  * synchronising `stream`.  The only call that synchronises. */

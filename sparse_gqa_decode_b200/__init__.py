@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "lib", "quantize_kv", "oam_select", "decode_attn", "plan_segments", "workspace_status",
+    "lib", "quantize_kv", "oam_select", "decode_attn", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "n_parts", "SGD_F32", "SGD_BF16", "SGD_I8",
     "SCHEME_A", "SCHEME_B", "STATUS_BITS",
 ]
@@ -67,6 +67,7 @@ lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
+lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]
 
 _DT = {torch.float32: SGD_F32, torch.bfloat16: SGD_BF16, torch.int8: SGD_I8}
 
@@ -197,6 +198,27 @@ def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_se
                                int(kept_total_), schedule, n_splits, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
                                _stream(stream)), "sgd_decode_attn")
     return o, lse, ws
+
+
+def decode_attn_noalloc(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                        k_scale=None, v_scale=None, scheme: str = "A", n_parts_: int = 0,
+                        idx=None, cu_kept=None, kept_total_: int = 0, schedule: int = 0, n_splits: int = 0,
+                        out=None, status=None, stream=None):
+    """decode_attn without a workspace: the library's built-in device scratch array is used
+    (for callers that cannot allocate).  ``out`` = (out, lse) and ``status`` ([1] int32) are
+    optional preallocated device outputs.  Returns (out, lse)."""
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, sch, n_parts_)
+    B = cu_seqlens.numel() - 1
+    if out is None:
+        o = torch.empty((B, k.shape[0] * G, k.shape[2]), dtype=torch.float32, device=k.device)
+        lse = torch.empty((B, k.shape[0] * G), dtype=torch.float32, device=k.device)
+    else:
+        o, lse = out
+    _check(lib.sgd_decode_attn_noalloc(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
+                                       int(kept_total_), schedule, n_splits, _ptr(o), _ptr(lse), _ptr(status),
+                                       _stream(stream)), "sgd_decode_attn_noalloc")
+    return o, lse
 
 
 def decode_num_ctas(k, v, cu_seqlens, G: int, indexed: bool = False, schedule: int = 0, n_splits: int = 0) -> int:

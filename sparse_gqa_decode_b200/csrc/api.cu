@@ -142,6 +142,7 @@ const char *sgd_error_string(int code) {
         case SGD_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
         case SGD_ERR_DEVICE: return "the current device is not an sm_100 GPU";
         case SGD_ERR_ARG: return "invalid argument";
+        case SGD_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than SGD_NOALLOC_SCRATCH_BYTES";
         default: return "unknown status";
     }
 }
