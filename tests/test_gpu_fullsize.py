@@ -1,0 +1,121 @@
+"""Full-size workloads in the launch configuration bench.py times (automatic split over all SMs),
+CUDA path vs the fp64 oracle.  The GPU computes every row; the oracle recomputes sampled
+(sequence, KV head) rows one by one (including the shortest and longest), and the INT8 codes and
+scales and the kept index sets are compared in full."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 1e-2
+LSE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def sgd():
+    from sparse_gqa_decode_b200 import build
+    build.build()
+    import sparse_gqa_decode_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return m
+
+
+def sample_rows(bt, n_extra=3, seed=0):
+    L = bt.lengths
+    rows = {(int(np.argmin(L)), 0), (int(np.argmax(L)), bt.wl.Hkv - 1)}
+    rng = np.random.default_rng(seed)
+    while len(rows) < 2 + n_extra:
+        rows.add((int(rng.integers(bt.wl.B)), int(rng.integers(bt.wl.Hkv))))
+    return sorted(rows)
+
+
+def compare_rows(out, lse, ref_out, ref_lse, rows, G):
+    out = out.double().cpu().numpy()
+    lse = lse.double().cpu().numpy()
+    for b, h in rows:
+        sl = slice(h * G, (h + 1) * G)
+        scale = np.abs(ref_out[b, sl]).max()
+        assert np.abs(out[b, sl] - ref_out[b, sl]).max() <= OUT_TOL * scale, (b, h)
+        assert np.abs(lse[b, sl] - ref_lse[b, sl]).max() <= LSE_TOL, (b, h)
+
+
+def test_config2_bf16_32k(sgd):
+    bt = workloads.generate(workloads.config(2))
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    out, lse, ws = sgd.decode_attn(q, 8, k, v, cu)
+    assert sgd.workspace_status(ws) == 0
+    rows = sample_rows(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, rows=rows)
+    compare_rows(out, lse, *ref, rows, 8)
+
+
+def test_config3_ragged_both_schedules(sgd):
+    bt = workloads.generate(workloads.config(3))
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    o0, l0, ws0 = sgd.decode_attn(q, 8, k, v, cu, schedule=0)
+    o1, l1, ws1 = sgd.decode_attn(q, 8, k, v, cu, schedule=1)
+    assert sgd.workspace_status(ws0) == 0 and sgd.workspace_status(ws1) == 0
+    rows = sample_rows(bt, n_extra=4)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, rows=rows)
+    compare_rows(o0, l0, *ref, rows, 8)
+    compare_rows(o1, l1, *ref, rows, 8)
+    # the two schedules agree on every row
+    scale = o1.abs().max().item()
+    assert (o0 - o1).abs().max().item() <= OUT_TOL * scale
+    assert (l0 - l1).abs().max().item() <= LSE_TOL
+
+
+@pytest.mark.parametrize("scheme", ["A", "B"])
+def test_config4_int8_128k(sgd, scheme):
+    bt = workloads.generate(workloads.config(4))
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, wsq = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+    del k, v
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=scheme,
+                                   n_parts_=sgd.n_parts(bt.lengths))
+    assert sgd.workspace_status(wsq) == 0 and sgd.workspace_status(ws) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    assert np.array_equal(ks.cpu().numpy().reshape(quant[2].shape), quant[2])
+    assert np.array_equal(vs.cpu().numpy(), quant[3])
+    for h in range(bt.wl.Hkv):  # every code, one head at a time
+        assert np.array_equal(kc[h].cpu().numpy(), quant[0][h]), h
+        assert np.array_equal(vc[h].cpu().numpy(), quant[1][h]), h
+    rows = sample_rows(bt, n_extra=2)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, quant=(*quant, scheme), rows=rows)
+    compare_rows(out, lse, *ref, rows, 8)
+
+
+def test_config5_oam_int8a(sgd):
+    wl = workloads.config(5)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    idx, cu_kept, wss = sgd.oam_select(q, k, v, cu, wl.G, wl.beta, wl.eps, wl.keep_num, wl.keep_den, bt.lengths)
+    out, lse, ws = sgd.decode_attn(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                   n_parts_=sgd.n_parts(bt.lengths), idx=idx, cu_kept=cu_kept,
+                                   kept_total_=idx.shape[1])
+    assert sgd.workspace_status(wss) == 0 and sgd.workspace_status(ws) == 0
+    # every row's kept set against the oracle's top-K (near-ties within 1e-4 exempt)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, wl.beta, wl.eps,
+                                                wl.keep_num, wl.keep_den)
+    assert cu_kept.cpu().tolist() == ref_cu.tolist()
+    got = idx.cpu().numpy()
+    n_diff = 0
+    for (b, h), s in scores.items():
+        a, e = int(ref_cu[b]), int(ref_cu[b + 1])
+        kth = np.sort(s)[::-1][e - a - 1]
+        g, w = set(got[h, a:e].tolist()), set(ref_idx[h, a:e].tolist())
+        assert (np.diff(got[h, a:e]) > 0).all()
+        for t in g ^ w:
+            assert abs(s[t] - kth) <= 1e-4, (b, h, t)
+        n_diff += len(g ^ w)
+    assert n_diff <= 8
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    rows = sample_rows(bt, n_extra=3)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
+                        quant=(*quant, "A"), rows=rows)
+    compare_rows(out, lse, *ref, rows, wl.G)
