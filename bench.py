@@ -63,11 +63,17 @@ def algorithmic_bytes(wl, lengths):
     q = B * Hkv * G * D * 2
     out = B * Hkv * G * (D + 1) * 4
     st = {}
-    if wl.scheme:
-        st["quantize"] = kv_bf16 + 2 * Hkv * T * D + (Hkv * P * 4 if wl.scheme == "A" else 4) + 4
+    codes_out = 2 * Hkv * T * D + (Hkv * P * 4 if wl.scheme == "A" else 4) + 4
     if wl.oam:
         Kt = sum(kept_of(L, wl.keep_num, wl.keep_den) for L in lengths)
-        st["select"] = kv_bf16 + q + Hkv * Kt * 4 + (B + 1) * 4
+        sel_out = q + Hkv * Kt * 4 + (B + 1) * 4
+    if wl.scheme and wl.oam:  # one call reads K and V once for both
+        st["quantize_select"] = kv_bf16 + codes_out + sel_out
+    elif wl.scheme:
+        st["quantize"] = kv_bf16 + codes_out
+    elif wl.oam:
+        st["select"] = kv_bf16 + sel_out
+    if wl.oam:
         n_att = Kt
         idx_bytes = Hkv * Kt * 4
     else:
@@ -158,15 +164,23 @@ class Pipeline:
                 record[name][i].record()
 
         kc, vc, ks, vs = self.k, self.v, None, None
-        if wl.scheme:
+        idx = cu_kept = None
+        Kt = 0
+        if wl.scheme and wl.oam:
+            ev("quantize_select", 0)
+            kc, vc, ks, vs, idx, cu_kept, self.ws_q = sgd.quantize_select(
+                self.q, self.k, self.v, self.cu, wl.G, wl.beta, wl.eps, wl.keep_num, wl.keep_den, wl.scheme,
+                self.lengths, out=self.qout, workspace=self.ws_q)
+            self.qout = (kc, vc, ks, vs, idx, cu_kept)
+            Kt = idx.shape[1]
+            ev("quantize_select", 1)
+        elif wl.scheme:
             ev("quantize", 0)
             kc, vc, ks, vs, self.ws_q = sgd.quantize_kv(self.k, self.v, self.cu, wl.scheme, self.lengths,
                                                         out=self.qout, workspace=self.ws_q)
             self.qout = (kc, vc, ks, vs)
             ev("quantize", 1)
-        idx = cu_kept = None
-        Kt = 0
-        if wl.oam:
+        elif wl.oam:
             ev("select", 0)
             idx, cu_kept, self.ws_s = sgd.oam_select(self.q, self.k, self.v, self.cu, wl.G, wl.beta, wl.eps,
                                                      wl.keep_num, wl.keep_den, self.lengths, out=self.sel_out,
@@ -184,6 +198,8 @@ class Pipeline:
         return o, lse
 
     def launches_per_step(self):
+        if self.wl.scheme and self.wl.oam:
+            return 4 + 3  # plan, score+quantize, V codes, top-K; plan, decode, merge
         return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 3
 
 
@@ -274,7 +290,7 @@ def run_ours(args, rank, world, local_rank):
     if st:
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
-    names = [n for n in ("quantize", "select", "decode") if n in stages]
+    names = [n for n in ("quantize_select", "quantize", "select", "decode") if n in stages]
     K = args.steps
     rec = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
            for _ in range(K)]
@@ -345,10 +361,13 @@ def run_ours(args, rank, world, local_rank):
     med = {n: statistics.median(v) for n, v in stage_ms.items()}
     dom = max(med, key=lambda n: med[n])
     achieved = stages[dom] / (med[dom] / 1e3) / 1e9
-    kernels = {"quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
+    kernels = {"quantize_select": "sgd_quantize_select (plan + fused OAM score/K quantise + V codes + top-K)",
+               "quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
                "select": "sgd_oam_select (plan + OAM score + top-K kernels)",
                "decode": "sgd_decode_attn (plan + split decode + merge kernels)"}
-    srcs = {"quantize": ["sparse_gqa_decode_b200/csrc/quantize.cu"],
+    srcs = {"quantize_select": ["sparse_gqa_decode_b200/csrc/decode.cu", "sparse_gqa_decode_b200/csrc/quantize.cu",
+                                "sparse_gqa_decode_b200/csrc/oam.cu"],
+            "quantize": ["sparse_gqa_decode_b200/csrc/quantize.cu"],
             "select": ["sparse_gqa_decode_b200/csrc/decode.cu", "sparse_gqa_decode_b200/csrc/oam.cu"],
             "decode": ["sparse_gqa_decode_b200/csrc/decode.cu"]}
     traffic = load_traffic(dom, wl.name)
@@ -374,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
             "workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D, "lengths": pipe.lengths,
             "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
             "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": args.workload,
-            "step": "quantize_kv -> oam_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn",
+            "step": "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn",
             "l2": "flushed between steps (256 MiB write, untimed); inputs > L2",
             "parallelism": f"dp{world} (independent copies, no collective)",
         },

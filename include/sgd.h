@@ -106,6 +106,7 @@ typedef struct {
 #define SGD_OP_QUANTIZE 0
 #define SGD_OP_OAM_SELECT 1
 #define SGD_OP_DECODE 2
+#define SGD_OP_QUANTIZE_SELECT 3
 
 /*
  * sgd_quantize_kv -- INT8 KV cache ([TD] section 6).
@@ -143,6 +144,23 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                    float beta, float eps, int keep_num, int keep_den,
                    int32_t *idx, int32_t *cu_kept, int64_t kept_total,
                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_quantize_select -- sgd_quantize_kv and sgd_oam_select of one cache in one call, with the
+ * same outputs ([TD] sections 6 and 3; the pages' pipeline, section 7, runs both on the same
+ * cache).  With a BF16 cache and BF16 q (D in {64, 128}) the K and V of every token are read
+ * from HBM once for both: the OAM score pass also writes the scheme-A K codes and scales (or
+ * takes max|K| for scheme B) and max|V|; a second pass writes the V codes (and the scheme-B K
+ * codes), then the top-K runs.  Other dtypes run the two calls one after the other.
+ * Arguments as in sgd_quantize_kv and sgd_oam_select; kv must be BF16 or F32.
+ * Workspace: sgd_workspace_size(SGD_OP_QUANTIZE_SELECT, ...).
+ */
+int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                        float beta, float eps, int keep_num, int keep_den,
+                        sgd_scheme scheme, int64_t n_parts,
+                        int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                        int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * sgd_decode_attn -- split-KV flash-decoding ([TD] section 5, [CD] eq. 5-7).

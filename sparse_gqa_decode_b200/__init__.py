@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "lib", "quantize_kv", "oam_select", "decode_attn", "decode_attn_noalloc", "plan_segments", "workspace_status",
+    "lib", "quantize_kv", "oam_select", "quantize_select", "decode_attn", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "n_parts", "SGD_F32", "SGD_BF16", "SGD_I8",
     "SCHEME_A", "SCHEME_B", "STATUS_BITS",
 ]
@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libsgd.so")
 
 SGD_F32, SGD_BF16, SGD_I8 = 0, 1, 2
 SCHEME_A, SCHEME_B = 0, 1
-OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE = 0, 1, 2
+OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE, OP_QUANTIZE_SELECT = 0, 1, 2, 3
 PARTITION = 64
 STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index"}
 
@@ -67,6 +67,8 @@ lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
+lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
+                                    _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]
 
 _DT = {torch.float32: SGD_F32, torch.bfloat16: SGD_BF16, torch.int8: SGD_I8}
@@ -176,6 +178,32 @@ def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
     _check(lib.sgd_oam_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, _ptr(idx),
                               _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)), "sgd_oam_select")
     return idx, cu_kept, ws
+
+
+def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                    beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
+                    out=None, workspace=None, stream=None):
+    """quantize_kv and oam_select of one cache in one call (K and V read once for both).
+    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws)."""
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    Hkv, T, D = k.shape
+    parts = n_parts(lengths) if sch == SCHEME_A else 0
+    Kt = kept_total(lengths, keep_num, keep_den)
+    kv = _kv(k, v, cu_seqlens)
+    if out is None:
+        kc = torch.empty((Hkv, T, D), dtype=torch.int8, device=k.device)
+        vc = torch.empty_like(kc)
+        ks = torch.empty((Hkv, parts) if sch == SCHEME_A else (1,), dtype=torch.float32, device=k.device)
+        vs = torch.empty(1, dtype=torch.float32, device=k.device)
+        idx = torch.empty((Hkv, Kt), dtype=torch.int32, device=k.device)
+        cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
+    else:
+        kc, vc, ks, vs, idx, cu_kept = out
+    ws = _workspace(workspace_size(OP_QUANTIZE_SELECT, kv, G), k.device, workspace)
+    _check(lib.sgd_quantize_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, sch,
+                                   parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(idx), _ptr(cu_kept), Kt,
+                                   _ptr(ws), ws.numel(), _stream(stream)), "sgd_quantize_select")
+    return kc, vc, ks, vs, idx, cu_kept, ws
 
 
 def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,

@@ -154,6 +154,7 @@ size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_s
     DevInfo *dev;
     if (current_device(&dev) != SGD_OK) return 0;
     int n_req = 0;
+    if (op == SGD_OP_QUANTIZE_SELECT) op = SGD_OP_OAM_SELECT;  // the fused call needs the select layout
     const bool score = op == SGD_OP_OAM_SELECT;
     if (op != SGD_OP_DECODE && !score) return 0;
     // indexed or not does not change the count
@@ -243,6 +244,78 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
     a.plan = pv;
     a.status = &hdr->status;
     int e = launch_decode(a, kv->dtype, q_dtype, false, true, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
+                    &hdr->status, s);
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
+                        int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
+                        int8_t *v_codes, float *k_scale, float *v_scale, int32_t *idx, int32_t *cu_kept,
+                        int64_t kept_total, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    if (!q || !idx || !cu_kept || !workspace || !k_codes || !v_codes || !k_scale || !v_scale) return SGD_ERR_NULL;
+    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (scheme != SGD_SCHEME_A && scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+    if (scheme == SGD_SCHEME_A && (n_parts < kv->B || n_parts > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
+    if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
+    if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
+    if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
+    if (!aligned16(q) || !aligned16(workspace) || !aligned16(k_codes) || !aligned16(v_codes)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u) ||
+        (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        return SGD_ERR_ALIGN;
+    if (decode_family(kv->dtype, q_dtype, kv->D, true) != kFamilyMma) {
+        // no fused kernel for this dtype: the two passes one after the other
+        rc = sgd_quantize_kv(kv, scheme, n_parts, k_codes, v_codes, k_scale, v_scale, workspace, workspace_bytes,
+                             stream);
+        if (rc != SGD_OK) return rc;
+        return sgd_oam_select(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, idx, cu_kept, kept_total, workspace,
+                              workspace_bytes, stream);
+    }
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    // tiles of the fused pass must be whole 64-token partitions: plan granule 64
+    launch_plan(kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, kAutoMinChunk, 0, pv, hdr, s, kPart);
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.cu_seq = kv->cu_seqlens;
+    a.k = kv->k;
+    a.v = kv->v;
+    a.B = kv->B;
+    a.Hkv = kv->Hkv;
+    a.G = G;
+    a.D = kv->D;
+    a.T = kv->T;
+    a.n_parts = scheme == SGD_SCHEME_A ? n_parts : 0;
+    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
+    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
+    a.beta = beta;
+    a.eps = eps;
+    a.scores = reinterpret_cast<float *>(ws + L.scores);
+    a.qscheme = scheme;
+    a.k_codes = k_codes;
+    a.k_scale_out = k_scale;
+    a.amax_bits = hdr->amax_bits;
+    a.plan = pv;
+    a.status = &hdr->status;
+    int e = launch_score_quantize(a, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    e = launch_quantize_global(kv->k, kv->v, kv->dtype, kv->Hkv, kv->D, kv->T, scheme, k_codes, v_codes, k_scale,
+                               v_scale, hdr, dev->sms, s);
     if (e != 0) return SGD_ERR_CUDA;
     e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
                     &hdr->status, s);

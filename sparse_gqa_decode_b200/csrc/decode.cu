@@ -34,6 +34,7 @@
 
 #include "internal.h"
 #include "plan.cuh"
+#include "quant.cuh"
 
 namespace sgd {
 
@@ -53,7 +54,7 @@ template <int D_, int GT_, bool I8_, bool IDX_, int MODE_>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
-    static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score
+    static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
     static constexpr int NW = 4;        // consumer warps
     static constexpr int SUB = I8 ? 2 : 1;  // 16-token sub-tiles per consumer warp per stage
     static constexpr int ROWS = NW * 16 * SUB;
@@ -64,12 +65,14 @@ struct MmaCfg {
     static constexpr int TILE = ROWS * ROWB;  // bytes of one tensor per stage
     static constexpr int STAGES = 3;
     static constexpr int KB = D / 16;
-    static constexpr int THREADS = (NW + 1) * 32;
+    static constexpr int NQ = (MODE == 2) ? 4 : 0;  // K-quantising warps (mode 2)
+    static constexpr int THREADS = (NW + NQ + 1) * 32;
     static constexpr int SMEM_STAGES = STAGES * 2 * TILE;
-    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16;
+    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + 2 * 4 * 4;
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
-    static_assert(!(I8 && MODE == 1), "scores read the unquantised cache");
+    static_assert(!(I8 && MODE >= 1), "scores read the unquantised cache");
+    static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
 // ------------------------------------------------------------------------------------------
@@ -295,6 +298,153 @@ __device__ __forceinline__ void pv_subtile(uint32_t vbase, int rb, int lane, con
     }
 }
 
+// Score mode for one 16-token sub-tile: OAM score of every token (max over the group's heads
+// of the logit, plus beta * ln(|v| + eps)); mode 2 also quantises the K rows of the tile (one
+// scheme-A partition: the four warps' maxima meet through shared memory) or accumulates max|K|
+// (scheme B), and accumulates max|V|.  Every consumer warp calls this for every tile.
+template <class C>
+__device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbase, uint32_t vbase, int rb,
+                                              int32_t j0, int32_t t, int32_t t1, bool ready, int b, int kvh,
+                                              int pA, int t4, int lane, int warp,
+                                              const uint32_t (&qf)[C::GT][C::KB][2], float &run_kmax,
+                                              float &run_vmax, float *kmxs, int parity) {
+    const bool act = ready && j0 < t1;
+    float sacc[C::GT][4];
+    if (act) {
+        qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
+    } else {
+#pragma unroll
+        for (int gt = 0; gt < C::GT; ++gt) sacc[gt][0] = sacc[gt][1] = sacc[gt][2] = sacc[gt][3] = 0.f;
+    }
+    float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+    for (int gt = 0; gt < C::GT; ++gt) {
+        const int g0 = 8 * gt + 2 * t4;
+        if (g0 < a.G) {
+            mA = fmaxf(mA, sacc[gt][0]);
+            mB = fmaxf(mB, sacc[gt][2]);
+        }
+        if (g0 + 1 < a.G) {
+            mA = fmaxf(mA, sacc[gt][1]);
+            mB = fmaxf(mB, sacc[gt][3]);
+        }
+    }
+    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+    // lane pair (rho, half) owns half of the row rb + rho of the K and V tiles
+    const int rho = lane >> 1, half = lane & 1;
+    const int vr = rb + rho;
+    const int32_t j = j0 + rho;
+    const bool vrow = act && j < t1;
+    constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
+    constexpr int NH = CPR / 2;
+    float ss = 0.f, vmx = 0.f;
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const int c = half * NH + i, bx = c >> 3, cc = c & 7;
+        const uint4 w = lds128(vbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
+            if constexpr (C::MODE == 2) vmx = fmaxf(vmx, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const int src = 4 * mma_row_perm(rho & 7);
+    const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
+    const float rmax = (rho < 8) ? rA : rB;
+    if (half == 0 && vrow) {
+        float sc = rmax * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
+        if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
+        a.scores[(int64_t)kvh * a.T + a.cu_seq[b] + j] = sc;
+    }
+    if constexpr (C::MODE == 2) {
+        if (vrow) run_vmax = fmaxf(run_vmax, vmx);
+    }
+}
+
+// Mode 2, K-quantising warp qw: rows 16*qw .. 16*qw+15 of every tile (a tile is one scheme-A
+// partition).  Scheme A: the tile's max|K| is met across the NQ warps through shared memory,
+// then each warp writes the codes of its rows and warp 0 the partition scale.  Scheme B: only
+// the running max|K|.  Every quantising warp takes every tile.
+template <class C>
+__device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                               volatile int32_t *abort_flag, float *kmxs, const int32_t *cu_rows,
+                                               int cta, int qw, int lane) {
+    SegCursor cur;
+    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    int stage = 0, tile_no = 0;
+    uint32_t phase = 0;
+    int row, slot;
+    int32_t t0, t1;
+    float run_kmax = 0.f;
+    constexpr int CPR = C::ROWB / 16, NH = CPR / 2;
+    const int rho = lane >> 1, half = lane & 1;
+    const int vr = 16 * qw + rho;
+    while (cur.next(row, t0, t1, slot)) {
+        const int b = row % a.B, kvh = row / a.B;
+        for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
+            const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
+            const uint32_t kbase = smem_u32(smem + stage * 2 * C::TILE);
+            const int32_t j = t + vr;
+            const bool vrow = ready && j < t1;
+            uint4 kw[NH];
+            float kmx = 0.f;
+#pragma unroll
+            for (int i = 0; i < NH; ++i) {
+                const int c = half * NH + i, bx = c >> 3, cc = c & 7;
+                kw[i] = lds128(kbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
+                const uint32_t ww[4] = {kw[i].x, kw[i].y, kw[i].z, kw[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    kmx = fmaxf(kmx, fmaxf(fabsf(__uint_as_float(ww[e] << 16)),
+                                           fabsf(__uint_as_float(ww[e] & 0xffff0000u))));
+            }
+            if (!vrow) kmx = 0.f;
+            if (a.qscheme == SGD_SCHEME_B) {
+                run_kmax = fmaxf(run_kmax, kmx);
+            } else {
+                kmx = warp_max(kmx);
+                const int parity = tile_no & 1;
+                if (lane == 0) kmxs[parity * C::NQ + qw] = kmx;
+                named_barrier_sync(2, C::NQ * 32);
+                float tm = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::NQ; ++w) tm = fmaxf(tm, kmxs[parity * C::NQ + w]);
+                const float sc = __fdiv_rn(tm, 127.f);
+                const float r = (sc != 0.f) ? __frcp_rn(sc) : 0.f;
+                if (vrow) {
+                    int8_t *dst = a.k_codes + ((int64_t)kvh * a.T + a.cu_seq[b] + j) * C::D + half * (C::D / 2);
+#pragma unroll
+                    for (int i = 0; i < NH; ++i) {
+                        float x[8];
+                        Vec<__nv_bfloat16>::unpack(kw[i], x);
+                        store_codes<8>(dst + i * 8, x, sc, r);
+                    }
+                }
+                // (the partition count was checked against the host's n_parts before any write)
+                if (qw == 0 && lane == 0 && ready)
+                    a.k_scale_out[(int64_t)kvh * a.n_parts + a.plan.seq_part0[b] + t / kPart] = sc;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+    if (a.qscheme == SGD_SCHEME_B) {
+        run_kmax = warp_max(run_kmax);
+        if (lane == 0) atomicMax(&a.amax_bits[0], __float_as_uint(run_kmax));
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
@@ -308,12 +458,13 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     uint64_t *empty = full + C::STAGES;
     float *ml = reinterpret_cast<float *>(empty + C::STAGES);  // [NW][NG][2]: m, l
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(ml + C::NW * C::NG * 2);
+    float *kmxs = ml + C::NW * C::NG * 2 + 4;  // [2][NW] per-warp max|K| of the current tile (mode 2)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], C::IDX ? 32u : 1u);
-            mbar_init(&empty[s], (uint32_t)C::NW);
+            mbar_init(&empty[s], (uint32_t)(C::NW + C::NQ));
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -321,11 +472,24 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     __syncthreads();
     const int cta = blockIdx.x;
     if (a.plan.cta_begin[cta] >= a.plan.cta_begin[cta + 1]) return;
+    if constexpr (C::MODE == 2) {
+        // scheme-A scales are written at kvh * n_parts + (partition): the device count must agree
+        if (a.qscheme == SGD_SCHEME_A && a.plan.seq_part0[a.B] != a.n_parts) {
+            if (threadIdx.x == 0) atomicOr(a.status, SGD_STATUS_SIZE_MISMATCH);
+            return;
+        }
+    }
     const int32_t *cu_rows = C::IDX ? a.cu_kept : a.cu_seq;
 
-    if (warp == C::NW) {
+    if (warp == C::NW + C::NQ) {
         mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, cu_rows, cta, lane);
         return;
+    }
+    if constexpr (C::NQ > 0) {
+        if (warp >= C::NW) {
+            quant_consumer<C>(a, smem, full, empty, abort_flag, kmxs, cu_rows, cta, warp - C::NW, lane);
+            return;
+        }
     }
 
     const int g4 = lane >> 2, t4 = lane & 3;
@@ -336,6 +500,8 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     uint32_t phase = 0;
     int row, slot;
     int32_t t0, t1;
+    float run_kmax = 0.f, run_vmax = 0.f;  // mode 2
+    int tile_no = 0;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
         const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
@@ -364,56 +530,16 @@ __global__ void __launch_bounds__(C::THREADS, 2)
             for (int s = 0; s < C::SUB; ++s) {
                 const int rb = 16 * (s * C::NW + warp);
                 const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
+                if constexpr (C::MODE >= 1) {
+                    score_subtile<C>(a, kbase, vbase, rb, j0, t, t1, ready, b, kvh, pA, t4, lane, warp, qf, run_kmax,
+                                     run_vmax, kmxs, tile_no & 1);
+                    continue;
+                }
                 if (j0 >= t1 || !ready) continue;
                 float sacc[C::GT][4];
                 qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
                 const bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
-                if constexpr (C::MODE == 1) {
-                    // OAM score: max over the group's heads of the logit, plus beta * ln(|v| + eps)
-                    float mA = -INFINITY, mB = -INFINITY;
-#pragma unroll
-                    for (int gt = 0; gt < C::GT; ++gt) {
-                        const int g0 = 8 * gt + 2 * t4;
-                        if (g0 < a.G) {
-                            mA = fmaxf(mA, sacc[gt][0]);
-                            mB = fmaxf(mB, sacc[gt][2]);
-                        }
-                        if (g0 + 1 < a.G) {
-                            mA = fmaxf(mA, sacc[gt][1]);
-                            mB = fmaxf(mB, sacc[gt][3]);
-                        }
-                    }
-                    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
-                    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
-                    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
-                    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-                    const int rho = lane >> 1, half = lane & 1;
-                    const int vr = rb + rho;
-                    float ss = 0.f;
-                    constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
-#pragma unroll
-                    for (int i = 0; i < CPR / 2; ++i) {
-                        const int c = half * (CPR / 2) + i, bx = c >> 3, cc = c & 7;
-                        const uint4 w = lds128(vbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
-                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
-                            ss = fmaf(lo, lo, ss);
-                            ss = fmaf(hi, hi, ss);
-                        }
-                    }
-                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                    const int src = 4 * mma_row_perm(rho & 7);
-                    const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
-                    const float rmax = (rho < 8) ? rA : rB;
-                    const int32_t j = j0 + rho;
-                    if (half == 0 && j < t1) {
-                        float sc = rmax * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
-                        if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
-                        a.scores[(int64_t)kvh * a.T + a.cu_seq[b] + j] = sc;
-                    }
-                } else {
+                {
                     // row (token) factors: scheme-A K scale of the token's 64-token partition
                     float rfA = 1.f, rfB = 1.f;
                     if constexpr (C::I8) {
@@ -475,6 +601,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                     pv_subtile<C>(vbase, rb, lane, pb, o);
                 }
             }
+            ++tile_no;
             const bool last = (t + C::ROWS >= t1);
             if (C::MODE == 0 && last) {
                 // ---- segment epilogue: combine the four warps' (m, l, O) in this stage's memory ----
@@ -535,6 +662,10 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                 phase ^= 1;
             }
         }
+    }
+    if constexpr (C::MODE == 2) {
+        run_vmax = warp_max(run_vmax);
+        if (lane == 0) atomicMax(&a.amax_bits[1], __float_as_uint(run_vmax));
     }
 }
 
@@ -852,6 +983,14 @@ int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, 
         default:
             return a.D == 128 ? launch_generic<128, int8_t, 0>(a, indexed, n_cta, s) : launch_generic<64, int8_t, 0>(a, indexed, n_cta, s);
     }
+}
+
+int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s) {
+    if (n_cta <= 0) return 0;
+    const bool g2 = a.G > 8;
+    if (a.D == 128)
+        return g2 ? launch_mma<MmaCfg<128, 2, false, false, 2>>(a, n_cta, s) : launch_mma<MmaCfg<128, 1, false, false, 2>>(a, n_cta, s);
+    return g2 ? launch_mma<MmaCfg<64, 2, false, false, 2>>(a, n_cta, s) : launch_mma<MmaCfg<64, 1, false, false, 2>>(a, n_cta, s);
 }
 
 int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s) {

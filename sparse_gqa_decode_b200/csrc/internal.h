@@ -22,6 +22,11 @@ struct DecodeArgs {
     float sm_scale;          // 1 / sqrt(D)
     float beta, eps;         // score mode
     float *scores;           // score mode output [Hkv, T]
+    // score + quantize mode (fused first pass of sgd_quantize_select)
+    int qscheme;             // SGD_SCHEME_A: K codes and partition scales here; B: max|K| only
+    int8_t *k_codes;         // [Hkv, T, D]
+    float *k_scale_out;      // [Hkv, n_parts]
+    uint32_t *amax_bits;     // [2]: max|K| (scheme B), max|V| as float bits
     PlanView plan;
     float *o_part;           // [slots, G, D]
     float *lse_part;         // [slots, G]
@@ -33,7 +38,7 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 
 // plan.cu
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
-                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s);
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 
@@ -45,9 +50,16 @@ int decode_ctas_per_sm(sgd_dtype kv_dtype, sgd_dtype q_dtype, int D, int G, bool
 // Launches the split decode (or score) kernel over n_cta CTAs; returns a cudaError_t.
 int launch_decode(const DecodeArgs &a, sgd_dtype kv_dtype, sgd_dtype q_dtype, bool indexed, bool score,
                   int n_cta, cudaStream_t s);
+// Fused first pass of sgd_quantize_select (bf16 cache, bf16 q): OAM scores, scheme-A K codes
+// and scales (or max|K| for scheme B) and max|V|.  Needs a plan built with granule kPart.
+int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s);
 int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s);
 
 // quantize.cu
+// Second pass: codes of V (and of K for scheme B) with the global scales in hdr->amax_bits.
+int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
+                           sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
+                           const WsHeader *hdr, int sm_count, cudaStream_t s);
 int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
                     int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
                     float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s);

@@ -1,5 +1,6 @@
 // plan.cu -- the split-KV partition kernel (one CTA) and its inspection kernel.
-// The rule is stated in plan.cuh.
+// The rule is stated in plan.cuh (granule 16 for decode; 64 for the fused score+quantize
+// pass, whose tiles must coincide with the 64-token scheme-A partitions).
 #include "internal.h"
 #include "plan.cuh"
 #include "scan.cuh"
@@ -10,12 +11,15 @@ namespace sgd {
 // cu_seq: cu_seqlens (for the scheme-A partition offsets of each sequence).
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu_len,
                                                     const int32_t *__restrict__ cu_seq, int B, int Hkv,
-                                                    int n_req, int min_chunk, int mode, PlanView pv,
-                                                    WsHeader *hdr) {
+                                                    int n_req, int min_chunk, int mode, int granule,
+                                                    PlanView pv, WsHeader *hdr) {
     __shared__ int32_t sm[33];
     const int tid = threadIdx.x;
     const int R = B * Hkv;
-    if (tid == 0) hdr->status = 0;
+    if (tid == 0) {
+        hdr->status = 0;
+        hdr->amax_bits[0] = hdr->amax_bits[1] = 0u;
+    }
 
     // 1. padded stream position of every row
     int32_t carry = 0;
@@ -26,7 +30,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
             const int b = r % B;
             const int32_t L = cu_len[b + 1] - cu_len[b];
             if (L < 1) atomicOr(&hdr->status, SGD_STATUS_EMPTY_SEQUENCE);
-            v = (int32_t)align_up(max(L, 0), kGranule);
+            v = (int32_t)align_up(max(L, 0), granule);
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
@@ -39,7 +43,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     int64_t S = 0;
     int ncta;
     if (mode == 0) {
-        S = align_up((W + (int64_t)n_req - 1) / n_req, kGranule);
+        S = align_up((W + (int64_t)n_req - 1) / n_req, granule);
         if (S < min_chunk) S = min_chunk;
         ncta = (int)((W + S - 1) / S);
     } else {
@@ -145,8 +149,8 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 }
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
-                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s) {
-    plan_kernel<<<1, 1024, 0, s>>>(cu_len, cu_seq, B, Hkv, n_req, min_chunk, mode, pv, hdr);
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule) {
+    plan_kernel<<<1, 1024, 0, s>>>(cu_len, cu_seq, B, Hkv, n_req, min_chunk, mode, granule, pv, hdr);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

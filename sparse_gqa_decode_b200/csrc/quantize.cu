@@ -22,63 +22,10 @@
 // half-integer.  Whenever q' is within 1e-4 of one (or is not finite) the IEEE
 // division __fdiv_rn(x, s) is taken instead.
 #include "internal.h"
+#include "quant.cuh"
 #include "scan.cuh"
 
 namespace sgd {
-
-__device__ __forceinline__ int code_of(float x, float s, float r) {
-    float q = x * r;
-    float n = rintf(q);
-    if (!(fabsf(q - n) < 0.4999f)) {
-        q = __fdiv_rn(x, s);
-        n = rintf(q);
-    }
-    n = fminf(fmaxf(n, -127.f), 127.f);
-    return (int)n;
-}
-
-template <typename T>
-struct Vec;  // 16 bytes of input -> VE elements -> VE code bytes
-template <>
-struct Vec<__nv_bfloat16> {
-    static constexpr int VE = 8;
-    __device__ static void unpack(const uint4 &w, float (&x)[8]) {
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[2 * i] = __uint_as_float(ww[i] << 16);
-            x[2 * i + 1] = __uint_as_float(ww[i] & 0xffff0000u);
-        }
-    }
-};
-template <>
-struct Vec<float> {
-    static constexpr int VE = 4;
-    __device__ static void unpack(const uint4 &w, float (&x)[4]) {
-        x[0] = __uint_as_float(w.x);
-        x[1] = __uint_as_float(w.y);
-        x[2] = __uint_as_float(w.z);
-        x[3] = __uint_as_float(w.w);
-    }
-};
-
-template <int VE>
-__device__ __forceinline__ void store_codes(int8_t *dst, const float (&x)[VE], float s, float r) {
-    uint32_t w[VE / 4];
-#pragma unroll
-    for (int i = 0; i < VE / 4; ++i) {
-        uint32_t b = 0;
-        if (s != 0.f) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) b |= (uint32_t)(code_of(x[4 * i + j], s, r) & 0xff) << (8 * j);
-        }
-        w[i] = b;
-    }
-    if constexpr (VE == 8)
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
-    else
-        *reinterpret_cast<uint32_t *>(dst) = w[0];
-}
 
 __device__ __forceinline__ float block_max(float v, float *sm) {
     v = warp_max(v);
@@ -264,6 +211,28 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
         quant_global_kernel<T><<<grid_stream, 256, 0, s>>>(k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
     }
     return (int)cudaGetLastError();
+}
+
+template <typename T>
+static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t Ttot, sgd_scheme scheme, int8_t *kc,
+                                int8_t *vc, float *k_scale, float *v_scale, const WsHeader *hdr, int sm_count,
+                                cudaStream_t s) {
+    const int64_t nvec = (int64_t)Hkv * Ttot * D / Vec<T>::VE;
+    if (scheme == SGD_SCHEME_A)
+        quant_global_kernel<T><<<sm_count * 8, 256, 0, s>>>(v, vc, v_scale, 1, nullptr, nullptr, nullptr, 0, nvec, hdr);
+    else
+        quant_global_kernel<T><<<sm_count * 8, 256, 0, s>>>(k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
+    return (int)cudaGetLastError();
+}
+
+int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
+                           sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
+                           const WsHeader *hdr, int sm_count, cudaStream_t s) {
+    if (dt == SGD_BF16)
+        return quantize_global_impl(static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
+                                    Hkv, D, T, scheme, kc, vc, k_scale, v_scale, hdr, sm_count, s);
+    return quantize_global_impl(static_cast<const float *>(k), static_cast<const float *>(v), Hkv, D, T, scheme, kc,
+                                vc, k_scale, v_scale, hdr, sm_count, s);
 }
 
 int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,

@@ -278,6 +278,31 @@ def test_oam_then_decode_over_kept(sgd, kvdt):
 
 
 # ---------------------------------------------------------------------------------------------
+# fused quantise + select
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("G,D,dtype", [(8, 128, "bf16"), (4, 64, "bf16"), (16, 128, "bf16"), (1, 128, "bf16"),
+                                       (8, 128, "f32")])
+def test_quantize_select_equals_separate_calls(sgd, scheme, G, D, dtype):
+    bt = make((1, 63, 64, 65, 700, 4099), G=G, D=D, Hkv=3, dtype=dtype, dist="outlier", seed=91 + G + D)
+    q, k, v, cu = dev(bt)
+    if dtype == "f32":
+        q = q.float()
+    fused = sgd.quantize_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+    idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, bt.lengths)
+    for a, b in zip(fused[:6], (kc, vc, ks, vs, idx, cu_kept)):
+        assert torch.equal(a, b)
+    check_status(sgd, fused[6])
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    assert np.array_equal(fused[0].cpu().numpy(), rkc) and np.array_equal(fused[1].cpu().numpy(), rvc)
+    assert np.array_equal(fused[2].cpu().numpy().reshape(rks.shape), rks)
+    assert np.array_equal(fused[3].cpu().numpy(), rvs)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 8)
+    check_selection(fused[4], fused[5].cpu(), ref_idx, ref_cu, scores, bt.wl.B, 3)
+
+
+# ---------------------------------------------------------------------------------------------
 # device status reporting
 # ---------------------------------------------------------------------------------------------
 def test_empty_sequence_is_reported(sgd):
