@@ -112,6 +112,10 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+__device__ __forceinline__ void cp_async_4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -186,6 +190,24 @@ __device__ __forceinline__ uint32_t biased_pair_to_f16x2(uint32_t a, uint32_t b,
     const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
     __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&x), bias);
     return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// max(|lo|, |hi|) of a running bf16x2 maximum folded into float (bf16 values are exact in float)
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t m, uint32_t w) {
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&w), b = *reinterpret_cast<__nv_bfloat162 *>(&m);
+    __nv_bfloat162 r = __hmax2(__habs2(a), b);
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ float bf16x2_fold_max(uint32_t m) {
+    return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
+}
+
+// ss += lo(w)^2 + hi(w)^2 for the two bf16 of w, as a packed f32x2 FMA on (even, odd) partial sums
+__device__ __forceinline__ uint64_t bf16x2_sumsq(uint64_t acc, uint32_t w) {
+    const uint64_t x = (uint64_t)(w << 16) | ((uint64_t)(w & 0xffff0000u) << 32);
+    asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(x));
+    return acc;
 }
 
 __device__ __forceinline__ float warp_max(float v) {

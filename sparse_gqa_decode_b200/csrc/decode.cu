@@ -68,7 +68,9 @@ struct MmaCfg {
     static constexpr int NQ = (MODE == 2) ? 4 : 0;  // K-quantising warps (mode 2)
     static constexpr int THREADS = (NW + NQ + 1) * 32;
     static constexpr int SMEM_STAGES = STAGES * 2 * TILE;
-    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + 2 * 4 * 4;
+    static constexpr bool ROW_SCALE = I8 && IDX;  // per-row K scales fetched by the producer
+    static constexpr int SMEM_ROWSCALE = ROW_SCALE ? STAGES * ROWS * 4 : 0;
+    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + 2 * 4 * 4 + SMEM_ROWSCALE;
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE >= 1), "scores read the unquantised cache");
@@ -81,8 +83,8 @@ struct MmaCfg {
 template <class C>
 __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUtensorMap *tmV, const DecodeArgs &a,
                                              uint8_t *smem, uint64_t *full, uint64_t *empty,
-                                             volatile int32_t *abort_flag, const int32_t *cu_rows, int cta,
-                                             int lane) {
+                                             volatile int32_t *abort_flag, float *row_scale, const int32_t *cu_rows,
+                                             int cta, int lane) {
     if (!C::IDX && lane != 0) return;
     uint64_t pol = 0;
     if constexpr (!C::IDX) {
@@ -102,6 +104,8 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
         const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
         const int32_t *ip = nullptr;
         if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
+        const float *ksc = nullptr;
+        if constexpr (C::ROW_SCALE) ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
             uint8_t *sk = smem + stage * 2 * C::TILE;
@@ -115,9 +119,15 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                     tma_load_2d(sv + bx * C::ROWS * 128, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
                 }
             } else if (Lb >= 1) {
-                for (int rr = lane; rr < C::ROWS; rr += 32) {
-                    const int32_t j = min(t + rr, t1 - 1);  // rows past the segment repeat its last token
-                    int32_t tok = __ldg(ip + j);
+                constexpr int RPL = C::ROWS / 32;  // rows per producer lane
+                int32_t toks[RPL];
+#pragma unroll
+                for (int qi = 0; qi < RPL; ++qi)  // every index load first, then the copies
+                    toks[qi] = __ldg(ip + min(t + lane + 32 * qi, t1 - 1));  // rows past the segment repeat its last token
+#pragma unroll
+                for (int qi = 0; qi < RPL; ++qi) {
+                    const int rr = lane + 32 * qi;
+                    int32_t tok = toks[qi];
                     if (tok < 0 || tok >= Lb) {
                         atomicOr(a.status, SGD_STATUS_BAD_INDEX);
                         tok = min(max(tok, 0), Lb - 1);
@@ -132,6 +142,9 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                             cp_async_16(sk + off, gk + bx * 128 + c * 16);
                             cp_async_16(sv + off, gv + bx * 128 + c * 16);
                         }
+                    if constexpr (C::ROW_SCALE) {
+                        if (a.scheme == SGD_SCHEME_A) cp_async_4(row_scale + stage * C::ROWS + rr, ksc + tok / kPart);
+                    }
                 }
                 cp_async_mbar_arrive_noinc(&full[stage]);
             } else {
@@ -299,15 +312,13 @@ __device__ __forceinline__ void pv_subtile(uint32_t vbase, int rb, int lane, con
 }
 
 // Score mode for one 16-token sub-tile: OAM score of every token (max over the group's heads
-// of the logit, plus beta * ln(|v| + eps)); mode 2 also quantises the K rows of the tile (one
-// scheme-A partition: the four warps' maxima meet through shared memory) or accumulates max|K|
-// (scheme B), and accumulates max|V|.  Every consumer warp calls this for every tile.
+// of the logit, plus beta * ln(|v| + eps)); mode 2 also accumulates max|V|.  Every score warp
+// calls this for every tile.
 template <class C>
 __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbase, uint32_t vbase, int rb,
-                                              int32_t j0, int32_t t, int32_t t1, bool ready, int b, int kvh,
-                                              int pA, int t4, int lane, int warp,
-                                              const uint32_t (&qf)[C::GT][C::KB][2], float &run_kmax,
-                                              float &run_vmax, float *kmxs, int parity) {
+                                              int32_t j0, int32_t t1, bool ready, int64_t tok_base, int pA,
+                                              int t4, int lane, const uint32_t (&qf)[C::GT][C::KB][2],
+                                              float &run_vmax) {
     const bool act = ready && j0 < t1;
     float sacc[C::GT][4];
     if (act) {
@@ -340,7 +351,8 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     const bool vrow = act && j < t1;
     constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
     constexpr int NH = CPR / 2;
-    float ss = 0.f, vmx = 0.f;
+    uint64_t ss2 = 0;  // (even, odd) partial sums of squares
+    uint32_t vm2 = 0;  // running max |v| as bf16x2 (mode 2)
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
         const int c = half * NH + i, bx = c >> 3, cc = c & 7;
@@ -348,12 +360,12 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
-            ss = fmaf(lo, lo, ss);
-            ss = fmaf(hi, hi, ss);
-            if constexpr (C::MODE == 2) vmx = fmaxf(vmx, fmaxf(fabsf(lo), fabsf(hi)));
+            ss2 = bf16x2_sumsq(ss2, ww[e]);
+            if constexpr (C::MODE == 2) vm2 = bf16x2_absmax(vm2, ww[e]);
         }
     }
+    float ss = __uint_as_float((uint32_t)ss2) + __uint_as_float((uint32_t)(ss2 >> 32));
+    const float vmx = bf16x2_fold_max(vm2);
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     const int src = 4 * mma_row_perm(rho & 7);
     const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
@@ -361,7 +373,7 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     if (half == 0 && vrow) {
         float sc = rmax * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
         if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
-        a.scores[(int64_t)kvh * a.T + a.cu_seq[b] + j] = sc;
+        a.scores[tok_base + j] = sc;
     }
     if constexpr (C::MODE == 2) {
         if (vrow) run_vmax = fmaxf(run_vmax, vmx);
@@ -388,23 +400,25 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
     const int vr = 16 * qw + rho;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
+        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + a.cu_seq[b]) * C::D + half * (C::D / 2);
+        float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
             const uint32_t kbase = smem_u32(smem + stage * 2 * C::TILE);
             const int32_t j = t + vr;
             const bool vrow = ready && j < t1;
             uint4 kw[NH];
-            float kmx = 0.f;
+            uint32_t km2 = 0;
 #pragma unroll
             for (int i = 0; i < NH; ++i) {
                 const int c = half * NH + i, bx = c >> 3, cc = c & 7;
                 kw[i] = lds128(kbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
-                const uint32_t ww[4] = {kw[i].x, kw[i].y, kw[i].z, kw[i].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    kmx = fmaxf(kmx, fmaxf(fabsf(__uint_as_float(ww[e] << 16)),
-                                           fabsf(__uint_as_float(ww[e] & 0xffff0000u))));
+                km2 = bf16x2_absmax(km2, kw[i].x);
+                km2 = bf16x2_absmax(km2, kw[i].y);
+                km2 = bf16x2_absmax(km2, kw[i].z);
+                km2 = bf16x2_absmax(km2, kw[i].w);
             }
+            float kmx = bf16x2_fold_max(km2);
             if (!vrow) kmx = 0.f;
             if (a.qscheme == SGD_SCHEME_B) {
                 run_kmax = fmaxf(run_kmax, kmx);
@@ -419,17 +433,22 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
                 const float sc = __fdiv_rn(tm, 127.f);
                 const float r = (sc != 0.f) ? __frcp_rn(sc) : 0.f;
                 if (vrow) {
-                    int8_t *dst = a.k_codes + ((int64_t)kvh * a.T + a.cu_seq[b] + j) * C::D + half * (C::D / 2);
+                    uint4 *dst = reinterpret_cast<uint4 *>(codes_row0 + (int64_t)j * C::D);
 #pragma unroll
-                    for (int i = 0; i < NH; ++i) {
-                        float x[8];
+                    for (int i = 0; i < NH; i += 2) {  // 16 codes per 16-byte store
+                        float x[8], y[8];
                         Vec<__nv_bfloat16>::unpack(kw[i], x);
-                        store_codes<8>(dst + i * 8, x, sc, r);
+                        Vec<__nv_bfloat16>::unpack(kw[i + 1], y);
+                        uint4 w;
+                        w.x = (sc != 0.f) ? codes4(x, sc, r) : 0u;
+                        w.y = (sc != 0.f) ? codes4(x + 4, sc, r) : 0u;
+                        w.z = (sc != 0.f) ? codes4(y, sc, r) : 0u;
+                        w.w = (sc != 0.f) ? codes4(y + 4, sc, r) : 0u;
+                        dst[i / 2] = w;
                     }
                 }
                 // (the partition count was checked against the host's n_parts before any write)
-                if (qw == 0 && lane == 0 && ready)
-                    a.k_scale_out[(int64_t)kvh * a.n_parts + a.plan.seq_part0[b] + t / kPart] = sc;
+                if (qw == 0 && lane == 0 && ready) scale_row0[t / kPart] = sc;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -458,7 +477,8 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     uint64_t *empty = full + C::STAGES;
     float *ml = reinterpret_cast<float *>(empty + C::STAGES);  // [NW][NG][2]: m, l
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(ml + C::NW * C::NG * 2);
-    float *kmxs = ml + C::NW * C::NG * 2 + 4;  // [2][NW] per-warp max|K| of the current tile (mode 2)
+    float *kmxs = ml + C::NW * C::NG * 2 + 4;  // [2][NQ] per-warp max|K| of the current tile (mode 2)
+    float *row_scale = kmxs + 8;               // [STAGES][ROWS] K scale of each gathered row (INT8 gathers)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -482,7 +502,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     const int32_t *cu_rows = C::IDX ? a.cu_kept : a.cu_seq;
 
     if (warp == C::NW + C::NQ) {
-        mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, cu_rows, cta, lane);
+        mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, row_scale, cu_rows, cta, lane);
         return;
     }
     if constexpr (C::NQ > 0) {
@@ -504,7 +524,9 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     int tile_no = 0;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
+        const int32_t seq_start = a.cu_seq[b];
+        const int32_t Lb = a.cu_seq[b + 1] - seq_start;
+        const int64_t tok_base = (int64_t)kvh * a.T + seq_start;  // cache row of token 0 of the sequence
         uint32_t qf[C::GT][C::KB][2];
         float colf[C::GT][2];
         load_q_frags<C>(a, b, kvh, g4, t4, qf, colf);
@@ -522,6 +544,17 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
 
         for (int32_t t = t0; t < t1; t += C::ROWS) {
+            // dense scheme A: the K scale of each sub-tile's partition, loaded before the wait
+            float rf_pre[C::SUB];
+#pragma unroll
+            for (int s = 0; s < C::SUB; ++s) rf_pre[s] = 1.f;
+            if constexpr (C::I8 && !C::IDX) {
+                if (a.scheme == SGD_SCHEME_A) {
+#pragma unroll
+                    for (int s = 0; s < C::SUB; ++s)
+                        rf_pre[s] = __ldg(ksc + min(t + 16 * (s * C::NW + warp), Lb - 1) / kPart);
+                }
+            }
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
             uint8_t *sk = smem + stage * 2 * C::TILE;
             uint8_t *sv = sk + C::TILE;
@@ -531,8 +564,7 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                 const int rb = 16 * (s * C::NW + warp);
                 const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
                 if constexpr (C::MODE >= 1) {
-                    score_subtile<C>(a, kbase, vbase, rb, j0, t, t1, ready, b, kvh, pA, t4, lane, warp, qf, run_kmax,
-                                     run_vmax, kmxs, tile_no & 1);
+                    score_subtile<C>(a, kbase, vbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, run_vmax);
                     continue;
                 }
                 if (j0 >= t1 || !ready) continue;
@@ -541,17 +573,11 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                 const bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
                 {
                     // row (token) factors: scheme-A K scale of the token's 64-token partition
-                    float rfA = 1.f, rfB = 1.f;
-                    if constexpr (C::I8) {
+                    float rfA = rf_pre[s], rfB = rf_pre[s];
+                    if constexpr (C::ROW_SCALE) {
                         if (a.scheme == SGD_SCHEME_A) {
-                            if constexpr (!C::IDX) {
-                                rfA = rfB = __ldg(ksc + min(j0, Lb - 1) / kPart);
-                            } else {
-                                const int32_t tA = __ldg(ip + min(j0 + pA, t1 - 1));
-                                const int32_t tB = __ldg(ip + min(j0 + pA + 8, t1 - 1));
-                                rfA = __ldg(ksc + min(max(tA, 0), Lb - 1) / kPart);
-                                rfB = __ldg(ksc + min(max(tB, 0), Lb - 1) / kPart);
-                            }
+                            rfA = row_scale[stage * C::ROWS + rb + pA];
+                            rfB = row_scale[stage * C::ROWS + rb + pA + 8];
                         }
                     }
                     uint32_t pb[C::GT][2];
@@ -825,35 +851,32 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const DecodeArgs a)
 // exact LSE merge: per (sequence, query head), lse = ln sum_c exp(lse_c),
 // out = sum_c exp(lse_c - lse) o_c
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) merge_kernel(const DecodeArgs a, float *__restrict__ out,
+__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a, float *__restrict__ out,
                                                     float *__restrict__ lse) {
-    const int r = blockIdx.x;
+    // one block per (row, query head of the group), one thread per channel
+    const int r = blockIdx.x / a.G, g = blockIdx.x - r * a.G;
     const int b = r % a.B, kvh = r / a.B;
     const int s0 = a.plan.row_slot0[r], n = a.plan.row_slot0[r + 1] - s0;
     const int Hq = a.Hkv * a.G;
-    for (int e = threadIdx.x; e < a.G * a.D; e += blockDim.x) {
-        const int g = e / a.D, d = e - g * a.D;
-        const int64_t oi = ((int64_t)b * Hq + kvh * a.G + g) * a.D + d;
-        float L, O;
-        if (n <= 0) {
-            L = -INFINITY;
-            O = 0.f;
-        } else if (n == 1) {
-            L = a.lse_part[(int64_t)s0 * a.G + g];
-            O = a.o_part[((int64_t)s0 * a.G + g) * a.D + d];
+    const int64_t h = (int64_t)b * Hq + kvh * a.G + g;
+    const float *lp = a.lse_part + (int64_t)s0 * a.G + g;
+    const float *op = a.o_part + ((int64_t)s0 * a.G + g) * a.D;
+    float M = -INFINITY;
+    for (int c = 0; c < n; ++c) M = fmaxf(M, __ldg(lp + (int64_t)c * a.G));
+    float S = 0.f;
+    for (int c = 0; c < n; ++c) S += expf(__ldg(lp + (int64_t)c * a.G) - M);
+    const float L = (n > 0) ? M + logf(S) : -INFINITY;
+    for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
+        float O = 0.f;
+        if (n == 1) {
+            O = __ldg(op + d);
         } else {
-            float M = -INFINITY;
-            for (int c = 0; c < n; ++c) M = fmaxf(M, a.lse_part[(int64_t)(s0 + c) * a.G + g]);
-            float S = 0.f;
-            for (int c = 0; c < n; ++c) S += expf(a.lse_part[(int64_t)(s0 + c) * a.G + g] - M);
-            L = M + logf(S);
-            O = 0.f;
             for (int c = 0; c < n; ++c)
-                O += expf(a.lse_part[(int64_t)(s0 + c) * a.G + g] - L) * a.o_part[((int64_t)(s0 + c) * a.G + g) * a.D + d];
+                O += expf(__ldg(lp + (int64_t)c * a.G) - L) * __ldg(op + (int64_t)c * a.G * a.D + d);
         }
-        out[oi] = O;
-        if (d == 0) lse[(int64_t)b * Hq + kvh * a.G + g] = L;
+        out[h * a.D + d] = O;
     }
+    if (threadIdx.x == 0) lse[h] = (n == 1) ? __ldg(lp) : L;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -888,9 +911,17 @@ static bool make_map(CUtensorMap *map, const void *base, bool i8, int D, int64_t
 }
 
 template <class C>
+static cudaError_t set_smem_attrs() {
+    auto k = decode_mma_kernel<C>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
+template <class C>
 static int ctas_per_sm_mma() {
     auto k = decode_mma_kernel<C>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) return 0;
+    if (set_smem_attrs<C>() != cudaSuccess) return 0;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::THREADS, C::SMEM) != cudaSuccess) return 0;
     return n;
@@ -908,7 +939,7 @@ static int launch_mma(const DecodeArgs &a, int n_cta, cudaStream_t s) {
             return (int)cudaErrorInvalidValue;
     }
     auto k = decode_mma_kernel<C>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = set_smem_attrs<C>();
     if (e != cudaSuccess) return (int)e;
     k<<<n_cta, C::THREADS, C::SMEM, s>>>(mk, mv, a);
     return (int)cudaGetLastError();
@@ -994,7 +1025,7 @@ int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s) {
 }
 
 int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s) {
-    merge_kernel<<<a.B * a.Hkv, 256, 0, s>>>(a, out, lse);
+    merge_kernel<<<a.B * a.Hkv * a.G, 128, 0, s>>>(a, out, lse);
     return (int)cudaGetLastError();
 }
 
