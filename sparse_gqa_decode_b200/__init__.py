@@ -5,7 +5,7 @@ This module is a thin binding over the C ABI of ``libsgd.so`` (``include/sgd.h``
 torch tensors into device pointers, allocates outputs and the workspace with torch, and
 passes the current CUDA stream.  Every step of the computation runs in the library's CUDA
 kernels; there is no CPU or PyTorch fallback, and importing fails loudly when the library
-has not been built (``python -m sparse_gqa_decode_b200.build``).
+has not been built (``python sparse_gqa_decode_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -31,7 +31,7 @@ PARTITION = 64
 STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index"}
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_gqa_decode_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_gqa_decode_b200/build.py` "
                       "(there is no fallback implementation)")
 
 

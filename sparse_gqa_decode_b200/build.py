@@ -1,6 +1,8 @@
 """Build libsgd.so in-tree from csrc/*.cu for sm_100a (nvcc; no GPU needed to build).
 
-    python -m sparse_gqa_decode_b200.build [--force] [--ptxas-verbose]
+    python sparse_gqa_decode_b200/build.py [--force] [--ptxas-verbose]
+
+(Run it by path: importing the package itself requires the library this script builds.)
 """
 from __future__ import annotations
 

@@ -119,31 +119,37 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                     tma_load_2d(sv + bx * C::ROWS * 128, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
                 }
             } else if (Lb >= 1) {
-                constexpr int RPL = C::ROWS / 32;  // rows per producer lane
+                // Row indices: lane l loads those of rows l, l+32, ...  Copies: one warp
+                // instruction moves whole rows (CPR lanes per row, one 16-byte chunk each), so
+                // every row reaches L2 as one contiguous request per tensor.
+                constexpr int RPL = C::ROWS / 32;  // row indices held per lane
+                constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
+                constexpr int RPI = 32 / CPR;      // rows per copy instruction
                 int32_t toks[RPL];
 #pragma unroll
-                for (int qi = 0; qi < RPL; ++qi)  // every index load first, then the copies
-                    toks[qi] = __ldg(ip + min(t + lane + 32 * qi, t1 - 1));  // rows past the segment repeat its last token
-#pragma unroll
-                for (int qi = 0; qi < RPL; ++qi) {
-                    const int rr = lane + 32 * qi;
-                    int32_t tok = toks[qi];
+                for (int qi = 0; qi < RPL; ++qi) {  // every index load first, then the copies
+                    int32_t tok = __ldg(ip + min(t + lane + 32 * qi, t1 - 1));  // rows past the segment repeat its last token
                     if (tok < 0 || tok >= Lb) {
                         atomicOr(a.status, SGD_STATUS_BAD_INDEX);
                         tok = min(max(tok, 0), Lb - 1);
                     }
-                    const uint8_t *gk = static_cast<const uint8_t *>(a.k) + (seq0 + tok) * C::ROWB;
-                    const uint8_t *gv = static_cast<const uint8_t *>(a.v) + (seq0 + tok) * C::ROWB;
+                    toks[qi] = tok;
+                }
+                const int c = lane % CPR, bx = c >> 3, cc = c & 7;
 #pragma unroll
-                    for (int bx = 0; bx < C::BOXES; ++bx)
+                for (int it = 0; it < C::ROWS / RPI; ++it) {
+                    const int rr = it * RPI + lane / CPR;  // this lane's row in this instruction
+                    const int32_t tok = __shfl_sync(0xffffffffu, toks[(it * RPI) / 32], rr & 31);
+                    const int64_t src = (seq0 + tok) * C::ROWB + c * 16;
+                    const int off = bx * C::ROWS * 128 + rr * 128 + ((cc ^ (rr & 7)) << 4);
+                    cp_async_16(sk + off, static_cast<const uint8_t *>(a.k) + src);
+                    cp_async_16(sv + off, static_cast<const uint8_t *>(a.v) + src);
+                }
+                if constexpr (C::ROW_SCALE) {
+                    if (a.scheme == SGD_SCHEME_A) {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const int off = bx * C::ROWS * 128 + rr * 128 + ((c ^ (rr & 7)) << 4);
-                            cp_async_16(sk + off, gk + bx * 128 + c * 16);
-                            cp_async_16(sv + off, gv + bx * 128 + c * 16);
-                        }
-                    if constexpr (C::ROW_SCALE) {
-                        if (a.scheme == SGD_SCHEME_A) cp_async_4(row_scale + stage * C::ROWS + rr, ksc + tok / kPart);
+                        for (int qi = 0; qi < RPL; ++qi)
+                            cp_async_4(row_scale + stage * C::ROWS + lane + 32 * qi, ksc + toks[qi] / kPart);
                     }
                 }
                 cp_async_mbar_arrive_noinc(&full[stage]);
@@ -344,8 +350,9 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
     mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
     mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-    // lane pair (rho, half) owns half of the row rb + rho of the K and V tiles
-    const int rho = lane >> 1, half = lane & 1;
+    // lanes rho and rho + 16 own the two halves of row rb + rho of the V tile (a quarter-warp
+    // then reads eight rows at one swizzled chunk: eight distinct bank groups)
+    const int rho = lane & 15, half = lane >> 4;
     const int vr = rb + rho;
     const int32_t j = j0 + rho;
     const bool vrow = act && j < t1;
@@ -366,7 +373,7 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     }
     float ss = __uint_as_float((uint32_t)ss2) + __uint_as_float((uint32_t)(ss2 >> 32));
     const float vmx = bf16x2_fold_max(vm2);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
     const int src = 4 * mma_row_perm(rho & 7);
     const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
     const float rmax = (rho < 8) ? rA : rB;
@@ -396,7 +403,7 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
     int32_t t0, t1;
     float run_kmax = 0.f;
     constexpr int CPR = C::ROWB / 16, NH = CPR / 2;
-    const int rho = lane >> 1, half = lane & 1;
+    const int rho = lane & 15, half = lane >> 4;  // lanes rho, rho + 16: the two halves of one row
     const int vr = 16 * qw + rho;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
@@ -408,17 +415,18 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
             const int32_t j = t + vr;
             const bool vrow = ready && j < t1;
             uint4 kw[NH];
-            uint32_t km2 = 0;
+            uint32_t km2[4] = {0u, 0u, 0u, 0u};  // four independent running maxima
 #pragma unroll
             for (int i = 0; i < NH; ++i) {
                 const int c = half * NH + i, bx = c >> 3, cc = c & 7;
                 kw[i] = lds128(kbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
-                km2 = bf16x2_absmax(km2, kw[i].x);
-                km2 = bf16x2_absmax(km2, kw[i].y);
-                km2 = bf16x2_absmax(km2, kw[i].z);
-                km2 = bf16x2_absmax(km2, kw[i].w);
+                km2[0] = bf16x2_absmax(km2[0], kw[i].x);
+                km2[1] = bf16x2_absmax(km2[1], kw[i].y);
+                km2[2] = bf16x2_absmax(km2[2], kw[i].z);
+                km2[3] = bf16x2_absmax(km2[3], kw[i].w);
             }
-            float kmx = bf16x2_fold_max(km2);
+            float kmx = fmaxf(fmaxf(bf16x2_fold_max(km2[0]), bf16x2_fold_max(km2[1])),
+                              fmaxf(bf16x2_fold_max(km2[2]), bf16x2_fold_max(km2[3])));
             if (!vrow) kmx = 0.f;
             if (a.qscheme == SGD_SCHEME_B) {
                 run_kmax = fmaxf(run_kmax, kmx);
@@ -435,15 +443,16 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
                 if (vrow) {
                     uint4 *dst = reinterpret_cast<uint4 *>(codes_row0 + (int64_t)j * C::D);
 #pragma unroll
+#pragma unroll
                     for (int i = 0; i < NH; i += 2) {  // 16 codes per 16-byte store
                         float x[8], y[8];
                         Vec<__nv_bfloat16>::unpack(kw[i], x);
                         Vec<__nv_bfloat16>::unpack(kw[i + 1], y);
                         uint4 w;
-                        w.x = (sc != 0.f) ? codes4(x, sc, r) : 0u;
-                        w.y = (sc != 0.f) ? codes4(x + 4, sc, r) : 0u;
-                        w.z = (sc != 0.f) ? codes4(y, sc, r) : 0u;
-                        w.w = (sc != 0.f) ? codes4(y + 4, sc, r) : 0u;
+                        w.x = (sc != 0.f) ? codes4<true>(x, sc, r) : 0u;
+                        w.y = (sc != 0.f) ? codes4<true>(x + 4, sc, r) : 0u;
+                        w.z = (sc != 0.f) ? codes4<true>(y, sc, r) : 0u;
+                        w.w = (sc != 0.f) ? codes4<true>(y + 4, sc, r) : 0u;
                         dst[i / 2] = w;
                     }
                 }

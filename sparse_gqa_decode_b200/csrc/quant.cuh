@@ -59,10 +59,19 @@ struct Vec<float> {
 // |e| < 0.4999 keeps the fast result; otherwise (near a half-integer, or not finite) code_of's
 // IEEE division decides.  |x*r| <= 127.0001 for the group's own scale, so the fast integer
 // already lies in [-127, 127].
+// The rare exact path of codes4, kept out of line so that the unrolled fast path stays compact.
+static __device__ __noinline__ uint32_t codes4_exact(float x0, float x1, float x2, float x3, float s, float r) {
+    return (uint32_t)(code_of(x0, s, r) & 0xff) | ((uint32_t)(code_of(x1, s, r) & 0xff) << 8) |
+           ((uint32_t)(code_of(x2, s, r) & 0xff) << 16) | ((uint32_t)(code_of(x3, s, r) & 0xff) << 24);
+}
+
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
 }
 
+// OUTLINE: take the rare exact path through an out-of-line call (keeps a large unrolled caller
+// compact; a small grid-stride loop is faster with it inline).
+template <bool OUTLINE = false>
 __device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
     const uint64_t rr = f32x2(r, r), mm = f32x2(12582912.f, 12582912.f);
     uint64_t t01, t23, n01, n23, e01, e23;
@@ -80,9 +89,13 @@ __device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
     const bool fast = fabsf(e[0]) < 0.4999f && fabsf(e[1]) < 0.4999f && fabsf(e[2]) < 0.4999f &&
                       fabsf(e[3]) < 0.4999f;
     if (!fast) {
-        w = 0;
+        if constexpr (OUTLINE) {
+            w = codes4_exact(x[0], x[1], x[2], x[3], s, r);
+        } else {
+            w = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w |= (uint32_t)(code_of(x[j], s, r) & 0xff) << (8 * j);
+            for (int j = 0; j < 4; ++j) w |= (uint32_t)(code_of(x[j], s, r) & 0xff) << (8 * j);
+        }
     }
     return w;
 }

@@ -179,13 +179,15 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
     const uint4 *p0 = reinterpret_cast<const uint4 *>(x0);
     const uint4 *p1 = reinterpret_cast<const uint4 *>(x1);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += stride) {
-        float x[VE];
-        Vec<T>::unpack(__ldcs(p0 + i), x);
-        store_codes<VE>(c0 + i * VE, x, s0, r0);
-        if (x1) {
-            Vec<T>::unpack(__ldcs(p1 + i), x);
-            store_codes<VE>(c1 + i * VE, x, s1, r1);
+    {
+        for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += stride) {
+            float x[VE];
+            Vec<T>::unpack(__ldcs(p0 + i), x);
+            store_codes<VE>(c0 + i * VE, x, s0, r0);
+            if (x1) {
+                Vec<T>::unpack(__ldcs(p1 + i), x);
+                store_codes<VE>(c1 + i * VE, x, s1, r1);
+            }
         }
     }
 }

@@ -12,9 +12,8 @@ HEADER = os.path.join(ROOT, "include", "sgd.h")
 
 @pytest.fixture(scope="module")
 def sgd():
-    from sparse_gqa_decode_b200 import build
-    build.build()
-    import sparse_gqa_decode_b200 as m
+    from conftest import build_library
+    m = build_library()
     return m
 
 

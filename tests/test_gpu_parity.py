@@ -21,9 +21,8 @@ TIE_WINDOW = 1e-4
 
 @pytest.fixture(scope="module")
 def sgd():
-    from sparse_gqa_decode_b200 import build
-    build.build()
-    import sparse_gqa_decode_b200 as m
+    from conftest import build_library
+    m = build_library()
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return m
 
@@ -285,6 +284,10 @@ def test_oam_then_decode_over_kept(sgd, kvdt):
                                        (8, 128, "f32")])
 def test_quantize_select_equals_separate_calls(sgd, scheme, G, D, dtype):
     bt = make((1, 63, 64, 65, 700, 4099), G=G, D=D, Hkv=3, dtype=dtype, dist="outlier", seed=91 + G + D)
+    # exact rounding ties in partition 1 of sequence 5, head 2 (max |x| = 127: scale 1)
+    s0 = int(bt.cu_seqlens[5])
+    bt.k[2, s0 + 64:s0 + 128] = 0
+    bt.k[2, s0 + 64:s0 + 80, :6] = torch.tensor([2.5, 3.5, -2.5, 126.5, 127.0, -0.5]).to(bt.k.dtype)
     q, k, v, cu = dev(bt)
     if dtype == "f32":
         q = q.float()
@@ -293,6 +296,8 @@ def test_quantize_select_equals_separate_calls(sgd, scheme, G, D, dtype):
     idx, cu_kept, _ = sgd.oam_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, bt.lengths)
     for a, b in zip(fused[:6], (kc, vc, ks, vs, idx, cu_kept)):
         assert torch.equal(a, b)
+    if scheme == "A":
+        assert fused[0][2, s0 + 64, :6].tolist() == [2, 4, -2, 126, 127, 0]
     check_status(sgd, fused[6])
     rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
     assert np.array_equal(fused[0].cpu().numpy(), rkc) and np.array_equal(fused[1].cpu().numpy(), rvc)

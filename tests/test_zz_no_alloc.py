@@ -22,9 +22,8 @@ LSE_TOL = 1e-3
 
 @pytest.fixture(scope="module")
 def sgd():
-    from sparse_gqa_decode_b200 import build
-    build.build()
-    import sparse_gqa_decode_b200 as m
+    from conftest import build_library
+    m = build_library()
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return m
 
