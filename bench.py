@@ -373,11 +373,6 @@ def run_ours(args, rank, world, local_rank):
                "quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
                "select": "sgd_oam_select (plan + OAM score + top-K kernels)",
                "decode": "sgd_decode_attn (plan + split decode + merge kernels)"}
-    srcs = {"quantize_select": ["sparse_gqa_decode_b200/csrc/decode.cu", "sparse_gqa_decode_b200/csrc/quantize.cu",
-                                "sparse_gqa_decode_b200/csrc/oam.cu"],
-            "quantize": ["sparse_gqa_decode_b200/csrc/quantize.cu"],
-            "select": ["sparse_gqa_decode_b200/csrc/decode.cu", "sparse_gqa_decode_b200/csrc/oam.cu"],
-            "decode": ["sparse_gqa_decode_b200/csrc/decode.cu"]}
     traffic = load_traffic(dom, wl.name)
     stage_report = {}
     for n in names:
