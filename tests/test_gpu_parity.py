@@ -243,6 +243,40 @@ def test_oam_ties_keep_lowest_indices(sgd):
         assert idx[h, 15:].tolist() == list(range(125))
 
 
+def test_oam_few_distinct_scores_take_the_radix_path(sgd):
+    # q = 0 and value-row norms cycling through 1, 2, 4: three distinct scores spread apart, so the
+    # threshold bin of the linear histogram holds thousands of keys and the exact radix select
+    # decides; the kept set is the first K tokens of the top score, across all 8 CTAs of the row
+    bt = make((20000, 7), G=4, D=64, Hkv=2, seed=52)
+    bt.q.zero_()
+    bt.v[:] = 0
+    cu = bt.cu_seqlens.tolist()
+    norms = torch.tensor([1.0, 2.0, 4.0])
+    for h in range(2):
+        for b in range(2):
+            t = torch.arange(cu[b + 1] - cu[b])
+            bt.v[h, cu[b]:cu[b + 1], 0] = norms[(t + h) % 3].to(bt.v.dtype)
+    q, k, v, cu_d = dev(bt)
+    idx, cu_kept, ws = sgd.oam_select(q, k, v, cu_d, 4, 1.0, 1e-6, 1, 8, bt.lengths)
+    check_status(sgd, ws)
+    assert cu_kept.tolist() == [0, 2500, 2501]
+    for h in range(2):
+        top = [t for t in range(20000) if (t + h) % 3 == 2][:2500]
+        assert idx[h, :2500].tolist() == top
+        assert idx[h, 2500:].tolist() == [[2, 1][h]]
+
+
+def test_oam_long_row_beyond_the_shared_memory_stage(sgd):
+    # 140000 tokens: each of the row's 8 CTAs holds more keys than it stages in shared memory,
+    # so the rest is read again from global memory and the compaction works from the keys
+    bt = make((140000, 300), G=8, D=128, Hkv=1, dist="outlier", seed=53)
+    q, k, v, cu = dev(bt)
+    idx, cu_kept, ws = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, bt.lengths)
+    check_status(sgd, ws)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 1.0, 1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, 2, 1)
+
+
 def test_oam_keep_all_then_decode_equals_dense(sgd):
     bt = make((33, 700), G=8, D=128, Hkv=2, seed=61)
     q, k, v, cu = dev(bt)
