@@ -204,6 +204,9 @@ int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedul
  * segs      [max_segs, 4] device int32 output: (cta, row, row-local start, length)
  *           in stream order
  * n_segs    [2] device int32 output: number of segments, number of CTAs used
+ * workspace device scratch, 16-byte aligned, of at least
+ *           2048 + 4 * (B + 2 * B * Hkv + 3 * n_req + 6) + 32 * B * Hkv bytes
+ *           (mode 1: n_req = B * Hkv); SGD_ERR_WORKSPACE when smaller
  */
 int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode,
                       int32_t *segs, int64_t max_segs, int32_t *n_segs,

@@ -262,7 +262,8 @@ def plan_segments(cu: torch.Tensor, B: int, Hkv: int, n_req: int, min_chunk: int
     cap = n_req + R + 8
     segs = torch.full((cap, 4), -1, dtype=torch.int32, device=cu.device)
     nseg = torch.zeros(2, dtype=torch.int32, device=cu.device)
-    nbytes = 256 + 4 * 256 + 8 * (R + n_req + B + 8) + 4096
+    n = R if mode == 1 else n_req
+    nbytes = 2048 + 4 * (B + 2 * R + 3 * n + 6) + 32 * R  # the bound sgd.h states
     ws = torch.empty(nbytes, dtype=torch.uint8, device=cu.device)
     _check(lib.sgd_plan_segments(_ptr(cu), B, Hkv, n_req, min_chunk, mode, _ptr(segs), cap, _ptr(nseg), _ptr(ws),
                                  ws.numel(), _stream(stream)), "sgd_plan_segments")

@@ -60,7 +60,7 @@ int check_kv(const sgd_kv *kv) {
 
 // workspace layout
 struct Layout {
-    size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, seq_part0 = 0;
+    size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, cta_row0 = 0, row_info = 0, seq_part0 = 0;
     size_t o_part = 0, lse_part = 0, scores = 0, total = 0;
 };
 
@@ -80,6 +80,8 @@ Layout layout(int op, int B, int Hkv, int G, int D, int64_t T, int n_req) {
         L.row_slot0 = take(off, (size_t)(R + 1) * 4);
         L.cta_begin = take(off, (size_t)(n_req + 1) * 4);
         L.cta_slot0 = take(off, (size_t)(n_req + 1) * 4);
+        L.cta_row0 = take(off, (size_t)(n_req + 1) * 4);
+        L.row_info = take(off, (size_t)R * sizeof(RowInfo));
     }
     if (op == SGD_OP_DECODE) {
         const int64_t slots = (int64_t)n_req + R;
@@ -97,6 +99,8 @@ PlanView plan_view(uint8_t *ws, const Layout &L) {
     pv.row_slot0 = reinterpret_cast<int32_t *>(ws + L.row_slot0);
     pv.cta_begin = reinterpret_cast<int32_t *>(ws + L.cta_begin);
     pv.cta_slot0 = reinterpret_cast<int32_t *>(ws + L.cta_slot0);
+    pv.cta_row0 = reinterpret_cast<int32_t *>(ws + L.cta_row0);
+    pv.row_info = reinterpret_cast<RowInfo *>(ws + L.row_info);
     pv.seq_part0 = reinterpret_cast<int32_t *>(ws + L.seq_part0);
     return pv;
 }

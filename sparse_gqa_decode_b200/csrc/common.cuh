@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/sgd.h"
 
 namespace sgd {
@@ -34,6 +36,32 @@ constexpr int kPart = SGD_PARTITION;
 constexpr long long kWaitLimit = 1 << 22;  // bounded mbarrier polls before giving up
 
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------------------------------
+// host: launch `kern` through cudaLaunchKernelEx, as clusters of `cluster` CTAs along x when
+// cluster > 1.  Returns the launch's cudaError_t.
+// ------------------------------------------------------------------------------------------
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            unsigned cluster, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    unsigned n = 0;
+    if (cluster > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        n = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------------------------------
 // PTX wrappers
@@ -225,11 +253,24 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ------------------------------------------------------------------------------------------
 // internal launch interface (host side)
 // ------------------------------------------------------------------------------------------
+struct RowInfo {        // per-row record written by the plan kernel (32 bytes)
+    int32_t pos;        // padded stream position of the row
+    int32_t len;        // attended tokens (kept count, or the sequence length)
+    int32_t seq_start;  // cu_seqlens[b]
+    int32_t seq_len;    // sequence length
+    int32_t len_start;  // start of the attended row (cu_kept[b], or cu_seqlens[b])
+    int32_t part0;      // scheme-A partition offset of the sequence
+    int32_t pad[2];
+};
+static_assert(sizeof(RowInfo) == 32, "row record is two int4");
+
 struct PlanView {  // device arrays of a plan inside a workspace
     int32_t *row_pos;    // [R+1] padded stream position of each row
     int32_t *row_slot0;  // [R+1] first partial slot of each row
     int32_t *cta_begin;  // [N+1] stream position where each CTA starts
     int32_t *cta_slot0;  // [N+1] first partial slot of each CTA
+    int32_t *cta_row0;   // [N] first row each CTA range reaches (R for an empty range)
+    RowInfo *row_info;   // [R] per-row record
     int32_t *seq_part0;  // [B+1] scheme-A partition offset of each sequence
 };
 

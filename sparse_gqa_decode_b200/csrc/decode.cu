@@ -83,7 +83,7 @@ struct MmaCfg {
 template <class C>
 __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUtensorMap *tmV, const DecodeArgs &a,
                                              uint8_t *smem, uint64_t *full, uint64_t *empty,
-                                             volatile int32_t *abort_flag, float *row_scale, const int32_t *cu_rows,
+                                             volatile int32_t *abort_flag, float *row_scale,
                                              int cta, int lane) {
     if (!C::IDX && lane != 0) return;
     uint64_t pol = 0;
@@ -93,19 +93,34 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
         pol = l2_evict_first_policy();
     }
     SegCursor cur;
-    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    cur.init(a.plan, a.B * a.Hkv, cta);
     int stage = 0;
     uint32_t phase = 0;
     int row, slot;
     int32_t t0, t1;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        const int64_t seq0 = (int64_t)kvh * a.T + a.cu_seq[b];
-        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
+        const int64_t seq0 = (int64_t)kvh * a.T + cur.ri.seq_start;
+        const int32_t Lb = cur.ri.seq_len;
         const int32_t *ip = nullptr;
-        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
+        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start;
         const float *ksc = nullptr;
-        if constexpr (C::ROW_SCALE) ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
+        if constexpr (C::ROW_SCALE) ksc = a.k_scale + (int64_t)kvh * a.n_parts + cur.ri.part0;
+        // Gathers: the row indices of the next kPrefetch tiles are loaded ahead in registers
+        // (lane l holds those of rows l, l+32, ... of a tile), so a segment waits for its index
+        // loads once and not before every tile.
+        constexpr int RPL = C::IDX ? C::ROWS / 32 : 1;  // row indices held per lane and tile
+        constexpr int kPrefetch = 2;
+        int32_t tk[kPrefetch + 1][RPL];
+        auto load_tile_idx = [&](int32_t (&dst)[RPL], int32_t tt) {
+#pragma unroll
+            for (int qi = 0; qi < RPL; ++qi)  // rows past the segment repeat its last token
+                dst[qi] = (tt < t1) ? __ldg(ip + min(tt + lane + 32 * qi, t1 - 1)) : 0;
+        };
+        if constexpr (C::IDX) {
+#pragma unroll
+            for (int j = 0; j <= kPrefetch; ++j) load_tile_idx(tk[j], t0 + j * C::ROWS);
+        }
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
             uint8_t *sk = smem + stage * 2 * C::TILE;
@@ -122,13 +137,12 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                 // Row indices: lane l loads those of rows l, l+32, ...  Copies: one warp
                 // instruction moves whole rows (CPR lanes per row, one 16-byte chunk each), so
                 // every row reaches L2 as one contiguous request per tensor.
-                constexpr int RPL = C::ROWS / 32;  // row indices held per lane
                 constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
                 constexpr int RPI = 32 / CPR;      // rows per copy instruction
                 int32_t toks[RPL];
 #pragma unroll
-                for (int qi = 0; qi < RPL; ++qi) {  // every index load first, then the copies
-                    int32_t tok = __ldg(ip + min(t + lane + 32 * qi, t1 - 1));  // rows past the segment repeat its last token
+                for (int qi = 0; qi < RPL; ++qi) {
+                    int32_t tok = tk[0][qi];
                     if (tok < 0 || tok >= Lb) {
                         atomicOr(a.status, SGD_STATUS_BAD_INDEX);
                         tok = min(max(tok, 0), Lb - 1);
@@ -157,6 +171,13 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                 // rows of an empty sequence (inconsistent kept counts): nothing to fetch
                 if (lane == 0) atomicOr(a.status, SGD_STATUS_SIZE_MISMATCH);
                 mbar_arrive(&full[stage]);
+            }
+            if constexpr (C::IDX) {
+#pragma unroll
+                for (int j = 0; j < kPrefetch; ++j)
+#pragma unroll
+                    for (int qi = 0; qi < RPL; ++qi) tk[j][qi] = tk[j + 1][qi];
+                load_tile_idx(tk[kPrefetch], t + (kPrefetch + 1) * C::ROWS);
             }
             if (++stage == C::STAGES) {
                 stage = 0;
@@ -393,10 +414,10 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
 // the running max|K|.  Every quantising warp takes every tile.
 template <class C>
 __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty,
-                                               volatile int32_t *abort_flag, float *kmxs, const int32_t *cu_rows,
+                                               volatile int32_t *abort_flag, float *kmxs,
                                                int cta, int qw, int lane) {
     SegCursor cur;
-    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    cur.init(a.plan, a.B * a.Hkv, cta);
     int stage = 0, tile_no = 0;
     uint32_t phase = 0;
     int row, slot;
@@ -407,8 +428,8 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
     const int vr = 16 * qw + rho;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + a.cu_seq[b]) * C::D + half * (C::D / 2);
-        float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
+        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + cur.ri.seq_start) * C::D + half * (C::D / 2);
+        float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + cur.ri.part0;
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
             const uint32_t kbase = smem_u32(smem + stage * 2 * C::TILE);
@@ -508,15 +529,14 @@ __global__ void __launch_bounds__(C::THREADS, 2)
             return;
         }
     }
-    const int32_t *cu_rows = C::IDX ? a.cu_kept : a.cu_seq;
 
     if (warp == C::NW + C::NQ) {
-        mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, row_scale, cu_rows, cta, lane);
+        mma_producer<C>(&tmK, &tmV, a, smem, full, empty, abort_flag, row_scale, cta, lane);
         return;
     }
     if constexpr (C::NQ > 0) {
         if (warp >= C::NW) {
-            quant_consumer<C>(a, smem, full, empty, abort_flag, kmxs, cu_rows, cta, warp - C::NW, lane);
+            quant_consumer<C>(a, smem, full, empty, abort_flag, kmxs, cta, warp - C::NW, lane);
             return;
         }
     }
@@ -524,17 +544,18 @@ __global__ void __launch_bounds__(C::THREADS, 2)
     const int g4 = lane >> 2, t4 = lane & 3;
     const int pA = mma_row_perm(g4);
     SegCursor cur;
-    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    cur.init(a.plan, a.B * a.Hkv, cta);
     int stage = 0;
     uint32_t phase = 0;
     int row, slot;
     int32_t t0, t1;
     float run_kmax = 0.f, run_vmax = 0.f;  // mode 2
     int tile_no = 0;
+    const float vfac = (C::I8 && C::MODE == 0) ? __ldg(a.v_scale) : 1.f;  // loaded once, used per segment
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        const int32_t seq_start = a.cu_seq[b];
-        const int32_t Lb = a.cu_seq[b + 1] - seq_start;
+        const int32_t seq_start = cur.ri.seq_start;
+        const int32_t Lb = cur.ri.seq_len;
         const int64_t tok_base = (int64_t)kvh * a.T + seq_start;  // cache row of token 0 of the sequence
         uint32_t qf[C::GT][C::KB][2];
         float colf[C::GT][2];
@@ -549,8 +570,8 @@ __global__ void __launch_bounds__(C::THREADS, 2)
         }
         const float *ksc = nullptr;
         const int32_t *ip = nullptr;
-        if constexpr (C::I8) ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
-        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b];
+        if constexpr (C::I8) ksc = a.k_scale + (int64_t)kvh * a.n_parts + cur.ri.part0;
+        if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start;
 
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             // dense scheme A: the K scale of each sub-tile's partition, loaded before the wait
@@ -669,7 +690,6 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                     }
                 }
                 named_barrier_sync(1, C::NW * 32);
-                const float vfac = C::I8 ? __ldg(a.v_scale) : 1.f;
                 for (int e = threadIdx.x; e < a.G * C::D; e += C::NW * 32) {
                     const int g = e / C::D, d = e - g * C::D;
                     float M = -INFINITY;
@@ -724,16 +744,15 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const DecodeArgs a)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
     if (a.plan.cta_begin[cta] >= a.plan.cta_begin[cta + 1]) return;
-    const int32_t *cu_rows = IDX ? a.cu_kept : a.cu_seq;
     const int Hq = a.Hkv * a.G;
     SegCursor cur;
-    cur.init(a.plan, cu_rows, a.B, a.Hkv, cta);
+    cur.init(a.plan, a.B * a.Hkv, cta);
     int row, slot;
     int32_t t0, t1;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        const int32_t Lb = a.cu_seq[b + 1] - a.cu_seq[b];
-        const int64_t seq0 = (int64_t)kvh * a.T + a.cu_seq[b];
+        const int32_t Lb = cur.ri.seq_len;
+        const int64_t seq0 = (int64_t)kvh * a.T + cur.ri.seq_start;
         float q[MG][PER];
 #pragma unroll
         for (int g = 0; g < MG; ++g)
@@ -760,9 +779,9 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const DecodeArgs a)
         if constexpr (I8) {
             vfac = __ldg(a.v_scale);
             if (a.scheme == SGD_SCHEME_B) kfac = __ldg(a.k_scale);
-            else ksc = a.k_scale + (int64_t)kvh * a.n_parts + a.plan.seq_part0[b];
+            else ksc = a.k_scale + (int64_t)kvh * a.n_parts + cur.ri.part0;
         }
-        const int32_t *ip = IDX ? a.idx + (int64_t)kvh * a.Kt + a.cu_kept[b] : nullptr;
+        const int32_t *ip = IDX ? a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start : nullptr;
         for (int32_t j = t0 + warp; j < t1; j += NW) {
             int32_t tok = j;
             if constexpr (IDX) {
@@ -860,9 +879,29 @@ __global__ void __launch_bounds__(128) decode_generic_kernel(const DecodeArgs a)
 // exact LSE merge: per (sequence, query head), lse = ln sum_c exp(lse_c),
 // out = sum_c exp(lse_c - lse) o_c
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a, float *__restrict__ out,
-                                                    float *__restrict__ lse) {
-    // one block per (row, query head of the group), one thread per channel
+constexpr int kMergeThreads = 128;
+constexpr int kMergeChunk = 512;  // combination weights staged in shared memory per round
+
+__device__ __forceinline__ float block_reduce_128(float v, bool is_max, float *red) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const float w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = is_max ? fmaxf(v, w) : v + w;
+    }
+    const int warp = threadIdx.x >> 5;
+    __syncthreads();  // red is reused
+    if ((threadIdx.x & 31) == 0) red[warp] = v;
+    __syncthreads();
+    return is_max ? fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) : (red[0] + red[1]) + (red[2] + red[3]);
+}
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a, float *__restrict__ out,
+                                                              float *__restrict__ lse) {
+    // one block per (row, query head of the group): the row's partial LSEs are read by all
+    // threads at once (no load waits on another), the weights exp(lse_c - lse) are staged in
+    // shared memory and thread d accumulates channel d over the slots with independent loads
+    __shared__ float w[kMergeChunk];
+    __shared__ float red[4];
     const int r = blockIdx.x / a.G, g = blockIdx.x - r * a.G;
     const int b = r % a.B, kvh = r / a.B;
     const int s0 = a.plan.row_slot0[r], n = a.plan.row_slot0[r + 1] - s0;
@@ -870,22 +909,33 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a, float *_
     const int64_t h = (int64_t)b * Hq + kvh * a.G + g;
     const float *lp = a.lse_part + (int64_t)s0 * a.G + g;
     const float *op = a.o_part + ((int64_t)s0 * a.G + g) * a.D;
-    float M = -INFINITY;
-    for (int c = 0; c < n; ++c) M = fmaxf(M, __ldg(lp + (int64_t)c * a.G));
-    float S = 0.f;
-    for (int c = 0; c < n; ++c) S += expf(__ldg(lp + (int64_t)c * a.G) - M);
-    const float L = (n > 0) ? M + logf(S) : -INFINITY;
-    for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
-        float O = 0.f;
-        if (n == 1) {
-            O = __ldg(op + d);
-        } else {
-            for (int c = 0; c < n; ++c)
-                O += expf(__ldg(lp + (int64_t)c * a.G) - L) * __ldg(op + (int64_t)c * a.G * a.D + d);
-        }
-        out[h * a.D + d] = O;
+    const int tid = threadIdx.x;
+    if (n == 1) {  // one segment: its partial is the result
+        for (int d = tid; d < a.D; d += kMergeThreads) out[h * a.D + d] = __ldg(op + d);
+        if (tid == 0) lse[h] = __ldg(lp);
+        return;
     }
-    if (threadIdx.x == 0) lse[h] = (n == 1) ? __ldg(lp) : L;
+    float M = -INFINITY;
+    for (int c = tid; c < n; c += kMergeThreads) M = fmaxf(M, __ldg(lp + (int64_t)c * a.G));
+    M = block_reduce_128(M, true, red);
+    float S = 0.f;
+    for (int c = tid; c < n; c += kMergeThreads) S += expf(__ldg(lp + (int64_t)c * a.G) - M);
+    S = block_reduce_128(S, false, red);
+    const float L = (n > 0) ? M + logf(S) : -INFINITY;
+    float O = 0.f;
+    for (int c0 = 0; c0 < n; c0 += kMergeChunk) {
+        const int m = min(kMergeChunk, n - c0);
+        __syncthreads();  // the previous round's weights are consumed
+        for (int c = tid; c < m; c += kMergeThreads) w[c] = expf(__ldg(lp + (int64_t)(c0 + c) * a.G) - L);
+        __syncthreads();
+        if (tid < a.D) {
+            const float *oc = op + (int64_t)c0 * a.G * a.D + tid;
+#pragma unroll 8
+            for (int c = 0; c < m; ++c) O += w[c] * __ldg(oc + (int64_t)c * a.G * a.D);
+        }
+    }
+    if (tid < a.D) out[h * a.D + tid] = O;
+    if (tid == 0) lse[h] = L;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -950,8 +1000,7 @@ static int launch_mma(const DecodeArgs &a, int n_cta, cudaStream_t s) {
     auto k = decode_mma_kernel<C>;
     cudaError_t e = set_smem_attrs<C>();
     if (e != cudaSuccess) return (int)e;
-    k<<<n_cta, C::THREADS, C::SMEM, s>>>(mk, mv, a);
-    return (int)cudaGetLastError();
+    return (int)launch_k(k, dim3(n_cta), dim3(C::THREADS), C::SMEM, s, 1, mk, mv, a);
 }
 
 template <int D, int GT, bool I8, int MODE>
@@ -967,10 +1016,8 @@ static int launch_mma_idx(const DecodeArgs &a, bool indexed, int n_cta, cudaStre
 template <int D, typename KT, int MODE>
 static int launch_generic(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
     if (indexed && MODE == 0)
-        decode_generic_kernel<D, KT, true, MODE><<<n_cta, 128, 0, s>>>(a);
-    else
-        decode_generic_kernel<D, KT, false, MODE><<<n_cta, 128, 0, s>>>(a);
-    return (int)cudaGetLastError();
+        return (int)launch_k(decode_generic_kernel<D, KT, true, MODE>, dim3(n_cta), dim3(128), 0, s, 1, a);
+    return (int)launch_k(decode_generic_kernel<D, KT, false, MODE>, dim3(n_cta), dim3(128), 0, s, 1, a);
 }
 
 Family decode_family(sgd_dtype kv, sgd_dtype q, int D, bool score) {
@@ -1034,8 +1081,7 @@ int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s) {
 }
 
 int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s) {
-    merge_kernel<<<a.B * a.Hkv * a.G, 128, 0, s>>>(a, out, lse);
-    return (int)cudaGetLastError();
+    return (int)launch_k(merge_kernel, dim3(a.B * a.Hkv * a.G), dim3(kMergeThreads), 0, s, 1, a, out, lse);
 }
 
 }  // namespace sgd

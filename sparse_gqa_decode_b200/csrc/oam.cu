@@ -547,20 +547,8 @@ int launch_topk_cfg(const float *scores, const int32_t *cu, int B, int Hkv, int6
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return (int)e;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(B * Hkv * CL));
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return (int)cudaLaunchKernelEx(&cfg, kern, scores, cu, B, T, keep_num, keep_den, idx, cu_kept, kept_total,
-                                   status, cap);
+    return (int)launch_k(kern, dim3((unsigned)(B * Hkv * CL)), dim3(NT), (size_t)smem, s, CL, scores, cu, B, T,
+                           keep_num, keep_den, idx, cu_kept, kept_total, status, cap);
 }
 
 int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t T, int keep_num, int keep_den,

@@ -7,19 +7,43 @@
 
 namespace sgd {
 
+constexpr size_t kPlanStageBytes = 48 * 1024;  // within the default dynamic shared-memory limit
+
 // cu_len: lengths of the attended rows (cu_seqlens, or cu_kept for a kept set);
 // cu_seq: cu_seqlens (for the scheme-A partition offsets of each sequence).
+// With `staged`, the per-sequence values are read once into dynamic shared memory and row_pos,
+// cta_begin and the partition offsets are built there (R + n_req + 2 + 5B int32) and copied out
+// at the end, so no step waits on a global-memory round trip after the first loads.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu_len,
                                                     const int32_t *__restrict__ cu_seq, int B, int Hkv,
                                                     int n_req, int min_chunk, int mode, int granule,
-                                                    PlanView pv, WsHeader *hdr) {
+                                                    PlanView pv, WsHeader *hdr, int staged) {
     __shared__ int32_t sm[33];
+    extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
     const int R = B * Hkv;
+    int32_t *row_pos = staged ? stage : pv.row_pos;
+    int32_t *cta_begin = staged ? stage + R + 1 : pv.cta_begin;
+    int32_t *seqv = stage + R + n_req + 2;  // staged: [5][B] length, sequence length, starts, part0
+    int32_t *part0 = staged ? seqv + 4 * B : pv.seq_part0;
     if (tid == 0) {
         hdr->status = 0;
         hdr->amax_bits[0] = hdr->amax_bits[1] = 0u;
     }
+    if (staged) {
+        for (int b = tid; b < B; b += blockDim.x) {  // all four loads of a thread in flight together
+            const int32_t a0 = cu_len[b], a1 = cu_len[b + 1], s0 = cu_seq[b], s1 = cu_seq[b + 1];
+            seqv[b] = a1 - a0;
+            seqv[B + b] = s1 - s0;
+            seqv[2 * B + b] = a0;
+            seqv[3 * B + b] = s0;
+        }
+        __syncthreads();
+    }
+    auto len_of = [&](int b) -> int32_t { return staged ? seqv[b] : cu_len[b + 1] - cu_len[b]; };
+    auto seq_len_of = [&](int b) -> int32_t { return staged ? seqv[B + b] : cu_seq[b + 1] - cu_seq[b]; };
+    auto len_start_of = [&](int b) -> int32_t { return staged ? seqv[2 * B + b] : cu_len[b]; };
+    auto seq_start_of = [&](int b) -> int32_t { return staged ? seqv[3 * B + b] : cu_seq[b]; };
 
     // 1. padded stream position of every row
     int32_t carry = 0;
@@ -27,18 +51,17 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         const int r = base + tid;
         int32_t v = 0;
         if (r < R) {
-            const int b = r % B;
-            const int32_t L = cu_len[b + 1] - cu_len[b];
+            const int32_t L = len_of(r % B);
             if (L < 1) atomicOr(&hdr->status, SGD_STATUS_EMPTY_SEQUENCE);
             v = (int32_t)align_up(max(L, 0), granule);
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
-        if (r < R) pv.row_pos[r] = carry + ex;
+        if (r < R) row_pos[r] = carry + ex;
         carry += total;
     }
     const int32_t W = carry;
-    if (tid == 0) pv.row_pos[R] = W;
+    if (tid == 0) row_pos[R] = W;
 
     int64_t S = 0;
     int ncta;
@@ -57,22 +80,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         if (mode == 0)
             a = (int32_t)(((int64_t)i * S < (int64_t)W) ? (int64_t)i * S : (int64_t)W);
         else
-            a = pv.row_pos[min(i, R)];
-        pv.cta_begin[i] = a;
+            a = row_pos[min(i, R)];
+        cta_begin[i] = a;
     }
     __syncthreads();
 
-    // 3. segments per CTA -> first slot of each CTA
+    // 3. segments per CTA -> first slot and first row of each CTA
     carry = 0;
     for (int base = 0; base < n_req; base += blockDim.x) {
         const int i = base + tid;
         int32_t v = 0;
         if (i < n_req) {
-            const int32_t a = pv.cta_begin[i], e = pv.cta_begin[i + 1];
+            const int32_t a = cta_begin[i], e = cta_begin[i + 1];
+            int r0 = R;
             if (a < e) {
-                for (int r = upper_bound_i32(pv.row_pos, R + 1, a) - 1; r < R && pv.row_pos[r] < e; ++r)
-                    v += (pv.row_pos[r + 1] > pv.row_pos[r]) ? 1 : 0;
+                r0 = upper_bound_i32(row_pos, R + 1, a) - 1;
+                for (int r = r0; r < R && row_pos[r] < e; ++r) v += (row_pos[r + 1] > row_pos[r]) ? 1 : 0;
             }
+            pv.cta_row0[i] = r0;
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
@@ -82,16 +107,37 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     const int32_t nslots_cta = carry;
     if (tid == 0) pv.cta_slot0[n_req] = nslots_cta;
 
-    // 4. segments per row -> first slot of each row (same stream order)
+    // 4. scheme-A partition offset of every sequence: sum_{b'<b} ceil(L_b' / 64)
+    carry = 0;
+    for (int base = 0; base < B; base += blockDim.x) {
+        const int b = base + tid;
+        int32_t v = 0;
+        if (b < B) v = (int32_t)((max(seq_len_of(b), 0) + kPart - 1) / kPart);
+        int32_t total;
+        const int32_t ex = block_exclusive_scan(v, total, sm);
+        if (b < B) {
+            part0[b] = carry + ex;
+            if (staged) pv.seq_part0[b] = carry + ex;
+        }
+        carry += total;
+    }
+    const int32_t n_parts = carry;
+    if (tid == 0) pv.seq_part0[B] = n_parts;
+    __syncthreads();  // part0 complete
+
+    // 5. segments per row -> first slot of each row (same stream order); the row records
     carry = 0;
     for (int base = 0; base < R; base += blockDim.x) {
         const int r = base + tid;
         int32_t v = 0;
         if (r < R) {
-            const int32_t p0 = pv.row_pos[r];
+            const int32_t p0 = row_pos[r];
             const int b = r % B;
-            const int32_t L = max(cu_len[b + 1] - cu_len[b], 0);
+            const int32_t Lr = len_of(b), L = max(Lr, 0);
             if (L > 0) v = (mode == 0) ? (int32_t)((p0 + L - 1) / S - p0 / S + 1) : 1;
+            int4 *ri = reinterpret_cast<int4 *>(pv.row_info + r);
+            ri[0] = make_int4(p0, Lr, seq_start_of(b), seq_len_of(b));
+            ri[1] = make_int4(len_start_of(b), part0[b], 0, 0);
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
@@ -101,26 +147,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     if (tid == 0) {
         pv.row_slot0[R] = carry;
         if (carry != nslots_cta) atomicOr(&hdr->status, SGD_STATUS_SIZE_MISMATCH);
-    }
-
-    // 5. scheme-A partition offset of every sequence: sum_{b'<b} ceil(L_b' / 64)
-    carry = 0;
-    for (int base = 0; base < B; base += blockDim.x) {
-        const int b = base + tid;
-        int32_t v = 0;
-        if (b < B) v = (int32_t)((max(cu_seq[b + 1] - cu_seq[b], 0) + kPart - 1) / kPart);
-        int32_t total;
-        const int32_t ex = block_exclusive_scan(v, total, sm);
-        if (b < B) pv.seq_part0[b] = carry + ex;
-        carry += total;
-    }
-    if (tid == 0) {
-        pv.seq_part0[B] = carry;
         hdr->plan_W = W;
         hdr->plan_S = S;
         hdr->plan_ncta = ncta;
         hdr->plan_nslots = nslots_cta;
-        hdr->n_parts = carry;
+        hdr->n_parts = n_parts;
+    }
+    if (staged) {  // copy the staged arrays out
+        __syncthreads();
+        for (int i = tid; i <= R; i += blockDim.x) pv.row_pos[i] = row_pos[i];
+        for (int i = tid; i <= n_req; i += blockDim.x) pv.cta_begin[i] = cta_begin[i];
     }
 }
 
@@ -134,7 +170,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
     }
     if (cta >= n_req) return;
     SegCursor cur;
-    cur.init(pv, cu, B, Hkv, cta);
+    cur.init(pv, B * Hkv, cta);
     int row, slot;
     int32_t t0, t1;
     while (cur.next(row, t0, t1, slot)) {
@@ -150,12 +186,16 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule) {
-    plan_kernel<<<1, 1024, 0, s>>>(cu_len, cu_seq, B, Hkv, n_req, min_chunk, mode, granule, pv, hdr);
+    const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
+    const int staged = stage_bytes <= kPlanStageBytes;
+    launch_k(plan_kernel, dim3(1), dim3(1024), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
+               min_chunk, mode, granule, pv, hdr, staged);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s) {
-    plan_dump_kernel<<<(n_req + 127) / 128, 128, 0, s>>>(pv, cu, B, Hkv, n_req, segs, max_segs, n_segs, hdr);
+    launch_k(plan_dump_kernel, dim3((n_req + 127) / 128), dim3(128), 0, s, 1, pv, cu, B, Hkv, n_req, segs, max_segs,
+               n_segs, hdr);
 }
 
 }  // namespace sgd

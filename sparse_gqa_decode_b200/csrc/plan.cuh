@@ -32,40 +32,48 @@ __device__ __forceinline__ int upper_bound_i32(const int32_t *a, int n, int32_t 
     return lo;
 }
 
-// Walks the segments of one CTA in stream order.
+// Walks the segments of one CTA in stream order.  init() is four independent loads; each
+// segment then costs one 32-byte row record, which also carries what the caller needs of the
+// segment's sequence, and the last segment is known without a further load.
 struct SegCursor {
-    const int32_t *row_pos;
-    const int32_t *cu;  // lengths of row r are cu[b+1] - cu[b], b = r % B
-    int R, B;
+    const RowInfo *info;
+    int R;
     int32_t end;  // CTA range end (stream position)
     int32_t pos;  // next stream position to cover
     int r;        // current row candidate
     int slot;     // slot of the next segment
+    int left;     // segments still to return
+    RowInfo ri;   // record of the row of the segment last returned
 
-    __device__ void init(const PlanView &pv, const int32_t *cu_, int B_, int Hkv, int cta) {
-        row_pos = pv.row_pos;
-        cu = cu_;
-        B = B_;
-        R = B_ * Hkv;
+    __device__ void init(const PlanView &pv, int R_, int cta) {
+        info = pv.row_info;
+        R = R_;
         pos = pv.cta_begin[cta];
         end = pv.cta_begin[cta + 1];
         slot = pv.cta_slot0[cta];
-        r = (pos < end) ? upper_bound_i32(row_pos, R + 1, pos) - 1 : R;
+        left = pv.cta_slot0[cta + 1] - slot;
+        r = pv.cta_row0[cta];
     }
 
     // Next segment: row, row-local token range [t0, t1), slot.  False when done.
     __device__ bool next(int &row, int32_t &t0, int32_t &t1, int &s) {
-        while (r < R && row_pos[r] < end) {
-            const int b = r % B;
-            const int32_t L = cu[b + 1] - cu[b];
-            const int32_t rp = row_pos[r];
-            const int32_t lo = max(pos, rp), hi = min(end, rp + max(L, 0));
+        while (left > 0 && r < R) {
+            const int4 *p = reinterpret_cast<const int4 *>(info + r);
+            const int4 x = __ldg(p), y = __ldg(p + 1);
+            ri.pos = x.x;
+            ri.len = x.y;
+            ri.seq_start = x.z;
+            ri.seq_len = x.w;
+            ri.len_start = y.x;
+            ri.part0 = y.y;
+            const int32_t lo = max(pos, ri.pos), hi = min(end, ri.pos + max(ri.len, 0));
             ++r;
             if (hi > lo) {
                 row = r - 1;
-                t0 = lo - rp;
-                t1 = hi - rp;
+                t0 = lo - ri.pos;
+                t1 = hi - ri.pos;
                 s = slot++;
+                --left;
                 pos = hi;
                 return true;
             }

@@ -198,21 +198,30 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
                          float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
     constexpr int VE = Vec<T>::VE;
     const int64_t nvec = (int64_t)Hkv * Ttot * D / VE;
-    quant_prep_kernel<<<1, 1024, 0, s>>>(cu, B, n_parts, scheme == SGD_SCHEME_A, seq_part0, hdr);
+    cudaError_t e = launch_k(quant_prep_kernel, dim3(1), dim3(1024), 0, s, 1, cu, B, n_parts,
+                               (int)(scheme == SGD_SCHEME_A), seq_part0, hdr);
+    if (e != cudaSuccess) return (int)e;
     const int grid_stream = sm_count * 8;
+    const T *none = nullptr;
+    int8_t *no_codes = nullptr;
+    float *no_scale = nullptr;
     if (scheme == SGD_SCHEME_A) {
         const int64_t total = (int64_t)Hkv * n_parts;
         const int grid = (int)std::min<int64_t>(total, (int64_t)sm_count * 8);
-        if (grid > 0)
-            quant_k_partition_kernel<T, D><<<grid, 256, 0, s>>>(k, v, cu, seq_part0, B, Hkv, Ttot, n_parts, kc,
-                                                                k_scale, hdr);
-        quant_global_kernel<T><<<grid_stream, 256, 0, s>>>(v, vc, v_scale, 1, nullptr, nullptr, nullptr, 0, nvec,
-                                                           hdr);
+        if (grid > 0) {
+            e = launch_k(quant_k_partition_kernel<T, D>, dim3(grid), dim3(256), 0, s, 1, k, v, cu,
+                           (const int32_t *)seq_part0, B, Hkv, Ttot, n_parts, kc, k_scale, hdr);
+            if (e != cudaSuccess) return (int)e;
+        }
+        e = launch_k(quant_global_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, v, vc, v_scale, 1, none,
+                       no_codes, no_scale, 0, nvec, (const WsHeader *)hdr);
     } else {
-        quant_amax_kernel<T><<<grid_stream, 256, 0, s>>>(k, v, nvec, hdr);
-        quant_global_kernel<T><<<grid_stream, 256, 0, s>>>(k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
+        e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
+        if (e != cudaSuccess) return (int)e;
+        e = launch_k(quant_global_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, kc, k_scale, 0, v, vc,
+                       v_scale, 1, nvec, (const WsHeader *)hdr);
     }
-    return (int)cudaGetLastError();
+    return (int)e;
 }
 
 template <typename T>
@@ -220,11 +229,14 @@ static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t 
                                 int8_t *vc, float *k_scale, float *v_scale, const WsHeader *hdr, int sm_count,
                                 cudaStream_t s) {
     const int64_t nvec = (int64_t)Hkv * Ttot * D / Vec<T>::VE;
+    const T *none = nullptr;
+    int8_t *no_codes = nullptr;
+    float *no_scale = nullptr;
     if (scheme == SGD_SCHEME_A)
-        quant_global_kernel<T><<<sm_count * 8, 256, 0, s>>>(v, vc, v_scale, 1, nullptr, nullptr, nullptr, 0, nvec, hdr);
-    else
-        quant_global_kernel<T><<<sm_count * 8, 256, 0, s>>>(k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
-    return (int)cudaGetLastError();
+        return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * 8), dim3(256), 0, s, 1, v, vc, v_scale, 1,
+                               none, no_codes, no_scale, 0, nvec, hdr);
+    return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * 8), dim3(256), 0, s, 1, k, kc, k_scale, 0, v, vc,
+                           v_scale, 1, nvec, hdr);
 }
 
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
