@@ -271,6 +271,20 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
     return nbytes / dt / 1e9, sample, dt
 
 
+def reduce_max(x, dev, world):
+    """The maximum of x over all ranks (x itself for one rank): every timing is the slowest rank's."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(step_bytes, steps, total_ms, world):
+    """Whole-job GB/s: each of `world` ranks moves step_bytes per step over `steps` steps, in the
+    slowest rank's total_ms (weak scaling: the per-rank work is fixed)."""
+    return world * step_bytes * steps / (total_ms / 1e3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_gqa_decode_b200 as sgd
 
@@ -320,13 +334,9 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     stage_ms = {n: [r[n][0].elapsed_time(r[n][1]) for r in rec] for n in names}
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = reduce_max(sum(step_ms), dev, world)
     ms_per_step = total_ms / K
-    value = world * step_bytes * K / (total_ms / 1e3) / 1e9
+    value = job_gbs(step_bytes, K, total_ms, world)
 
     # e2e: host buffers through the same calls, copies inside the timed region
     pin_q, pin_k, pin_v, pin_cu = (x.pin_memory() for x in (bt.q, bt.k, bt.v, bt.cu_seqlens))
@@ -357,11 +367,7 @@ def run_ours(args, rank, world, local_rank):
         h_lse.copy_(lse, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    et = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(et.item())
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, dev, world)
 
     if rank != 0:
         return None
@@ -406,7 +412,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": kernels[dom], "achieved": round(achieved, 1), "peak": peak,
                      "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": stages[dom]},
-        "e2e": {"value": round(world * step_bytes / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(job_gbs(step_bytes, 1, e2e_ms, world), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": pipe.launches_per_step() * K,
         "clocks": clk,

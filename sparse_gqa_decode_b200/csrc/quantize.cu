@@ -158,6 +158,8 @@ __global__ void __launch_bounds__(256) quant_amax_kernel(const T *__restrict__ k
     }
 }
 
+constexpr int kGlobalUnroll = 4;  // independent 16-byte loads per thread and tensor
+
 // Pass 2: codes of one or two whole tensors with their global scales.
 template <typename T>
 __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__ x0, int8_t *__restrict__ c0,
@@ -179,17 +181,51 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
     const uint4 *p0 = reinterpret_cast<const uint4 *>(x0);
     const uint4 *p1 = reinterpret_cast<const uint4 *>(x1);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    {
-        for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += stride) {
+    // kGlobalUnroll vectors per thread in flight per tensor, then their codes
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (; i + (kGlobalUnroll - 1) * stride < nvec; i += kGlobalUnroll * stride) {
+        uint4 w0[kGlobalUnroll], w1[kGlobalUnroll];
+#pragma unroll
+        for (int u = 0; u < kGlobalUnroll; ++u) w0[u] = __ldcs(p0 + i + u * stride);
+        if (x1) {
+#pragma unroll
+            for (int u = 0; u < kGlobalUnroll; ++u) w1[u] = __ldcs(p1 + i + u * stride);
+        }
+#pragma unroll
+        for (int u = 0; u < kGlobalUnroll; ++u) {
             float x[VE];
-            Vec<T>::unpack(__ldcs(p0 + i), x);
-            store_codes<VE>(c0 + i * VE, x, s0, r0);
+            Vec<T>::unpack(w0[u], x);
+            store_codes<VE>(c0 + (i + u * stride) * VE, x, s0, r0);
             if (x1) {
-                Vec<T>::unpack(__ldcs(p1 + i), x);
-                store_codes<VE>(c1 + i * VE, x, s1, r1);
+                Vec<T>::unpack(w1[u], x);
+                store_codes<VE>(c1 + (i + u * stride) * VE, x, s1, r1);
             }
         }
     }
+    for (; i < nvec; i += stride) {
+        float x[VE];
+        Vec<T>::unpack(__ldcs(p0 + i), x);
+        store_codes<VE>(c0 + i * VE, x, s0, r0);
+        if (x1) {
+            Vec<T>::unpack(__ldcs(p1 + i), x);
+            store_codes<VE>(c1 + i * VE, x, s1, r1);
+        }
+    }
+}
+
+// Resident CTAs per SM of quant_global_kernel<T> on the current device (cached per device).
+template <typename T>
+static int global_ctas_per_sm() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_global_kernel<T>, 256, 0) != cudaSuccess || n < 1)
+            n = 4;
+        cache[dev] = n;
+    }
+    return cache[dev];
 }
 
 template <typename T, int D>
@@ -213,13 +249,13 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
                            (const int32_t *)seq_part0, B, Hkv, Ttot, n_parts, kc, k_scale, hdr);
             if (e != cudaSuccess) return (int)e;
         }
-        e = launch_k(quant_global_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, v, vc, v_scale, 1, none,
-                       no_codes, no_scale, 0, nvec, (const WsHeader *)hdr);
+        e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v, vc,
+                     v_scale, 1, none, no_codes, no_scale, 0, nvec, (const WsHeader *)hdr);
     } else {
         e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
         if (e != cudaSuccess) return (int)e;
-        e = launch_k(quant_global_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, kc, k_scale, 0, v, vc,
-                       v_scale, 1, nvec, (const WsHeader *)hdr);
+        e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k, kc,
+                     k_scale, 0, v, vc, v_scale, 1, nvec, (const WsHeader *)hdr);
     }
     return (int)e;
 }
@@ -233,10 +269,10 @@ static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t 
     int8_t *no_codes = nullptr;
     float *no_scale = nullptr;
     if (scheme == SGD_SCHEME_A)
-        return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * 8), dim3(256), 0, s, 1, v, vc, v_scale, 1,
-                               none, no_codes, no_scale, 0, nvec, hdr);
-    return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * 8), dim3(256), 0, s, 1, k, kc, k_scale, 0, v, vc,
-                           v_scale, 1, nvec, hdr);
+        return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v,
+                             vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr);
+    return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k,
+                         kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
 }
 
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
