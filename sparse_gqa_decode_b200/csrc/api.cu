@@ -60,7 +60,8 @@ int check_kv(const sgd_kv *kv) {
 
 // workspace layout
 struct Layout {
-    size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, cta_row0 = 0, row_info = 0, seq_part0 = 0;
+    size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, cta_row0 = 0, row_info = 0, row_done = 0;
+    size_t seq_part0 = 0;
     size_t o_part = 0, lse_part = 0, scores = 0, total = 0;
 };
 
@@ -84,6 +85,7 @@ Layout layout(int op, int B, int Hkv, int G, int D, int64_t T, int n_req) {
         L.row_info = take(off, (size_t)R * sizeof(RowInfo));
     }
     if (op == SGD_OP_DECODE) {
+        L.row_done = take(off, (size_t)R * 4);
         const int64_t slots = (int64_t)n_req + R;
         L.o_part = take(off, (size_t)slots * G * D * 4);
         L.lse_part = take(off, (size_t)slots * G * 4);
@@ -101,6 +103,7 @@ PlanView plan_view(uint8_t *ws, const Layout &L) {
     pv.cta_slot0 = reinterpret_cast<int32_t *>(ws + L.cta_slot0);
     pv.cta_row0 = reinterpret_cast<int32_t *>(ws + L.cta_row0);
     pv.row_info = reinterpret_cast<RowInfo *>(ws + L.row_info);
+    pv.row_done = L.row_done ? reinterpret_cast<int32_t *>(ws + L.row_done) : nullptr;
     pv.seq_part0 = reinterpret_cast<int32_t *>(ws + L.seq_part0);
     return pv;
 }
@@ -359,7 +362,7 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     cudaStream_t s = as_stream(stream);
     const int min_chunk = (n_splits > 0 || schedule == 1) ? kGranule : kAutoMinChunk;
     launch_plan(indexed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
-                hdr, s);
+                hdr, s, kGranule, out, lse, G, kv->D);
     DecodeArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q;
@@ -384,9 +387,13 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     a.plan = pv;
     a.o_part = reinterpret_cast<float *>(ws + L.o_part);
     a.lse_part = reinterpret_cast<float *>(ws + L.lse_part);
+    a.out = out;
+    a.lse = lse;
     a.status = &hdr->status;
     int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
+    // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials
+    if (decode_family(kv->dtype, q_dtype, kv->D, false) == kFamilyMma) return SGD_OK;
     e = launch_merge(a, out, lse, s);
     return e == 0 ? SGD_OK : SGD_ERR_CUDA;
 }
@@ -400,13 +407,14 @@ int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chun
     if (n_req < 1 || min_chunk < kGranule || min_chunk % kGranule != 0 || max_segs < 0) return SGD_ERR_ARG;
     if (!aligned16(workspace)) return SGD_ERR_ALIGN;
     const Layout L = layout(SGD_OP_DECODE, B, Hkv, 1, 64, 1, n_req);
-    if (workspace_bytes < L.o_part) return SGD_ERR_WORKSPACE;
+    if (workspace_bytes < L.row_done) return SGD_ERR_WORKSPACE;  // the plan arrays only
     DevInfo *dev;
     int rc = current_device(&dev);
     if (rc != SGD_OK) return rc;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
-    const PlanView pv = plan_view(ws, L);
+    PlanView pv = plan_view(ws, L);
+    pv.row_done = nullptr;  // no decode follows
     cudaStream_t s = as_stream(stream);
     launch_plan(cu, cu, B, Hkv, n_req, min_chunk, mode, pv, hdr, s);
     launch_plan_dump(pv, cu, B, Hkv, n_req, segs, max_segs, n_segs, hdr, s);

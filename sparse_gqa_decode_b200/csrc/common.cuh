@@ -260,7 +260,8 @@ struct RowInfo {        // per-row record written by the plan kernel (32 bytes)
     int32_t seq_len;    // sequence length
     int32_t len_start;  // start of the attended row (cu_kept[b], or cu_seqlens[b])
     int32_t part0;      // scheme-A partition offset of the sequence
-    int32_t pad[2];
+    int32_t slot0;      // first partial slot of the row
+    int32_t nseg;       // segments (partial results) of the row
 };
 static_assert(sizeof(RowInfo) == 32, "row record is two int4");
 
@@ -271,6 +272,7 @@ struct PlanView {  // device arrays of a plan inside a workspace
     int32_t *cta_slot0;  // [N+1] first partial slot of each CTA
     int32_t *cta_row0;   // [N] first row each CTA range reaches (R for an empty range)
     RowInfo *row_info;   // [R] per-row record
+    int32_t *row_done;   // [R] decode: segments of the row finished (zeroed by the plan kernel), or NULL
     int32_t *seq_part0;  // [B+1] scheme-A partition offset of each sequence
 };
 

@@ -495,6 +495,91 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
 }
 
 // ------------------------------------------------------------------------------------------
+// in-kernel LSE merge of one row's partials (run by the CTA that finishes the row's last
+// outstanding segment; the 128 consumer threads, `scratch` = one stage of shared memory):
+// lse = ln sum_c exp(lse_c), out = sum_c exp(lse_c - lse) o_c, as merge_kernel computes it.
+// ------------------------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n, int b, int kvh, float *scratch) {
+    constexpr int NT = C::NW * 32;
+    const int G = a.G, tid = threadIdx.x;
+    float *Ls = scratch;                       // [16] per head: running max, then the lse
+    float *Ss = scratch + 16;                  // [16] running sum
+    float *w = scratch + 32;                   // [chunk][G] lse, then weights
+    const int chunk = (2 * C::TILE / 4 - 32) / G;
+    const float *lp = a.lse_part + (int64_t)slot0 * G;
+    const float *op = a.o_part + (int64_t)slot0 * G * C::D;
+    if (tid < G) {
+        Ls[tid] = -INFINITY;
+        Ss[tid] = 0.f;
+    }
+    for (int c0 = 0; c0 < n; c0 += chunk) {  // pass 1: max and sum of exp per head, online
+        const int m = min(chunk, n - c0);
+        named_barrier_sync(1, NT);
+        for (int p = tid; p < m * G; p += NT) w[p] = __ldcg(lp + (int64_t)c0 * G + p);
+        named_barrier_sync(1, NT);
+        if (tid < G) {
+            float M = Ls[tid], S = Ss[tid];
+            for (int c = 0; c < m; ++c) {
+                const float x = w[c * G + tid];
+                if (x > M) {
+                    S = S * expf(M - x) + 1.f;
+                    M = x;
+                } else {
+                    S += expf(x - M);
+                }
+            }
+            Ls[tid] = M;
+            Ss[tid] = S;
+        }
+    }
+    named_barrier_sync(1, NT);
+    if (tid < G) Ls[tid] = (n > 0) ? Ls[tid] + logf(Ss[tid]) : -INFINITY;
+    const int Hq = a.Hkv * G;
+    float *dst = a.out + ((int64_t)b * Hq + kvh * G) * C::D;
+    // pass 2: thread t owns float4 columns t, t + NT, ... of the row's [G][D] block and reads
+    // them from every slot of a chunk, kQ4 * 4 independent 16-byte loads in flight
+    constexpr int kQ4 = 16 * C::D / 4 / NT;  // float4 columns per thread at G = 16
+    const int Q = G * C::D / 4;
+    float4 *dst4 = reinterpret_cast<float4 *>(dst);
+    for (int c0 = 0; c0 < n; c0 += chunk) {
+        const int m = min(chunk, n - c0);
+        named_barrier_sync(1, NT);
+        for (int p = tid; p < m * G; p += NT) w[p] = expf(__ldcg(lp + (int64_t)c0 * G + p) - Ls[p % G]);
+        named_barrier_sync(1, NT);
+        const float4 *oc = reinterpret_cast<const float4 *>(op + (int64_t)c0 * G * C::D);
+        float4 acc[kQ4];
+#pragma unroll
+        for (int j = 0; j < kQ4; ++j) {
+            const int q = tid + j * NT;
+            acc[j] = (c0 > 0 && q < Q) ? dst4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll 4
+        for (int c = 0; c < m; ++c) {
+#pragma unroll
+            for (int j = 0; j < kQ4; ++j) {
+                const int q = tid + j * NT;
+                if (q < Q) {
+                    const float4 x = __ldcg(oc + (int64_t)c * Q + q);
+                    const float wc = w[c * G + (4 * q) / C::D];
+                    acc[j].x += wc * x.x;
+                    acc[j].y += wc * x.y;
+                    acc[j].z += wc * x.z;
+                    acc[j].w += wc * x.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kQ4; ++j) {
+            const int q = tid + j * NT;
+            if (q < Q) dst4[q] = acc[j];
+        }
+    }
+    if (tid < G) a.lse[(int64_t)b * Hq + kvh * G + tid] = Ls[tid];
+    named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
+}
+
+// ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
 template <class C>
@@ -690,22 +775,50 @@ __global__ void __launch_bounds__(C::THREADS, 2)
                     }
                 }
                 named_barrier_sync(1, C::NW * 32);
-                for (int e = threadIdx.x; e < a.G * C::D; e += C::NW * 32) {
-                    const int g = e / C::D, d = e - g * C::D;
-                    float M = -INFINITY;
+                const int tid = threadIdx.x;
+                if (tid < a.G) {  // head g: the warps' weights replace their m in ml; the lse replaces warp 0's l
+                    float M = -INFINITY, f[C::NW], L = 0.f;
 #pragma unroll
-                    for (int w = 0; w < C::NW; ++w) M = fmaxf(M, ml[(w * C::NG + g) * 2]);
-                    float L = 0.f, O = 0.f;
-                    if (M != -INFINITY) {
+                    for (int w = 0; w < C::NW; ++w) M = fmaxf(M, ml[(w * C::NG + tid) * 2]);
 #pragma unroll
-                        for (int w = 0; w < C::NW; ++w) {
-                            const float f = exp2f(ml[(w * C::NG + g) * 2] - M);
-                            L += f * ml[(w * C::NG + g) * 2 + 1];
-                            O += f * eo[(w * C::NG + g) * C::D + d];
-                        }
+                    for (int w = 0; w < C::NW; ++w) {
+                        f[w] = (M == -INFINITY) ? 0.f : exp2f(ml[(w * C::NG + tid) * 2] - M);
+                        L += f[w] * ml[(w * C::NG + tid) * 2 + 1];
                     }
-                    a.o_part[((int64_t)slot * a.G + g) * C::D + d] = (L > 0.f) ? O / L * vfac : 0.f;
-                    if (d == 0) a.lse_part[(int64_t)slot * a.G + g] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+                    const float inv = (L > 0.f) ? vfac / L : 0.f;
+#pragma unroll
+                    for (int w = 0; w < C::NW; ++w) ml[(w * C::NG + tid) * 2] = f[w] * inv;
+                    ml[tid * 2 + 1] = (L > 0.f) ? (M + log2f(L)) * kLn2 : -INFINITY;
+                }
+                named_barrier_sync(1, C::NW * 32);
+                // a row's only segment is its result; otherwise a partial in the segment's slot
+                const bool direct = cur.ri.nseg == 1;
+                const int Hq = a.Hkv * a.G;
+                float *dst = direct ? a.out + ((int64_t)b * Hq + kvh * a.G) * C::D
+                                    : a.o_part + (int64_t)slot * a.G * C::D;
+                for (int e = tid; e < a.G * C::D; e += C::NW * 32) {
+                    const int g = e / C::D, d = e - g * C::D;
+                    float O = 0.f;
+#pragma unroll
+                    for (int w = 0; w < C::NW; ++w) O += ml[(w * C::NG + g) * 2] * eo[(w * C::NG + g) * C::D + d];
+                    dst[e] = O;
+                }
+                if (tid < a.G) {
+                    const float lv = ml[tid * 2 + 1];
+                    if (direct) a.lse[(int64_t)b * Hq + kvh * a.G + tid] = lv;
+                    else a.lse_part[(int64_t)slot * a.G + tid] = lv;
+                }
+                if (!direct) {
+                    // the CTA that finishes the row's last outstanding segment merges the row
+                    volatile int *merge_flag = reinterpret_cast<volatile int *>(kmxs);
+                    __threadfence();
+                    named_barrier_sync(1, C::NW * 32);
+                    if (tid == 0) *merge_flag = atomicAdd(a.plan.row_done + row, 1) == cur.ri.nseg - 1;
+                    named_barrier_sync(1, C::NW * 32);
+                    if (*merge_flag) {
+                        __threadfence();
+                        merge_row<C>(a, cur.ri.slot0, cur.ri.nseg, b, kvh, reinterpret_cast<float *>(sk));
+                    }
                 }
                 fence_proxy_async_shared();
                 named_barrier_sync(1, C::NW * 32);

@@ -30,6 +30,8 @@ struct DecodeArgs {
     PlanView plan;
     float *o_part;           // [slots, G, D]
     float *lse_part;         // [slots, G]
+    float *out;              // decode: [B, Hq, D] result (written by the kernel itself on the MMA path)
+    float *lse;              // decode: [B, Hq]
     int32_t *status;
 };
 
@@ -37,8 +39,10 @@ struct DecodeArgs {
 enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 
 // plan.cu
+// out/lse (decode only, else NULL): rows without tokens get out = 0 and lse = -inf here.
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
-                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule);
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
+                 float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 

@@ -17,7 +17,8 @@ constexpr size_t kPlanStageBytes = 48 * 1024;  // within the default dynamic sha
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu_len,
                                                     const int32_t *__restrict__ cu_seq, int B, int Hkv,
                                                     int n_req, int min_chunk, int mode, int granule,
-                                                    PlanView pv, WsHeader *hdr, int staged) {
+                                                    PlanView pv, WsHeader *hdr, int staged, float *out,
+                                                    float *lse, int G, int D) {
     __shared__ int32_t sm[33];
     extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
@@ -133,15 +134,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         if (r < R) {
             const int32_t p0 = row_pos[r];
             const int b = r % B;
-            const int32_t Lr = len_of(b), L = max(Lr, 0);
+            const int32_t L = max(len_of(b), 0);
             if (L > 0) v = (mode == 0) ? (int32_t)((p0 + L - 1) / S - p0 / S + 1) : 1;
-            int4 *ri = reinterpret_cast<int4 *>(pv.row_info + r);
-            ri[0] = make_int4(p0, Lr, seq_start_of(b), seq_len_of(b));
-            ri[1] = make_int4(len_start_of(b), part0[b], 0, 0);
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
-        if (r < R) pv.row_slot0[r] = carry + ex;
+        if (r < R) {
+            const int b = r % B;
+            pv.row_slot0[r] = carry + ex;
+            int4 *ri = reinterpret_cast<int4 *>(pv.row_info + r);
+            ri[0] = make_int4(row_pos[r], len_of(b), seq_start_of(b), seq_len_of(b));
+            ri[1] = make_int4(len_start_of(b), part0[b], carry + ex, v);
+            if (pv.row_done) pv.row_done[r] = 0;
+            if (out && v == 0) {  // a row with no tokens (reported above): zero output, lse -inf
+                const int64_t h0 = (int64_t)b * Hkv * G + (r / B) * G;
+                for (int e = 0; e < G * D; ++e) out[h0 * D + e] = 0.f;
+                for (int g = 0; g < G; ++g) lse[h0 + g] = -INFINITY;
+            }
+        }
         carry += total;
     }
     if (tid == 0) {
@@ -185,11 +195,12 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 }
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
-                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule) {
+                 int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
+                 int G, int D) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     launch_k(plan_kernel, dim3(1), dim3(1024), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
-               min_chunk, mode, granule, pv, hdr, staged);
+               min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

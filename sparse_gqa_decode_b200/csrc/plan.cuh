@@ -66,6 +66,8 @@ struct SegCursor {
             ri.seq_len = x.w;
             ri.len_start = y.x;
             ri.part0 = y.y;
+            ri.slot0 = y.z;
+            ri.nseg = y.w;
             const int32_t lo = max(pos, ri.pos), hi = min(end, ri.pos + max(ri.len, 0));
             ++r;
             if (hi > lo) {

@@ -92,6 +92,20 @@ def test_bf16_multi_tile_several_ctas(sgd):
     check_status(sgd, ws)
 
 
+@pytest.mark.parametrize("G", [16, 3])
+def test_row_merged_from_hundreds_of_segments(sgd, G):
+    # 800 requested CTAs: ranges of 16 tokens, so the 11500-token row has 719 segments and the
+    # CTA finishing its last one merges them, in more than one shared-memory round at G = 16
+    bt = make((11500, 40), G=G, D=128, Hkv=1, seed=91)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G)
+    out, lse, ws = sgd.decode_attn(q, G, k, v, cu, n_splits=800)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
+    segs, _ = sgd.plan_segments(cu, 2, 1, 800, 16, 0)
+    assert int((segs[:, 1] == 0).sum()) > 510
+
+
 def test_ragged_equal_work_equals_one_cta_per_row(sgd):
     wl = workloads.config(3, length_range=(17, 6000))
     bt = workloads.generate(wl, seed=3)
