@@ -198,9 +198,10 @@ class Pipeline:
         return o, lse
 
     def launches_per_step(self):
+        # decode: plan + the tensor-core decode, which merges each row itself (D = 128, bf16 q)
         if self.wl.scheme and self.wl.oam:
-            return 4 + 3  # plan, score+quantize, V codes, top-K; plan, decode, merge
-        return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 3
+            return 4 + 2  # plan, score+quantize, V codes, top-K; plan, decode
+        return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 2
 
 
 def source_hash(paths):
