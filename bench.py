@@ -313,11 +313,29 @@ def run_ours(args, rank, world, local_rank):
     if st:
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
+    # The step's C-ABI calls captured once in a CUDA graph (the library is stream-ordered, allocates
+    # nothing and never synchronises); the timed steps replay it.
+    graph, launch = None, "CUDA graph replay of the step's C-ABI calls"
+    try:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            pipe.run()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            pipe.run()
+        graph = g
+    except RuntimeError as exc:
+        launch = "eager C-ABI calls (graph capture failed: " + str(exc).splitlines()[0][:120] + ")"
+    torch.cuda.synchronize()
+
     names = [n for n in ("quantize_select", "quantize", "select", "decode") if n in stages]
     K = args.steps
     rec = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
            for _ in range(K)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    eager_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = ClockSampler(local_rank)
     if world > 1:
         torch.distributed.barrier()
@@ -327,17 +345,29 @@ def run_ours(args, rank, world, local_rank):
     for i in range(K):
         flush_l2(i)
         step_ev[i][0].record()
-        pipe.run(rec[i])
+        if graph is not None:
+            graph.replay()
+        else:
+            pipe.run()
         step_ev[i][1].record()
+    for i in range(K):  # the same steps as eager calls, timed per stage
+        flush_l2(i)
+        eager_ev[i][0].record()
+        pipe.run(rec[i])
+        eager_ev[i][1].record()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
+    st = sgd.workspace_status(pipe.ws_d)
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the timed steps")
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     stage_ms = {n: [r[n][0].elapsed_time(r[n][1]) for r in rec] for n in names}
     total_ms = reduce_max(sum(step_ms), dev, world)
     ms_per_step = total_ms / K
     value = job_gbs(step_bytes, K, total_ms, world)
+    eager_ms = reduce_max(sum(a.elapsed_time(b) for a, b in eager_ev), dev, world) / K
 
     # e2e: host buffers through the same calls, copies inside the timed region
     pin_q, pin_k, pin_v, pin_cu = (x.pin_memory() for x in (bt.q, bt.k, bt.v, bt.cu_seqlens))
@@ -406,7 +436,9 @@ def run_ours(args, rank, world, local_rank):
             "step": "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn",
             "l2": "flushed between steps (untimed 256 MiB write then 256 MiB read: L2 left clean); inputs > L2",
             "parallelism": f"dp{world} (independent copies, no collective)",
+            "launch": launch,
         },
+        "eager_ms_per_step": round(eager_ms, 4),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "seq_heads_per_s": round(world * wl.B * wl.Hq / (ms_per_step / 1e3), 1),
         "stages": stage_report,

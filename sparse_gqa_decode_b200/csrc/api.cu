@@ -127,6 +127,12 @@ int decode_n_req(const DevInfo &dev, const sgd_kv *kv, sgd_dtype q_dtype, int G,
     return SGD_OK;
 }
 
+// CTAs of the fused score + quantise pass of sgd_quantize_select: every SM's worth of them.
+int fused_n_req(const DevInfo &dev, const sgd_kv *kv, int G) {
+    const int per = score_quantize_ctas_per_sm(kv->D, G);
+    return per > 0 ? dev.sms * per : 0;
+}
+
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
@@ -161,7 +167,8 @@ size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_s
     DevInfo *dev;
     if (current_device(&dev) != SGD_OK) return 0;
     int n_req = 0;
-    if (op == SGD_OP_QUANTIZE_SELECT) op = SGD_OP_OAM_SELECT;  // the fused call needs the select layout
+    const bool fused = op == SGD_OP_QUANTIZE_SELECT;
+    if (fused) op = SGD_OP_OAM_SELECT;  // the fused call needs the select layout
     const bool score = op == SGD_OP_OAM_SELECT;
     if (op != SGD_OP_DECODE && !score) return 0;
     // indexed or not does not change the count
@@ -172,6 +179,7 @@ size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_s
     if (decode_n_req(*dev, kv, SGD_F32, G, false, score, score ? 0 : schedule, score ? 0 : n_splits, &n_req_f32) ==
         SGD_OK)
         n_req = std::max(n_req, n_req_f32);
+    if (fused) n_req = std::max(n_req, fused_n_req(*dev, kv, G));
     return layout(op, kv->B, kv->Hkv, G, kv->D, kv->T, n_req).total;
 }
 
@@ -286,8 +294,8 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     }
     DevInfo *dev;
     if ((rc = current_device(&dev)) != SGD_OK) return rc;
-    int n_req = 0;
-    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
+    const int n_req = fused_n_req(*dev, kv, G);
+    if (n_req < 1) return SGD_ERR_CUDA;
     const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
     if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);

@@ -64,6 +64,7 @@ struct MmaCfg {
     static constexpr int BOX_ELEMS = 128 / EB;
     static constexpr int TILE = ROWS * ROWB;  // bytes of one tensor per stage
     static constexpr int STAGES = 3;
+    static constexpr int MINB = 2;  // CTAs per SM the registers must allow
     static constexpr int KB = D / 16;
     static constexpr int NQ = (MODE == 2) ? 4 : 0;  // K-quantising warps (mode 2)
     static constexpr int THREADS = (NW + NQ + 1) * 32;
@@ -583,7 +584,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
 // the kernel
 // ------------------------------------------------------------------------------------------
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 2)
+__global__ void __launch_bounds__(C::THREADS, C::MINB)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const DecodeArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -1154,6 +1155,12 @@ int decode_ctas_per_sm(sgd_dtype kv, sgd_dtype q, int D, int G, bool indexed, bo
     if (D == 128) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, false, false, 0>>();
     (void)indexed;
     return g2 ? ctas_per_sm_mma<MmaCfg<64, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<64, 1, false, false, 0>>();
+}
+
+int score_quantize_ctas_per_sm(int D, int G) {
+    const bool g2 = G > 8;
+    if (D == 128) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, false, false, 2>>() : ctas_per_sm_mma<MmaCfg<128, 1, false, false, 2>>();
+    return g2 ? ctas_per_sm_mma<MmaCfg<64, 2, false, false, 2>>() : ctas_per_sm_mma<MmaCfg<64, 1, false, false, 2>>();
 }
 
 int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, bool score, int n_cta,

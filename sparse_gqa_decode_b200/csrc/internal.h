@@ -54,6 +54,8 @@ int decode_ctas_per_sm(sgd_dtype kv_dtype, sgd_dtype q_dtype, int D, int G, bool
 // Launches the split decode (or score) kernel over n_cta CTAs; returns a cudaError_t.
 int launch_decode(const DecodeArgs &a, sgd_dtype kv_dtype, sgd_dtype q_dtype, bool indexed, bool score,
                   int n_cta, cudaStream_t s);
+// CTAs resident per SM for the fused first pass of sgd_quantize_select (0 on error).
+int score_quantize_ctas_per_sm(int D, int G);
 // Fused first pass of sgd_quantize_select (bf16 cache, bf16 q): OAM scores, scheme-A K codes
 // and scales (or max|K| for scheme B) and max|V|.  Needs a plan built with granule kPart.
 int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s);

@@ -1,6 +1,8 @@
 // plan.cu -- the split-KV partition kernel (one CTA) and its inspection kernel.
 // The rule is stated in plan.cuh (granule 16 for decode; 64 for the fused score+quantize
 // pass, whose tiles must coincide with the 64-token scheme-A partitions).
+#include <algorithm>
+
 #include "internal.h"
 #include "plan.cuh"
 #include "scan.cuh"
@@ -199,8 +201,12 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
                  int G, int D) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
-    launch_k(plan_kernel, dim3(1), dim3(1024), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
-               min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D);
+    // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
+    // block barriers cheaper (the loops stride over anything larger)
+    const int want = std::max(std::max(B * Hkv, n_req), B) + 1;
+    const int nt = std::min(1024, std::max(64, (want + 31) / 32 * 32));
+    launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
+             min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
