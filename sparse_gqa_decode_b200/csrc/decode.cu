@@ -50,6 +50,8 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
+
 template <int D_, int GT_, bool I8_, bool IDX_, int MODE_>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
@@ -66,12 +68,13 @@ struct MmaCfg {
     static constexpr int STAGES = 3;
     static constexpr int MINB = 2;  // CTAs per SM the registers must allow
     static constexpr int KB = D / 16;
-    static constexpr int NQ = (MODE == 2) ? 4 : 0;  // K-quantising warps (mode 2)
+    static constexpr int NQ = (MODE == 2) ? kQuantWarps : 0;  // K-quantising warps (mode 2)
     static constexpr int THREADS = (NW + NQ + 1) * 32;
     static constexpr int SMEM_STAGES = STAGES * 2 * TILE;
     static constexpr bool ROW_SCALE = I8 && IDX;  // per-row K scales fetched by the producer
     static constexpr int SMEM_ROWSCALE = ROW_SCALE ? STAGES * ROWS * 4 : 0;
-    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + 2 * 4 * 4 + SMEM_ROWSCALE;
+    static constexpr int SMEM_KMX = 2 * (NQ > 4 ? NQ : 4) * 4;  // [2][NQ] per-warp max|K| (mode 2)
+    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + SMEM_KMX + SMEM_ROWSCALE;
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE >= 1), "scores read the unquantised cache");
@@ -424,12 +427,14 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
     int row, slot;
     int32_t t0, t1;
     float run_kmax = 0.f;
-    constexpr int CPR = C::ROWB / 16, NH = CPR / 2;
-    const int rho = lane & 15, half = lane >> 4;  // lanes rho, rho + 16: the two halves of one row
-    const int vr = 16 * qw + rho;
+    // each warp takes RW rows of the 64-row tile, LPR lanes per row, NH 16-byte chunks per lane
+    constexpr int RW = C::ROWS / C::NQ, LPR = 32 / RW, CPR = C::ROWB / 16, NH = CPR / LPR;
+    static_assert(NH % 2 == 0 && RW * LPR == 32, "quantising lane map");
+    const int rho = lane % RW, half = lane / RW;  // lane: row rho of the warp, part `half` of it
+    const int vr = RW * qw + rho;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + cur.ri.seq_start) * C::D + half * (C::D / 2);
+        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + cur.ri.seq_start) * C::D + half * (C::D / LPR);
         float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + cur.ri.part0;
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
@@ -510,6 +515,55 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
     const int chunk = (2 * C::TILE / 4 - 32) / G;
     const float *lp = a.lse_part + (int64_t)slot0 * G;
     const float *op = a.o_part + (int64_t)slot0 * G * C::D;
+    const int Hq = a.Hkv * G;
+    float *dst = a.out + ((int64_t)b * Hq + kvh * G) * C::D;
+    constexpr int kQ4 = 16 * C::D / 4 / NT;  // float4 columns per thread at G = 16
+    const int Q = G * C::D / 4;
+    float4 *dst4 = reinterpret_cast<float4 *>(dst);
+    if (n <= chunk) {
+        // one round: every lse loaded once, the weights computed in place, then thread t reads
+        // its float4 columns t, t + NT, ... of every slot, eight slots' loads in flight
+        for (int p = tid; p < n * G; p += NT) w[p] = __ldcg(lp + p);
+        named_barrier_sync(1, NT);
+        if (tid < G) {
+            float M = -INFINITY, S = 0.f;
+            for (int c = 0; c < n; ++c) M = fmaxf(M, w[c * G + tid]);
+            for (int c = 0; c < n; ++c) S += expf(w[c * G + tid] - M);
+            Ls[tid] = (n > 0) ? M + logf(S) : -INFINITY;
+        }
+        named_barrier_sync(1, NT);
+        for (int p = tid; p < n * G; p += NT) w[p] = expf(w[p] - Ls[p % G]);
+        named_barrier_sync(1, NT);
+        const float4 *oc = reinterpret_cast<const float4 *>(op);
+        float4 acc[kQ4];
+#pragma unroll
+        for (int j = 0; j < kQ4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int c = 0; c < n; ++c) {
+#pragma unroll
+            for (int j = 0; j < kQ4; ++j) {
+                const int q = tid + j * NT;
+                if (q < Q) {
+                    const float4 x = __ldcg(oc + (int64_t)c * Q + q);
+                    const float wc = w[c * G + (4 * q) / C::D];
+                    acc[j].x += wc * x.x;
+                    acc[j].y += wc * x.y;
+                    acc[j].z += wc * x.z;
+                    acc[j].w += wc * x.w;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kQ4; ++j) {
+            const int q = tid + j * NT;
+            if (q < Q) dst4[q] = acc[j];
+        }
+        if (tid < G) a.lse[(int64_t)b * Hq + kvh * G + tid] = Ls[tid];
+        named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
+        return;
+    }
+    // more slots than one round of shared memory holds: running max and sum per head, then the
+    // weighted sum round by round, adding to what this thread wrote
     if (tid < G) {
         Ls[tid] = -INFINITY;
         Ss[tid] = 0.f;
@@ -536,13 +590,8 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
     }
     named_barrier_sync(1, NT);
     if (tid < G) Ls[tid] = (n > 0) ? Ls[tid] + logf(Ss[tid]) : -INFINITY;
-    const int Hq = a.Hkv * G;
-    float *dst = a.out + ((int64_t)b * Hq + kvh * G) * C::D;
     // pass 2: thread t owns float4 columns t, t + NT, ... of the row's [G][D] block and reads
     // them from every slot of a chunk, kQ4 * 4 independent 16-byte loads in flight
-    constexpr int kQ4 = 16 * C::D / 4 / NT;  // float4 columns per thread at G = 16
-    const int Q = G * C::D / 4;
-    float4 *dst4 = reinterpret_cast<float4 *>(dst);
     for (int c0 = 0; c0 < n; c0 += chunk) {
         const int m = min(chunk, n - c0);
         named_barrier_sync(1, NT);
@@ -594,7 +643,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     float *ml = reinterpret_cast<float *>(empty + C::STAGES);  // [NW][NG][2]: m, l
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(ml + C::NW * C::NG * 2);
     float *kmxs = ml + C::NW * C::NG * 2 + 4;  // [2][NQ] per-warp max|K| of the current tile (mode 2)
-    float *row_scale = kmxs + 8;               // [STAGES][ROWS] K scale of each gathered row (INT8 gathers)
+    float *row_scale = kmxs + C::SMEM_KMX / 4;  // [STAGES][ROWS] K scale of each gathered row (INT8 gathers)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
