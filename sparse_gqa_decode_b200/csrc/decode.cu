@@ -375,45 +375,54 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
     mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
     mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-    // lanes rho and rho + 16 own the two halves of row rb + rho of the V tile (a quarter-warp
-    // then reads eight rows at one swizzled chunk: eight distinct bank groups)
-    const int rho = lane & 15, half = lane >> 4;
-    const int vr = rb + rho;
-    const int32_t j = j0 + rho;
-    const bool vrow = act && j < t1;
-    constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
-    constexpr int NH = CPR / 2;
-    uint64_t ss2 = 0;  // (even, odd) partial sums of squares
-    uint32_t vm2 = 0;  // running max |v| as bf16x2 (mode 2)
+    // ||v||^2 of the sub-tile's 16 rows on the tensor cores, as the diagonal of V.V^T: the rows
+    // take the MMA order of qk_subtile (row g4 at rb + pA, g4 + 8 at rb + pA + 8), and the B
+    // operand of rows 0-7 (8-15) is the (a0, a2) ((a1, a3)) half of the A fragment, so no further
+    // loads are needed; products are exact and sums f32.  The same registers give max|v| (mode 2).
+    const int rA = rb + pA, rB = rA + 8;
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t vmA = 0, vmB = 0;  // running max |v| of rows rA and rB as bf16x2 (mode 2)
 #pragma unroll
-    for (int i = 0; i < NH; ++i) {
-        const int c = half * NH + i, bx = c >> 3, cc = c & 7;
-        const uint4 w = lds128(vbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            ss2 = bf16x2_sumsq(ss2, ww[e]);
-            if constexpr (C::MODE == 2) vm2 = bf16x2_absmax(vm2, ww[e]);
+    for (int h = 0; h < C::KB / 2; ++h) {
+        const int c = t4 + 4 * h, bx = c >> 3, cc = c & 7;
+        const uint32_t base = vbase + bx * C::ROWS * 128 + ((cc ^ pA) << 4);
+        const uint4 va = lds128(base + rA * 128), vb = lds128(base + rB * 128);
+        mma_bf16(d0, va.x, vb.x, va.y, vb.y, va.x, va.y);
+        mma_bf16(d1, va.x, vb.x, va.y, vb.y, vb.x, vb.y);
+        mma_bf16(d0, va.z, vb.z, va.w, vb.w, va.z, va.w);
+        mma_bf16(d1, va.z, vb.z, va.w, vb.w, vb.z, vb.w);
+        if constexpr (C::MODE == 2) {
+            vmA = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(vmA, va.x), va.y), va.z), va.w);
+            vmB = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(vmB, vb.x), vb.y), vb.z), vb.w);
         }
     }
-    float ss = __uint_as_float((uint32_t)ss2) + __uint_as_float((uint32_t)(ss2 >> 32));
-    const float vmx = bf16x2_fold_max(vm2);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-    const int src = 4 * mma_row_perm(rho & 7);
-    const float rA = __shfl_sync(0xffffffffu, mA, src), rB = __shfl_sync(0xffffffffu, mB, src);
-    const float rmax = (rho < 8) ? rA : rB;
+    // lane 4g + g/2 holds the diagonal of MMA rows g and g + 8
+    const int g4 = lane >> 2;
+    const float dlo = (g4 & 1) ? d0[1] : d0[0], dhi = (g4 & 1) ? d1[3] : d1[2];
+    // row rb + rho of the tile is MMA row gm (rho < 8) or gm + 8, gm = perm(rho mod 8); lane rho
+    // writes its score
+    const int rho = lane & 15, half = lane >> 4;
+    const int32_t j = j0 + rho;
+    const bool vrow = act && j < t1;
+    const int gm = mma_row_perm(rho & 7);
+    const int src = 4 * gm, dsrc = 4 * gm + (gm >> 1);
+    const float rAm = __shfl_sync(0xffffffffu, mA, src), rBm = __shfl_sync(0xffffffffu, mB, src);
+    const float slo = __shfl_sync(0xffffffffu, dlo, dsrc), shi = __shfl_sync(0xffffffffu, dhi, dsrc);
+    const float rmax = (rho < 8) ? rAm : rBm;
+    const float ss = (rho < 8) ? slo : shi;
     if (half == 0 && vrow) {
         float sc = rmax * a.sm_scale + a.beta * logf(sqrtf(ss) + a.eps);
         if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
         a.scores[tok_base + j] = sc;
     }
     if constexpr (C::MODE == 2) {
-        if (vrow) run_vmax = fmaxf(run_vmax, vmx);
+        const bool okA = act && j0 + pA < t1, okB = act && j0 + pA + 8 < t1;
+        run_vmax = fmaxf(run_vmax, fmaxf(okA ? bf16x2_fold_max(vmA) : 0.f, okB ? bf16x2_fold_max(vmB) : 0.f));
     }
 }
 
-// Mode 2, K-quantising warp qw: rows 16*qw .. 16*qw+15 of every tile (a tile is one scheme-A
-// partition).  Scheme A: the tile's max|K| is met across the NQ warps through shared memory,
+// Mode 2, K-quantising warp qw: rows RW*qw .. RW*qw + RW-1 of every tile (a tile is one scheme-A
+// partition, RW = 64 / NQ).  Scheme A: the tile's max|K| is met across the NQ warps through shared memory,
 // then each warp writes the codes of its rows and warp 0 the partition scale.  Scheme B: only
 // the running max|K|.  Every quantising warp takes every tile.
 template <class C>
