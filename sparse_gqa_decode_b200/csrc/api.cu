@@ -171,14 +171,18 @@ size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_s
     if (fused) op = SGD_OP_OAM_SELECT;  // the fused call needs the select layout
     const bool score = op == SGD_OP_OAM_SELECT;
     if (op != SGD_OP_DECODE && !score) return 0;
-    // indexed or not does not change the count
+    // the largest count over the kernels the call may pick: indexed or not, bf16 or f32 query
     if (decode_n_req(*dev, kv, SGD_BF16, G, false, score, score ? 0 : schedule, score ? 0 : n_splits, &n_req) !=
         SGD_OK)
         return 0;
-    int n_req_f32 = 0;  // an F32 query may pick another kernel family
-    if (decode_n_req(*dev, kv, SGD_F32, G, false, score, score ? 0 : schedule, score ? 0 : n_splits, &n_req_f32) ==
-        SGD_OK)
-        n_req = std::max(n_req, n_req_f32);
+    for (int ix = 0; ix < 2; ++ix) {
+        for (sgd_dtype qd : {SGD_BF16, SGD_F32}) {
+            int other = 0;
+            if (decode_n_req(*dev, kv, qd, G, ix == 1, score, score ? 0 : schedule, score ? 0 : n_splits, &other) ==
+                SGD_OK)
+                n_req = std::max(n_req, other);
+        }
+    }
     if (fused) n_req = std::max(n_req, fused_n_req(*dev, kv, G));
     return layout(op, kv->B, kv->Hkv, G, kv->D, kv->T, n_req).total;
 }

@@ -1208,10 +1208,11 @@ int decode_ctas_per_sm(sgd_dtype kv, sgd_dtype q, int D, int G, bool indexed, bo
         return n;
     }
     const bool g2 = G > 8;
-    // the shared-memory footprint decides residency; all variants of one dtype/D share it
+    // the shared-memory and register footprint decide residency
+    if (kv == SGD_I8 && indexed)
+        return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, true, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, true, 0>>();
     if (kv == SGD_I8) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, false, 0>>();
     if (D == 128) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, false, false, 0>>();
-    (void)indexed;
     return g2 ? ctas_per_sm_mma<MmaCfg<64, 2, false, false, 0>>() : ctas_per_sm_mma<MmaCfg<64, 1, false, false, 0>>();
 }
 
