@@ -100,6 +100,9 @@ typedef struct {
                                    sum_{b'<b} ceil(L_b'/64); B: [1] */
     const float *v_scale;       /* [1] */
     int64_t n_parts;            /* A: sum_b ceil(L_b / 64) (host value); B: ignored */
+    const float *v_norm;        /* I8, for sgd_oam_select: [Hkv, T] ||v_t||_2 of the values
+                                   before quantisation (the v_norm output of sgd_quantize_kv or
+                                   sgd_quantize_select); NULL otherwise */
 } sgd_kv;
 
 /* operations, for sgd_workspace_size */
@@ -119,10 +122,12 @@ typedef struct {
  * k_codes, v_codes   [Hkv, T, D] int8 outputs
  * k_scale  A: [Hkv, n_parts] (n_parts = sum_b ceil(L_b/64), passed below), B: [1]
  * v_scale  [1]
+ * v_norm   optional [Hkv, T] float32 output (NULL: not written): ||v_t||_2 of every value row,
+ *          so that sgd_oam_select can later score the INT8 cache without the original values
  * Codes and scales are bit-exact functions of the input.
  */
 int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts,
-                    int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                    int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
@@ -133,7 +138,9 @@ int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts,
  *   K_b = clamp(ceil(L_b * keep_num / keep_den), 1, L_b) highest-scoring
  *   tokens, ties broken by the lower token index.
  * q        [B, Hq, D], BF16 or F32 (q_dtype)
- * kv       the cache as the caller holds it before quantisation: BF16 or F32
+ * kv       BF16 or F32: the cache as the caller holds it before quantisation; or
+ *          I8 (BF16 q, D = 128): the quantised cache, scored on khat = code * scale with
+ *          ||v_t|| taken from kv->v_norm (required), so that only the K codes are read
  * idx      [Hkv, kept_total] int32 output: row (b, kvh) is
  *          idx[kvh, cu_kept[b] .. cu_kept[b+1]-1], kept token positions local
  *          to sequence b, ascending
@@ -158,7 +165,7 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
 int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                         float beta, float eps, int keep_num, int keep_den,
                         sgd_scheme scheme, int64_t n_parts,
-                        int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                        int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm,
                         int32_t *idx, int32_t *cu_kept, int64_t kept_total,
                         void *workspace, size_t workspace_bytes, void *stream);
 

@@ -267,6 +267,40 @@ def oam_select(q, k, v, cu_seqlens, G: int, beta: float, eps: float, keep_num: i
     return idx, cu_kept, scores
 
 
+def value_norms(v) -> np.ndarray:
+    """||v_t||_2 of every row of v [..., T, D] in float64 (the norm the OAM score takes)."""
+    x = _f64(v)
+    return np.sqrt(np.sum(x * x, axis=-1))
+
+
+def oam_select_int8(q, k_codes, k_scale, v, cu_seqlens, scheme: str, G: int, beta: float, eps: float,
+                    keep_num: int, keep_den: int, rows: Optional[Sequence] = None, part: int = PART):
+    """oam_select over a quantised cache ([TD] section 3 score on the section 6 codes, the
+    section 7 pipeline with the selection moved after quantisation): k_t is replaced by its
+    dequantised value code * scale; ||v_t|| is that of the values before quantisation.
+    Same outputs as oam_select."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = cu.size - 1
+    Hkv = k_codes.shape[0]
+    lengths = np.diff(cu)
+    cu_parts = np.concatenate([[0], np.cumsum((lengths + part - 1) // part)])
+    kept = np.array([kept_count(int(cu[b + 1] - cu[b]), keep_num, keep_den) for b in range(B)], np.int64)
+    cu_kept = np.concatenate([[0], np.cumsum(kept)]).astype(np.int32)
+    idx = np.full((Hkv, int(cu_kept[-1])), -1, np.int32)
+    scores = {}
+    kc = np.asarray(k_codes)
+    ks = np.asarray(k_scale, np.float32)
+    todo = rows if rows is not None else [(b, h) for h in range(Hkv) for b in range(B)]
+    for b, h in todo:
+        s0, e0 = int(cu[b]), int(cu[b + 1])
+        L = e0 - s0
+        khat = dequant_rows(kc[h, s0:e0], k_scale_of_tokens(ks, scheme, h, b, L, cu_parts, part))
+        s = oam_scores(q[b, h * G:(h + 1) * G], khat, v[h, s0:e0], beta, eps)
+        scores[(b, h)] = s
+        idx[h, cu_kept[b]:cu_kept[b + 1]] = topk(s, int(kept[b]))
+    return idx, cu_kept, scores
+
+
 # ----------------------------------------------------------------------------------------------
 # decode over a packed cache
 # ----------------------------------------------------------------------------------------------

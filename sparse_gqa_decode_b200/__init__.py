@@ -49,6 +49,7 @@ class SgdKv(ctypes.Structure):
         ("k_scale", ctypes.c_void_p),
         ("v_scale", ctypes.c_void_p),
         ("n_parts", ctypes.c_int64),
+        ("v_norm", ctypes.c_void_p),
     ]
 
 
@@ -62,13 +63,13 @@ lib.sgd_error_string.restype = ctypes.c_char_p
 lib.sgd_workspace_size.argtypes = [_i32, _kvp, _i32, _i32, _i32]
 lib.sgd_workspace_size.restype = _sz
 lib.sgd_decode_num_ctas.argtypes = [_kvp, _i32, _vp, _i32, _i32]
-lib.sgd_quantize_kv.argtypes = [_kvp, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.sgd_quantize_kv.argtypes = [_kvp, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
-                                    _vp, _vp, _i64, _vp, _sz, _vp]
+                                    _vp, _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]
 
 _DT = {torch.float32: SGD_F32, torch.bfloat16: SGD_BF16, torch.int8: SGD_I8}
@@ -102,7 +103,7 @@ def kept_total(lengths: Sequence[int], keep_num: int, keep_den: int) -> int:
     return int(sum(max(1, min(int(L), -(-int(L) * keep_num // keep_den))) for L in lengths))
 
 
-def _kv(k, v, cu_seqlens, k_scale=None, v_scale=None, scheme=SCHEME_A, parts=0) -> SgdKv:
+def _kv(k, v, cu_seqlens, k_scale=None, v_scale=None, scheme=SCHEME_A, parts=0, v_norm=None) -> SgdKv:
     if k.dim() != 3 or k.shape != v.shape or k.dtype != v.dtype:
         raise ValueError("k and v must both be [Hkv, T, D] of one dtype")
     if k.dtype not in _DT:
@@ -114,7 +115,8 @@ def _kv(k, v, cu_seqlens, k_scale=None, v_scale=None, scheme=SCHEME_A, parts=0) 
     Hkv, T, D = k.shape
     return SgdKv(_DT[k.dtype], cu_seqlens.numel() - 1, Hkv, D, T, cu_seqlens.data_ptr(), k.data_ptr(),
                  v.data_ptr(), scheme, None if k_scale is None else k_scale.data_ptr(),
-                 None if v_scale is None else v_scale.data_ptr(), int(parts))
+                 None if v_scale is None else v_scale.data_ptr(), int(parts),
+                 None if v_norm is None else v_norm.data_ptr())
 
 
 def workspace_size(op: int, kv: SgdKv, G: int = 1, schedule: int = 0, n_splits: int = 0) -> int:
@@ -140,10 +142,11 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
 
 
 def quantize_kv(k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, scheme: str,
-                lengths: Sequence[int], out=None, workspace=None, stream=None):
+                lengths: Sequence[int], out=None, workspace=None, stream=None, v_norm=None):
     """INT8 codes and scales of a bf16/f32 cache.  Returns (k_codes, v_codes, k_scale, v_scale, ws).
 
-    ``lengths`` are the host copies of the sequence lengths (buffer sizes only).
+    ``lengths`` are the host copies of the sequence lengths (buffer sizes only).  ``v_norm``: an
+    optional float32 [Hkv, T] tensor that receives ||v_t|| (for oam_select over the INT8 cache).
     """
     sch = SCHEME_A if scheme == "A" else SCHEME_B
     Hkv, T, D = k.shape
@@ -157,18 +160,22 @@ def quantize_kv(k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, sche
     else:
         kc, vc, ks, vs = out
     ws = _workspace(workspace_size(OP_QUANTIZE, kv), k.device, workspace)
-    _check(lib.sgd_quantize_kv(ctypes.byref(kv), sch, parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(ws),
-                               ws.numel(), _stream(stream)), "sgd_quantize_kv")
+    _check(lib.sgd_quantize_kv(ctypes.byref(kv), sch, parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(v_norm),
+                               _ptr(ws), ws.numel(), _stream(stream)), "sgd_quantize_kv")
     return kc, vc, ks, vs, ws
 
 
 def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
                beta: float, eps: float, keep_num: int, keep_den: int, lengths: Sequence[int],
-               out=None, workspace=None, stream=None):
-    """Kept token positions per (sequence, KV head).  Returns (idx [Hkv, Kt], cu_kept [B+1], ws)."""
+               out=None, workspace=None, stream=None, k_scale=None, v_scale=None, scheme: str = "A",
+               n_parts_: int = 0, v_norm=None):
+    """Kept token positions per (sequence, KV head).  Returns (idx [Hkv, Kt], cu_kept [B+1], ws).
+
+    k, v bf16/f32: the cache before quantisation.  k, v int8: the quantised cache, scored on
+    k_code * k_scale with ||v|| from ``v_norm`` (as written by quantize_kv / quantize_select)."""
     Hkv = k.shape[0]
     Kt = kept_total(lengths, keep_num, keep_den)
-    kv = _kv(k, v, cu_seqlens)
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, SCHEME_A if scheme == "A" else SCHEME_B, n_parts_, v_norm)
     if out is None:
         idx = torch.empty((Hkv, Kt), dtype=torch.int32, device=k.device)
         cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
@@ -182,9 +189,9 @@ def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
 
 def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
                     beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
-                    out=None, workspace=None, stream=None):
+                    out=None, workspace=None, stream=None, v_norm=None):
     """quantize_kv and oam_select of one cache in one call (K and V read once for both).
-    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws)."""
+    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws); ``v_norm`` as in quantize_kv."""
     sch = SCHEME_A if scheme == "A" else SCHEME_B
     Hkv, T, D = k.shape
     parts = n_parts(lengths) if sch == SCHEME_A else 0
@@ -201,8 +208,8 @@ def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
         kc, vc, ks, vs, idx, cu_kept = out
     ws = _workspace(workspace_size(OP_QUANTIZE_SELECT, kv, G), k.device, workspace)
     _check(lib.sgd_quantize_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, sch,
-                                   parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(idx), _ptr(cu_kept), Kt,
-                                   _ptr(ws), ws.numel(), _stream(stream)), "sgd_quantize_select")
+                                   parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(v_norm), _ptr(idx),
+                                   _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)), "sgd_quantize_select")
     return kc, vc, ks, vs, idx, cu_kept, ws
 
 

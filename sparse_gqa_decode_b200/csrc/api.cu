@@ -198,7 +198,8 @@ int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedul
 }
 
 int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes, int8_t *v_codes,
-                    float *k_scale, float *v_scale, void *workspace, size_t workspace_bytes, void *stream) {
+                    float *k_scale, float *v_scale, float *v_norm, void *workspace, size_t workspace_bytes,
+                    void *stream) {
     int rc = check_kv(in);
     if (rc != SGD_OK) return rc;
     if (!k_codes || !v_codes || !k_scale || !v_scale || !workspace) return SGD_ERR_NULL;
@@ -206,14 +207,16 @@ int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts, int8_t
     if (scheme != SGD_SCHEME_A && scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
     if (scheme == SGD_SCHEME_A && (n_parts < in->B || n_parts > in->T / SGD_PARTITION + in->B)) return SGD_ERR_SHAPE;
     if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace)) return SGD_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_norm) & 3u))
+        return SGD_ERR_ALIGN;
     const Layout L = layout(SGD_OP_QUANTIZE, in->B, in->Hkv, 0, in->D, in->T, 0);
     if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
     DevInfo *dev;
     if ((rc = current_device(&dev)) != SGD_OK) return rc;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const int e = launch_quantize(in->k, in->v, in->dtype, in->cu_seqlens, in->B, in->Hkv, in->D, in->T, scheme,
-                                  n_parts, k_codes, v_codes, k_scale, v_scale, reinterpret_cast<WsHeader *>(ws),
+                                  n_parts, k_codes, v_codes, k_scale, v_scale, v_norm, reinterpret_cast<WsHeader *>(ws),
                                   reinterpret_cast<int32_t *>(ws + L.seq_part0), dev->sms, as_stream(stream));
     return e == 0 ? SGD_OK : SGD_ERR_CUDA;
 }
@@ -225,8 +228,18 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
     if (rc != SGD_OK) return rc;
     if (!q || !idx || !cu_kept || !workspace) return SGD_ERR_NULL;
     if (G < 1 || G > 16) return SGD_ERR_SHAPE;
-    if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (kv->dtype == SGD_I8) {
+        // scoring the INT8 cache: khat = code * scale, ||v|| from the norms stored at quantisation
+        if (q_dtype != SGD_BF16 || kv->D != 128) return SGD_ERR_DTYPE;
+        if (!kv->k_scale || !kv->v_norm) return SGD_ERR_NULL;
+        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
+            return SGD_ERR_SHAPE;
+        if (reinterpret_cast<uintptr_t>(kv->v_norm) & 3u) return SGD_ERR_ALIGN;
+    } else if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) {
+        return SGD_ERR_DTYPE;
+    }
     if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
     if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
     if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
@@ -259,6 +272,12 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
     a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
     a.beta = beta;
     a.eps = eps;
+    if (kv->dtype == SGD_I8) {
+        a.k_scale = kv->k_scale;
+        a.scheme = kv->scheme;
+        a.n_parts = kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
+        a.v_norm = kv->v_norm;
+    }
     a.scores = reinterpret_cast<float *>(ws + L.scores);
     a.plan = pv;
     a.status = &hdr->status;
@@ -271,8 +290,9 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
 
 int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
                         int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
-                        int8_t *v_codes, float *k_scale, float *v_scale, int32_t *idx, int32_t *cu_kept,
-                        int64_t kept_total, void *workspace, size_t workspace_bytes, void *stream) {
+                        int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm, int32_t *idx,
+                        int32_t *cu_kept, int64_t kept_total, void *workspace, size_t workspace_bytes,
+                        void *stream) {
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !idx || !cu_kept || !workspace || !k_codes || !v_codes || !k_scale || !v_scale) return SGD_ERR_NULL;
@@ -286,12 +306,13 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
     if (!aligned16(q) || !aligned16(workspace) || !aligned16(k_codes) || !aligned16(v_codes)) return SGD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u) ||
-        (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_norm) & 3u))
         return SGD_ERR_ALIGN;
     if (decode_family(kv->dtype, q_dtype, kv->D, true) != kFamilyMma) {
         // no fused kernel for this dtype: the two passes one after the other
-        rc = sgd_quantize_kv(kv, scheme, n_parts, k_codes, v_codes, k_scale, v_scale, workspace, workspace_bytes,
-                             stream);
+        rc = sgd_quantize_kv(kv, scheme, n_parts, k_codes, v_codes, k_scale, v_scale, v_norm, workspace,
+                             workspace_bytes, stream);
         if (rc != SGD_OK) return rc;
         return sgd_oam_select(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, idx, cu_kept, kept_total, workspace,
                               workspace_bytes, stream);
@@ -334,7 +355,7 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     int e = launch_score_quantize(a, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
     e = launch_quantize_global(kv->k, kv->v, kv->dtype, kv->Hkv, kv->D, kv->T, scheme, k_codes, v_codes, k_scale,
-                               v_scale, hdr, dev->sms, s);
+                               v_scale, v_norm, hdr, dev->sms, s);
     if (e != 0) return SGD_ERR_CUDA;
     e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
                     &hdr->status, s);

@@ -77,7 +77,8 @@ struct MmaCfg {
     static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + SMEM_KMX + SMEM_ROWSCALE;
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
-    static_assert(!(I8 && MODE >= 1), "scores read the unquantised cache");
+    static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
+    static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
@@ -130,12 +131,13 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
             uint8_t *sk = smem + stage * 2 * C::TILE;
             uint8_t *sv = sk + C::TILE;
             if constexpr (!C::IDX) {
-                mbar_arrive_expect_tx(&full[stage], 2 * C::TILE);
+                mbar_arrive_expect_tx(&full[stage], (C::KONLY ? 1 : 2) * C::TILE);
                 const int y = (int)(seq0 + t);
 #pragma unroll
                 for (int bx = 0; bx < C::BOXES; ++bx) {
                     tma_load_2d(sk + bx * C::ROWS * 128, tmK, &full[stage], bx * C::BOX_ELEMS, y, pol);
-                    tma_load_2d(sv + bx * C::ROWS * 128, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
+                    if constexpr (!C::KONLY)
+                        tma_load_2d(sv + bx * C::ROWS * 128, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
                 }
             } else if (Lb >= 1) {
                 // Row indices: lane l loads those of rows l, l+32, ...  Copies: one warp
@@ -418,6 +420,55 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
     if constexpr (C::MODE == 2) {
         const bool okA = act && j0 + pA < t1, okB = act && j0 + pA + 8 < t1;
         run_vmax = fmaxf(run_vmax, fmaxf(okA ? bf16x2_fold_max(vmA) : 0.f, okB ? bf16x2_fold_max(vmB) : 0.f));
+    }
+}
+
+// OAM scores of a sub-tile of an INT8 cache (mode 1): khat = code * scale, so the logit of head g
+// is sacc * colf_g (log2 units, with the head's Q pre-scale) times the sub-tile's partition scale
+// rf >= 0 (scheme A; scheme B's scale is inside colf); ||v_t|| comes from the norms stored when
+// the cache was quantised, so the V codes are never read.
+template <class C>
+__device__ __forceinline__ void score_subtile_i8(const DecodeArgs &a, uint32_t kbase, int rb, int32_t j0, int32_t t1,
+                                                 bool ready, int64_t tok_base, int pA, int t4, int lane,
+                                                 const uint32_t (&qf)[C::GT][C::KB][2], const float (&colf)[C::GT][2],
+                                                 float rf) {
+    const bool act = ready && j0 < t1;
+    const int rho = lane & 15, half = lane >> 4;
+    const int32_t j = j0 + rho;
+    const bool vrow = act && j < t1;
+    float vn = 0.f;
+    if (half == 0 && vrow) vn = __ldg(a.v_norm + tok_base + j);  // in flight during the MMAs
+    float sacc[C::GT][4];
+    if (act) {
+        qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
+    } else {
+#pragma unroll
+        for (int gt = 0; gt < C::GT; ++gt) sacc[gt][0] = sacc[gt][1] = sacc[gt][2] = sacc[gt][3] = 0.f;
+    }
+    float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+    for (int gt = 0; gt < C::GT; ++gt) {
+        const int g0 = 8 * gt + 2 * t4;
+        if (g0 < a.G) {
+            mA = fmaxf(mA, sacc[gt][0] * colf[gt][0]);
+            mB = fmaxf(mB, sacc[gt][2] * colf[gt][0]);
+        }
+        if (g0 + 1 < a.G) {
+            mA = fmaxf(mA, sacc[gt][1] * colf[gt][1]);
+            mB = fmaxf(mB, sacc[gt][3] * colf[gt][1]);
+        }
+    }
+    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+    mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+    mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+    const int src = 4 * mma_row_perm(rho & 7);  // row rb + rho is MMA row perm(rho mod 8) (+ 8)
+    const float rAm = __shfl_sync(0xffffffffu, mA, src), rBm = __shfl_sync(0xffffffffu, mB, src);
+    const float rmax = (rho < 8) ? rAm : rBm;
+    if (half == 0 && vrow) {
+        float sc = rmax * rf * kLn2 + a.beta * logf(vn + a.eps);
+        if (sc == 0.f) sc = 0.f;  // one key for +0 and -0
+        a.scores[tok_base + j] = sc;
     }
 }
 
@@ -738,7 +789,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 const int rb = 16 * (s * C::NW + warp);
                 const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
                 if constexpr (C::MODE >= 1) {
-                    score_subtile<C>(a, kbase, vbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, run_vmax);
+                    if constexpr (C::I8)
+                        score_subtile_i8<C>(a, kbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, colf, rf_pre[s]);
+                    else
+                        score_subtile<C>(a, kbase, vbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, run_vmax);
                     continue;
                 }
                 if (j0 >= t1 || !ready) continue;
@@ -1195,7 +1249,7 @@ static int launch_generic(const DecodeArgs &a, bool indexed, int n_cta, cudaStre
 Family decode_family(sgd_dtype kv, sgd_dtype q, int D, bool score) {
     if (q != SGD_BF16) return kFamilyGeneric;
     if (kv == SGD_BF16 && (D == 64 || D == 128)) return kFamilyMma;
-    if (kv == SGD_I8 && D == 128 && !score) return kFamilyMma;
+    if (kv == SGD_I8 && D == 128) return kFamilyMma;
     return kFamilyGeneric;
 }
 
@@ -1228,6 +1282,7 @@ int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, 
     const bool g2 = a.G > 8;
     if (decode_family(kv, q, a.D, score) == kFamilyMma) {
         if (score) {
+            if (kv == SGD_I8) return g2 ? launch_mma_idx<128, 2, true, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, true, 1>(a, false, n_cta, s);
             if (a.D == 128) return g2 ? launch_mma_idx<128, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, false, 1>(a, false, n_cta, s);
             return g2 ? launch_mma_idx<64, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<64, 1, false, 1>(a, false, n_cta, s);
         }

@@ -22,6 +22,7 @@ struct DecodeArgs {
     float sm_scale;          // 1 / sqrt(D)
     float beta, eps;         // score mode
     float *scores;           // score mode output [Hkv, T]
+    const float *v_norm;     // score mode over an I8 cache: [Hkv, T] ||v_t||
     // score + quantize mode (fused first pass of sgd_quantize_select)
     int qscheme;             // SGD_SCHEME_A: K codes and partition scales here; B: max|K| only
     int8_t *k_codes;         // [Hkv, T, D]
@@ -63,12 +64,13 @@ int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s);
 
 // quantize.cu
 // Second pass: codes of V (and of K for scheme B) with the global scales in hdr->amax_bits.
+// vnorm (NULL: not wanted): [Hkv, T] L2 norm of every V row, written by the V-codes pass.
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
                            sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
-                           const WsHeader *hdr, int sm_count, cudaStream_t s);
+                           float *vnorm, const WsHeader *hdr, int sm_count, cudaStream_t s);
 int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
                     int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
-                    float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s);
+                    float *v_scale, float *vnorm, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s);
 
 // oam.cu
 int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t T, int keep_num, int keep_den,

@@ -160,12 +160,17 @@ __global__ void __launch_bounds__(256) quant_amax_kernel(const T *__restrict__ k
 
 constexpr int kGlobalUnroll = 4;  // independent 16-byte loads per thread and tensor
 
-// Pass 2: codes of one or two whole tensors with their global scales.
+// Pass 2: codes of one or two whole tensors with their global scales.  Optionally also the L2
+// norm of every row (token) of one of them (vnorm_of = 0 or 1: x0 or x1; -1: none) into vnorm:
+// a row's vpr 16-byte vectors sit on vpr consecutive lanes of one warp (vpr divides 32; the
+// grid-stride index keeps warps aligned), so the row's sum of squares is a shuffle tree over
+// them.  Loop bounds are taken per warp so that every lane reaches every shuffle.
 template <typename T>
 __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__ x0, int8_t *__restrict__ c0,
                                                            float *scale0, int which0, const T *__restrict__ x1,
                                                            int8_t *__restrict__ c1, float *scale1, int which1,
-                                                           int64_t nvec, const WsHeader *hdr) {
+                                                           int64_t nvec, const WsHeader *hdr,
+                                                           float *__restrict__ vnorm, int vnorm_of, int vpr) {
     constexpr int VE = Vec<T>::VE;
     const float s0 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which0]), 127.f);
     const float r0 = (s0 != 0.f) ? __frcp_rn(s0) : 0.f;
@@ -178,12 +183,21 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
         *scale0 = s0;
         if (x1) *scale1 = s1;
     }
+    const int lane = threadIdx.x & 31;
+    const bool norms = vnorm != nullptr;
+    auto row_norm = [&](const float (&x)[VE], int64_t iv, bool in) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) ss = fmaf(x[e], x[e], ss);
+        for (int o = vpr >> 1; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (in && lane % vpr == 0) vnorm[iv / vpr] = sqrtf(ss);
+    };
     const uint4 *p0 = reinterpret_cast<const uint4 *>(x0);
     const uint4 *p1 = reinterpret_cast<const uint4 *>(x1);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     // kGlobalUnroll vectors per thread in flight per tensor, then their codes
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    for (; i + (kGlobalUnroll - 1) * stride < nvec; i += kGlobalUnroll * stride) {
+    for (; (i - lane) + 31 + (kGlobalUnroll - 1) * stride < nvec; i += kGlobalUnroll * stride) {
         uint4 w0[kGlobalUnroll], w1[kGlobalUnroll];
 #pragma unroll
         for (int u = 0; u < kGlobalUnroll; ++u) w0[u] = __ldcs(p0 + i + u * stride);
@@ -196,19 +210,24 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
             float x[VE];
             Vec<T>::unpack(w0[u], x);
             store_codes<VE>(c0 + (i + u * stride) * VE, x, s0, r0);
+            if (norms && vnorm_of == 0) row_norm(x, i + u * stride, true);
             if (x1) {
                 Vec<T>::unpack(w1[u], x);
                 store_codes<VE>(c1 + (i + u * stride) * VE, x, s1, r1);
+                if (norms && vnorm_of == 1) row_norm(x, i + u * stride, true);
             }
         }
     }
-    for (; i < nvec; i += stride) {
+    for (; i - lane < nvec; i += stride) {  // the rest, every lane of the warp together
+        const bool in = i < nvec;
         float x[VE];
-        Vec<T>::unpack(__ldcs(p0 + i), x);
-        store_codes<VE>(c0 + i * VE, x, s0, r0);
+        Vec<T>::unpack(in ? __ldcs(p0 + i) : make_uint4(0, 0, 0, 0), x);
+        if (in) store_codes<VE>(c0 + i * VE, x, s0, r0);
+        if (norms && vnorm_of == 0) row_norm(x, i, in);
         if (x1) {
-            Vec<T>::unpack(__ldcs(p1 + i), x);
-            store_codes<VE>(c1 + i * VE, x, s1, r1);
+            Vec<T>::unpack(in ? __ldcs(p1 + i) : make_uint4(0, 0, 0, 0), x);
+            if (in) store_codes<VE>(c1 + i * VE, x, s1, r1);
+            if (norms && vnorm_of == 1) row_norm(x, i, in);
         }
     }
 }
@@ -231,7 +250,8 @@ static int global_ctas_per_sm() {
 template <typename T, int D>
 static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int Hkv, int64_t Ttot,
                          sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
-                         float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
+                         float *v_scale, float *vnorm, WsHeader *hdr, int32_t *seq_part0, int sm_count,
+                         cudaStream_t s) {
     constexpr int VE = Vec<T>::VE;
     const int64_t nvec = (int64_t)Hkv * Ttot * D / VE;
     cudaError_t e = launch_k(quant_prep_kernel, dim3(1), dim3(1024), 0, s, 1, cu, B, n_parts,
@@ -250,56 +270,56 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
             if (e != cudaSuccess) return (int)e;
         }
         e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v, vc,
-                     v_scale, 1, none, no_codes, no_scale, 0, nvec, (const WsHeader *)hdr);
+                     v_scale, 1, none, no_codes, no_scale, 0, nvec, (const WsHeader *)hdr, vnorm, 0, D / VE);
     } else {
         e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
         if (e != cudaSuccess) return (int)e;
         e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k, kc,
-                     k_scale, 0, v, vc, v_scale, 1, nvec, (const WsHeader *)hdr);
+                     k_scale, 0, v, vc, v_scale, 1, nvec, (const WsHeader *)hdr, vnorm, 1, D / VE);
     }
     return (int)e;
 }
 
 template <typename T>
 static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t Ttot, sgd_scheme scheme, int8_t *kc,
-                                int8_t *vc, float *k_scale, float *v_scale, const WsHeader *hdr, int sm_count,
-                                cudaStream_t s) {
+                                int8_t *vc, float *k_scale, float *v_scale, float *vnorm, const WsHeader *hdr,
+                                int sm_count, cudaStream_t s) {
     const int64_t nvec = (int64_t)Hkv * Ttot * D / Vec<T>::VE;
     const T *none = nullptr;
     int8_t *no_codes = nullptr;
     float *no_scale = nullptr;
     if (scheme == SGD_SCHEME_A)
         return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v,
-                             vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr);
+                             vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr, vnorm, 0, D / Vec<T>::VE);
     return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k,
-                         kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr);
+                         kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr, vnorm, 1, D / Vec<T>::VE);
 }
 
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
                            sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
-                           const WsHeader *hdr, int sm_count, cudaStream_t s) {
+                           float *vnorm, const WsHeader *hdr, int sm_count, cudaStream_t s) {
     if (dt == SGD_BF16)
         return quantize_global_impl(static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
-                                    Hkv, D, T, scheme, kc, vc, k_scale, v_scale, hdr, sm_count, s);
+                                    Hkv, D, T, scheme, kc, vc, k_scale, v_scale, vnorm, hdr, sm_count, s);
     return quantize_global_impl(static_cast<const float *>(k), static_cast<const float *>(v), Hkv, D, T, scheme, kc,
-                                vc, k_scale, v_scale, hdr, sm_count, s);
+                                vc, k_scale, v_scale, vnorm, hdr, sm_count, s);
 }
 
 int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
                     int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
-                    float *v_scale, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
+                    float *v_scale, float *vnorm, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s) {
     if (dt == SGD_BF16) {
         auto kk = static_cast<const __nv_bfloat16 *>(k), vv = static_cast<const __nv_bfloat16 *>(v);
         return D == 128 ? quantize_impl<__nv_bfloat16, 128>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale,
-                                                            v_scale, hdr, seq_part0, sm_count, s)
+                                                            v_scale, vnorm, hdr, seq_part0, sm_count, s)
                         : quantize_impl<__nv_bfloat16, 64>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale,
-                                                           v_scale, hdr, seq_part0, sm_count, s);
+                                                           v_scale, vnorm, hdr, seq_part0, sm_count, s);
     }
     auto kk = static_cast<const float *>(k), vv = static_cast<const float *>(v);
     return D == 128 ? quantize_impl<float, 128>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale, v_scale,
-                                                hdr, seq_part0, sm_count, s)
-                    : quantize_impl<float, 64>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale, v_scale, hdr,
-                                               seq_part0, sm_count, s);
+                                                vnorm, hdr, seq_part0, sm_count, s)
+                    : quantize_impl<float, 64>(kk, vv, cu, B, Hkv, T, scheme, n_parts, kc, vc, k_scale, v_scale,
+                                               vnorm, hdr, seq_part0, sm_count, s);
 }
 
 }  // namespace sgd

@@ -43,14 +43,15 @@ def test_error_strings_and_version(sgd):
 
 
 def test_struct_layout_matches_header(sgd):
-    # dtype, B, Hkv, D (4 x 4 bytes), T (8), 3 pointers, scheme (+pad), 2 pointers, n_parts
-    assert ctypes.sizeof(sgd.SgdKv) == 4 * 4 + 8 + 3 * 8 + 8 + 2 * 8 + 8
+    # dtype, B, Hkv, D (4 x 4 bytes), T (8), 3 pointers, scheme (+pad), 2 pointers, n_parts, v_norm
+    assert ctypes.sizeof(sgd.SgdKv) == 4 * 4 + 8 + 3 * 8 + 8 + 2 * 8 + 8 + 8
     assert sgd.SgdKv.T.offset == 16 and sgd.SgdKv.k_scale.offset == 56 and sgd.SgdKv.n_parts.offset == 72
+    assert sgd.SgdKv.v_norm.offset == 80
 
 
 def _kv(sgd, **kw):
     base = dict(dtype=sgd.SGD_BF16, B=2, Hkv=2, D=128, T=100, cu_seqlens=0x1000, k=0x10000, v=0x20000,
-                scheme=0, k_scale=None, v_scale=None, n_parts=0)
+                scheme=0, k_scale=None, v_scale=None, n_parts=0, v_norm=None)
     base.update(kw)
     return sgd.SgdKv(**base)
 
@@ -95,15 +96,15 @@ def test_quantize_and_select_reject_bad_args_on_host(sgd):
     L = sgd.lib
     kv = _kv(sgd)
     p = ctypes.c_void_p
-    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, None, p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, None, p(0x1000), p(0x2000), p(0x3000), None, p(0x4000), 4096,
                              None) == -1
     assert L.sgd_quantize_kv(ctypes.byref(_kv(sgd, dtype=sgd.SGD_I8)), 0, 3, p(0x1000), p(0x1000), p(0x2000),
-                             p(0x3000), p(0x4000), 4096, None) == -3
-    assert L.sgd_quantize_kv(ctypes.byref(kv), 5, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+                             p(0x3000), None, p(0x4000), 4096, None) == -3
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 5, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), None, p(0x4000), 4096,
                              None) == -3
-    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 1, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 4096,
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 1, p(0x1000), p(0x1000), p(0x2000), p(0x3000), None, p(0x4000), 4096,
                              None) == -2  # fewer partitions than sequences
-    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), p(0x4000), 16,
+    assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), None, p(0x4000), 16,
                              None) == -5  # workspace too small
     sel = lambda **kw: L.sgd_oam_select(p(0x3000), kw.get("qdt", sgd.SGD_BF16), kw.get("G", 8), ctypes.byref(kv),
                                         kw.get("beta", 1.0), 1e-6, kw.get("num", 1), kw.get("den", 8), p(0x1000),
@@ -113,3 +114,12 @@ def test_quantize_and_select_reject_bad_args_on_host(sgd):
     assert sel(kt=1) == -2
     assert sel(beta=float("nan")) == -8
     assert sel(G=20) == -2
+    # scoring an INT8 cache needs its K scales and the value norms, a bf16 query and D = 128
+    kv8 = _kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_scale=0x7100, n_parts=3)
+    sel8 = lambda k8, qdt=sgd.SGD_BF16: L.sgd_oam_select(p(0x3000), qdt, 8, ctypes.byref(k8), 1.0, 1e-6, 1, 8,
+                                                         p(0x1000), p(0x2000), 20, p(0x4000), 1 << 20, None)
+    assert sel8(kv8) == -1  # no v_norm
+    assert sel8(_kv(sgd, dtype=sgd.SGD_I8, v_norm=0x7200, n_parts=3)) == -1  # no k_scale
+    assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7200, n_parts=3, D=64)) == -3
+    assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7200, n_parts=3), sgd.SGD_F32) == -3
+    assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7202, n_parts=3)) == -4

@@ -325,6 +325,71 @@ def test_oam_then_decode_over_kept(sgd, kvdt):
 
 
 # ---------------------------------------------------------------------------------------------
+# OAM over the INT8 cache: value norms stored at quantisation, scores on code * scale
+# ---------------------------------------------------------------------------------------------
+# fp32 sum of D exact squares: relative error below D * 2^-24; the square root halves it
+VNORM_RTOL = 1e-5
+
+
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("bf16", 64), ("f32", 128), ("f32", 64)])
+def test_quantize_writes_value_norms(sgd, scheme, dtype, D):
+    bt = make((1, 63, 64, 65, 700, 2053), G=8, D=D, Hkv=2, dtype=dtype, dist="outlier", seed=21 + D)
+    q, k, v, cu = dev(bt)
+    vn = torch.full((2, int(bt.cu_seqlens[-1])), -1.0, dtype=torch.float32, device="cuda")
+    _, _, _, _, ws = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn)
+    check_status(sgd, ws)
+    ref = oracle.value_norms(bt.v)
+    rel = np.abs(vn.cpu().numpy() - ref) / np.maximum(ref, 1e-30)
+    assert rel.max() <= VNORM_RTOL, rel.max()
+
+
+def test_quantize_select_writes_the_same_value_norms(sgd):
+    bt = make((7, 64, 500, 3000), G=8, D=128, Hkv=2, dist="outlier", seed=23)
+    q, k, v, cu = dev(bt)
+    T = int(bt.cu_seqlens[-1])
+    vn1 = torch.empty((2, T), dtype=torch.float32, device="cuda")
+    vn2 = torch.empty((2, T), dtype=torch.float32, device="cuda")
+    sgd.quantize_kv(k, v, cu, "A", bt.lengths, v_norm=vn1)
+    sgd.quantize_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, "A", bt.lengths, v_norm=vn2)
+    assert torch.equal(vn1, vn2)
+
+
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("G", [8, 16, 1])
+def test_oam_select_over_the_int8_cache(sgd, scheme, G):
+    bt = make((1, 7, 64, 500, 5000), G=G, D=128, Hkv=2, dist="outlier", seed=33 + G)
+    q, k, v, cu = dev(bt)
+    vn = torch.empty((2, int(bt.cu_seqlens[-1])), dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn)
+    parts = sgd.n_parts(bt.lengths) if scheme == "A" else 0
+    idx, cu_kept, ws = sgd.oam_select(q, kc, vc, cu, G, 1.0, 1e-6, 1, 8, bt.lengths, k_scale=ks, v_scale=vs,
+                                      scheme=scheme, n_parts_=parts, v_norm=vn)
+    check_status(sgd, ws)
+    rkc, _, rks, _ = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    ref_idx, ref_cu, scores = oracle.oam_select_int8(bt.q, rkc, rks, bt.v, bt.cu_seqlens, scheme, G, 1.0, 1e-6,
+                                                     1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, bt.wl.B, 2)
+
+
+def test_int8_cache_selection_then_decode(sgd):
+    bt = make((90, 2000, 4500), G=8, D=128, Hkv=2, dist="outlier", seed=73)
+    q, k, v, cu = dev(bt)
+    vn = torch.empty((2, int(bt.cu_seqlens[-1])), dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths, v_norm=vn)
+    parts = sgd.n_parts(bt.lengths)
+    idx, cu_kept, _ = sgd.oam_select(q, kc, vc, cu, 8, 1.0, 1e-6, 1, 8, bt.lengths, k_scale=ks, v_scale=vs,
+                                     scheme="A", n_parts_=parts, v_norm=vn)
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A", n_parts_=parts, idx=idx,
+                                   cu_kept=cu_kept, kept_total_=idx.shape[1])
+    check_status(sgd, ws)
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=idx.cpu().numpy(), cu_kept=cu_kept.cpu().numpy(),
+                        quant=(*quant, "A"))
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------------------------
 # fused quantise + select
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("scheme", ["A", "B"])

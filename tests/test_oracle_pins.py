@@ -324,6 +324,49 @@ def test_beta_zero_is_classic_qk_ranking_and_q_zero_is_norm_ranking():
     assert np.array_equal(oracle.topk(su, 15), np.sort(np.argsort(-qk, kind="stable")[:15]))
 
 
+def test_value_norms_closed_form_and_library():
+    v = np.zeros((2, 3, 8))
+    v[0, 0, :2] = (3.0, 4.0)  # 5
+    v[1, 2, :] = 1.0  # sqrt(8)
+    n = oracle.value_norms(v)
+    assert n[0, 0] == 5.0 and n[1, 2] == math.sqrt(8.0) and n[0, 1] == 0.0
+    w = np.random.default_rng(3).standard_normal((4, 50, 64))
+    assert np.allclose(oracle.value_norms(w), np.linalg.norm(w, axis=-1), rtol=1e-14, atol=0)
+
+
+def test_int8_selection_with_exact_codes_is_the_plain_selection():
+    # keys = integer codes * 2^e with every 64-token partition reaching |127| * 2^e: the partition
+    # scale is exactly 2^e (a different e per partition and head) and the codes are the integers,
+    # so the dequantised keys equal the keys and the INT8-cache selection must equal the plain one
+    rng = np.random.default_rng(11)
+    lengths = [70, 200, 5]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    Hkv, G, D = 2, 4, 64
+    T = int(cu[-1])
+    codes = rng.integers(-127, 128, size=(Hkv, T, D)).astype(np.float32)
+    k = np.empty_like(codes)
+    want_scales = []
+    for h in range(Hkv):
+        row = []
+        for b in range(3):
+            for p0 in range(0, lengths[b], 64):
+                e = int(rng.integers(-3, 4))
+                sl = slice(cu[b] + p0, cu[b] + min(p0 + 64, lengths[b]))
+                codes[h, sl.start, 0] = 127.0
+                k[h, sl] = codes[h, sl] * 2.0 ** e
+                row.append(2.0 ** e)
+        want_scales.append(row)
+    v = rng.standard_normal((Hkv, T, D)).astype(np.float32)
+    q = rng.standard_normal((3, Hkv * G, D)).astype(np.float32)
+    kc, _, ks, _ = oracle.quantize_kv(k, v, cu, "A")
+    assert np.array_equal(ks, np.array(want_scales, np.float32)) and np.array_equal(kc.astype(np.float32), codes)
+    got = oracle.oam_select_int8(q, kc, ks, v, cu, "A", G, 1.0, 1e-6, 1, 4)
+    want = oracle.oam_select(q, k, v, cu, G, 1.0, 1e-6, 1, 4)
+    assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+    for key in want[2]:
+        assert np.array_equal(got[2][key], want[2][key])
+
+
 def test_keep_all_selection_equals_dense_decode():
     bt = _tiny_batch(G=4, D=16, lengths=(9, 40), Hkv=2, dtype="bf16")
     idx, cu_kept, _ = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 4, 1.0, 1e-6, 1, 1)
