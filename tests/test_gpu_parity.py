@@ -384,8 +384,10 @@ def test_int8_cache_selection_then_decode(sgd):
                                    cu_kept=cu_kept, kept_total_=idx.shape[1])
     check_status(sgd, ws)
     quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
-    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=idx.cpu().numpy(), cu_kept=cu_kept.cpu().numpy(),
-                        quant=(*quant, "A"))
+    ref_idx, ref_cu, scores = oracle.oam_select_int8(bt.q, quant[0], quant[2], bt.v, bt.cu_seqlens, "A", 8, 1.0,
+                                                     1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, 3, 2)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=ref_idx, cu_kept=ref_cu, quant=(*quant, "A"))
     assert_close(out, lse, *ref, OUT_TOL["bf16"])
 
 
