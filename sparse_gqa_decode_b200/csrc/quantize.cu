@@ -165,7 +165,7 @@ constexpr int kGlobalUnroll = 4;  // independent 16-byte loads per thread and te
 // a row's vpr 16-byte vectors sit on vpr consecutive lanes of one warp (vpr divides 32; the
 // grid-stride index keeps warps aligned), so the row's sum of squares is a shuffle tree over
 // them.  Loop bounds are taken per warp so that every lane reaches every shuffle.
-template <typename T>
+template <typename T, bool NORMS>
 __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__ x0, int8_t *__restrict__ c0,
                                                            float *scale0, int which0, const T *__restrict__ x1,
                                                            int8_t *__restrict__ c1, float *scale1, int which1,
@@ -183,8 +183,7 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
         *scale0 = s0;
         if (x1) *scale1 = s1;
     }
-    const int lane = threadIdx.x & 31;
-    const bool norms = vnorm != nullptr;
+    const int lane = NORMS ? (threadIdx.x & 31) : 0;  // without norms no loop bound is taken per warp
     auto row_norm = [&](const float (&x)[VE], int64_t iv, bool in) {
         float ss = 0.f;
 #pragma unroll
@@ -197,7 +196,7 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     // kGlobalUnroll vectors per thread in flight per tensor, then their codes
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    for (; (i - lane) + 31 + (kGlobalUnroll - 1) * stride < nvec; i += kGlobalUnroll * stride) {
+    for (; (i - lane) + (NORMS ? 31 : 0) + (kGlobalUnroll - 1) * stride < nvec; i += kGlobalUnroll * stride) {
         uint4 w0[kGlobalUnroll], w1[kGlobalUnroll];
 #pragma unroll
         for (int u = 0; u < kGlobalUnroll; ++u) w0[u] = __ldcs(p0 + i + u * stride);
@@ -210,24 +209,24 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
             float x[VE];
             Vec<T>::unpack(w0[u], x);
             store_codes<VE>(c0 + (i + u * stride) * VE, x, s0, r0);
-            if (norms && vnorm_of == 0) row_norm(x, i + u * stride, true);
+            if (NORMS && vnorm_of == 0) row_norm(x, i + u * stride, true);
             if (x1) {
                 Vec<T>::unpack(w1[u], x);
                 store_codes<VE>(c1 + (i + u * stride) * VE, x, s1, r1);
-                if (norms && vnorm_of == 1) row_norm(x, i + u * stride, true);
+                if (NORMS && vnorm_of == 1) row_norm(x, i + u * stride, true);
             }
         }
     }
-    for (; i - lane < nvec; i += stride) {  // the rest, every lane of the warp together
+    for (; i - lane < nvec; i += stride) {  // the rest (with norms: every lane of the warp together)
         const bool in = i < nvec;
         float x[VE];
         Vec<T>::unpack(in ? __ldcs(p0 + i) : make_uint4(0, 0, 0, 0), x);
         if (in) store_codes<VE>(c0 + i * VE, x, s0, r0);
-        if (norms && vnorm_of == 0) row_norm(x, i, in);
+        if (NORMS && vnorm_of == 0) row_norm(x, i, in);
         if (x1) {
             Vec<T>::unpack(in ? __ldcs(p1 + i) : make_uint4(0, 0, 0, 0), x);
             if (in) store_codes<VE>(c1 + i * VE, x, s1, r1);
-            if (norms && vnorm_of == 1) row_norm(x, i, in);
+            if (NORMS && vnorm_of == 1) row_norm(x, i, in);
         }
     }
 }
@@ -240,7 +239,7 @@ static int global_ctas_per_sm() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
     if (cache[dev] == 0) {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_global_kernel<T>, 256, 0) != cudaSuccess || n < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_global_kernel<T, false>, 256, 0) != cudaSuccess || n < 1)
             n = 4;
         cache[dev] = n;
     }
@@ -269,12 +268,12 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
                            (const int32_t *)seq_part0, B, Hkv, Ttot, n_parts, kc, k_scale, hdr);
             if (e != cudaSuccess) return (int)e;
         }
-        e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v, vc,
+        e = launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v, vc,
                      v_scale, 1, none, no_codes, no_scale, 0, nvec, (const WsHeader *)hdr, vnorm, 0, D / VE);
     } else {
         e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
         if (e != cudaSuccess) return (int)e;
-        e = launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k, kc,
+        e = launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k, kc,
                      k_scale, 0, v, vc, v_scale, 1, nvec, (const WsHeader *)hdr, vnorm, 1, D / VE);
     }
     return (int)e;
@@ -289,9 +288,9 @@ static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t 
     int8_t *no_codes = nullptr;
     float *no_scale = nullptr;
     if (scheme == SGD_SCHEME_A)
-        return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v,
+        return (int)launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v,
                              vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr, vnorm, 0, D / Vec<T>::VE);
-    return (int)launch_k(quant_global_kernel<T>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k,
+    return (int)launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k,
                          kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr, vnorm, 1, D / Vec<T>::VE);
 }
 
