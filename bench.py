@@ -41,7 +41,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -67,7 +67,9 @@ def algorithmic_bytes(wl, lengths):
     if wl.oam:
         Kt = sum(kept_of(L, wl.keep_num, wl.keep_den) for L in lengths)
         sel_out = q + Hkv * Kt * 4 + (B + 1) * 4
-    if wl.scheme and wl.oam:  # one call reads K and V once for both
+    if wl.select_on_codes:  # the cache is already INT8: the selection reads K codes and the norms
+        st["select"] = Hkv * T * D + Hkv * T * 4 + (Hkv * P * 4 if wl.scheme == "A" else 4) + sel_out
+    elif wl.scheme and wl.oam:  # one call reads K and V once for both
         st["quantize_select"] = kv_bf16 + codes_out + sel_out
     elif wl.scheme:
         st["quantize"] = kv_bf16 + codes_out
@@ -154,6 +156,19 @@ class Pipeline:
         self.sel_out = None
         self.dec_out = None
         self.stage_events = {}
+        if wl.select_on_codes:
+            # a cache quantised once, before the steps (untimed), with its value norms
+            self.vn = torch.empty(self.k.shape[:2], dtype=torch.float32, device=dev)
+            self.kc, self.vc, self.ks, self.vs, _ = sgd.quantize_kv(self.k, self.v, self.cu, wl.scheme,
+                                                                    self.lengths, v_norm=self.vn)
+            torch.cuda.synchronize(dev)
+            del self.k, self.v
+
+    def inputs(self):
+        """The device tensors a step reads (for the end-to-end copies)."""
+        if self.wl.select_on_codes:
+            return [self.q, self.kc, self.vc, self.ks, self.vs, self.vn, self.cu]
+        return [self.q, self.k, self.v, self.cu]
 
     def run(self, record=None):
         """One step.  record: dict stage -> (start_event, end_event) to time each stage."""
@@ -163,10 +178,19 @@ class Pipeline:
             if record is not None:
                 record[name][i].record()
 
-        kc, vc, ks, vs = self.k, self.v, None, None
         idx = cu_kept = None
         Kt = 0
-        if wl.scheme and wl.oam:
+        if wl.select_on_codes:  # the cache is INT8 already: select on its codes
+            kc, vc, ks, vs = self.kc, self.vc, self.ks, self.vs
+            ev("select", 0)
+            idx, cu_kept, self.ws_s = sgd.oam_select(self.q, kc, vc, self.cu, wl.G, wl.beta, wl.eps, wl.keep_num,
+                                                     wl.keep_den, self.lengths, out=self.sel_out,
+                                                     workspace=self.ws_s, k_scale=ks, v_scale=vs,
+                                                     scheme=wl.scheme, n_parts_=self.parts, v_norm=self.vn)
+            self.sel_out = (idx, cu_kept)
+            Kt = idx.shape[1]
+            ev("select", 1)
+        elif wl.scheme and wl.oam:
             ev("quantize_select", 0)
             kc, vc, ks, vs, idx, cu_kept, self.ws_q = sgd.quantize_select(
                 self.q, self.k, self.v, self.cu, wl.G, wl.beta, wl.eps, wl.keep_num, wl.keep_den, wl.scheme,
@@ -181,6 +205,7 @@ class Pipeline:
             self.qout = (kc, vc, ks, vs)
             ev("quantize", 1)
         elif wl.oam:
+            kc, vc, ks, vs = self.k, self.v, None, None
             ev("select", 0)
             idx, cu_kept, self.ws_s = sgd.oam_select(self.q, self.k, self.v, self.cu, wl.G, wl.beta, wl.eps,
                                                      wl.keep_num, wl.keep_den, self.lengths, out=self.sel_out,
@@ -188,6 +213,8 @@ class Pipeline:
             self.sel_out = (idx, cu_kept)
             Kt = idx.shape[1]
             ev("select", 1)
+        else:
+            kc, vc, ks, vs = self.k, self.v, None, None
         ev("decode", 0)
         o, lse, self.ws_d = sgd.decode_attn(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
                                             scheme=wl.scheme or "A", n_parts_=self.parts, idx=idx,
@@ -199,6 +226,8 @@ class Pipeline:
 
     def launches_per_step(self):
         # decode: plan + the tensor-core decode, which merges each row itself (D = 128, bf16 q)
+        if self.wl.select_on_codes:
+            return 3 + 2  # plan, INT8 score, top-K; plan, decode
         if self.wl.scheme and self.wl.oam:
             return 4 + 2  # plan, score+quantize, V codes, top-K; plan, decode
         return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 2
@@ -256,7 +285,10 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
         if wl.scheme:
             quant = oracle.quantize_kv(kk, vv, one, wl.scheme)
         idx = cu_kept = None
-        if wl.oam:
+        if wl.oam and wl.select_on_codes:
+            idx, cu_kept, _ = oracle.oam_select_int8(qrow, quant[0], quant[2], vv, one, wl.scheme, wl.G, wl.beta,
+                                                     wl.eps, wl.keep_num, wl.keep_den)
+        elif wl.oam:
             idx, cu_kept, _ = oracle.oam_select(qrow, kk, vv, one, wl.G, wl.beta, wl.eps, wl.keep_num,
                                                 wl.keep_den)
         oracle.decode(qrow, kk, vv, one, wl.G, idx=idx, cu_kept=cu_kept,
@@ -370,18 +402,17 @@ def run_ours(args, rank, world, local_rank):
     eager_ms = reduce_max(sum(a.elapsed_time(b) for a, b in eager_ev), dev, world) / K
 
     # e2e: host buffers through the same calls, copies inside the timed region
-    pin_q, pin_k, pin_v, pin_cu = (x.pin_memory() for x in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    dev_in = pipe.inputs()
+    pin_in = [x.cpu().pin_memory() for x in dev_in]
     B, Hq, D = bt.q.shape
     h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
     h_lse = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in (pin_q, pin_k, pin_v, pin_cu))
+    h2d = sum(x.numel() * x.element_size() for x in pin_in)
     d2h = h_out.numel() * 4 + h_lse.numel() * 4
     e2e_steps = max(2, min(K, 5))
     for _ in range(2):
-        pipe.q.copy_(pin_q, non_blocking=True)
-        pipe.k.copy_(pin_k, non_blocking=True)
-        pipe.v.copy_(pin_v, non_blocking=True)
-        pipe.cu.copy_(pin_cu, non_blocking=True)
+        for d_t, h_t in zip(dev_in, pin_in):
+            d_t.copy_(h_t, non_blocking=True)
         o, lse = pipe.run()
         h_out.copy_(o, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
@@ -389,10 +420,8 @@ def run_ours(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
-        pipe.q.copy_(pin_q, non_blocking=True)
-        pipe.k.copy_(pin_k, non_blocking=True)
-        pipe.v.copy_(pin_v, non_blocking=True)
-        pipe.cu.copy_(pin_cu, non_blocking=True)
+        for d_t, h_t in zip(dev_in, pin_in):
+            d_t.copy_(h_t, non_blocking=True)
         o, lse = pipe.run()
         h_out.copy_(o, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
@@ -433,7 +462,9 @@ def run_ours(args, rank, world, local_rank):
             "workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D, "lengths": pipe.lengths,
             "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
             "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": args.workload,
-            "step": "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn",
+            "step": ("oam_select(int8 cache, stored norms) -> decode_attn(kept); cache quantised once, untimed"
+                     if wl.select_on_codes else
+                     "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn"),
             "l2": "flushed between steps (untimed 256 MiB write then 256 MiB read: L2 left clean); inputs > L2",
             "parallelism": f"dp{world} (independent copies, no collective)",
             "launch": launch,

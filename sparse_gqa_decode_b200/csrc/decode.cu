@@ -57,6 +57,7 @@ struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
     static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
+    static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static constexpr int NW = 4;        // consumer warps
     static constexpr int SUB = I8 ? 2 : 1;  // 16-token sub-tiles per consumer warp per stage
     static constexpr int ROWS = NW * 16 * SUB;
@@ -66,11 +67,14 @@ struct MmaCfg {
     static constexpr int BOX_ELEMS = 128 / EB;
     static constexpr int TILE = ROWS * ROWB;  // bytes of one tensor per stage
     static constexpr int STAGES = 3;
-    static constexpr int MINB = 2;  // CTAs per SM the registers must allow
+    // CTAs per SM the registers must allow: the K-only score of an INT8 cache has half-size stages
+    // and is issue-bound, so a third CTA (more consumer warps) fits and pays
+    static constexpr int MINB = KONLY ? 3 : 2;
     static constexpr int KB = D / 16;
     static constexpr int NQ = (MODE == 2) ? kQuantWarps : 0;  // K-quantising warps (mode 2)
     static constexpr int THREADS = (NW + NQ + 1) * 32;
-    static constexpr int SMEM_STAGES = STAGES * 2 * TILE;
+    static constexpr int STAGE_BYTES = (KONLY ? 1 : 2) * TILE;  // K tile, then V tile
+    static constexpr int SMEM_STAGES = STAGES * STAGE_BYTES;
     static constexpr bool ROW_SCALE = I8 && IDX;  // per-row K scales fetched by the producer
     static constexpr int SMEM_ROWSCALE = ROW_SCALE ? STAGES * ROWS * 4 : 0;
     static constexpr int SMEM_KMX = 2 * (NQ > 4 ? NQ : 4) * 4;  // [2][NQ] per-warp max|K| (mode 2)
@@ -78,7 +82,6 @@ struct MmaCfg {
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
-    static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
@@ -128,7 +131,7 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
         }
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
-            uint8_t *sk = smem + stage * 2 * C::TILE;
+            uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
             if constexpr (!C::IDX) {
                 mbar_arrive_expect_tx(&full[stage], (C::KONLY ? 1 : 2) * C::TILE);
@@ -425,19 +428,17 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
 
 // OAM scores of a sub-tile of an INT8 cache (mode 1): khat = code * scale, so the logit of head g
 // is sacc * colf_g (log2 units, with the head's Q pre-scale) times the sub-tile's partition scale
-// rf >= 0 (scheme A; scheme B's scale is inside colf); ||v_t|| comes from the norms stored when
-// the cache was quantised, so the V codes are never read.
+// rf >= 0 (scheme A; scheme B's scale is inside colf); ||v_t|| (vn, lanes 0-15: row rb + lane)
+// comes from the norms stored when the cache was quantised, so the V codes are never read.
 template <class C>
 __device__ __forceinline__ void score_subtile_i8(const DecodeArgs &a, uint32_t kbase, int rb, int32_t j0, int32_t t1,
                                                  bool ready, int64_t tok_base, int pA, int t4, int lane,
                                                  const uint32_t (&qf)[C::GT][C::KB][2], const float (&colf)[C::GT][2],
-                                                 float rf) {
+                                                 float rf, float vn) {
     const bool act = ready && j0 < t1;
     const int rho = lane & 15, half = lane >> 4;
     const int32_t j = j0 + rho;
     const bool vrow = act && j < t1;
-    float vn = 0.f;
-    if (half == 0 && vrow) vn = __ldg(a.v_norm + tok_base + j);  // in flight during the MMAs
     float sacc[C::GT][4];
     if (act) {
         qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
@@ -498,7 +499,7 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
         float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + cur.ri.part0;
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
-            const uint32_t kbase = smem_u32(smem + stage * 2 * C::TILE);
+            const uint32_t kbase = smem_u32(smem + stage * C::STAGE_BYTES);
             const int32_t j = t + vr;
             const bool vrow = ready && j < t1;
             uint4 kw[NH];
@@ -767,6 +768,16 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         const int32_t *ip = nullptr;
         if constexpr (C::I8) ksc = a.k_scale + (int64_t)kvh * a.n_parts + cur.ri.part0;
         if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start;
+        // scores of an INT8 cache: the value norms of each sub-tile row, loaded one tile ahead
+        float vn_cur[C::SUB], vn_nxt[C::SUB];
+        auto load_norms = [&](float (&dst)[C::SUB], int32_t tt) {
+#pragma unroll
+            for (int s = 0; s < C::SUB; ++s) {
+                const int32_t j = tt + 16 * (s * C::NW + warp) + (lane & 15);
+                dst[s] = (lane < 16 && j < t1) ? __ldg(a.v_norm + tok_base + j) : 0.f;
+            }
+        };
+        if constexpr (C::KONLY) load_norms(vn_cur, t0);
 
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             // dense scheme A: the K scale of each sub-tile's partition, loaded before the wait
@@ -780,8 +791,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                         rf_pre[s] = __ldg(ksc + min(t + 16 * (s * C::NW + warp), Lb - 1) / kPart);
                 }
             }
+            if constexpr (C::KONLY) load_norms(vn_nxt, t + C::ROWS);
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
-            uint8_t *sk = smem + stage * 2 * C::TILE;
+            uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
             const uint32_t kbase = smem_u32(sk), vbase = smem_u32(sv);
 #pragma unroll
@@ -790,7 +802,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
                 if constexpr (C::MODE >= 1) {
                     if constexpr (C::I8)
-                        score_subtile_i8<C>(a, kbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, colf, rf_pre[s]);
+                        score_subtile_i8<C>(a, kbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, colf, rf_pre[s],
+                                            vn_cur[s]);
                     else
                         score_subtile<C>(a, kbase, vbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, run_vmax);
                     continue;
@@ -856,6 +869,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
             }
             ++tile_no;
+            if constexpr (C::KONLY) {
+#pragma unroll
+                for (int s = 0; s < C::SUB; ++s) vn_cur[s] = vn_nxt[s];
+            }
             const bool last = (t + C::ROWS >= t1);
             if (C::MODE == 0 && last) {
                 // ---- segment epilogue: combine the four warps' (m, l, O) in this stage's memory ----
@@ -1263,6 +1280,8 @@ int decode_ctas_per_sm(sgd_dtype kv, sgd_dtype q, int D, int G, bool indexed, bo
     }
     const bool g2 = G > 8;
     // the shared-memory and register footprint decide residency
+    if (kv == SGD_I8 && score)
+        return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, false, 1>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, false, 1>>();
     if (kv == SGD_I8 && indexed)
         return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, true, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, true, 0>>();
     if (kv == SGD_I8) return g2 ? ctas_per_sm_mma<MmaCfg<128, 2, true, false, 0>>() : ctas_per_sm_mma<MmaCfg<128, 1, true, false, 0>>();

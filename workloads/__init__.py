@@ -63,6 +63,7 @@ class Workload:
     keep_num: int = 1  # keep ceil(L_b * keep_num / keep_den) tokens per (sequence, KV head)
     keep_den: int = 8
     n_splits: int = 0  # 0 = equal-work split over all SMs; >0 forces that many CTAs
+    select_on_codes: bool = False  # the cache is quantised beforehand; OAM scores its INT8 K codes
 
     @property
     def Hq(self) -> int:
@@ -72,7 +73,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five seeded workloads.  Seed = workload number.
+# The seeded workloads.  Seed = workload number.
 CONFIGS = {
     1: Workload("tiny_dense_f32_L256", B=1, Hkv=1, G=4, D=64, kv_dtype="f32", dist="normal",
                 lengths=(256,), n_splits=4),
@@ -84,11 +85,13 @@ CONFIGS = {
                 lengths=(131072,) * 8, scheme="A"),
     5: Workload("oam_int8A_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True),
+    6: Workload("oam_on_int8cache_A_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
+                dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, select_on_codes=True),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..5), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..6), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
