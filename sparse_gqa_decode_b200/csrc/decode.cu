@@ -69,7 +69,7 @@ struct MmaCfg {
     static constexpr int STAGES = 3;
     // CTAs per SM the registers must allow: the K-only score of an INT8 cache has half-size stages
     // and is issue-bound, so a third CTA (more consumer warps) fits and pays
-    static constexpr int MINB = KONLY ? 3 : 2;
+    static constexpr int MINB = KONLY ? 4 : 2;
     static constexpr int KB = D / 16;
     static constexpr int NQ = (MODE == 2) ? kQuantWarps : 0;  // K-quantising warps (mode 2)
     static constexpr int THREADS = (NW + NQ + 1) * 32;
