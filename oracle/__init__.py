@@ -142,6 +142,37 @@ def quantize(x, scale) -> np.ndarray:
     return out
 
 
+def quantize_q(q, mode: str):
+    """Query-side INT8 ([TD] section 6: schemes A and B also quantise Q per token partition).
+
+    A decode query is one token per sequence, so its partition is that token: ``mode`` "token"
+    gives every (sequence, query head) row of q [B, Hq, D] its own scale over D; "tensor" gives
+    all of q one scale (the per-tensor baseline).  Scale and code rules as for K and V.
+    Returns (codes int8 [B, Hq, D], scales float32 [B, Hq] or [1])."""
+    x = _f32(q)
+    if mode == "tensor":
+        s = scale_from_amax(amax(x))
+        return quantize(x, s), np.array([s], np.float32)
+    if mode != "token":
+        raise ValueError("mode is 'token' or 'tensor'")
+    B, Hq, D = x.shape
+    codes = np.empty((B, Hq, D), np.int8)
+    scales = np.empty((B, Hq), np.float32)
+    for b in range(B):
+        for h in range(Hq):
+            scales[b, h] = scale_from_amax(amax(x[b, h]))
+            codes[b, h] = quantize(x[b, h], scales[b, h])
+    return codes, scales
+
+
+def dequant_q(codes, scales) -> np.ndarray:
+    """code * scale of a quantised query (float64, exact), scales [B, Hq] or [1]."""
+    s = np.asarray(scales, np.float64)
+    if s.size == 1:
+        return np.asarray(codes, np.float64) * s[0]
+    return np.asarray(codes, np.float64) * s[..., None]
+
+
 def n_parts(lengths: Sequence[int], part: int = PART) -> np.ndarray:
     return np.array([(int(L) + part - 1) // part for L in lengths], dtype=np.int64)
 

@@ -243,6 +243,22 @@ def test_quantize_zero_group_gives_zero_scale_and_codes():
     assert s == 0.0 and not oracle.quantize(x, s).any()
 
 
+def test_query_quantisation_per_row_and_per_tensor():
+    # row 0 reaches 127: scale 1, codes are the rounded values (ties to even); row 1 is row 0 times
+    # 2^-3 (scale 2^-3, the same codes); per tensor, the one scale is 1 and row 1's codes shrink
+    q = np.zeros((1, 2, 8), np.float32)
+    q[0, 0] = [127.0, 2.5, -3.5, 0.5, -0.5, 1.49, 64.0, 0.0]
+    q[0, 1] = q[0, 0] * 0.125
+    codes, scales = oracle.quantize_q(q, "token")
+    assert scales.tolist() == [[1.0, 0.125]]
+    assert codes[0, 0].tolist() == [127, 2, -4, 0, 0, 1, 64, 0]
+    assert codes[0, 1].tolist() == codes[0, 0].tolist()
+    tcodes, ts = oracle.quantize_q(q, "tensor")
+    assert ts.tolist() == [1.0] and tcodes[0, 0].tolist() == codes[0, 0].tolist()
+    assert tcodes[0, 1].tolist() == [16, 0, 0, 0, 0, 0, 8, 0]  # 15.875 -> 16, 0.3125 -> 0, 8 -> 8
+    assert np.array_equal(oracle.dequant_q(codes, scales)[0, 1], codes[0, 1] * 0.125)
+
+
 def test_scheme_a_partitions_start_at_each_sequence():
     bt = _tiny_batch(G=2, D=8, lengths=(70, 64, 3, 129), Hkv=2, dtype="bf16")
     kc, vc, ks, vs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
