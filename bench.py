@@ -41,7 +41,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -219,7 +219,7 @@ class Pipeline:
         o, lse, self.ws_d = sgd.decode_attn(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
                                             scheme=wl.scheme or "A", n_parts_=self.parts, idx=idx,
                                             cu_kept=cu_kept, kept_total_=Kt, out=self.dec_out,
-                                            workspace=self.ws_d)
+                                            workspace=self.ws_d, q_quant=wl.q_quant or "none")
         self.dec_out = (o, lse)
         ev("decode", 1)
         return o, lse
@@ -291,6 +291,8 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
         elif wl.oam:
             idx, cu_kept, _ = oracle.oam_select(qrow, kk, vv, one, wl.G, wl.beta, wl.eps, wl.keep_num,
                                                 wl.keep_den)
+        if wl.q_quant:  # the attention sees the query's code * scale
+            qrow = oracle.dequant_q(*oracle.quantize_q(qrow, wl.q_quant))
         oracle.decode(qrow, kk, vv, one, wl.G, idx=idx, cu_kept=cu_kept,
                       quant=None if quant is None else (*quant, wl.scheme))
         done.append((b, h, L))
@@ -324,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = workloads.config(args.workload)
-    bt = workloads.generate(wl, seed=args.workload)  # the same batch on every rank
+    bt = workloads.generate(wl, seed=wl.seed if wl.seed is not None else args.workload)  # the same batch on every rank
     pipe = Pipeline(sgd, wl, bt, dev)
     stages = algorithmic_bytes(wl, pipe.lengths)
     step_bytes = sum(stages.values())
@@ -461,7 +463,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D, "lengths": pipe.lengths,
             "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
-            "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": args.workload,
+            "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": wl.seed if wl.seed is not None else args.workload, "q_quant": wl.q_quant,
             "step": ("oam_select(int8 cache, stored norms) -> decode_attn(kept); cache quantised once, untimed"
                      if wl.select_on_codes else
                      "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn"),
@@ -495,7 +497,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     wl = workloads.config(args.workload)
-    bt = workloads.generate(wl, seed=args.workload)
+    bt = workloads.generate(wl, seed=wl.seed if wl.seed is not None else args.workload)
     cu = bt.cu_seqlens.numpy()
     rows = [(b, h) for h in range(wl.Hkv) for b in range(wl.B)]
     shortest = min(rows, key=lambda r: int(cu[r[0] + 1] - cu[r[0]]))

@@ -177,16 +177,20 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
  *   are the cache values (I8: code * scale).  The work of all (sequence, KV
  *   head) rows is cut into equal token ranges, one per CTA (schedule 0: as many
  *   CTAs as fill the GPU, or n_splits when > 0; schedule 1: one CTA per row);
- *   each range emits partial (o_c, lse_c) per row it touches and a merge
- *   kernel combines them exactly: lse = ln sum_c exp(lse_c),
- *   out = sum_c exp(lse_c - lse) o_c.
+ *   each range emits partial (o_c, lse_c) per row it touches and they are
+ *   combined exactly: lse = ln sum_c exp(lse_c), out = sum_c exp(lse_c - lse) o_c.
  * q        [B, Hq, D], BF16 (F32 only with an F32 cache)
  * idx, cu_kept, kept_total   as produced by sgd_oam_select, or NULL/NULL/0
+ * q_quant  query-side INT8 ([TD] section 6, schemes A and B quantise Q too), I8 cache with
+ *          D = 128 and a BF16 q only: 0 = q as given; 1 = q replaced by code * scale with one
+ *          scale per (sequence, query head) row, max|q_row| / 127; 2 = one scale for all of q
+ *          (the per-tensor baseline).  Codes follow the K rule (IEEE quotient, ties to even,
+ *          clamp to +-127); q.k is then an exact integer dot product of the codes.
  * out      [B, Hq, D] float32;  lse [B, Hq] float32
  */
 int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                     const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
-                    int schedule, int n_splits, float *out, float *lse,
+                    int schedule, int n_splits, int q_quant, float *out, float *lse,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /* Workspace bytes an operation needs for this cache shape (>= 256). For
@@ -241,7 +245,7 @@ int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chun
 #define SGD_NOALLOC_SCRATCH_BYTES (4u << 20)
 int sgd_decode_attn_noalloc(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                             const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
-                            int schedule, int n_splits, float *out, float *lse, int32_t *status,
+                            int schedule, int n_splits, int q_quant, float *out, float *lse, int32_t *status,
                             void *stream);
 
 /* Copies the device status word of `workspace` to *status (host) after

@@ -65,14 +65,16 @@ lib.sgd_workspace_size.restype = _sz
 lib.sgd_decode_num_ctas.argtypes = [_kvp, _i32, _vp, _i32, _i32]
 lib.sgd_quantize_kv.argtypes = [_kvp, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _vp, _i64, _vp, _sz, _vp]
-lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _vp, _sz, _vp]
-lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp, _vp]
+lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp,
+                                        _vp]
 
 _DT = {torch.float32: SGD_F32, torch.bfloat16: SGD_BF16, torch.int8: SGD_I8}
+_QQ = {"none": 0, "token": 1, "tensor": 2}
 
 
 class SgdError(RuntimeError):
@@ -216,8 +218,11 @@ def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
 def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                 k_scale=None, v_scale=None, scheme: str = "A", n_parts_: int = 0,
                 idx=None, cu_kept=None, kept_total_: int = 0, schedule: int = 0, n_splits: int = 0,
-                out=None, workspace=None, stream=None):
-    """Attention output and log-sum-exp per query head.  Returns (out [B,Hq,D] f32, lse [B,Hq] f32, ws)."""
+                out=None, workspace=None, stream=None, q_quant: str = "none"):
+    """Attention output and log-sum-exp per query head.  Returns (out [B,Hq,D] f32, lse [B,Hq] f32, ws).
+
+    ``q_quant`` (INT8 cache, bf16 q, D = 128): "none", "token" (one query scale per (sequence,
+    head) row) or "tensor" (one scale for all of q); q.k then runs on the INT8 codes."""
     sch = SCHEME_A if scheme == "A" else SCHEME_B
     kv = _kv(k, v, cu_seqlens, k_scale, v_scale, sch, n_parts_)
     B = cu_seqlens.numel() - 1
@@ -230,7 +235,8 @@ def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_se
         o, lse = out
     ws = _workspace(workspace_size(OP_DECODE, kv, G, schedule, n_splits), k.device, workspace)
     _check(lib.sgd_decode_attn(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
-                               int(kept_total_), schedule, n_splits, _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                               int(kept_total_), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse), _ptr(ws),
+                               ws.numel(),
                                _stream(stream)), "sgd_decode_attn")
     return o, lse, ws
 
@@ -238,7 +244,7 @@ def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_se
 def decode_attn_noalloc(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                         k_scale=None, v_scale=None, scheme: str = "A", n_parts_: int = 0,
                         idx=None, cu_kept=None, kept_total_: int = 0, schedule: int = 0, n_splits: int = 0,
-                        out=None, status=None, stream=None):
+                        out=None, status=None, stream=None, q_quant: str = "none"):
     """decode_attn without a workspace: the library's built-in device scratch array is used
     (for callers that cannot allocate).  ``out`` = (out, lse) and ``status`` ([1] int32) are
     optional preallocated device outputs.  Returns (out, lse)."""
@@ -251,7 +257,8 @@ def decode_attn_noalloc(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tenso
     else:
         o, lse = out
     _check(lib.sgd_decode_attn_noalloc(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
-                                       int(kept_total_), schedule, n_splits, _ptr(o), _ptr(lse), _ptr(status),
+                                       int(kept_total_), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse),
+                                       _ptr(status),
                                        _stream(stream)), "sgd_decode_attn_noalloc")
     return o, lse
 

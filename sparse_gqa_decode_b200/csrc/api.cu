@@ -363,8 +363,8 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
 }
 
 int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, const int32_t *idx,
-                    const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, float *out, float *lse,
-                    void *workspace, size_t workspace_bytes, void *stream) {
+                    const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, int q_quant, float *out,
+                    float *lse, void *workspace, size_t workspace_bytes, void *stream) {
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
@@ -380,6 +380,9 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
         if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
             return SGD_ERR_SHAPE;
     }
+    if (q_quant < 0 || q_quant > 2) return SGD_ERR_ARG;
+    if (q_quant != 0 && (kv->dtype != SGD_I8 || q_dtype != SGD_BF16)) return SGD_ERR_DTYPE;
+    if (q_quant != 0 && kv->D != 128) return SGD_ERR_SHAPE;
     if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SGD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (indexed && (reinterpret_cast<uintptr_t>(idx) & 3u)))
         return SGD_ERR_ALIGN;
@@ -395,7 +398,8 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     cudaStream_t s = as_stream(stream);
     const int min_chunk = (n_splits > 0 || schedule == 1) ? kGranule : kAutoMinChunk;
     launch_plan(indexed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
-                hdr, s, kGranule, out, lse, G, kv->D);
+                hdr, s, kGranule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
+                (int64_t)kv->B * kv->Hkv * G * kv->D);
     DecodeArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q;
@@ -423,6 +427,8 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     a.out = out;
     a.lse = lse;
     a.status = &hdr->status;
+    a.q_quant = q_quant;
+    a.q_scale = &hdr->q_scale;
     int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
     // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials

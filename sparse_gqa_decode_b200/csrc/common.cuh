@@ -27,7 +27,8 @@ struct WsHeader {
     int32_t plan_ncta;    // plan: CTAs with work
     int32_t plan_nslots;  // plan: segments (partial results)
     int32_t n_parts;      // quantize/decode: partitions counted on the device
-    int32_t pad1[53];
+    float q_scale;        // decode with a per-tensor query scale: max|q| / 127
+    int32_t pad1[52];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -184,6 +185,16 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1,
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D += A(16x32, s8) * B(32x8, s8), int32 accumulation
+__device__ __forceinline__ void mma_s8(int32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 

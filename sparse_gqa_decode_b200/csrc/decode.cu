@@ -52,10 +52,11 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 
 constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
 
-template <int D_, int GT_, bool I8_, bool IDX_, int MODE_>
+template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
+    static constexpr bool QI8 = QI8_;  // INT8 query codes: S^T = K_codes . Q_codes^T on s8 MMAs
     static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
     static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static constexpr int NW = 4;        // consumer warps
@@ -82,6 +83,7 @@ struct MmaCfg {
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
+    static_assert(!QI8 || (I8 && MODE == 0 && D == 128), "query codes meet INT8 keys in the decode");
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
@@ -243,6 +245,27 @@ __device__ __forceinline__ void load_q_frags(const DecodeArgs &a, int b, int kvh
             }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            if constexpr (C::QI8) {
+                // the head's query codes ([TD] section 6 on Q): scale max|q|/127 of this (sequence,
+                // head) row, or the tensor's; the lane's chunk c = t4 + 4h gives two s8 MMAs (bytes
+                // 0-7, 8-15), in the k order qk_subtile reads the K chunk in
+                const float sq = a.q_quant == 2 ? __ldg(a.q_scale) : __fdiv_rn(mx, 127.f);
+                const float rq = (sq != 0.f) ? __frcp_rn(sq) : 0.f;
+#pragma unroll
+                for (int h = 0; h < C::KB / 4; ++h)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) {
+                        qf[gt][2 * h + m][0] = (sq != 0.f) ? codes4(&x[h][8 * m], sq, rq) : 0u;
+                        qf[gt][2 * h + m][1] = (sq != 0.f) ? codes4(&x[h][8 * m + 4], sq, rq) : 0u;
+                    }
+                const float s0 = __shfl_sync(0xffffffffu, sq, 4 * (2 * t4));
+                const float s1 = __shfl_sync(0xffffffffu, sq, 4 * (2 * t4 + 1));
+                float f = a.sm_scale_log2;
+                if (a.scheme == SGD_SCHEME_B) f *= __ldg(a.k_scale);
+                colf[gt][0] = f * s0;
+                colf[gt][1] = f * s1;
+                continue;
+            }
             int ex = 0;
             if (mx > 0.f) frexpf(mx, &ex);
             const int sh = 14 - ex;  // max |q| * 2^sh < 2^14: inside f16 range
@@ -285,6 +308,27 @@ __device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t
                 mma_bf16(sacc[gt], ka.z, kb.z, ka.w, kb.w, qf[gt][2 * h + 1][0], qf[gt][2 * h + 1][1]);
             }
         }
+    } else if constexpr (C::QI8) {
+        // s8 x s8 -> s32: two m16n8k32 MMAs per 16-byte chunk of the row (its bytes 0-7 and 8-15 are
+        // k 0..3 / 16..19 and so on of one MMA: the query codes follow the same order)
+        int32_t ia[C::GT][4];
+#pragma unroll
+        for (int gt = 0; gt < C::GT; ++gt) ia[gt][0] = ia[gt][1] = ia[gt][2] = ia[gt][3] = 0;
+#pragma unroll
+        for (int h = 0; h < C::KB / 4; ++h) {
+            const int c = t4 + 4 * h;
+            const uint32_t base = kbase + ((c ^ pA) << 4);
+            const uint4 ka = lds128(base + rA * 128), kb = lds128(base + rB * 128);
+#pragma unroll
+            for (int gt = 0; gt < C::GT; ++gt) {
+                mma_s8(ia[gt], ka.x, kb.x, ka.y, kb.y, qf[gt][2 * h][0], qf[gt][2 * h][1]);
+                mma_s8(ia[gt], ka.z, kb.z, ka.w, kb.w, qf[gt][2 * h + 1][0], qf[gt][2 * h + 1][1]);
+            }
+        }
+#pragma unroll
+        for (int gt = 0; gt < C::GT; ++gt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sacc[gt][j] = (float)ia[gt][j];  // |sum| < 2^24: exact
     } else {
 #pragma unroll
         for (int h = 0; h < C::KB / 4; ++h) {
@@ -1246,13 +1290,13 @@ static int launch_mma(const DecodeArgs &a, int n_cta, cudaStream_t s) {
     return (int)launch_k(k, dim3(n_cta), dim3(C::THREADS), C::SMEM, s, 1, mk, mv, a);
 }
 
-template <int D, int GT, bool I8, int MODE>
+template <int D, int GT, bool I8, int MODE, bool QI8 = false>
 static int launch_mma_idx(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
     if constexpr (MODE == 1) {
         return launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
     } else {
-        return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE>>(a, n_cta, s)
-                       : launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
+        return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE, QI8>>(a, n_cta, s)
+                       : launch_mma<MmaCfg<D, GT, I8, false, MODE, QI8>>(a, n_cta, s);
     }
 }
 
@@ -1305,6 +1349,8 @@ int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, 
             if (a.D == 128) return g2 ? launch_mma_idx<128, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, false, 1>(a, false, n_cta, s);
             return g2 ? launch_mma_idx<64, 2, false, 1>(a, false, n_cta, s) : launch_mma_idx<64, 1, false, 1>(a, false, n_cta, s);
         }
+        if (kv == SGD_I8 && a.q_quant)
+            return g2 ? launch_mma_idx<128, 2, true, 0, true>(a, indexed, n_cta, s) : launch_mma_idx<128, 1, true, 0, true>(a, indexed, n_cta, s);
         if (kv == SGD_I8)
             return g2 ? launch_mma_idx<128, 2, true, 0>(a, indexed, n_cta, s) : launch_mma_idx<128, 1, true, 0>(a, indexed, n_cta, s);
         if (a.D == 128)

@@ -15,6 +15,8 @@ struct DecodeArgs {
     const float *k_scale;    // I8
     const float *v_scale;    // I8
     int scheme;              // I8: SGD_SCHEME_A / SGD_SCHEME_B
+    int q_quant;             // I8 decode: 0 bf16 query, 1 query codes per (sequence, head), 2 per tensor
+    const float *q_scale;    // q_quant == 2: the per-tensor query scale (in the workspace header)
     int B, Hkv, G, D;
     int64_t T, Kt, n_parts;
     int q_f32;               // q is float32 (otherwise bf16)
@@ -41,9 +43,11 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 
 // plan.cu
 // out/lse (decode only, else NULL): rows without tokens get out = 0 and lse = -inf here.
+// q_bf16 (decode with a per-tensor query scale, else NULL): hdr->q_scale = max|q| / 127.
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
-                 float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0);
+                 float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0, const void *q_bf16 = nullptr,
+                 int64_t q_elems = 0);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 

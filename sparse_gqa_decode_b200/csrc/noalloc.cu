@@ -44,7 +44,7 @@ int scratch_address(void **addr) {
 
 extern "C" int sgd_decode_attn_noalloc(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                                        const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
-                                       int schedule, int n_splits, float *out, float *lse, int32_t *status,
+                                       int schedule, int n_splits, int q_quant, float *out, float *lse, int32_t *status,
                                        void *stream) {
     void *scratch = nullptr;
     int rc = scratch_address(&scratch);
@@ -54,7 +54,8 @@ extern "C" int sgd_decode_attn_noalloc(const void *q, sgd_dtype q_dtype, int G, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the previous call's header is still there: start from a clear status word
     if (cudaMemsetAsync(scratch, 0, sizeof(sgd::WsHeader), s) != cudaSuccess) return SGD_ERR_CUDA;
-    rc = sgd_decode_attn(q, q_dtype, G, kv, idx, cu_kept, kept_total, schedule, n_splits, out, lse, scratch,
+    rc = sgd_decode_attn(q, q_dtype, G, kv, idx, cu_kept, kept_total, schedule, n_splits, q_quant, out, lse,
+                         scratch,
                          SGD_NOALLOC_SCRATCH_BYTES, stream);
     if (rc == SGD_OK && status) {
         if (cudaMemcpyAsync(status, static_cast<uint8_t *>(scratch) + SGD_WS_STATUS_OFFSET, sizeof(int32_t),

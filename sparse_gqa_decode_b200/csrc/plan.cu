@@ -20,7 +20,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
                                                     const int32_t *__restrict__ cu_seq, int B, int Hkv,
                                                     int n_req, int min_chunk, int mode, int granule,
                                                     PlanView pv, WsHeader *hdr, int staged, float *out,
-                                                    float *lse, int G, int D) {
+                                                    float *lse, int G, int D, const __nv_bfloat16 *q,
+                                                    int64_t q_elems) {
     __shared__ int32_t sm[33];
     extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
@@ -32,6 +33,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     if (tid == 0) {
         hdr->status = 0;
         hdr->amax_bits[0] = hdr->amax_bits[1] = 0u;
+    }
+    if (q) {  // per-tensor query scale for the decode: max|q| / 127 (IEEE division)
+        __shared__ uint32_t qmax;  // float bits: non-negative floats order as integers
+        float m = 0.f;
+        for (int64_t i = tid; i < q_elems; i += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(q[i])));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (tid == 0) qmax = 0u;
+        __syncthreads();
+        if ((tid & 31) == 0) atomicMax(&qmax, __float_as_uint(m));
+        __syncthreads();
+        if (tid == 0) hdr->q_scale = __fdiv_rn(__uint_as_float(qmax), 127.f);
     }
     if (staged) {
         for (int b = tid; b < B; b += blockDim.x) {  // all four loads of a thread in flight together
@@ -198,7 +211,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
-                 int G, int D) {
+                 int G, int D, const void *q_bf16, int64_t q_elems) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
@@ -206,7 +219,8 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
     const int want = std::max(std::max(B * Hkv, n_req), B) + 1;
     const int nt = std::min(1024, std::max(64, (want + 31) / 32 * 32));
     launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
-             min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D);
+             min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D,
+             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

@@ -62,7 +62,7 @@ def _kv(sgd, **kw):
 ])
 def test_decode_rejects_bad_cache_on_host(sgd, kw, code):
     kv = _kv(sgd, **kw)
-    rc = sgd.lib.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv), None, None, 0, 0, 0,
+    rc = sgd.lib.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv), None, None, 0, 0, 0, 0,
                                  ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000), 1 << 20,
                                  None)
     assert rc == code
@@ -72,10 +72,11 @@ def test_decode_rejects_bad_args_on_host(sgd):
     kv = _kv(sgd)
     L = sgd.lib
 
-    def call(q=0x3000, qdt=sgd.SGD_BF16, G=8, idx=None, cu_kept=None, kt=0, out=0x4000, lse=0x5000, ws=0x6000):
-        return L.sgd_decode_attn(ctypes.c_void_p(q) if q else None, qdt, G, ctypes.byref(kv),
+    def call(q=0x3000, qdt=sgd.SGD_BF16, G=8, idx=None, cu_kept=None, kt=0, out=0x4000, lse=0x5000, ws=0x6000,
+             qq=0, cache=kv):
+        return L.sgd_decode_attn(ctypes.c_void_p(q) if q else None, qdt, G, ctypes.byref(cache),
                                  ctypes.c_void_p(idx) if idx else None, ctypes.c_void_p(cu_kept) if cu_kept else None,
-                                 kt, 0, 0, ctypes.c_void_p(out) if out else None,
+                                 kt, 0, 0, qq, ctypes.c_void_p(out) if out else None,
                                  ctypes.c_void_p(lse) if lse else None, ctypes.c_void_p(ws) if ws else None,
                                  1 << 20, None)
 
@@ -87,9 +88,14 @@ def test_decode_rejects_bad_args_on_host(sgd):
     assert call(idx=0x7000, cu_kept=0x8000, kt=1) == -2  # fewer kept tokens than sequences
     assert call(q=0x3004) == -4
     kv8 = _kv(sgd, dtype=sgd.SGD_I8)
-    assert L.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv8), None, None, 0, 0, 0,
+    assert L.sgd_decode_attn(ctypes.c_void_p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv8), None, None, 0, 0, 0, 0,
                              ctypes.c_void_p(0x4000), ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000), 1 << 20,
                              None) == -1  # int8 cache without scales
+    # query codes: an INT8 cache with D = 128 and a bf16 query only; modes 0..2
+    kv8s = _kv(sgd, dtype=sgd.SGD_I8, k_scale=0x30000, v_scale=0x40000, scheme=1)
+    assert call(qq=3, cache=kv8s) == -8 and call(qq=-1, cache=kv8s) == -8
+    assert call(qq=1) == -3  # bf16 cache
+    assert call(qq=2, cache=_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x30000, v_scale=0x40000, scheme=1, D=64)) == -2
 
 
 def test_quantize_and_select_reject_bad_args_on_host(sgd):

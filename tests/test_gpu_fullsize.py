@@ -118,3 +118,14 @@ def test_config5_oam_int8a(sgd):
     ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
                         quant=(*quant, "A"), rows=rows)
     compare_rows(out, lse, *ref, rows, wl.G)
+    # the same selection decoded with INT8 query codes, one scale per (sequence, head): the
+    # query-codes workload (same sizes, q_quant = "token")
+    assert workloads.config(7).with_(name=wl.name, q_quant=None, seed=None) == wl
+    out, lse, ws = sgd.decode_attn(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                   n_parts_=sgd.n_parts(bt.lengths), idx=idx, cu_kept=cu_kept,
+                                   kept_total_=idx.shape[1], q_quant="token")
+    assert sgd.workspace_status(ws) == 0
+    qd = oracle.dequant_q(*oracle.quantize_q(bt.q, "token"))
+    ref = oracle.decode(qd, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
+                        quant=(*quant, "A"), rows=rows)
+    compare_rows(out, lse, *ref, rows, wl.G)

@@ -195,6 +195,38 @@ def test_int8_decode(sgd, scheme, G):
         check_status(sgd, ws)
 
 
+# query codes: q.k becomes an exact integer dot product of the codes times the two scales, so
+# the result is compared with the oracle attending with the dequantised query code * scale; the
+# oracle with the unquantised query must sit measurably further away (the kernel really used codes)
+@pytest.mark.parametrize("mode", ["token", "tensor"])
+@pytest.mark.parametrize("G", [8, 16])
+@pytest.mark.parametrize("indexed", [False, True])
+def test_int8_decode_query_codes(sgd, mode, G, indexed):
+    bt = make((1, 65, 700, 3000), G=G, D=128, Hkv=2, dist="outlier", seed=91 + G)
+    q, k, v, cu = dev(bt)
+    scheme = "A" if mode == "token" else "B"
+    quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme), scheme)
+    sel = {}
+    if indexed:
+        ref_idx, ref_cu, _ = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)
+        sel = dict(idx=ref_idx, cu_kept=ref_cu)
+    qd = oracle.dequant_q(*oracle.quantize_q(bt.q, mode))
+    ref = oracle.decode(qd, bt.k, bt.v, bt.cu_seqlens, G, quant=quant, **sel)
+    ref_raw = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G, quant=quant, **sel)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+    extra = {}
+    if indexed:
+        extra = dict(idx=torch.from_numpy(ref_idx).int().cuda(), cu_kept=torch.from_numpy(ref_cu).int().cuda(),
+                     kept_total_=ref_idx.shape[1])
+    for n_splits in (0, 7):
+        out, lse, ws = sgd.decode_attn(q, G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=scheme,
+                                       n_parts_=sgd.n_parts(bt.lengths), n_splits=n_splits, q_quant=mode, **extra)
+        _, lerr = assert_close(out, lse, *ref, OUT_TOL["bf16"])
+        check_status(sgd, ws)
+        gap = np.abs(ref[1] - ref_raw[1]).max()
+        assert lerr < 0.25 * gap, f"lse error {lerr:.2e} vs quantisation effect {gap:.2e}"
+
+
 def test_int8_d64_uses_cuda_core_path(sgd):
     bt = make((5, 300), G=8, D=64, Hkv=2, dist="outlier", seed=5)
     q, k, v, cu = dev(bt)

@@ -43,7 +43,7 @@ def _noalloc_via_abi(sgd, q, G, k, v, cu, **kw):
     lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=k.device)
     status = torch.full((1,), -1, dtype=torch.int32, device=k.device)
     rc = sgd.lib.sgd_decode_attn_noalloc(
-        ctypes.c_void_p(q.data_ptr()), sgd.SGD_BF16, G, ctypes.byref(kv), None, None, 0, 0, 0,
+        ctypes.c_void_p(q.data_ptr()), sgd.SGD_BF16, G, ctypes.byref(kv), None, None, 0, 0, 0, 0,
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), ctypes.c_void_p(status.data_ptr()),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     return rc, out, lse, status

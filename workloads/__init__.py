@@ -64,6 +64,8 @@ class Workload:
     keep_den: int = 8
     n_splits: int = 0  # 0 = equal-work split over all SMs; >0 forces that many CTAs
     select_on_codes: bool = False  # the cache is quantised beforehand; OAM scores its INT8 K codes
+    q_quant: Optional[str] = None  # None, "token" or "tensor": the attention's q.k runs on INT8 query codes
+    seed: Optional[int] = None  # the draw's seed when it is not the workload's number
 
     @property
     def Hq(self) -> int:
@@ -87,11 +89,15 @@ CONFIGS = {
                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True),
     6: Workload("oam_on_int8cache_A_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, select_on_codes=True),
+    # workload 5 with INT8 query codes, drawn from workload 5's seed: the same batch, so the
+    # two decode stages compare directly
+    7: Workload("oam_int8A_qcodes_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
+                dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, q_quant="token", seed=5),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..6), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..7), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
@@ -138,7 +144,7 @@ def _cast(x: np.ndarray, dtype: str) -> torch.Tensor:
 def generate(wl: Workload, seed: Optional[int] = None) -> Batch:
     """Draw one instance of ``wl`` (see the module docstring for the exact recipe)."""
     if seed is None:
-        seed = next((n for n, c in CONFIGS.items() if c.name == wl.name), 0)
+        seed = wl.seed if wl.seed is not None else next((n for n, c in CONFIGS.items() if c.name == wl.name), 0)
     streams = np.random.SeedSequence(seed).spawn(1 + 2 * wl.Hkv)
     rng = np.random.default_rng(streams[0])
     lengths = draw_lengths(wl, rng)
