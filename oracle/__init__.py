@@ -342,22 +342,26 @@ def decode_row(q, k, v, cu_seqlens, G: int, b: int, h: int, idx=None, cu_kept=No
     cache code * scale instead of k, v.  ``idx``/``cu_kept``: attend only over the kept
     tokens of the row.
     """
+    _, kr, vr = _row_kv(k, v, cu_seqlens, b, h, idx, cu_kept, quant)
+    return attend(q[b, h * G:(h + 1) * G], kr, vr)
+
+
+def _row_kv(k, v, cu_seqlens, b: int, h: int, idx=None, cu_kept=None, quant=None):
+    """The attended tokens of row (b, h): (positions in the sequence, keys [n, D], values [n, D])
+    in float64, dequantised when ``quant`` is given, restricted to the kept tokens with ``idx``."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     s0, e0 = int(cu[b]), int(cu[b + 1])
     L = e0 - s0
     sel = np.arange(L) if idx is None else np.asarray(idx[h, int(cu_kept[b]):int(cu_kept[b + 1])], np.int64)
-    qg = q[b, h * G:(h + 1) * G]
     if quant is None:
-        kr = _f64(k[h, s0:e0])[sel]
-        vr = _f64(v[h, s0:e0])[sel]
-    else:
-        kc, vc, k_scale, v_scale, scheme = quant
-        lengths = np.diff(cu)
-        cu_parts = np.concatenate([[0], np.cumsum(n_parts(lengths))])
-        ks = k_scale_of_tokens(np.asarray(k_scale), scheme, h, b, L, cu_parts)
-        kr = dequant_rows(np.asarray(kc[h, s0:e0])[sel], ks[sel])
-        vr = dequant_rows(np.asarray(vc[h, s0:e0])[sel], np.full(sel.size, np.asarray(v_scale).ravel()[0]))
-    return attend(qg, kr, vr)
+        return sel, _f64(k[h, s0:e0])[sel], _f64(v[h, s0:e0])[sel]
+    kc, vc, k_scale, v_scale, scheme = quant
+    lengths = np.diff(cu)
+    cu_parts = np.concatenate([[0], np.cumsum(n_parts(lengths))])
+    ks = k_scale_of_tokens(np.asarray(k_scale), scheme, h, b, L, cu_parts)
+    kr = dequant_rows(np.asarray(kc[h, s0:e0])[sel], ks[sel])
+    vr = dequant_rows(np.asarray(vc[h, s0:e0])[sel], np.full(sel.size, np.asarray(v_scale).ravel()[0]))
+    return sel, kr, vr
 
 
 def decode(q, k, v, cu_seqlens, G: int, idx=None, cu_kept=None, quant=None, rows=None):
@@ -379,6 +383,36 @@ def decode(q, k, v, cu_seqlens, G: int, idx=None, cu_kept=None, quant=None, rows
 
 # ----------------------------------------------------------------------------------------------
 # equal-work partition ([TD] section 5)
+def decode_multi(q, k, v, cu_seqlens, G: int, M: int, idx=None, cu_kept=None, quant=None, rows=None):
+    """Decode of M query tokens per sequence in one step (speculative verification, [CD] "decode":
+    the draft tokens raise the GEMM M dimension from G to (1 + n_draft) * G).
+
+    The M new tokens' keys and values are the last M entries of each sequence's cache, and query
+    token m (0-based) attends causally: sequence positions p <= L_b - M + m (of the kept tokens,
+    with ``idx``).  A query that sees no token gets out 0 and lse -inf.
+    q [B, M, Hq, D] -> out [B, M, Hq, D], lse [B, M, Hq] in float64 (rows not computed: NaN).
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = cu.size - 1
+    Hkv = (k if quant is None else quant[0]).shape[0]
+    D = q.shape[-1]
+    out = np.full((B, M, Hkv * G, D), np.nan)
+    lse = np.full((B, M, Hkv * G), np.nan)
+    todo = rows if rows is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for b, h in todo:
+        L = int(cu[b + 1] - cu[b])
+        pos, kr, vr = _row_kv(k, v, cu, b, h, idx, cu_kept, quant)
+        for m in range(M):
+            vis = pos <= L - M + m
+            heads = slice(h * G, (h + 1) * G)
+            if not vis.any():
+                out[b, m, heads] = 0.0
+                lse[b, m, heads] = -np.inf
+                continue
+            out[b, m, heads], lse[b, m, heads] = attend(q[b, m, heads], kr[vis], vr[vis])
+    return out, lse
+
+
 # ----------------------------------------------------------------------------------------------
 def plan(row_lengths, n_req: int, granule: int, min_chunk: int, mode: int):
     """Segments (cta, row, start, length) of the split-KV partition, and the CTA count."""

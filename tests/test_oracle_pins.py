@@ -457,3 +457,68 @@ def test_plan_covers_every_token_once_with_equal_work(seed):
     assert work.max() <= S
     one = oracle.plan(lens, 0, gran, gran, 1)
     assert one["n_cta"] == R and one["len"].tolist() == lens.tolist()
+
+
+# ---------------------------------------------------------------------------------------------
+# decode_multi: M query tokens per sequence, causal over the last M cache entries
+# ---------------------------------------------------------------------------------------------
+def _multi_batch(M, G=2, D=16, lengths=(9, 40, 3), Hkv=2, seed=3, dtype="f32"):
+    wl = workloads.Workload("tiny-multi", B=len(lengths), Hkv=Hkv, G=G, D=D, kv_dtype=dtype,
+                            dist="normal", lengths=tuple(lengths), M=M)
+    return workloads.generate(wl, seed)
+
+
+def test_multi_token_with_one_token_is_decode():
+    bt = _multi_batch(1)
+    q = bt.q[:, None]
+    out, lse = oracle.decode_multi(q, bt.k, bt.v, bt.cu_seqlens, 2, 1)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 2)
+    assert np.array_equal(out[:, 0], ref[0]) and np.array_equal(lse[:, 0], ref[1])
+
+
+@pytest.mark.parametrize("M", [2, 4])
+def test_multi_token_query_m_is_decode_over_the_truncated_cache(M):
+    # query m sees the first L - M + m + 1 tokens: the single-token decode of a repacked cache
+    # holding only that prefix of every sequence must give the same numbers
+    bt = _multi_batch(M)
+    out, lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, M)
+    cu = bt.cu_seqlens.numpy().astype(np.int64)
+    for m in range(M):
+        keep = [max(0, int(cu[b + 1] - cu[b]) - M + m + 1) for b in range(bt.wl.B)]
+        live = [b for b in range(bt.wl.B) if keep[b] > 0]
+        k = torch.cat([bt.k[:, cu[b]:cu[b] + keep[b]] for b in live], dim=1)
+        v = torch.cat([bt.v[:, cu[b]:cu[b] + keep[b]] for b in live], dim=1)
+        cu2 = np.concatenate([[0], np.cumsum([keep[b] for b in live])])
+        ref = oracle.decode(bt.q[live, m], k, v, cu2, 2)
+        assert np.array_equal(out[live, m], ref[0]) and np.array_equal(lse[live, m], ref[1])
+        for b in set(range(bt.wl.B)) - set(live):  # L < M: this query sees nothing
+            assert (out[b, m] == 0).all() and np.isneginf(lse[b, m]).all()
+
+
+def test_multi_token_matches_sdpa_with_a_causal_offset_mask():
+    M, G, D = 3, 2, 16
+    bt = _multi_batch(M, G=G, D=D, lengths=(11,), Hkv=1)
+    out, lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M)
+    L = 11
+    allowed = torch.arange(L)[None, :] <= (L - M + torch.arange(M))[:, None]  # [M, L]
+    q = bt.q[0].double().permute(1, 0, 2)  # [G, M, D]
+    kk, vv = bt.k[0].double(), bt.v[0].double()
+    ref = torch.nn.functional.scaled_dot_product_attention(q, kk[None].expand(G, -1, -1),
+                                                           vv[None].expand(G, -1, -1), attn_mask=allowed)
+    assert np.allclose(out[0], ref.permute(1, 0, 2).numpy(), atol=1e-12)
+    z = (q @ kk.T) / math.sqrt(D)
+    ref_lse = torch.logsumexp(z.masked_fill(~allowed, -math.inf), dim=-1)  # [G, M]
+    assert np.allclose(lse[0], ref_lse.T.numpy(), atol=1e-12)
+    assert allowed.sum().item() == 3 * (L - M) + 1 + 2 + 3
+
+
+def test_multi_token_over_kept_tokens_masks_by_position():
+    M = 2
+    bt = _multi_batch(M, lengths=(30,), Hkv=1)
+    idx = np.array([[0, 5, 28, 29]], np.int32)
+    cu_kept = np.array([0, 4], np.int32)
+    out, lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, M, idx=idx, cu_kept=cu_kept)
+    # query 0 sees positions 0, 5, 28; query 1 all four
+    for m, sel in ((0, [0, 5, 28]), (1, [0, 5, 28, 29])):
+        ref = oracle.attend(bt.q[0, m, 0:2], bt.k[0, sel], bt.v[0, sel])
+        assert np.array_equal(out[0, m], ref[0]) and np.array_equal(lse[0, m], ref[1])

@@ -15,7 +15,7 @@ numpy PCG64 streams: stream 0 draws, in this order,
   1. ragged lengths (only for workloads with a length range),
   2. the outlier channels of K (only for the "outlier" distribution): ``n_outlier`` distinct
      channels, the same for every head and sequence,
-  3. q, as one [B, Hq, D] float32 standard-normal draw;
+  3. q, as one [B, Hq, D] float32 standard-normal draw ([B, M, Hq, D] with M > 1 query tokens);
 stream 1 + kvh draws k[kvh] as one [T, D] float32 standard-normal draw; stream 1 + Hkv + kvh
 draws v[kvh] as one [T, D] float32 standard-normal draw followed (outlier distribution only)
 by one [T] LogNormal(0, 1) draw of per-token magnitudes s_t, V[t] = N(0,1)^D * s_t.
@@ -66,6 +66,7 @@ class Workload:
     select_on_codes: bool = False  # the cache is quantised beforehand; OAM scores its INT8 K codes
     q_quant: Optional[str] = None  # None, "token" or "tensor": the attention's q.k runs on INT8 query codes
     seed: Optional[int] = None  # the draw's seed when it is not the workload's number
+    M: int = 1  # query tokens per sequence and step (speculative decode: 1 + draft tokens)
 
     @property
     def Hq(self) -> int:
@@ -109,7 +110,7 @@ class Batch:
     seed: int
     lengths: np.ndarray  # int64 [B]
     cu_seqlens: torch.Tensor  # int32 [B+1]
-    q: torch.Tensor  # [B, Hq, D] float32 or bfloat16
+    q: torch.Tensor  # [B, Hq, D] (M = 1) or [B, M, Hq, D], float32 or bfloat16
     k: torch.Tensor  # [Hkv, T, D] float32 or bfloat16
     v: torch.Tensor  # [Hkv, T, D]
     outlier_channels: Optional[np.ndarray]
@@ -158,7 +159,8 @@ def generate(wl: Workload, seed: Optional[int] = None) -> Batch:
         outl = np.sort(rng.choice(wl.D, size=wl.n_outlier, replace=False))
     elif wl.dist != "normal":
         raise ValueError(f"unknown distribution {wl.dist}")
-    q = _cast(rng.standard_normal((wl.B, wl.Hq, wl.D), dtype=np.float32),
+    qshape = (wl.B, wl.Hq, wl.D) if wl.M == 1 else (wl.B, wl.M, wl.Hq, wl.D)
+    q = _cast(rng.standard_normal(qshape, dtype=np.float32),
               "f32" if wl.kv_dtype == "f32" else "bf16")
     tdt = torch.float32 if wl.kv_dtype == "f32" else torch.bfloat16
     k = torch.empty((wl.Hkv, T, wl.D), dtype=tdt)
