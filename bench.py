@@ -41,7 +41,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -83,7 +83,7 @@ def algorithmic_bytes(wl, lengths):
         idx_bytes = 0
     eb = 1 if wl.scheme else 2
     scales = (Hkv * P * 4 if wl.scheme == "A" else 8) if wl.scheme else 0
-    st["decode"] = 2 * Hkv * n_att * D * eb + idx_bytes + scales + q + out
+    st["decode"] = 2 * Hkv * n_att * D * eb + idx_bytes + scales + wl.M * (q + out)  # M query tokens
     return st
 
 
@@ -216,7 +216,8 @@ class Pipeline:
         else:
             kc, vc, ks, vs = self.k, self.v, None, None
         ev("decode", 0)
-        o, lse, self.ws_d = sgd.decode_attn(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
+        decode = sgd.decode_attn if wl.M == 1 else sgd.decode_attn_multi
+        o, lse, self.ws_d = decode(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
                                             scheme=wl.scheme or "A", n_parts_=self.parts, idx=idx,
                                             cu_kept=cu_kept, kept_total_=Kt, out=self.dec_out,
                                             workspace=self.ws_d, q_quant=wl.q_quant or "none")
@@ -280,7 +281,7 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
         kk = bt.k[h:h + 1, s:e]
         vv = bt.v[h:h + 1, s:e]
         one = np.array([0, L], np.int64)
-        qrow = bt.q[b:b + 1, h * wl.G:(h + 1) * wl.G]
+        qrow = bt.q[b:b + 1, ..., h * wl.G:(h + 1) * wl.G, :]  # [1, (M,) G, D]
         quant = None
         if wl.scheme:
             quant = oracle.quantize_kv(kk, vv, one, wl.scheme)
@@ -293,8 +294,12 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
                                                 wl.keep_den)
         if wl.q_quant:  # the attention sees the query's code * scale
             qrow = oracle.dequant_q(*oracle.quantize_q(qrow, wl.q_quant))
-        oracle.decode(qrow, kk, vv, one, wl.G, idx=idx, cu_kept=cu_kept,
-                      quant=None if quant is None else (*quant, wl.scheme))
+        if wl.M > 1:
+            oracle.decode_multi(qrow, kk, vv, one, wl.G, wl.M, idx=idx, cu_kept=cu_kept,
+                                quant=None if quant is None else (*quant, wl.scheme))
+        else:
+            oracle.decode(qrow, kk, vv, one, wl.G, idx=idx, cu_kept=cu_kept,
+                          quant=None if quant is None else (*quant, wl.scheme))
         done.append((b, h, L))
         rowwl = wl.with_(B=1, Hkv=1, lengths=(L,), length_range=None)
         nbytes += sum(algorithmic_bytes(rowwl, [L]).values())
@@ -406,9 +411,8 @@ def run_ours(args, rank, world, local_rank):
     # e2e: host buffers through the same calls, copies inside the timed region
     dev_in = pipe.inputs()
     pin_in = [x.cpu().pin_memory() for x in dev_in]
-    B, Hq, D = bt.q.shape
-    h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
-    h_lse = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    h_out = torch.empty(tuple(bt.q.shape), dtype=torch.float32).pin_memory()  # [B, (M,) Hq, D]
+    h_lse = torch.empty(tuple(bt.q.shape[:-1]), dtype=torch.float32).pin_memory()
     h2d = sum(x.numel() * x.element_size() for x in pin_in)
     d2h = h_out.numel() * 4 + h_lse.numel() * 4
     e2e_steps = max(2, min(K, 5))
@@ -464,6 +468,7 @@ def run_ours(args, rank, world, local_rank):
             "workload": wl.name, "B": wl.B, "Hkv": wl.Hkv, "G": wl.G, "D": wl.D, "lengths": pipe.lengths,
             "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
             "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": wl.seed if wl.seed is not None else args.workload, "q_quant": wl.q_quant,
+            "query_tokens": wl.M,
             "step": ("oam_select(int8 cache, stored norms) -> decode_attn(kept); cache quantised once, untimed"
                      if wl.select_on_codes else
                      "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn"),

@@ -193,6 +193,24 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                     int schedule, int n_splits, int q_quant, float *out, float *lse,
                     void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * sgd_decode_attn_multi -- M query tokens per sequence in one step ([CD] "decode": speculative
+ * decoding verifies n_draft drafted tokens at once, raising the GEMM M dimension of decode from
+ * G to (1 + n_draft) * G).  The M new tokens' keys and values are the last M entries of each
+ * sequence's cache; query token m (0-based) attends causally, to sequence positions
+ * p <= L_b - M + m (of the kept tokens when idx is given).  A query token that sees no token
+ * (L_b < M - m) gets out = 0 and lse = -inf.  M = 1 is sgd_decode_attn.
+ * q        [B, M, Hq, D] BF16;  out [B, M, Hq, D] float32;  lse [B, M, Hq] float32
+ * M        1 <= M and G * M <= 16; with M > 1 the cache is BF16 (D 64 or 128) or I8 (D 128)
+ *          (SGD_ERR_DTYPE otherwise)
+ * workspace   sgd_workspace_size(SGD_OP_DECODE, kv, G * M, schedule, n_splits) bytes
+ * Every other argument, and the error behaviour, as in sgd_decode_attn.
+ */
+int sgd_decode_attn_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv,
+                          const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
+                          int schedule, int n_splits, int q_quant, float *out, float *lse,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* Workspace bytes an operation needs for this cache shape (>= 256). For
  * SGD_OP_DECODE, `schedule` and `n_splits` as in sgd_decode_attn; for the
  * other ops they are ignored.  Returns 0 on invalid arguments. */

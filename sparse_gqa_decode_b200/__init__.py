@@ -66,6 +66,8 @@ lib.sgd_decode_num_ctas.argtypes = [_kvp, _i32, _vp, _i32, _i32]
 lib.sgd_quantize_kv.argtypes = [_kvp, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
+lib.sgd_decode_attn_multi.argtypes = [_vp, _i32, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp,
+                                      _sz, _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
@@ -238,6 +240,29 @@ def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_se
                                int(kept_total_), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse), _ptr(ws),
                                ws.numel(),
                                _stream(stream)), "sgd_decode_attn")
+    return o, lse, ws
+
+
+def decode_attn_multi(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                      k_scale=None, v_scale=None, scheme: str = "A", n_parts_: int = 0,
+                      idx=None, cu_kept=None, kept_total_: int = 0, schedule: int = 0, n_splits: int = 0,
+                      out=None, workspace=None, stream=None, q_quant: str = "none"):
+    """M query tokens per sequence, q [B, M, Hq, D]; token m attends causally to positions
+    <= L_b - M + m.  Returns (out [B, M, Hq, D] f32, lse [B, M, Hq] f32, ws)."""
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, sch, n_parts_)
+    B, M = q.shape[0], q.shape[1]
+    Hq = k.shape[0] * G
+    D = k.shape[2]
+    if out is None:
+        o = torch.empty((B, M, Hq, D), dtype=torch.float32, device=k.device)
+        lse = torch.empty((B, M, Hq), dtype=torch.float32, device=k.device)
+    else:
+        o, lse = out
+    ws = _workspace(workspace_size(OP_DECODE, kv, G * M, schedule, n_splits), k.device, workspace)
+    _check(lib.sgd_decode_attn_multi(_ptr(q), _DT[q.dtype], G, M, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
+                                     int(kept_total_), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse),
+                                     _ptr(ws), ws.numel(), _stream(stream)), "sgd_decode_attn_multi")
     return o, lse, ws
 
 

@@ -266,6 +266,7 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
     a.B = kv->B;
     a.Hkv = kv->Hkv;
     a.G = G;
+    a.M = 1;
     a.D = kv->D;
     a.T = kv->T;
     a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
@@ -338,6 +339,7 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     a.B = kv->B;
     a.Hkv = kv->Hkv;
     a.G = G;
+    a.M = 1;
     a.D = kv->D;
     a.T = kv->T;
     a.n_parts = scheme == SGD_SCHEME_A ? n_parts : 0;
@@ -365,10 +367,20 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
 int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, const int32_t *idx,
                     const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, int q_quant, float *out,
                     float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    return sgd_decode_attn_multi(q, q_dtype, G, 1, kv, idx, cu_kept, kept_total, schedule, n_splits, q_quant, out,
+                                 lse, workspace, workspace_bytes, stream);
+}
+
+int sgd_decode_attn_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, const int32_t *idx,
+                          const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, int q_quant,
+                          float *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
-    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
+    const int NC = G * M;  // the kernels' columns per KV head: (query token, head) pairs
+    // several query tokens run on the tensor-core kernel only
+    if (M > 1 && decode_family(kv->dtype, q_dtype, kv->D, false) != kFamilyMma) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (q_dtype == SGD_F32 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
     const bool indexed = idx != nullptr;
@@ -389,8 +401,8 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     DevInfo *dev;
     if ((rc = current_device(&dev)) != SGD_OK) return rc;
     int n_req = 0;
-    if ((rc = decode_n_req(*dev, kv, q_dtype, G, indexed, false, schedule, n_splits, &n_req)) != SGD_OK) return rc;
-    const Layout L = layout(SGD_OP_DECODE, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if ((rc = decode_n_req(*dev, kv, q_dtype, NC, indexed, false, schedule, n_splits, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_DECODE, kv->B, kv->Hkv, NC, kv->D, kv->T, n_req);
     if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
@@ -399,7 +411,7 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     const int min_chunk = (n_splits > 0 || schedule == 1) ? kGranule : kAutoMinChunk;
     launch_plan(indexed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
                 hdr, s, kGranule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
-                (int64_t)kv->B * kv->Hkv * G * kv->D);
+                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M);
     DecodeArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q;
@@ -415,6 +427,7 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
     a.B = kv->B;
     a.Hkv = kv->Hkv;
     a.G = G;
+    a.M = M;
     a.D = kv->D;
     a.T = kv->T;
     a.Kt = indexed ? kept_total : 0;

@@ -52,11 +52,12 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 
 constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
 
-template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false>
+template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false, bool CAUSAL_ = false>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
     static constexpr bool QI8 = QI8_;  // INT8 query codes: S^T = K_codes . Q_codes^T on s8 MMAs
+    static constexpr bool CAUSAL = CAUSAL_;  // several query tokens: causal limit per column
     static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
     static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static constexpr int NW = 4;        // consumer warps
@@ -84,6 +85,7 @@ struct MmaCfg {
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
     static_assert(!QI8 || (I8 && MODE == 0 && D == 128), "query codes meet INT8 keys in the decode");
+    static_assert(!CAUSAL || MODE == 0, "several query tokens: decode only");
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
@@ -201,18 +203,23 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
 // ------------------------------------------------------------------------------------------
 // consumer helpers
 // ------------------------------------------------------------------------------------------
+// Element offset of column n's row in q [B, M, Hq, D] (and out): the columns of KV head kvh are
+// its M * G (query token, head) pairs, n = m * G + g.
+__device__ __forceinline__ int64_t col_row(const DecodeArgs &a, int b, int kvh, int n) {
+    const int m = (a.M == 1) ? 0 : n / a.G, g = n - m * a.G;
+    return (((int64_t)b * a.M + m) * a.Hkv + kvh) * a.G + g;
+}
+
 // Q of one KV group as MMA B fragments (k <-> d order matching the K fragments) and the
 // per-column logit factor (log2 units; INT8 also undoes the power-of-two Q pre-scale).
 template <class C>
 __device__ __forceinline__ void load_q_frags(const DecodeArgs &a, int b, int kvh, int g4, int t4,
                                              uint32_t (&qf)[C::GT][C::KB][2], float (&colf)[C::GT][2]) {
-    const int Hq = a.Hkv * a.G;
 #pragma unroll
     for (int gt = 0; gt < C::GT; ++gt) {
         const int g = 8 * gt + g4;
-        const bool live = g < a.G;
-        const __nv_bfloat16 *qrow =
-            static_cast<const __nv_bfloat16 *>(a.q) + ((int64_t)b * Hq + kvh * a.G + (live ? g : 0)) * C::D;
+        const bool live = g < a.G * a.M;
+        const __nv_bfloat16 *qrow = static_cast<const __nv_bfloat16 *>(a.q) + col_row(a, b, kvh, live ? g : 0) * C::D;
         if constexpr (!C::I8) {
 #pragma unroll
             for (int h = 0; h < C::KB / 2; ++h) {
@@ -613,18 +620,20 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
 template <class C>
 __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n, int b, int kvh, float *scratch) {
     constexpr int NT = C::NW * 32;
-    const int G = a.G, tid = threadIdx.x;
+    const int G = a.G * a.M, tid = threadIdx.x;  // G here: the row's columns, (query token, head) pairs
     float *Ls = scratch;                       // [16] per head: running max, then the lse
     float *Ss = scratch + 16;                  // [16] running sum
     float *w = scratch + 32;                   // [chunk][G] lse, then weights
     const int chunk = (2 * C::TILE / 4 - 32) / G;
     const float *lp = a.lse_part + (int64_t)slot0 * G;
     const float *op = a.o_part + (int64_t)slot0 * G * C::D;
-    const int Hq = a.Hkv * G;
-    float *dst = a.out + ((int64_t)b * Hq + kvh * G) * C::D;
-    constexpr int kQ4 = 16 * C::D / 4 / NT;  // float4 columns per thread at G = 16
+    constexpr int kQ4 = C::NG * C::D / 4 / NT;  // float4 columns per thread at the most columns
     const int Q = G * C::D / 4;
-    float4 *dst4 = reinterpret_cast<float4 *>(dst);
+    // float4 q of the row's [G][D] block -> its place in out (column n = 4q / D)
+    auto dst4 = [&](int q) -> float4 & {
+        const int n = (4 * q) / C::D;
+        return *reinterpret_cast<float4 *>(a.out + col_row(a, b, kvh, n) * C::D + (4 * q - n * C::D));
+    };
     if (n <= chunk) {
         // one round: every lse loaded once, the weights computed in place, then thread t reads
         // its float4 columns t, t + NT, ... of every slot, eight slots' loads in flight
@@ -633,11 +642,12 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
         if (tid < G) {
             float M = -INFINITY, S = 0.f;
             for (int c = 0; c < n; ++c) M = fmaxf(M, w[c * G + tid]);
-            for (int c = 0; c < n; ++c) S += expf(w[c * G + tid] - M);
-            Ls[tid] = (n > 0) ? M + logf(S) : -INFINITY;
+            if (M > -INFINITY)  // else no partial saw a token (a query token past a short row)
+                for (int c = 0; c < n; ++c) S += expf(w[c * G + tid] - M);
+            Ls[tid] = (S > 0.f) ? M + logf(S) : -INFINITY;
         }
         named_barrier_sync(1, NT);
-        for (int p = tid; p < n * G; p += NT) w[p] = expf(w[p] - Ls[p % G]);
+        for (int p = tid; p < n * G; p += NT) w[p] = (Ls[p % G] > -INFINITY) ? expf(w[p] - Ls[p % G]) : 0.f;
         named_barrier_sync(1, NT);
         const float4 *oc = reinterpret_cast<const float4 *>(op);
         float4 acc[kQ4];
@@ -661,9 +671,9 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
 #pragma unroll
         for (int j = 0; j < kQ4; ++j) {
             const int q = tid + j * NT;
-            if (q < Q) dst4[q] = acc[j];
+            if (q < Q) dst4(q) = acc[j];
         }
-        if (tid < G) a.lse[(int64_t)b * Hq + kvh * G + tid] = Ls[tid];
+        if (tid < G) a.lse[col_row(a, b, kvh, tid)] = Ls[tid];
         named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
         return;
     }
@@ -685,7 +695,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
                 if (x > M) {
                     S = S * expf(M - x) + 1.f;
                     M = x;
-                } else {
+                } else if (x > -INFINITY) {
                     S += expf(x - M);
                 }
             }
@@ -694,20 +704,21 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
         }
     }
     named_barrier_sync(1, NT);
-    if (tid < G) Ls[tid] = (n > 0) ? Ls[tid] + logf(Ss[tid]) : -INFINITY;
+    if (tid < G) Ls[tid] = (Ss[tid] > 0.f) ? Ls[tid] + logf(Ss[tid]) : -INFINITY;
     // pass 2: thread t owns float4 columns t, t + NT, ... of the row's [G][D] block and reads
     // them from every slot of a chunk, kQ4 * 4 independent 16-byte loads in flight
     for (int c0 = 0; c0 < n; c0 += chunk) {
         const int m = min(chunk, n - c0);
         named_barrier_sync(1, NT);
-        for (int p = tid; p < m * G; p += NT) w[p] = expf(__ldcg(lp + (int64_t)c0 * G + p) - Ls[p % G]);
+        for (int p = tid; p < m * G; p += NT)
+            w[p] = (Ls[p % G] > -INFINITY) ? expf(__ldcg(lp + (int64_t)c0 * G + p) - Ls[p % G]) : 0.f;
         named_barrier_sync(1, NT);
         const float4 *oc = reinterpret_cast<const float4 *>(op + (int64_t)c0 * G * C::D);
         float4 acc[kQ4];
 #pragma unroll
         for (int j = 0; j < kQ4; ++j) {
             const int q = tid + j * NT;
-            acc[j] = (c0 > 0 && q < Q) ? dst4[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+            acc[j] = (c0 > 0 && q < Q) ? dst4(q) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll 4
         for (int c = 0; c < m; ++c) {
@@ -727,10 +738,10 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
 #pragma unroll
         for (int j = 0; j < kQ4; ++j) {
             const int q = tid + j * NT;
-            if (q < Q) dst4[q] = acc[j];
+            if (q < Q) dst4(q) = acc[j];
         }
     }
-    if (tid < G) a.lse[(int64_t)b * Hq + kvh * G + tid] = Ls[tid];
+    if (tid < G) a.lse[col_row(a, b, kvh, tid)] = Ls[tid];
     named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
 }
 
@@ -856,6 +867,28 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 float sacc[C::GT][4];
                 qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
                 const bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
+                // several query tokens: token m sees sequence positions <= L_b - M + m; bit 4 gt + e
+                // keeps element e of column tile gt (only sub-tiles reaching the last M - 1
+                // positions mask anything)
+                uint32_t cm = ~0u;
+                if constexpr (C::CAUSAL) {
+                    int32_t pa = j0 + pA, pb = pa + 8;
+                    if constexpr (C::IDX) {
+                        pa = vA ? __ldg(ip + j0 + pA) : 0;
+                        pb = vB ? __ldg(ip + j0 + pA + 8) : 0;
+                    }
+                    const int32_t lim0 = Lb - a.M;
+                    if (__any_sync(0xffffffffu, max(pa, pb) > lim0)) {
+                        cm = 0u;
+#pragma unroll
+                        for (int gt = 0; gt < C::GT; ++gt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int32_t lim = lim0 + (8 * gt + 2 * t4 + (e & 1)) / a.G;
+                                cm |= (uint32_t)((e < 2 ? pa : pb) <= lim) << (4 * gt + e);
+                            }
+                    }
+                }
                 {
                     // row (token) factors: scheme-A K scale of the token's 64-token partition
                     float rfA = rf_pre[s], rfB = rf_pre[s];
@@ -868,10 +901,17 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                     uint32_t pb[C::GT][2];
 #pragma unroll
                     for (int gt = 0; gt < C::GT; ++gt) {
-                        const float z0 = vA ? sacc[gt][0] * rfA * colf[gt][0] : -INFINITY;
-                        const float z1 = vA ? sacc[gt][1] * rfA * colf[gt][1] : -INFINITY;
-                        const float z2 = vB ? sacc[gt][2] * rfB * colf[gt][0] : -INFINITY;
-                        const float z3 = vB ? sacc[gt][3] * rfB * colf[gt][1] : -INFINITY;
+                        bool k0 = vA, k1 = vA, k2 = vB, k3 = vB;
+                        if constexpr (C::CAUSAL) {
+                            k0 = k0 && (cm >> (4 * gt) & 1u);
+                            k1 = k1 && (cm >> (4 * gt + 1) & 1u);
+                            k2 = k2 && (cm >> (4 * gt + 2) & 1u);
+                            k3 = k3 && (cm >> (4 * gt + 3) & 1u);
+                        }
+                        const float z0 = k0 ? sacc[gt][0] * rfA * colf[gt][0] : -INFINITY;
+                        const float z1 = k1 ? sacc[gt][1] * rfA * colf[gt][1] : -INFINITY;
+                        const float z2 = k2 ? sacc[gt][2] * rfB * colf[gt][0] : -INFINITY;
+                        const float z3 = k3 ? sacc[gt][3] * rfB * colf[gt][1] : -INFINITY;
                         float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
 #pragma unroll
                         for (int off = 4; off < 32; off <<= 1) {
@@ -950,7 +990,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
                 named_barrier_sync(1, C::NW * 32);
                 const int tid = threadIdx.x;
-                if (tid < a.G) {  // head g: the warps' weights replace their m in ml; the lse replaces warp 0's l
+                const int NC = a.G * a.M;  // columns: (query token, head) pairs
+                if (tid < NC) {  // column n: the warps' weights replace their m in ml; the lse replaces warp 0's l
                     float M = -INFINITY, f[C::NW], L = 0.f;
 #pragma unroll
                     for (int w = 0; w < C::NW; ++w) M = fmaxf(M, ml[(w * C::NG + tid) * 2]);
@@ -967,20 +1008,19 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 named_barrier_sync(1, C::NW * 32);
                 // a row's only segment is its result; otherwise a partial in the segment's slot
                 const bool direct = cur.ri.nseg == 1;
-                const int Hq = a.Hkv * a.G;
-                float *dst = direct ? a.out + ((int64_t)b * Hq + kvh * a.G) * C::D
-                                    : a.o_part + (int64_t)slot * a.G * C::D;
-                for (int e = tid; e < a.G * C::D; e += C::NW * 32) {
+                float *part = a.o_part + (int64_t)slot * NC * C::D;
+                for (int e = tid; e < NC * C::D; e += C::NW * 32) {
                     const int g = e / C::D, d = e - g * C::D;
                     float O = 0.f;
 #pragma unroll
                     for (int w = 0; w < C::NW; ++w) O += ml[(w * C::NG + g) * 2] * eo[(w * C::NG + g) * C::D + d];
-                    dst[e] = O;
+                    if (direct) a.out[col_row(a, b, kvh, g) * C::D + d] = O;
+                    else part[e] = O;
                 }
-                if (tid < a.G) {
+                if (tid < NC) {
                     const float lv = ml[tid * 2 + 1];
-                    if (direct) a.lse[(int64_t)b * Hq + kvh * a.G + tid] = lv;
-                    else a.lse_part[(int64_t)slot * a.G + tid] = lv;
+                    if (direct) a.lse[col_row(a, b, kvh, tid)] = lv;
+                    else a.lse_part[(int64_t)slot * NC + tid] = lv;
                 }
                 if (!direct) {
                     // the CTA that finishes the row's last outstanding segment merges the row
@@ -1294,6 +1334,9 @@ template <int D, int GT, bool I8, int MODE, bool QI8 = false>
 static int launch_mma_idx(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
     if constexpr (MODE == 1) {
         return launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
+    } else if (a.M > 1) {  // several query tokens per sequence: the causally masked instantiation
+        return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE, QI8, true>>(a, n_cta, s)
+                       : launch_mma<MmaCfg<D, GT, I8, false, MODE, QI8, true>>(a, n_cta, s);
     } else {
         return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE, QI8>>(a, n_cta, s)
                        : launch_mma<MmaCfg<D, GT, I8, false, MODE, QI8>>(a, n_cta, s);
@@ -1342,7 +1385,7 @@ int score_quantize_ctas_per_sm(int D, int G) {
 int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, bool score, int n_cta,
                   cudaStream_t s) {
     if (n_cta <= 0) return 0;
-    const bool g2 = a.G > 8;
+    const bool g2 = a.G * a.M > 8;  // columns: (query token, head) pairs of a KV head
     if (decode_family(kv, q, a.D, score) == kFamilyMma) {
         if (score) {
             if (kv == SGD_I8) return g2 ? launch_mma_idx<128, 2, true, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, true, 1>(a, false, n_cta, s);

@@ -7,7 +7,7 @@ namespace sgd {
 
 // Arguments of the decode / score kernels (device pointers unless noted).
 struct DecodeArgs {
-    const void *q;           // [B, Hq, D]
+    const void *q;           // [B, M, Hq, D]
     const int32_t *cu_seq;   // cu_seqlens [B+1]
     const int32_t *cu_kept;  // kept-set prefix sums [B+1] (indexed mode)
     const int32_t *idx;      // [Hkv, Kt] kept positions (indexed mode)
@@ -18,6 +18,8 @@ struct DecodeArgs {
     int q_quant;             // I8 decode: 0 bf16 query, 1 query codes per (sequence, head), 2 per tensor
     const float *q_scale;    // q_quant == 2: the per-tensor query scale (in the workspace header)
     int B, Hkv, G, D;
+    int M;                   // decode: query tokens per sequence (>= 1), causal over the cache's last M;
+                             // the kernel's columns are the M * G (token, head) pairs of a KV head
     int64_t T, Kt, n_parts;
     int q_f32;               // q is float32 (otherwise bf16)
     float sm_scale_log2;     // log2(e) / sqrt(D)
@@ -31,10 +33,10 @@ struct DecodeArgs {
     float *k_scale_out;      // [Hkv, n_parts]
     uint32_t *amax_bits;     // [2]: max|K| (scheme B), max|V| as float bits
     PlanView plan;
-    float *o_part;           // [slots, G, D]
-    float *lse_part;         // [slots, G]
-    float *out;              // decode: [B, Hq, D] result (written by the kernel itself on the MMA path)
-    float *lse;              // decode: [B, Hq]
+    float *o_part;           // [slots, M * G, D]
+    float *lse_part;         // [slots, M * G]
+    float *out;              // decode: [B, M, Hq, D] result (written by the kernel itself on the MMA path)
+    float *lse;              // decode: [B, M, Hq]
     int32_t *status;
 };
 
@@ -44,10 +46,11 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 // plan.cu
 // out/lse (decode only, else NULL): rows without tokens get out = 0 and lse = -inf here.
 // q_bf16 (decode with a per-tensor query scale, else NULL): hdr->q_scale = max|q| / 127.
+// M: query tokens per sequence of the decode (out is [B, M, Hkv * G, D]).
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
                  float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0, const void *q_bf16 = nullptr,
-                 int64_t q_elems = 0);
+                 int64_t q_elems = 0, int M = 1);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 

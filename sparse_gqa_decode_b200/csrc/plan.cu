@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
                                                     int n_req, int min_chunk, int mode, int granule,
                                                     PlanView pv, WsHeader *hdr, int staged, float *out,
                                                     float *lse, int G, int D, const __nv_bfloat16 *q,
-                                                    int64_t q_elems) {
+                                                    int64_t q_elems, int M) {
     __shared__ int32_t sm[33];
     extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
@@ -162,9 +162,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
             ri[1] = make_int4(len_start_of(b), part0[b], carry + ex, v);
             if (pv.row_done) pv.row_done[r] = 0;
             if (out && v == 0) {  // a row with no tokens (reported above): zero output, lse -inf
-                const int64_t h0 = (int64_t)b * Hkv * G + (r / B) * G;
-                for (int e = 0; e < G * D; ++e) out[h0 * D + e] = 0.f;
-                for (int g = 0; g < G; ++g) lse[h0 + g] = -INFINITY;
+                for (int m = 0; m < M; ++m) {
+                    const int64_t h0 = ((int64_t)b * M + m) * Hkv * G + (r / B) * G;
+                    for (int e = 0; e < G * D; ++e) out[h0 * D + e] = 0.f;
+                    for (int g = 0; g < G; ++g) lse[h0 + g] = -INFINITY;
+                }
             }
         }
         carry += total;
@@ -211,7 +213,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
-                 int G, int D, const void *q_bf16, int64_t q_elems) {
+                 int G, int D, const void *q_bf16, int64_t q_elems, int M) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
@@ -220,7 +222,7 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
     const int nt = std::min(1024, std::max(64, (want + 31) / 32 * 32));
     launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
              min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D,
-             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems);
+             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

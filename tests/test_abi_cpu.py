@@ -26,7 +26,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("sgd_oam_select", "sgd_quantize_kv", "sgd_decode_attn", "sgd_workspace_size",
-                     "sgd_error_string", "sgd_plan_segments", "sgd_workspace_status"):
+                     "sgd_error_string", "sgd_plan_segments", "sgd_workspace_status", "sgd_decode_attn_multi"):
         assert required in names
 
 
@@ -96,6 +96,20 @@ def test_decode_rejects_bad_args_on_host(sgd):
     assert call(qq=3, cache=kv8s) == -8 and call(qq=-1, cache=kv8s) == -8
     assert call(qq=1) == -3  # bf16 cache
     assert call(qq=2, cache=_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x30000, v_scale=0x40000, scheme=1, D=64)) == -2
+
+
+def test_multi_token_decode_rejects_bad_args_on_host(sgd):
+    L = sgd.lib
+    p = ctypes.c_void_p
+
+    def call(G=8, M=2, cache=None, qdt=sgd.SGD_BF16):
+        kv = cache or _kv(sgd)
+        return L.sgd_decode_attn_multi(p(0x3000), qdt, G, M, ctypes.byref(kv), None, None, 0, 0, 0, 0, p(0x4000),
+                                       p(0x5000), p(0x6000), 1 << 20, None)
+
+    assert call(M=0) == -2 and call(M=3) == -2 and call(G=16, M=2) == -2  # G * M <= 16
+    assert call(cache=_kv(sgd, dtype=sgd.SGD_F32), qdt=sgd.SGD_F32) == -3  # tensor-core path only
+    assert call(cache=_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x30000, v_scale=0x40000, scheme=1, D=64)) == -3
 
 
 def test_quantize_and_select_reject_bad_args_on_host(sgd):

@@ -465,3 +465,100 @@ def test_empty_sequence_is_reported(sgd):
     out, lse, ws = sgd.decode_attn(q3, 8, k, v, cu)
     assert sgd.workspace_status(ws) & 0x1
     assert torch.isinf(lse[1]).all() and (out[1] == 0).all()
+
+
+# ---------------------------------------------------------------------------------------------
+# multi-token (speculative) decode: M query tokens per sequence, causal over the last M entries
+# ---------------------------------------------------------------------------------------------
+def make_multi(lengths, M, G, D=128, Hkv=2, dist="outlier", seed=0):
+    wl = workloads.Workload("t-multi", B=len(lengths), Hkv=Hkv, G=G, D=D, kv_dtype="bf16", dist=dist,
+                            lengths=tuple(lengths), M=M)
+    return workloads.generate(wl, seed)
+
+
+def assert_close_multi(out, lse, ref_out, ref_lse, tol):
+    """Queries that see no token: exactly out 0 and lse -inf; the rest as assert_close."""
+    o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
+    blind = np.isneginf(ref_lse)
+    assert np.isneginf(l[blind]).all() and (o[blind] == 0).all()
+    seen = ~blind
+    scale = np.abs(ref_out[seen]).max()
+    err = np.abs(o[seen] - ref_out[seen]).max()
+    lerr = np.abs(l[seen] - ref_lse[seen]).max()
+    assert err <= tol * scale, f"out error {err:.3e} > {tol} * {scale:.3e}"
+    assert lerr <= LSE_TOL, f"lse error {lerr:.3e}"
+
+
+def kept_with_tail(lengths, Hkv, M, seed):
+    """A seeded kept set per (sequence, KV head): a random eighth of the positions plus the last
+    M (so the causal limit cuts through kept tokens), ascending."""
+    rng = np.random.default_rng(seed)
+    rows, counts = {}, []
+    for b, L in enumerate(lengths):
+        K = max(min(L, M), (L + 7) // 8)
+        counts.append(K)
+        for h in range(Hkv):
+            tail = np.arange(max(0, L - M), L)
+            rest = np.setdiff1d(np.arange(L), tail)
+            pick = rng.choice(rest, size=K - tail.size, replace=False) if K > tail.size else []
+            rows[(b, h)] = np.sort(np.concatenate([tail, pick]).astype(np.int32))
+    cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    idx = np.zeros((Hkv, int(cu[-1])), np.int32)
+    for (b, h), r in rows.items():
+        idx[h, cu[b]:cu[b + 1]] = r
+    return idx, cu
+
+
+@pytest.mark.parametrize("kvdt", ["bf16", "int8A"])
+@pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (16, 1)])
+@pytest.mark.parametrize("indexed", [False, True])
+def test_multi_token_decode(sgd, kvdt, M, G, indexed):
+    lengths = (1, 3, 70, 700, 3001)
+    bt = make_multi(lengths, M, G, seed=31 + M)
+    q, k, v, cu = dev(bt)
+    sel, extra = {}, {}
+    if indexed:
+        idx, cu_kept = kept_with_tail(lengths, 2, M, seed=7)
+        sel = dict(idx=idx, cu_kept=cu_kept)
+        extra = dict(idx=torch.from_numpy(idx).cuda(), cu_kept=torch.from_numpy(cu_kept).cuda(),
+                     kept_total_=idx.shape[1])
+    quant, kw = None, {}
+    kk, vv = k, v
+    if kvdt == "int8A":
+        quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A"), "A")
+        kk, vv, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+        kw = dict(k_scale=ks, v_scale=vs, scheme="A", n_parts_=sgd.n_parts(bt.lengths))
+    ref = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, quant=quant, **sel)
+    for n_splits in (0, 7, 300):
+        out, lse, ws = sgd.decode_attn_multi(q, G, kk, vv, cu, n_splits=n_splits, **kw, **extra)
+        assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
+        check_status(sgd, ws)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_multi_token_bf16_head_dims_and_one_token_equals_decode(sgd, D):
+    bt = make_multi((5, 129, 1000), 2, 8, D=D, dist="normal", seed=3)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 2)
+    out, lse, _ = sgd.decode_attn_multi(q, 8, k, v, cu)
+    assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
+    # M = 1 through the multi entry is the single-token decode, bit for bit
+    q1 = q[:, :1].contiguous()
+    o1, l1, _ = sgd.decode_attn_multi(q1, 8, k, v, cu)
+    o0, l0, _ = sgd.decode_attn(q1[:, 0].contiguous(), 8, k, v, cu)
+    assert torch.equal(o1[:, 0], o0) and torch.equal(l1[:, 0], l0)
+
+
+def test_multi_token_with_query_codes(sgd):
+    M, G = 2, 8
+    lengths = (2, 90, 2500)
+    bt = make_multi(lengths, M, G, seed=77)
+    q, k, v, cu = dev(bt)
+    quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A"), "A")
+    qd = oracle.dequant_q(*oracle.quantize_q(bt.q.reshape(len(lengths) * M, 2 * G, 128), "token"))
+    ref = oracle.decode_multi(qd.reshape(len(lengths), M, 2 * G, 128), bt.k, bt.v, bt.cu_seqlens, G, M, quant=quant)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    out, lse, ws = sgd.decode_attn_multi(q, G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                         n_parts_=sgd.n_parts(bt.lengths), n_splits=9, q_quant="token")
+    assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)

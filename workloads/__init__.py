@@ -94,11 +94,14 @@ CONFIGS = {
     # two decode stages compare directly
     7: Workload("oam_int8A_qcodes_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, q_quant="token", seed=5),
+    # workload 4 with two query tokens per sequence (one draft token): 16 columns per KV head
+    8: Workload("spec_M2_int8_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                lengths=(131072,) * 8, scheme="A", M=2, seed=4),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..7), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..8), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
