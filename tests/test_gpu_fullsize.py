@@ -129,3 +129,21 @@ def test_config5_oam_int8a(sgd):
     ref = oracle.decode(qd, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
                         quant=(*quant, "A"), rows=rows)
     compare_rows(out, lse, *ref, rows, wl.G)
+
+
+def test_config8_two_query_tokens_int8_128k(sgd):
+    # the speculative-decode workload: workload 4's cache, two query tokens per sequence
+    wl = workloads.config(8)
+    bt = workloads.generate(wl)
+    assert bt.q.shape == (wl.B, 2, wl.Hq, wl.D)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, wsq = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    del k, v
+    out, lse, ws = sgd.decode_attn_multi(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                         n_parts_=sgd.n_parts(bt.lengths))
+    assert sgd.workspace_status(wsq) == 0 and sgd.workspace_status(ws) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    rows = sample_rows(bt, n_extra=1)
+    ref_out, ref_lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, 2, quant=(*quant, "A"), rows=rows)
+    for m in range(2):
+        compare_rows(out[:, m], lse[:, m], ref_out[:, m], ref_lse[:, m], rows, wl.G)
