@@ -332,6 +332,60 @@ def oam_select_int8(q, k_codes, k_scale, v, cu_seqlens, scheme: str, G: int, bet
     return idx, cu_kept, scores
 
 
+def block_scores(s, block: int = PART) -> np.ndarray:
+    """Block-granular importance ([NSA] section 2.1 selected attention: 64-token blocks scored as a
+    whole): S_j = max of the token scores of block j (tokens j*block .. j*block + block - 1, the
+    last block of a row ragged)."""
+    s = _f64(s)
+    nb = -(-s.size // block)
+    return np.array([s[j * block:(j + 1) * block].max() for j in range(nb)], np.float64)
+
+
+def select_blocks(scores, cu_seqlens, Hkv: int, keep_num: int, keep_den: int, block: int = PART):
+    """Keep, per (sequence, KV head), the top ceil(nb * keep_num / keep_den) blocks of that row's
+    token scores under (block score desc, block index asc), ascending.  ``scores`` = {(b, h): s}
+    as the oam_select functions return it (rows not in it stay -1).
+
+    -> (blk int32 [Hkv, sum_b NB_b], cu_kept_blocks int32 [B+1], {(b, h): block scores})."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = cu.size - 1
+    nblk = [-(-int(cu[b + 1] - cu[b]) // block) for b in range(B)]
+    kept = np.array([kept_count(nblk[b], keep_num, keep_den) for b in range(B)], np.int64)
+    cu_kept = np.concatenate([[0], np.cumsum(kept)]).astype(np.int32)
+    blk = np.full((Hkv, int(cu_kept[-1])), -1, np.int32)
+    bs = {}
+    for (b, h), srow in scores.items():
+        bs[(b, h)] = block_scores(srow, block)
+        blk[h, cu_kept[b]:cu_kept[b + 1]] = topk(bs[(b, h)], int(kept[b]))
+    return blk, cu_kept, bs
+
+
+def decode_blocks(q, k, v, cu_seqlens, G: int, blk, cu_kept_blocks, block: int = PART, quant=None, rows=None):
+    """Decode attending, per (sequence, KV head), to every token of that row's kept blocks
+    (the last block of a sequence holds fewer than ``block`` tokens): out [B, Hq, D], lse [B, Hq]."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    ckb = np.asarray(cu_kept_blocks, dtype=np.int64)
+    B = cu.size - 1
+    Hkv = (k if quant is None else quant[0]).shape[0]
+    D = q.shape[-1]
+    out = np.full((B, Hkv * G, D), np.nan)
+    lse = np.full((B, Hkv * G), np.nan)
+    todo = rows if rows is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for b, h in todo:
+        L = int(cu[b + 1] - cu[b])
+        toks = np.concatenate([np.arange(j * block, min((j + 1) * block, L))
+                               for j in np.asarray(blk[h, ckb[b]:ckb[b + 1]], np.int64)]).astype(np.int32)
+        # one row's kept tokens as a one-row index list for decode_row
+        idx = np.zeros((Hkv, toks.size), np.int32)
+        idx[h] = toks
+        cu_k = np.zeros(B + 1, np.int64)
+        cu_k[b + 1:] = toks.size
+        o, l = decode_row(q, k, v, cu, G, b, h, idx, cu_k, quant)
+        out[b, h * G:(h + 1) * G] = o
+        lse[b, h * G:(h + 1) * G] = l
+    return out, lse
+
+
 # ----------------------------------------------------------------------------------------------
 # decode over a packed cache
 # ----------------------------------------------------------------------------------------------

@@ -522,3 +522,62 @@ def test_multi_token_over_kept_tokens_masks_by_position():
     for m, sel in ((0, [0, 5, 28]), (1, [0, 5, 28, 29])):
         ref = oracle.attend(bt.q[0, m, 0:2], bt.k[0, sel], bt.v[0, sel])
         assert np.array_equal(out[0, m], ref[0]) and np.array_equal(lse[0, m], ref[1])
+
+
+# ---------------------------------------------------------------------------------------------
+# block-granular selection: 64-token blocks scored by the max of their token scores
+# ---------------------------------------------------------------------------------------------
+def test_block_scores_brute_force_with_ragged_last_block():
+    s = _rand(130, 5)
+    bs = oracle.block_scores(s, 64)
+    assert bs.size == 3
+    assert bs[0] == max(s[:64]) and bs[1] == max(s[64:128]) and bs[2] == max(s[128], s[129])
+
+
+def test_block_selection_with_one_token_blocks_is_token_selection():
+    bt = _tiny_batch(G=2, D=16, lengths=(9, 40, 1), Hkv=2, dtype="bf16")
+    idx, cu_kept, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, 1.0, 1e-6, 3, 8)
+    blk, cu_b, _ = oracle.select_blocks(scores, bt.cu_seqlens, 2, 3, 8, block=1)
+    assert np.array_equal(blk, idx) and np.array_equal(cu_b, cu_kept)
+
+
+def test_block_selection_hand_example_and_ties():
+    # one sequence of 130 tokens: blocks of 64, 64 and 2 tokens; keep ceil(3 / 3) = 1 block
+    s = np.zeros(130)
+    s[10], s[100], s[129] = 1.0, 2.0, 3.0  # the ragged last block holds the best token
+    blk, cu_b, bs = oracle.select_blocks({(0, 0): s}, [0, 130], 1, 1, 3)
+    assert cu_b.tolist() == [0, 1] and blk.tolist() == [[2]] and bs[(0, 0)].tolist() == [1.0, 2.0, 3.0]
+    # keep 2 of 3 with blocks 0 and 2 tied: the lower block index wins the tie, output ascending
+    s = np.zeros(130)
+    s[5], s[70], s[128] = 5.0, 7.0, 5.0
+    blk, cu_b, _ = oracle.select_blocks({(0, 0): s}, [0, 130], 1, 2, 3)
+    assert blk.tolist() == [[0, 1]]
+
+
+def test_block_selection_brute_force_ranking():
+    rng = np.random.default_rng(11)
+    cu = [0, 300, 1000]
+    scores = {(b, h): np.round(rng.standard_normal(cu[b + 1] - cu[b]), 1) for b in range(2) for h in range(2)}
+    blk, cu_b, _ = oracle.select_blocks(scores, cu, 2, 1, 4)
+    for (b, h), s in scores.items():
+        nb = -(-s.size // 64)
+        S = [max(s[64 * j:64 * j + 64]) for j in range(nb)]
+        K = -(-nb // 4)
+        want = sorted(sorted(range(nb), key=lambda j: (-S[j], j))[:K])
+        assert blk[h, cu_b[b]:cu_b[b + 1]].tolist() == want
+
+
+def test_decode_over_blocks_is_attention_over_their_tokens():
+    bt = _tiny_batch(G=2, D=8, lengths=(150, 64), Hkv=2)
+    blk = np.array([[0, 2, 0], [1, 2, 0]], np.int32)  # sequence 0 keeps 2 blocks, sequence 1 one
+    cu_b = np.array([0, 2, 3], np.int32)
+    out, lse = oracle.decode_blocks(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, blk, cu_b)
+    # head 1 of sequence 0: blocks 1 and 2 = tokens 64..127 and the ragged 128..149
+    sel = list(range(64, 150))
+    ref = oracle.attend(bt.q[0, 2:4], bt.k[1, sel], bt.v[1, sel])
+    assert np.array_equal(out[0, 2:4], ref[0]) and np.array_equal(lse[0, 2:4], ref[1])
+    # keeping every block is the dense decode
+    dense = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 2)
+    allb = np.array([[0, 1, 2, 0], [0, 1, 2, 0]], np.int32)
+    o2, l2 = oracle.decode_blocks(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, allb, np.array([0, 3, 4], np.int32))
+    assert np.allclose(o2, dense[0], atol=1e-13) and np.allclose(l2, dense[1], atol=1e-13)
