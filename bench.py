@@ -41,7 +41,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -65,7 +65,10 @@ def algorithmic_bytes(wl, lengths):
     st = {}
     codes_out = 2 * Hkv * T * D + (Hkv * P * 4 if wl.scheme == "A" else 4) + 4
     if wl.oam:
-        Kt = sum(kept_of(L, wl.keep_num, wl.keep_den) for L in lengths)
+        # kept tokens (block selection: kept blocks, each counted as the 64 tokens its tile reads)
+        nb = [(int(L) + 63) // 64 for L in lengths]
+        Kt = (sum(kept_of(n, wl.keep_num, wl.keep_den) for n in nb) if wl.blocks
+              else sum(kept_of(L, wl.keep_num, wl.keep_den) for L in lengths))
         sel_out = q + Hkv * Kt * 4 + (B + 1) * 4
     if wl.select_on_codes:  # the cache is already INT8: the selection reads K codes and the norms
         st["select"] = Hkv * T * D + Hkv * T * 4 + (Hkv * P * 4 if wl.scheme == "A" else 4) + sel_out
@@ -76,7 +79,7 @@ def algorithmic_bytes(wl, lengths):
     elif wl.oam:
         st["select"] = kv_bf16 + sel_out
     if wl.oam:
-        n_att = Kt
+        n_att = 64 * Kt if wl.blocks else Kt
         idx_bytes = Hkv * Kt * 4
     else:
         n_att = T
@@ -183,10 +186,11 @@ class Pipeline:
         if wl.select_on_codes:  # the cache is INT8 already: select on its codes
             kc, vc, ks, vs = self.kc, self.vc, self.ks, self.vs
             ev("select", 0)
-            idx, cu_kept, self.ws_s = sgd.oam_select(self.q, kc, vc, self.cu, wl.G, wl.beta, wl.eps, wl.keep_num,
-                                                     wl.keep_den, self.lengths, out=self.sel_out,
-                                                     workspace=self.ws_s, k_scale=ks, v_scale=vs,
-                                                     scheme=wl.scheme, n_parts_=self.parts, v_norm=self.vn)
+            select = sgd.oam_select_blocks if wl.blocks else sgd.oam_select
+            idx, cu_kept, self.ws_s = select(self.q, kc, vc, self.cu, wl.G, wl.beta, wl.eps, wl.keep_num,
+                                             wl.keep_den, self.lengths, out=self.sel_out, workspace=self.ws_s,
+                                             k_scale=ks, v_scale=vs, scheme=wl.scheme, n_parts_=self.parts,
+                                             v_norm=self.vn)
             self.sel_out = (idx, cu_kept)
             Kt = idx.shape[1]
             ev("select", 1)
@@ -216,6 +220,13 @@ class Pipeline:
         else:
             kc, vc, ks, vs = self.k, self.v, None, None
         ev("decode", 0)
+        if wl.blocks:
+            o, lse, self.ws_d = sgd.decode_attn_blocks(self.q, wl.G, kc, vc, self.cu, idx, cu_kept, k_scale=ks,
+                                                       v_scale=vs, scheme=wl.scheme, n_parts_=self.parts,
+                                                       out=self.dec_out, workspace=self.ws_d)
+            self.dec_out = (o, lse)
+            ev("decode", 1)
+            return o, lse
         decode = sgd.decode_attn if wl.M == 1 else sgd.decode_attn_multi
         o, lse, self.ws_d = decode(self.q, wl.G, kc, vc, self.cu, k_scale=ks, v_scale=vs,
                                             scheme=wl.scheme or "A", n_parts_=self.parts, idx=idx,
@@ -227,8 +238,8 @@ class Pipeline:
 
     def launches_per_step(self):
         # decode: plan + the tensor-core decode, which merges each row itself (D = 128, bf16 q)
-        if self.wl.select_on_codes:
-            return 3 + 2  # plan, INT8 score, top-K; plan, decode
+        if self.wl.select_on_codes:  # plan, INT8 score, (block max,) top-K; plan, decode
+            return (4 if self.wl.blocks else 3) + 2
         if self.wl.scheme and self.wl.oam:
             return 4 + 2  # plan, score+quantize, V codes, top-K; plan, decode
         return (3 if self.wl.scheme else 0) + (3 if self.wl.oam else 0) + 2
@@ -287,8 +298,17 @@ def cpu_baseline_sample(bt, wl, budget_s=20.0, max_rows=None, rows=None):
             quant = oracle.quantize_kv(kk, vv, one, wl.scheme)
         idx = cu_kept = None
         if wl.oam and wl.select_on_codes:
-            idx, cu_kept, _ = oracle.oam_select_int8(qrow, quant[0], quant[2], vv, one, wl.scheme, wl.G, wl.beta,
-                                                     wl.eps, wl.keep_num, wl.keep_den)
+            idx, cu_kept, sc = oracle.oam_select_int8(qrow, quant[0], quant[2], vv, one, wl.scheme, wl.G, wl.beta,
+                                                      wl.eps, wl.keep_num, wl.keep_den)
+            if wl.blocks:
+                blk, cu_b, _ = oracle.select_blocks(sc, one, 1, wl.keep_num, wl.keep_den)
+                oracle.decode_blocks(qrow, kk, vv, one, wl.G, blk, cu_b, quant=(*quant, wl.scheme))
+                done.append((b, h, L))
+                rowwl = wl.with_(B=1, Hkv=1, lengths=(L,), length_range=None)
+                nbytes += sum(algorithmic_bytes(rowwl, [L]).values())
+                if time.perf_counter() - t0 > budget_s:
+                    break
+                continue
         elif wl.oam:
             idx, cu_kept, _ = oracle.oam_select(qrow, kk, vv, one, wl.G, wl.beta, wl.eps, wl.keep_num,
                                                 wl.keep_den)
@@ -469,7 +489,9 @@ def run_ours(args, rank, world, local_rank):
             "T": int(sum(pipe.lengths)), "scheme": wl.scheme, "oam": wl.oam, "beta": wl.beta, "eps": wl.eps,
             "keep": f"{wl.keep_num}/{wl.keep_den}", "seed": wl.seed if wl.seed is not None else args.workload, "q_quant": wl.q_quant,
             "query_tokens": wl.M,
-            "step": ("oam_select(int8 cache, stored norms) -> decode_attn(kept); cache quantised once, untimed"
+            "step": ("oam_select_blocks(int8 cache, stored norms) -> decode_attn_blocks(kept 64-token blocks); "
+                     "cache quantised once, untimed" if wl.blocks else
+                     "oam_select(int8 cache, stored norms) -> decode_attn(kept); cache quantised once, untimed"
                      if wl.select_on_codes else
                      "quantize_select -> decode_attn(kept)" if wl.oam else "quantize_kv -> decode_attn"),
             "l2": "flushed between steps (untimed 256 MiB write then 256 MiB read: L2 left clean); inputs > L2",

@@ -153,6 +153,26 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * sgd_oam_select_blocks -- block-granular token dropping: whole 64-token blocks are kept
+ * ([NSA] section 2.1 selects 64-token blocks so that the kept KV is read contiguously; here a
+ * block is ranked by the best OAM score s_t of its tokens).  Block j of sequence b holds tokens
+ * 64j .. min(64j + 63, L_b - 1) (the last block may be ragged).  Per (b, kvh) the
+ * NB_b = clamp(ceil(nb_b * keep_num / keep_den), 1, nb_b) best of the nb_b = ceil(L_b / 64)
+ * blocks are kept, ties broken by the lower block index.
+ * q, kv, beta, eps, keep_num, keep_den   as in sgd_oam_select
+ * n_blocks        sum_b nb_b (host value; checked on the device)
+ * blk             [Hkv, kept_blocks_total] int32 output: row (b, kvh) is
+ *                 blk[kvh, cu_kept_blocks[b] .. cu_kept_blocks[b+1]-1], block numbers local
+ *                 to sequence b, ascending
+ * cu_kept_blocks  [B+1] int32 output, prefix sums of NB_b;  kept_blocks_total = sum_b NB_b
+ * workspace       sgd_workspace_size(SGD_OP_OAM_SELECT, kv, G, 0, 0) bytes
+ */
+int sgd_oam_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                          float beta, float eps, int keep_num, int keep_den, int64_t n_blocks,
+                          int32_t *blk, int32_t *cu_kept_blocks, int64_t kept_blocks_total,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * sgd_quantize_select -- sgd_quantize_kv and sgd_oam_select of one cache in one call, with the
  * same outputs ([TD] sections 6 and 3; the pages' pipeline, section 7, runs both on the same
  * cache).  With a BF16 cache and BF16 q (D in {64, 128}) the K and V of every token are read
@@ -210,6 +230,22 @@ int sgd_decode_attn_multi(const void *q, sgd_dtype q_dtype, int G, int M, const 
                           const int32_t *idx, const int32_t *cu_kept, int64_t kept_total,
                           int schedule, int n_splits, int q_quant, float *out, float *lse,
                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_decode_attn_blocks -- sgd_decode_attn over kept 64-token blocks (the output of
+ * sgd_oam_select_blocks): every row attends to all tokens of its kept blocks (a sequence's
+ * ragged last block contributes only its L_b - 64 j tokens), renormalised over them.  Each
+ * block is one contiguous run of the cache, fetched as whole tiles (no per-token gathers).
+ * blk, cu_kept_blocks, kept_blocks_total   as produced by sgd_oam_select_blocks; a block number
+ *          outside [0, nb_b) sets SGD_STATUS_BAD_INDEX and is clamped
+ * The cache is BF16 (D 64 or 128) or I8 (D 128) with a BF16 q (SGD_ERR_DTYPE otherwise);
+ * workspace, schedule, n_splits, q_quant, out, lse and errors as in sgd_decode_attn.
+ */
+int sgd_decode_attn_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                           const int32_t *blk, const int32_t *cu_kept_blocks,
+                           int64_t kept_blocks_total, int schedule, int n_splits, int q_quant,
+                           float *out, float *lse, void *workspace, size_t workspace_bytes,
+                           void *stream);
 
 /* Workspace bytes an operation needs for this cache shape (>= 256). For
  * SGD_OP_DECODE, `schedule` and `n_splits` as in sgd_decode_attn; for the

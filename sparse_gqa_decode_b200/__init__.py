@@ -68,6 +68,10 @@ lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_decode_attn_multi.argtypes = [_vp, _i32, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp,
                                       _sz, _vp]
+lib.sgd_oam_select_blocks.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i64, _vp, _vp, _i64, _vp, _sz,
+                                      _vp]
+lib.sgd_decode_attn_blocks.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
+                                       _vp]
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
@@ -105,6 +109,12 @@ def n_parts(lengths: Sequence[int]) -> int:
 def kept_total(lengths: Sequence[int], keep_num: int, keep_den: int) -> int:
     """Size of the kept-index buffer per KV head: sum_b clamp(ceil(L_b*num/den), 1, L_b)."""
     return int(sum(max(1, min(int(L), -(-int(L) * keep_num // keep_den))) for L in lengths))
+
+
+def kept_blocks_total(lengths: Sequence[int], keep_num: int, keep_den: int) -> int:
+    """Size of the kept-block buffer per KV head: sum_b clamp(ceil(nb_b*num/den), 1, nb_b) with
+    nb_b = ceil(L_b / 64) blocks."""
+    return kept_total([(int(L) + PARTITION - 1) // PARTITION for L in lengths], keep_num, keep_den)
 
 
 def _kv(k, v, cu_seqlens, k_scale=None, v_scale=None, scheme=SCHEME_A, parts=0, v_norm=None) -> SgdKv:
@@ -191,6 +201,27 @@ def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
     return idx, cu_kept, ws
 
 
+def oam_select_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                      beta: float, eps: float, keep_num: int, keep_den: int, lengths: Sequence[int],
+                      out=None, workspace=None, stream=None, k_scale=None, v_scale=None, scheme: str = "A",
+                      n_parts_: int = 0, v_norm=None):
+    """Kept 64-token blocks per (sequence, KV head), ranked by their best token's OAM score.
+    Returns (blk [Hkv, NBt], cu_kept_blocks [B+1], ws); the cache arguments as in oam_select."""
+    Hkv = k.shape[0]
+    NBt = kept_blocks_total(lengths, keep_num, keep_den)
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, SCHEME_A if scheme == "A" else SCHEME_B, n_parts_, v_norm)
+    if out is None:
+        blk = torch.empty((Hkv, NBt), dtype=torch.int32, device=k.device)
+        cu_kb = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
+    else:
+        blk, cu_kb = out
+    ws = _workspace(workspace_size(OP_OAM_SELECT, kv, G), k.device, workspace)
+    _check(lib.sgd_oam_select_blocks(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den,
+                                     n_parts(lengths), _ptr(blk), _ptr(cu_kb), NBt, _ptr(ws), ws.numel(),
+                                     _stream(stream)), "sgd_oam_select_blocks")
+    return blk, cu_kb, ws
+
+
 def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
                     beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
                     out=None, workspace=None, stream=None, v_norm=None):
@@ -263,6 +294,29 @@ def decode_attn_multi(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor,
     _check(lib.sgd_decode_attn_multi(_ptr(q), _DT[q.dtype], G, M, ctypes.byref(kv), _ptr(idx), _ptr(cu_kept),
                                      int(kept_total_), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse),
                                      _ptr(ws), ws.numel(), _stream(stream)), "sgd_decode_attn_multi")
+    return o, lse, ws
+
+
+def decode_attn_blocks(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                       blk: torch.Tensor, cu_kept_blocks: torch.Tensor, k_scale=None, v_scale=None,
+                       scheme: str = "A", n_parts_: int = 0, schedule: int = 0, n_splits: int = 0, out=None,
+                       workspace=None, stream=None, q_quant: str = "none"):
+    """Decode over kept 64-token blocks (as oam_select_blocks returns them).
+    Returns (out [B, Hq, D] f32, lse [B, Hq] f32, ws)."""
+    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, sch, n_parts_)
+    B = cu_seqlens.numel() - 1
+    Hq = k.shape[0] * G
+    D = k.shape[2]
+    if out is None:
+        o = torch.empty((B, Hq, D), dtype=torch.float32, device=k.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=k.device)
+    else:
+        o, lse = out
+    ws = _workspace(workspace_size(OP_DECODE, kv, G, schedule, n_splits), k.device, workspace)
+    _check(lib.sgd_decode_attn_blocks(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), _ptr(blk), _ptr(cu_kept_blocks),
+                                      int(blk.shape[1]), schedule, n_splits, _QQ[q_quant], _ptr(o), _ptr(lse),
+                                      _ptr(ws), ws.numel(), _stream(stream)), "sgd_decode_attn_blocks")
     return o, lse, ws
 
 

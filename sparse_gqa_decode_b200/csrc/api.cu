@@ -62,7 +62,7 @@ int check_kv(const sgd_kv *kv) {
 struct Layout {
     size_t row_pos = 0, row_slot0 = 0, cta_begin = 0, cta_slot0 = 0, cta_row0 = 0, row_info = 0, row_done = 0;
     size_t seq_part0 = 0;
-    size_t o_part = 0, lse_part = 0, scores = 0, total = 0;
+    size_t o_part = 0, lse_part = 0, scores = 0, bscores = 0, total = 0;
 };
 
 size_t take(size_t &off, size_t bytes) {
@@ -90,7 +90,10 @@ Layout layout(int op, int B, int Hkv, int G, int D, int64_t T, int n_req) {
         L.o_part = take(off, (size_t)slots * G * D * 4);
         L.lse_part = take(off, (size_t)slots * G * 4);
     }
-    if (op == SGD_OP_OAM_SELECT) L.scores = take(off, (size_t)Hkv * T * 4);
+    if (op == SGD_OP_OAM_SELECT) {
+        L.scores = take(off, (size_t)Hkv * T * 4);
+        L.bscores = take(off, (size_t)Hkv * (T / kPart + B) * 4);  // block selection: per-block scores
+    }
     L.total = off;
     return L;
 }
@@ -139,6 +142,176 @@ cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 }  // namespace sgd
 
 using namespace sgd;
+
+namespace {
+
+// The decode behind sgd_decode_attn, _multi and _blocks.  blocks: idx / cu_kept / kept_total
+// list kept 64-token blocks (the tensor-core kernel reads each as one box per tensor).
+int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, const int32_t *idx,
+                const int32_t *cu_kept, int64_t kept_total, bool blocks, int schedule, int n_splits, int q_quant,
+                float *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
+    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
+    const int NC = G * M;  // the kernels' columns per KV head: (query token, head) pairs
+    // several query tokens, and kept blocks, run on the tensor-core kernel only
+    if ((M > 1 || blocks) && decode_family(kv->dtype, q_dtype, kv->D, false) != kFamilyMma) return SGD_ERR_DTYPE;
+    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (q_dtype == SGD_F32 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
+    const bool listed = idx != nullptr;  // kept tokens or kept blocks
+    if (listed != (cu_kept != nullptr)) return SGD_ERR_NULL;
+    if (listed && (kept_total < kv->B || kept_total > (blocks ? kv->T / SGD_PARTITION + kv->B : kv->T)))
+        return SGD_ERR_SHAPE;
+    const bool indexed = listed && !blocks;  // token gathers
+    if (kv->dtype == SGD_I8) {
+        if (!kv->k_scale || !kv->v_scale) return SGD_ERR_NULL;
+        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
+            return SGD_ERR_SHAPE;
+    }
+    if (q_quant < 0 || q_quant > 2) return SGD_ERR_ARG;
+    if (q_quant != 0 && (kv->dtype != SGD_I8 || q_dtype != SGD_BF16)) return SGD_ERR_DTYPE;
+    if (q_quant != 0 && kv->D != 128) return SGD_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (indexed && (reinterpret_cast<uintptr_t>(idx) & 3u)))
+        return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    if ((rc = decode_n_req(*dev, kv, q_dtype, NC, indexed, false, schedule, n_splits, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_DECODE, kv->B, kv->Hkv, NC, kv->D, kv->T, n_req);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    // blocks: segments start and end on block boundaries (granule 64), lengths counted in blocks
+    const int granule = blocks ? kPart : kGranule;
+    const int min_chunk = (n_splits > 0 || schedule == 1) ? granule : kAutoMinChunk;
+    launch_plan(listed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
+                hdr, s, granule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
+                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M, blocks ? kPart : 1);
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.q_f32 = q_dtype == SGD_F32;
+    a.cu_seq = kv->cu_seqlens;
+    a.cu_kept = cu_kept;
+    a.idx = idx;
+    a.k = kv->k;
+    a.v = kv->v;
+    a.k_scale = kv->k_scale;
+    a.v_scale = kv->v_scale;
+    a.scheme = kv->scheme;
+    a.B = kv->B;
+    a.Hkv = kv->Hkv;
+    a.G = G;
+    a.M = M;
+    a.D = kv->D;
+    a.T = kv->T;
+    a.Kt = listed ? kept_total : 0;
+    a.blk = blocks ? 1 : 0;
+    a.n_parts = kv->dtype == SGD_I8 && kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
+    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
+    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
+    a.plan = pv;
+    a.o_part = reinterpret_cast<float *>(ws + L.o_part);
+    a.lse_part = reinterpret_cast<float *>(ws + L.lse_part);
+    a.out = out;
+    a.lse = lse;
+    a.status = &hdr->status;
+    a.q_quant = q_quant;
+    a.q_scale = &hdr->q_scale;
+    int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials
+    if (decode_family(kv->dtype, q_dtype, kv->D, false) == kFamilyMma) return SGD_OK;
+    e = launch_merge(a, out, lse, s);
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+
+// The selection behind sgd_oam_select and sgd_oam_select_blocks.  blocks: rank the 64-token
+// blocks by their best token's score and keep whole blocks (n_blocks = sum_b ceil(L_b / 64)).
+int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps, int keep_num,
+                int keep_den, bool blocks, int64_t n_blocks, int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_kv(kv);
+    if (rc != SGD_OK) return rc;
+    if (!q || !idx || !cu_kept || !workspace) return SGD_ERR_NULL;
+    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
+    if (kv->dtype == SGD_I8) {
+        // scoring the INT8 cache: khat = code * scale, ||v|| from the norms stored at quantisation
+        if (q_dtype != SGD_BF16 || kv->D != 128) return SGD_ERR_DTYPE;
+        if (!kv->k_scale || !kv->v_norm) return SGD_ERR_NULL;
+        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
+        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
+            return SGD_ERR_SHAPE;
+        if (reinterpret_cast<uintptr_t>(kv->v_norm) & 3u) return SGD_ERR_ALIGN;
+    } else if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) {
+        return SGD_ERR_DTYPE;
+    }
+    if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
+    if (blocks && (n_blocks < kv->B || n_blocks > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
+    if (kept_total < kv->B || kept_total > (blocks ? n_blocks : kv->T)) return SGD_ERR_SHAPE;
+    if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
+    if (!aligned16(q) || !aligned16(workspace)) return SGD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u)) return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    if ((rc = current_device(&dev)) != SGD_OK) return rc;
+    int n_req = 0;
+    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    const PlanView pv = plan_view(ws, L);
+    cudaStream_t s = as_stream(stream);
+    launch_plan(kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, kAutoMinChunk, 0, pv, hdr, s);
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.q_f32 = q_dtype == SGD_F32;
+    a.cu_seq = kv->cu_seqlens;
+    a.k = kv->k;
+    a.v = kv->v;
+    a.B = kv->B;
+    a.Hkv = kv->Hkv;
+    a.G = G;
+    a.M = 1;
+    a.D = kv->D;
+    a.T = kv->T;
+    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
+    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
+    a.beta = beta;
+    a.eps = eps;
+    if (kv->dtype == SGD_I8) {
+        a.k_scale = kv->k_scale;
+        a.scheme = kv->scheme;
+        a.n_parts = kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
+        a.v_norm = kv->v_norm;
+    }
+    a.scores = reinterpret_cast<float *>(ws + L.scores);
+    a.plan = pv;
+    a.status = &hdr->status;
+    int e = launch_decode(a, kv->dtype, q_dtype, false, true, n_req, s);
+    if (e != 0) return SGD_ERR_CUDA;
+    if (blocks) {  // block scores, then the top blocks of each row (the plan's partition offsets = block offsets)
+        float *bs = reinterpret_cast<float *>(ws + L.bscores);
+        e = launch_block_max(a.scores, kv->cu_seqlens, pv.seq_part0, kv->B, kv->Hkv, kv->T, n_blocks, bs,
+                             &hdr->status, s);
+        if (e != 0) return SGD_ERR_CUDA;
+        e = launch_topk(bs, pv.seq_part0, kv->B, kv->Hkv, n_blocks, keep_num, keep_den, idx, cu_kept, kept_total,
+                        &hdr->status, s);
+        return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+    }
+    e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
+                    &hdr->status, s);
+    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+}  // namespace
 
 extern "C" {
 
@@ -224,69 +397,15 @@ int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts, int8_t
 int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps, int keep_num,
                    int keep_den, int32_t *idx, int32_t *cu_kept, int64_t kept_total, void *workspace,
                    size_t workspace_bytes, void *stream) {
-    int rc = check_kv(kv);
-    if (rc != SGD_OK) return rc;
-    if (!q || !idx || !cu_kept || !workspace) return SGD_ERR_NULL;
-    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
-    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
-    if (kv->dtype == SGD_I8) {
-        // scoring the INT8 cache: khat = code * scale, ||v|| from the norms stored at quantisation
-        if (q_dtype != SGD_BF16 || kv->D != 128) return SGD_ERR_DTYPE;
-        if (!kv->k_scale || !kv->v_norm) return SGD_ERR_NULL;
-        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
-        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
-            return SGD_ERR_SHAPE;
-        if (reinterpret_cast<uintptr_t>(kv->v_norm) & 3u) return SGD_ERR_ALIGN;
-    } else if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) {
-        return SGD_ERR_DTYPE;
-    }
-    if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
-    if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
-    if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
-    if (!aligned16(q) || !aligned16(workspace)) return SGD_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u)) return SGD_ERR_ALIGN;
-    DevInfo *dev;
-    if ((rc = current_device(&dev)) != SGD_OK) return rc;
-    int n_req = 0;
-    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
-    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
-    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
-    const PlanView pv = plan_view(ws, L);
-    cudaStream_t s = as_stream(stream);
-    launch_plan(kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, kAutoMinChunk, 0, pv, hdr, s);
-    DecodeArgs a;
-    memset(&a, 0, sizeof(a));
-    a.q = q;
-    a.q_f32 = q_dtype == SGD_F32;
-    a.cu_seq = kv->cu_seqlens;
-    a.k = kv->k;
-    a.v = kv->v;
-    a.B = kv->B;
-    a.Hkv = kv->Hkv;
-    a.G = G;
-    a.M = 1;
-    a.D = kv->D;
-    a.T = kv->T;
-    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
-    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
-    a.beta = beta;
-    a.eps = eps;
-    if (kv->dtype == SGD_I8) {
-        a.k_scale = kv->k_scale;
-        a.scheme = kv->scheme;
-        a.n_parts = kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
-        a.v_norm = kv->v_norm;
-    }
-    a.scores = reinterpret_cast<float *>(ws + L.scores);
-    a.plan = pv;
-    a.status = &hdr->status;
-    int e = launch_decode(a, kv->dtype, q_dtype, false, true, n_req, s);
-    if (e != 0) return SGD_ERR_CUDA;
-    e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
-                    &hdr->status, s);
-    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+    return select_impl(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, false, 0, idx, cu_kept, kept_total, workspace,
+                       workspace_bytes, stream);
+}
+
+int sgd_oam_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
+                          int keep_num, int keep_den, int64_t n_blocks, int32_t *blk, int32_t *cu_kept_blocks,
+                          int64_t kept_blocks_total, void *workspace, size_t workspace_bytes, void *stream) {
+    return select_impl(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, true, n_blocks, blk, cu_kept_blocks,
+                       kept_blocks_total, workspace, workspace_bytes, stream);
 }
 
 int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
@@ -374,80 +493,17 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, c
 int sgd_decode_attn_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, const int32_t *idx,
                           const int32_t *cu_kept, int64_t kept_total, int schedule, int n_splits, int q_quant,
                           float *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
-    int rc = check_kv(kv);
-    if (rc != SGD_OK) return rc;
-    if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
-    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
-    const int NC = G * M;  // the kernels' columns per KV head: (query token, head) pairs
-    // several query tokens run on the tensor-core kernel only
-    if (M > 1 && decode_family(kv->dtype, q_dtype, kv->D, false) != kFamilyMma) return SGD_ERR_DTYPE;
-    if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
-    if (q_dtype == SGD_F32 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
-    const bool indexed = idx != nullptr;
-    if (indexed != (cu_kept != nullptr)) return SGD_ERR_NULL;
-    if (indexed && (kept_total < kv->B || kept_total > kv->T)) return SGD_ERR_SHAPE;
-    if (kv->dtype == SGD_I8) {
-        if (!kv->k_scale || !kv->v_scale) return SGD_ERR_NULL;
-        if (kv->scheme != SGD_SCHEME_A && kv->scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
-        if (kv->scheme == SGD_SCHEME_A && (kv->n_parts < kv->B || kv->n_parts > kv->T / SGD_PARTITION + kv->B))
-            return SGD_ERR_SHAPE;
-    }
-    if (q_quant < 0 || q_quant > 2) return SGD_ERR_ARG;
-    if (q_quant != 0 && (kv->dtype != SGD_I8 || q_dtype != SGD_BF16)) return SGD_ERR_DTYPE;
-    if (q_quant != 0 && kv->D != 128) return SGD_ERR_SHAPE;
-    if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return SGD_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (indexed && (reinterpret_cast<uintptr_t>(idx) & 3u)))
-        return SGD_ERR_ALIGN;
-    DevInfo *dev;
-    if ((rc = current_device(&dev)) != SGD_OK) return rc;
-    int n_req = 0;
-    if ((rc = decode_n_req(*dev, kv, q_dtype, NC, indexed, false, schedule, n_splits, &n_req)) != SGD_OK) return rc;
-    const Layout L = layout(SGD_OP_DECODE, kv->B, kv->Hkv, NC, kv->D, kv->T, n_req);
-    if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
-    const PlanView pv = plan_view(ws, L);
-    cudaStream_t s = as_stream(stream);
-    const int min_chunk = (n_splits > 0 || schedule == 1) ? kGranule : kAutoMinChunk;
-    launch_plan(indexed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
-                hdr, s, kGranule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
-                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M);
-    DecodeArgs a;
-    memset(&a, 0, sizeof(a));
-    a.q = q;
-    a.q_f32 = q_dtype == SGD_F32;
-    a.cu_seq = kv->cu_seqlens;
-    a.cu_kept = cu_kept;
-    a.idx = idx;
-    a.k = kv->k;
-    a.v = kv->v;
-    a.k_scale = kv->k_scale;
-    a.v_scale = kv->v_scale;
-    a.scheme = kv->scheme;
-    a.B = kv->B;
-    a.Hkv = kv->Hkv;
-    a.G = G;
-    a.M = M;
-    a.D = kv->D;
-    a.T = kv->T;
-    a.Kt = indexed ? kept_total : 0;
-    a.n_parts = kv->dtype == SGD_I8 && kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
-    a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
-    a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
-    a.plan = pv;
-    a.o_part = reinterpret_cast<float *>(ws + L.o_part);
-    a.lse_part = reinterpret_cast<float *>(ws + L.lse_part);
-    a.out = out;
-    a.lse = lse;
-    a.status = &hdr->status;
-    a.q_quant = q_quant;
-    a.q_scale = &hdr->q_scale;
-    int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
-    if (e != 0) return SGD_ERR_CUDA;
-    // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials
-    if (decode_family(kv->dtype, q_dtype, kv->D, false) == kFamilyMma) return SGD_OK;
-    e = launch_merge(a, out, lse, s);
-    return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+    return decode_impl(q, q_dtype, G, M, kv, idx, cu_kept, kept_total, false, schedule, n_splits, q_quant, out, lse,
+                       workspace, workspace_bytes, stream);
+}
+
+int sgd_decode_attn_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, const int32_t *blk,
+                           const int32_t *cu_kept_blocks, int64_t kept_blocks_total, int schedule, int n_splits,
+                           int q_quant, float *out, float *lse, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    if (!blk || !cu_kept_blocks) return SGD_ERR_NULL;
+    return decode_impl(q, q_dtype, G, 1, kv, blk, cu_kept_blocks, kept_blocks_total, true, schedule, n_splits,
+                       q_quant, out, lse, workspace, workspace_bytes, stream);
 }
 
 int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode, int32_t *segs,

@@ -52,12 +52,14 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 
 constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
 
-template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false, bool CAUSAL_ = false>
+template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false, bool CAUSAL_ = false,
+          bool BLK_ = false>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
     static constexpr bool QI8 = QI8_;  // INT8 query codes: S^T = K_codes . Q_codes^T on s8 MMAs
     static constexpr bool CAUSAL = CAUSAL_;  // several query tokens: causal limit per column
+    static constexpr bool BLK = BLK_;  // kept 64-token blocks: one TMA box per block, at its start
     static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
     static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static constexpr int NW = 4;        // consumer warps
@@ -67,6 +69,7 @@ struct MmaCfg {
     static constexpr int ROWB = D * EB;
     static constexpr int BOXES = ROWB / 128;
     static constexpr int BOX_ELEMS = 128 / EB;
+    static constexpr int BOX_ROWS = BLK ? kPart : ROWS;  // rows of one TMA box
     static constexpr int TILE = ROWS * ROWB;  // bytes of one tensor per stage
     static constexpr int STAGES = 3;
     // CTAs per SM the registers must allow: the K-only score of an INT8 cache has half-size stages
@@ -86,6 +89,7 @@ struct MmaCfg {
     static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
     static_assert(!QI8 || (I8 && MODE == 0 && D == 128), "query codes meet INT8 keys in the decode");
     static_assert(!CAUSAL || MODE == 0, "several query tokens: decode only");
+    static_assert(!BLK || (MODE == 0 && !IDX && !CAUSAL && ROWS % kPart == 0), "a tile is whole blocks");
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
 };
 
@@ -133,11 +137,59 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
 #pragma unroll
             for (int j = 0; j <= kPrefetch; ++j) load_tile_idx(tk[j], t0 + j * C::ROWS);
         }
+        // kept blocks: the block numbers of this tile and the next (-1 past the segment), checked
+        constexpr int NBT = C::BLK ? C::ROWS / kPart : 1;
+        int32_t blk_cur[NBT], blk_nxt[NBT];
+        const int32_t *bp = nullptr;
+        if constexpr (C::BLK) bp = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start / kPart;
+        const int32_t nblk = (Lb + kPart - 1) / kPart;
+#pragma unroll
+        for (int i = 0; i < NBT; ++i) blk_nxt[i] = -1;
+        auto load_tile_blk = [&](int32_t tt) {
+#pragma unroll
+            for (int i = 0; i < NBT; ++i) {
+                blk_cur[i] = blk_nxt[i];
+                const int32_t u = tt + i * kPart;
+                int32_t v = -1;
+                if (u < t1) {
+                    v = __ldg(bp + u / kPart);
+                    if (v < 0 || v >= nblk) {  // out of range: reported, clamped (nothing loaded if none)
+                        atomicOr(a.status, SGD_STATUS_BAD_INDEX);
+                        v = (nblk > 0) ? min(max(v, 0), nblk - 1) : -1;
+                    }
+                }
+                blk_nxt[i] = v;
+            }
+        };
+        if constexpr (C::BLK) {
+            load_tile_blk(t0);
+            load_tile_blk(t0 + C::ROWS);
+        }
         for (int32_t t = t0; t < t1; t += C::ROWS) {
             if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
             uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
-            if constexpr (!C::IDX) {
+            if constexpr (C::BLK) {
+                // the tile's kept blocks (t and t1 are multiples of 64 in the row's padded block
+                // stream), each one box per tensor and 128-byte column, at its own cache row
+                constexpr int NB = C::ROWS / kPart;
+                int nload = 0;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) nload += (blk_cur[i] >= 0) ? 1 : 0;
+                mbar_arrive_expect_tx(&full[stage], nload * 2 * (C::TILE / NB));
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    if (blk_cur[i] < 0) continue;
+                    const int y = (int)(seq0 + (int64_t)blk_cur[i] * kPart);
+#pragma unroll
+                    for (int bx = 0; bx < C::BOXES; ++bx) {
+                        const int off = bx * C::ROWS * 128 + i * kPart * 128;
+                        tma_load_2d(sk + off, tmK, &full[stage], bx * C::BOX_ELEMS, y, pol);
+                        tma_load_2d(sv + off, tmV, &full[stage], bx * C::BOX_ELEMS, y, pol);
+                    }
+                }
+                load_tile_blk(t + 2 * C::ROWS);
+            } else if constexpr (!C::IDX) {
                 mbar_arrive_expect_tx(&full[stage], (C::KONLY ? 1 : 2) * C::TILE);
                 const int y = (int)(seq0 + t);
 #pragma unroll
@@ -823,6 +875,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         const int32_t *ip = nullptr;
         if constexpr (C::I8) ksc = a.k_scale + (int64_t)kvh * a.n_parts + cur.ri.part0;
         if constexpr (C::IDX) ip = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start;
+        if constexpr (C::BLK) ip = a.idx + (int64_t)kvh * a.Kt + cur.ri.len_start / kPart;
         // scores of an INT8 cache: the value norms of each sub-tile row, loaded one tile ahead
         float vn_cur[C::SUB], vn_nxt[C::SUB];
         auto load_norms = [&](float (&dst)[C::SUB], int32_t tt) {
@@ -839,7 +892,23 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             float rf_pre[C::SUB];
 #pragma unroll
             for (int s = 0; s < C::SUB; ++s) rf_pre[s] = 1.f;
-            if constexpr (C::I8 && !C::IDX) {
+            // kept blocks: the sequence position of each sub-tile's row 0 (a 16-row sub-tile lies in
+            // one block) and, for scheme A, that block's K scale (blocks are the K partitions)
+            int32_t bpos[C::SUB];
+            if constexpr (C::BLK) {
+                const int32_t nb = (Lb + kPart - 1) / kPart;
+#pragma unroll
+                for (int s = 0; s < C::SUB; ++s) {
+                    const int32_t u = t + 16 * (s * C::NW + warp);
+                    int32_t v = (u < t1) ? __ldg(ip + u / kPart) : 0;
+                    v = min(max(v, 0), max(nb - 1, 0));
+                    bpos[s] = v * kPart + (u % kPart);
+                    if constexpr (C::I8) {
+                        if (a.scheme == SGD_SCHEME_A && nb > 0) rf_pre[s] = __ldg(ksc + v);
+                    }
+                }
+            }
+            if constexpr (C::I8 && !C::IDX && !C::BLK) {
                 if (a.scheme == SGD_SCHEME_A) {
 #pragma unroll
                     for (int s = 0; s < C::SUB; ++s)
@@ -866,7 +935,11 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 if (j0 >= t1 || !ready) continue;
                 float sacc[C::GT][4];
                 qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
-                const bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
+                bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
+                if constexpr (C::BLK) {  // the last block of a sequence is ragged
+                    vA = bpos[s] + pA < Lb;
+                    vB = bpos[s] + pA + 8 < Lb;
+                }
                 // several query tokens: token m sees sequence positions <= L_b - M + m; bit 4 gt + e
                 // keeps element e of column tile gt (only sub-tiles reaching the last M - 1
                 // positions mask anything)
@@ -1320,8 +1393,8 @@ static int launch_mma(const DecodeArgs &a, int n_cta, cudaStream_t s) {
     memset(&mv, 0, sizeof(mv));
     if constexpr (!C::IDX) {
         const int64_t rows = (int64_t)a.Hkv * a.T;
-        if (!make_map(&mk, a.k, C::I8, C::D, rows, C::BOX_ELEMS, C::ROWS) ||
-            !make_map(&mv, a.v, C::I8, C::D, rows, C::BOX_ELEMS, C::ROWS))
+        if (!make_map(&mk, a.k, C::I8, C::D, rows, C::BOX_ELEMS, C::BOX_ROWS) ||
+            !make_map(&mv, a.v, C::I8, C::D, rows, C::BOX_ELEMS, C::BOX_ROWS))
             return (int)cudaErrorInvalidValue;
     }
     auto k = decode_mma_kernel<C>;
@@ -1334,6 +1407,8 @@ template <int D, int GT, bool I8, int MODE, bool QI8 = false>
 static int launch_mma_idx(const DecodeArgs &a, bool indexed, int n_cta, cudaStream_t s) {
     if constexpr (MODE == 1) {
         return launch_mma<MmaCfg<D, GT, I8, false, MODE>>(a, n_cta, s);
+    } else if (a.blk) {  // kept 64-token blocks: one TMA box per block
+        return launch_mma<MmaCfg<D, GT, I8, false, MODE, QI8, false, true>>(a, n_cta, s);
     } else if (a.M > 1) {  // several query tokens per sequence: the causally masked instantiation
         return indexed ? launch_mma<MmaCfg<D, GT, I8, true, MODE, QI8, true>>(a, n_cta, s)
                        : launch_mma<MmaCfg<D, GT, I8, false, MODE, QI8, true>>(a, n_cta, s);

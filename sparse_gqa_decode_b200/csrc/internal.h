@@ -20,6 +20,7 @@ struct DecodeArgs {
     int B, Hkv, G, D;
     int M;                   // decode: query tokens per sequence (>= 1), causal over the cache's last M;
                              // the kernel's columns are the M * G (token, head) pairs of a KV head
+    int blk;                 // decode: idx / cu_kept / Kt list kept 64-token blocks, not tokens
     int64_t T, Kt, n_parts;
     int q_f32;               // q is float32 (otherwise bf16)
     float sm_scale_log2;     // log2(e) / sqrt(D)
@@ -47,10 +48,11 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 // out/lse (decode only, else NULL): rows without tokens get out = 0 and lse = -inf here.
 // q_bf16 (decode with a per-tensor query scale, else NULL): hdr->q_scale = max|q| / 127.
 // M: query tokens per sequence of the decode (out is [B, M, Hkv * G, D]).
+// len_unit: tokens per unit of cu_len (64 when cu_len counts kept 64-token blocks).
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
                  float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0, const void *q_bf16 = nullptr,
-                 int64_t q_elems = 0, int M = 1);
+                 int64_t q_elems = 0, int M = 1, int len_unit = 1);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 
@@ -82,5 +84,9 @@ int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *c
 // oam.cu
 int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t T, int keep_num, int keep_den,
                 int32_t *idx, int32_t *cu_kept, int64_t kept_total, int32_t *status, cudaStream_t s);
+// Block scores of 64-token blocks: bscores[h * Tb + j] = max of the token scores of block j
+// (sequence b's blocks are cu_blk[b] .. cu_blk[b+1]; its last block may be ragged).
+int launch_block_max(const float *scores, const int32_t *cu_seq, const int32_t *cu_blk, int B, int Hkv, int64_t T,
+                     int64_t Tb, float *bscores, int32_t *status, cudaStream_t s);
 
 }  // namespace sgd

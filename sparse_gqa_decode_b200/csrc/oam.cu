@@ -32,6 +32,7 @@
 #include <cooperative_groups.h>
 
 #include "internal.h"
+#include "plan.cuh"
 #include "scan.cuh"
 
 namespace cg = cooperative_groups;
@@ -556,6 +557,50 @@ int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t 
     // 512 threads, 8-CTA clusters, two CTAs per SM: every row of a 32-row batch resident at once
     return launch_topk_cfg<512, 8, 2>(scores, cu, B, Hkv, T, keep_num, keep_den, idx, cu_kept, kept_total, status,
                                    kTopkChunk, s);
+}
+
+// ------------------------------------------------------------------------------------------
+// block scores for block-granular selection ([NSA] section 2.1: 64-token selection blocks): one
+// warp per (KV head, block), two coalesced loads per lane, the block's best token score
+// ------------------------------------------------------------------------------------------
+constexpr int kBlockMaxWarps = 8;
+
+__global__ void __launch_bounds__(kBlockMaxWarps * 32)
+    block_max_kernel(const float *__restrict__ scores, const int32_t *__restrict__ cu_seq,
+                     const int32_t *__restrict__ cu_blk, int B, int Hkv, int64_t T, int64_t Tb,
+                     float *__restrict__ bscores, int32_t *status) {
+    const int64_t w = (int64_t)blockIdx.x * kBlockMaxWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= (int64_t)Hkv * Tb) return;
+    const int h = (int)(w / Tb);
+    const int32_t j = (int32_t)(w - (int64_t)h * Tb);
+    const int b = upper_bound_i32(cu_blk, B + 1, j) - 1;  // sequence of block j
+    if (b < 0 || b >= B) {  // the caller's block count exceeds the lengths' (or the lengths are bad)
+        if (lane == 0) {
+            bscores[(int64_t)h * Tb + j] = -INFINITY;
+            atomicOr(status, SGD_STATUS_SIZE_MISMATCH);
+        }
+        return;
+    }
+    if (j == 0 && h == 0 && lane == 0 && __ldg(cu_blk + B) != Tb) atomicOr(status, SGD_STATUS_SIZE_MISMATCH);
+    const int32_t s0 = __ldg(cu_seq + b), s1 = __ldg(cu_seq + b + 1);
+    const int32_t t0 = s0 + (j - __ldg(cu_blk + b)) * kPart;
+    const int32_t n = min(kPart, s1 - t0);
+    const float *row = scores + (int64_t)h * T + t0;
+    float m = -INFINITY;
+    if (lane < n) m = __ldg(row + lane);
+    if (lane + 32 < n) m = fmaxf(m, __ldg(row + lane + 32));
+    m = warp_max(m);
+    if (lane == 0) bscores[(int64_t)h * Tb + j] = m;
+}
+
+int launch_block_max(const float *scores, const int32_t *cu_seq, const int32_t *cu_blk, int B, int Hkv, int64_t T,
+                     int64_t Tb, float *bscores, int32_t *status, cudaStream_t s) {
+    const int64_t warps = (int64_t)Hkv * Tb;
+    if (warps <= 0) return 0;
+    const unsigned grid = (unsigned)((warps + kBlockMaxWarps - 1) / kBlockMaxWarps);
+    return (int)launch_k(block_max_kernel, dim3(grid), dim3(kBlockMaxWarps * 32), 0, s, 1, scores, cu_seq, cu_blk,
+                         B, Hkv, T, Tb, bscores, status);
 }
 
 }  // namespace sgd

@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
                                                     int n_req, int min_chunk, int mode, int granule,
                                                     PlanView pv, WsHeader *hdr, int staged, float *out,
                                                     float *lse, int G, int D, const __nv_bfloat16 *q,
-                                                    int64_t q_elems, int M) {
+                                                    int64_t q_elems, int M, int len_unit) {
     __shared__ int32_t sm[33];
     extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     }
     if (staged) {
         for (int b = tid; b < B; b += blockDim.x) {  // all four loads of a thread in flight together
-            const int32_t a0 = cu_len[b], a1 = cu_len[b + 1], s0 = cu_seq[b], s1 = cu_seq[b + 1];
+            const int32_t a0 = cu_len[b] * len_unit, a1 = cu_len[b + 1] * len_unit, s0 = cu_seq[b], s1 = cu_seq[b + 1];
             seqv[b] = a1 - a0;
             seqv[B + b] = s1 - s0;
             seqv[2 * B + b] = a0;
@@ -56,9 +56,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         }
         __syncthreads();
     }
-    auto len_of = [&](int b) -> int32_t { return staged ? seqv[b] : cu_len[b + 1] - cu_len[b]; };
+    auto len_of = [&](int b) -> int32_t { return staged ? seqv[b] : (cu_len[b + 1] - cu_len[b]) * len_unit; };
     auto seq_len_of = [&](int b) -> int32_t { return staged ? seqv[B + b] : cu_seq[b + 1] - cu_seq[b]; };
-    auto len_start_of = [&](int b) -> int32_t { return staged ? seqv[2 * B + b] : cu_len[b]; };
+    auto len_start_of = [&](int b) -> int32_t { return staged ? seqv[2 * B + b] : cu_len[b] * len_unit; };
     auto seq_start_of = [&](int b) -> int32_t { return staged ? seqv[3 * B + b] : cu_seq[b]; };
 
     // 1. padded stream position of every row
@@ -213,7 +213,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
-                 int G, int D, const void *q_bf16, int64_t q_elems, int M) {
+                 int G, int D, const void *q_bf16, int64_t q_elems, int M, int len_unit) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
@@ -222,7 +222,7 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
     const int nt = std::min(1024, std::max(64, (want + 31) / 32 * 32));
     launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
              min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D,
-             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M);
+             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M, len_unit);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

@@ -143,3 +143,25 @@ def test_quantize_and_select_reject_bad_args_on_host(sgd):
     assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7200, n_parts=3, D=64)) == -3
     assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7200, n_parts=3), sgd.SGD_F32) == -3
     assert sel8(_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x7000, v_norm=0x7202, n_parts=3)) == -4
+
+
+def test_block_entry_points_reject_bad_args_on_host(sgd):
+    L = sgd.lib
+    p = ctypes.c_void_p
+    kv = _kv(sgd)  # B = 2, T = 100: at most 100 / 64 + 2 = 3 blocks
+
+    def sel(n_blocks=3, kept=2, blk=0x7000):
+        return L.sgd_oam_select_blocks(p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv), 1.0, 1e-6, 1, 8, n_blocks,
+                                       p(blk) if blk else None, p(0x8000), kept, p(0x6000), 1 << 20, None)
+
+    assert sel(n_blocks=1) == -2 and sel(n_blocks=4) == -2  # between B and T / 64 + B
+    assert sel(kept=4) == -2 and sel(kept=1) == -2  # kept blocks between B and n_blocks
+    assert sel(blk=0) == -1
+
+    def dec(blk=0x7000, cache=kv, kept=2):
+        return L.sgd_decode_attn_blocks(p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(cache), p(blk) if blk else None,
+                                        p(0x8000), kept, 0, 0, 0, p(0x4000), p(0x5000), p(0x6000), 1 << 20, None)
+
+    assert dec(blk=0) == -1
+    assert dec(kept=4) == -2
+    assert dec(cache=_kv(sgd, dtype=sgd.SGD_F32)) == -3  # tensor-core path only

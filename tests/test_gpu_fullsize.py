@@ -147,3 +147,46 @@ def test_config8_two_query_tokens_int8_128k(sgd):
     ref_out, ref_lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, 2, quant=(*quant, "A"), rows=rows)
     for m in range(2):
         compare_rows(out[:, m], lse[:, m], ref_out[:, m], ref_lse[:, m], rows, wl.G)
+
+
+@pytest.mark.parametrize("n", [6, 9])
+def test_config6_and_9_selection_over_the_int8_cache(sgd, n):
+    # workload 6 keeps tokens, workload 9 whole 64-token blocks, both scored on the INT8 K codes
+    wl = workloads.config(n)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    vn = torch.empty(k.shape[:2], dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths, v_norm=vn)
+    del k, v
+    parts = sgd.n_parts(bt.lengths)
+    kw = dict(k_scale=ks, v_scale=vs, scheme="A", n_parts_=parts)
+    select = sgd.oam_select_blocks if wl.blocks else sgd.oam_select
+    idx, cu_kept, wss = select(q, kc, vc, cu, wl.G, wl.beta, wl.eps, wl.keep_num, wl.keep_den, bt.lengths,
+                               v_norm=vn, **kw)
+    assert sgd.workspace_status(wss) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    ref_idx, ref_cu, scores = oracle.oam_select_int8(bt.q, quant[0], quant[2], bt.v, bt.cu_seqlens, "A", wl.G,
+                                                     wl.beta, wl.eps, wl.keep_num, wl.keep_den)
+    if wl.blocks:
+        ref_idx, ref_cu, scores = oracle.select_blocks(scores, bt.cu_seqlens, wl.Hkv, wl.keep_num, wl.keep_den)
+    assert cu_kept.cpu().tolist() == ref_cu.tolist()
+    got = idx.cpu().numpy()
+    for (b, h), s in scores.items():
+        a, e = int(ref_cu[b]), int(ref_cu[b + 1])
+        kth = np.sort(s)[::-1][e - a - 1]
+        assert (np.diff(got[h, a:e]) > 0).all()
+        for t in set(got[h, a:e].tolist()) ^ set(ref_idx[h, a:e].tolist()):
+            assert abs(s[t] - kth) <= 1e-4, (b, h, t)
+    # the decode over the oracle's selection, in the bench's launch configuration
+    ti, tc = torch.from_numpy(ref_idx).cuda(), torch.from_numpy(ref_cu).cuda()
+    rows = sample_rows(bt, n_extra=2)
+    if wl.blocks:
+        out, lse, ws = sgd.decode_attn_blocks(q, wl.G, kc, vc, cu, ti, tc, **kw)
+        ref = oracle.decode_blocks(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, ref_idx, ref_cu, quant=(*quant, "A"),
+                                   rows=rows)
+    else:
+        out, lse, ws = sgd.decode_attn(q, wl.G, kc, vc, cu, idx=ti, cu_kept=tc, kept_total_=ref_idx.shape[1], **kw)
+        ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
+                            quant=(*quant, "A"), rows=rows)
+    assert sgd.workspace_status(ws) == 0
+    compare_rows(out, lse, *ref, rows, wl.G)

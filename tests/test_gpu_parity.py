@@ -562,3 +562,81 @@ def test_multi_token_with_query_codes(sgd):
                                          n_parts_=sgd.n_parts(bt.lengths), n_splits=9, q_quant="token")
     assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
     check_status(sgd, ws)
+
+
+# ---------------------------------------------------------------------------------------------
+# block-granular selection (64-token blocks ranked by their best token) and decode over blocks
+# ---------------------------------------------------------------------------------------------
+BLOCK_LENGTHS = (1, 64, 65, 130, 700, 4099)
+
+
+@pytest.mark.parametrize("cache", ["bf16", "int8A", "int8B"])
+@pytest.mark.parametrize("G,D", [(8, 128), (4, 64)])
+def test_block_selection_matches_oracle(sgd, cache, G, D):
+    if cache != "bf16" and D != 128:
+        pytest.skip("the INT8 cache is scored at D = 128")
+    bt = make(BLOCK_LENGTHS, G=G, D=D, Hkv=2, dist="outlier", seed=41 + G)
+    q, k, v, cu = dev(bt)
+    if cache == "bf16":
+        blk, cu_kb, ws = sgd.oam_select_blocks(q, k, v, cu, G, 1.0, 1e-6, 1, 4, bt.lengths)
+        _, _, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)
+    else:
+        scheme = cache[-1]
+        vn = torch.empty((2, bt.T), dtype=torch.float32, device="cuda")
+        kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn)
+        blk, cu_kb, ws = sgd.oam_select_blocks(q, kc, vc, cu, G, 1.0, 1e-6, 1, 4, bt.lengths, k_scale=ks,
+                                               v_scale=vs, scheme=scheme, n_parts_=sgd.n_parts(bt.lengths),
+                                               v_norm=vn)
+        rkc, _, rks, _ = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+        _, _, scores = oracle.oam_select_int8(bt.q, rkc, rks, bt.v, bt.cu_seqlens, scheme, G, 1.0, 1e-6, 1, 4)
+    ref_blk, ref_cu, bscores = oracle.select_blocks(scores, bt.cu_seqlens, 2, 1, 4)
+    check_selection(blk, cu_kb.cpu(), ref_blk, ref_cu, bscores, bt.wl.B, 2)
+    check_status(sgd, ws)
+
+
+@pytest.mark.parametrize("cache", ["bf16", "int8A", "int8B"])
+@pytest.mark.parametrize("G,D", [(8, 128), (16, 128), (4, 64)])
+def test_decode_over_blocks_matches_oracle(sgd, cache, G, D):
+    if cache != "bf16" and D != 128:
+        pytest.skip("the INT8 cache decodes on tensor cores at D = 128")
+    bt = make(BLOCK_LENGTHS, G=G, D=D, Hkv=2, dist="outlier", seed=43 + G)
+    q, k, v, cu = dev(bt)
+    # a seeded kept-block set: a quarter of each row's blocks, always with its ragged last block
+    rng = np.random.default_rng(5)
+    nb = [-(-int(L) // 64) for L in BLOCK_LENGTHS]
+    keep = [max(1, -(-n // 4)) for n in nb]
+    cu_kb = np.concatenate([[0], np.cumsum(keep)]).astype(np.int32)
+    blk = np.zeros((2, int(cu_kb[-1])), np.int32)
+    for b, (n, K) in enumerate(zip(nb, keep)):
+        for h in range(2):
+            pick = rng.choice(n - 1, size=K - 1, replace=False) if K > 1 else []
+            blk[h, cu_kb[b]:cu_kb[b + 1]] = np.sort(np.concatenate([pick, [n - 1]])).astype(np.int32)
+    quant, kw, kk, vv = None, {}, k, v
+    if cache != "bf16":
+        scheme = cache[-1]
+        quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme), scheme)
+        kk, vv, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+        kw = dict(k_scale=ks, v_scale=vs, scheme=scheme, n_parts_=sgd.n_parts(bt.lengths))
+    ref = oracle.decode_blocks(bt.q, bt.k, bt.v, bt.cu_seqlens, G, blk, cu_kb, quant=quant)
+    tb, tcu = torch.from_numpy(blk).cuda(), torch.from_numpy(cu_kb).cuda()
+    for n_splits in (0, 7, 300):
+        out, lse, ws = sgd.decode_attn_blocks(q, G, kk, vv, cu, tb, tcu, n_splits=n_splits, **kw)
+        assert_close(out, lse, *ref, OUT_TOL["bf16"])
+        check_status(sgd, ws)
+    # every block kept: the dense decode
+    allb = np.concatenate([np.arange(n, dtype=np.int32) for n in nb])
+    cu_all = np.concatenate([[0], np.cumsum(nb)]).astype(np.int32)
+    tall = torch.from_numpy(np.stack([allb, allb])).cuda()
+    out, lse, _ = sgd.decode_attn_blocks(q, G, kk, vv, cu, tall, torch.from_numpy(cu_all).cuda(), **kw)
+    dense = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, G, quant=quant)
+    assert_close(out, lse, *dense, OUT_TOL["bf16"])
+
+
+def test_decode_over_blocks_reports_a_block_number_out_of_range(sgd):
+    bt = make((130, 300), G=8, D=128, Hkv=1, seed=3)
+    q, k, v, cu = dev(bt)
+    blk = torch.tensor([[0, 7, 1]], dtype=torch.int32, device="cuda")  # sequence 0 has blocks 0..2
+    cu_kb = torch.tensor([0, 2, 3], dtype=torch.int32, device="cuda")
+    out, lse, ws = sgd.decode_attn_blocks(q, 8, k, v, cu, blk, cu_kb)
+    assert sgd.workspace_status(ws) & 0x8  # bad index
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()

@@ -67,6 +67,7 @@ class Workload:
     q_quant: Optional[str] = None  # None, "token" or "tensor": the attention's q.k runs on INT8 query codes
     seed: Optional[int] = None  # the draw's seed when it is not the workload's number
     M: int = 1  # query tokens per sequence and step (speculative decode: 1 + draft tokens)
+    blocks: bool = False  # OAM keeps whole 64-token blocks (ranked by their best token)
 
     @property
     def Hq(self) -> int:
@@ -97,11 +98,15 @@ CONFIGS = {
     # workload 4 with two query tokens per sequence (one draft token): 16 columns per KV head
     8: Workload("spec_M2_int8_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
                 lengths=(131072,) * 8, scheme="A", M=2, seed=4),
+    # workload 6 with block-granular selection: whole 64-token blocks kept, read as contiguous tiles
+    9: Workload("oam_blocks_on_int8cache_A_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
+                dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, select_on_codes=True,
+                blocks=True, seed=6),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..8), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..9), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
