@@ -83,7 +83,12 @@ struct MmaCfg {
     static constexpr bool ROW_SCALE = I8 && IDX;  // per-row K scales fetched by the producer
     static constexpr int SMEM_ROWSCALE = ROW_SCALE ? STAGES * ROWS * 4 : 0;
     static constexpr int SMEM_KMX = 2 * (NQ > 4 ? NQ : 4) * 4;  // [2][NQ] per-warp max|K| (mode 2)
-    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + SMEM_KMX + SMEM_ROWSCALE;
+    // two column tiles of the decode: the Q fragments wait in shared memory (each lane its own
+    // 8 bytes per fragment pair) instead of 32-64 registers that the softmax and PV phases need
+    static constexpr bool QS = GT == 2 && MODE == 0;
+    static constexpr int SMEM_Q = QS ? GT * KB * 32 * 8 : 0;
+    static constexpr int SMEM = 1024 + SMEM_STAGES + 2 * STAGES * 8 + NW * NG * 2 * 4 + 16 + SMEM_KMX + SMEM_ROWSCALE +
+                                SMEM_Q;
     static_assert(ROWB % 128 == 0, "rows are whole 128-byte boxes");
     static_assert(NW * NG * D * 4 <= 2 * TILE, "epilogue fits in one stage");
     static_assert(!(I8 && MODE == 2), "the fused pass reads the unquantised cache");
@@ -351,7 +356,13 @@ __device__ __forceinline__ void load_q_frags(const DecodeArgs &a, int b, int kvh
 // S^T = K_tile(16 x D) * Q^T(D x NG) for this warp's sub-tile.
 template <class C>
 __device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t4,
-                                           const uint32_t (&qf)[C::GT][C::KB][2], float (&sacc)[C::GT][4]) {
+                                           const uint32_t (&qf)[C::GT][C::KB][2], float (&sacc)[C::GT][4],
+                                           uint32_t qsm = 0) {
+    // fragment pair x of column tile gt: registers, or this lane's 8 bytes in shared memory
+    auto qv = [&](int gt, int x) -> uint2 {
+        if constexpr (C::QS) return lds64(qsm + (gt * C::KB + x) * 256);
+        else return make_uint2(qf[gt][x][0], qf[gt][x][1]);
+    };
 #pragma unroll
     for (int gt = 0; gt < C::GT; ++gt) sacc[gt][0] = sacc[gt][1] = sacc[gt][2] = sacc[gt][3] = 0.f;
     const int rA = rb + pA, rB = rA + 8;
@@ -363,8 +374,9 @@ __device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t
             const uint4 ka = lds128(base + rA * 128), kb = lds128(base + rB * 128);
 #pragma unroll
             for (int gt = 0; gt < C::GT; ++gt) {
-                mma_bf16(sacc[gt], ka.x, kb.x, ka.y, kb.y, qf[gt][2 * h][0], qf[gt][2 * h][1]);
-                mma_bf16(sacc[gt], ka.z, kb.z, ka.w, kb.w, qf[gt][2 * h + 1][0], qf[gt][2 * h + 1][1]);
+                const uint2 q0 = qv(gt, 2 * h), q1 = qv(gt, 2 * h + 1);
+                mma_bf16(sacc[gt], ka.x, kb.x, ka.y, kb.y, q0.x, q0.y);
+                mma_bf16(sacc[gt], ka.z, kb.z, ka.w, kb.w, q1.x, q1.y);
             }
         }
     } else if constexpr (C::QI8) {
@@ -380,8 +392,9 @@ __device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t
             const uint4 ka = lds128(base + rA * 128), kb = lds128(base + rB * 128);
 #pragma unroll
             for (int gt = 0; gt < C::GT; ++gt) {
-                mma_s8(ia[gt], ka.x, kb.x, ka.y, kb.y, qf[gt][2 * h][0], qf[gt][2 * h][1]);
-                mma_s8(ia[gt], ka.z, kb.z, ka.w, kb.w, qf[gt][2 * h + 1][0], qf[gt][2 * h + 1][1]);
+                const uint2 q0 = qv(gt, 2 * h), q1 = qv(gt, 2 * h + 1);
+                mma_s8(ia[gt], ka.x, kb.x, ka.y, kb.y, q0.x, q0.y);
+                mma_s8(ia[gt], ka.z, kb.z, ka.w, kb.w, q1.x, q1.y);
             }
         }
 #pragma unroll
@@ -401,8 +414,10 @@ __device__ __forceinline__ void qk_subtile(uint32_t kbase, int rb, int pA, int t
                 s8x4_to_f16x2x2(wa[j], a0, a2);
                 s8x4_to_f16x2x2(wb[j], a1, a3);
 #pragma unroll
-                for (int gt = 0; gt < C::GT; ++gt)
-                    mma_f16(sacc[gt], a0, a1, a2, a3, qf[gt][4 * h + j][0], qf[gt][4 * h + j][1]);
+                for (int gt = 0; gt < C::GT; ++gt) {
+                    const uint2 q = qv(gt, 4 * h + j);
+                    mma_f16(sacc[gt], a0, a1, a2, a3, q.x, q.y);
+                }
             }
         }
     }
@@ -812,6 +827,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
     volatile int32_t *abort_flag = reinterpret_cast<int32_t *>(ml + C::NW * C::NG * 2);
     float *kmxs = ml + C::NW * C::NG * 2 + 4;  // [2][NQ] per-warp max|K| of the current tile (mode 2)
     float *row_scale = kmxs + C::SMEM_KMX / 4;  // [STAGES][ROWS] K scale of each gathered row (INT8 gathers)
+    // [GT][KB][32 lanes] uint2: the Q fragments of the current segment (two column tiles)
+    const uint32_t qsm = smem_u32(row_scale + C::SMEM_ROWSCALE / 4) + (threadIdx.x & 31) * 8;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -863,6 +880,15 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         uint32_t qf[C::GT][C::KB][2];
         float colf[C::GT][2];
         load_q_frags<C>(a, b, kvh, g4, t4, qf, colf);
+        if constexpr (C::QS) {
+            // each lane stores, and later reads, only its own slots; every consumer warp writes the
+            // same values, and none still reads the previous segment's (the epilogue barriers)
+#pragma unroll
+            for (int gt = 0; gt < C::GT; ++gt)
+#pragma unroll
+                for (int x = 0; x < C::KB; ++x) sts64(qsm + (gt * C::KB + x) * 256, qf[gt][x][0], qf[gt][x][1]);
+            __syncwarp();
+        }
         float m[C::GT][2], l[C::GT][2], o[C::GT][C::KB][4];
 #pragma unroll
         for (int gt = 0; gt < C::GT; ++gt) {
@@ -934,7 +960,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
                 if (j0 >= t1 || !ready) continue;
                 float sacc[C::GT][4];
-                qk_subtile<C>(kbase, rb, pA, t4, qf, sacc);
+                qk_subtile<C>(kbase, rb, pA, t4, qf, sacc, qsm);
                 bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
                 if constexpr (C::BLK) {  // the last block of a sequence is ragged
                     vA = bpos[s] + pA < Lb;
