@@ -41,7 +41,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9, 10])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()

@@ -221,9 +221,12 @@ int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
  * p <= L_b - M + m (of the kept tokens when idx is given).  A query token that sees no token
  * (L_b < M - m) gets out = 0 and lse = -inf.  M = 1 is sgd_decode_attn.
  * q        [B, M, Hq, D] BF16;  out [B, M, Hq, D] float32;  lse [B, M, Hq] float32
- * M        1 <= M and G * M <= 16; with M > 1 the cache is BF16 (D 64 or 128) or I8 (D 128)
- *          (SGD_ERR_DTYPE otherwise)
- * workspace   sgd_workspace_size(SGD_OP_DECODE, kv, G * M, schedule, n_splits) bytes
+ * M        1 <= M and G * M <= 64; with M > 1 the cache is BF16 (D 64 or 128) or I8 (D 128)
+ *          (SGD_ERR_DTYPE otherwise).  Above 16 columns (G * M), each split range is run by
+ *          ceil(G * M / 16) CTAs, one per group of 16 (query token, head) columns, that read the
+ *          same K/V tiles (the later ones from L2)
+ * workspace   sgd_workspace_size(SGD_OP_DECODE, kv, G * M, schedule, n_splits) bytes (its G
+ *          argument takes up to 64 for SGD_OP_DECODE)
  * Every other argument, and the error behaviour, as in sgd_decode_attn.
  */
 int sgd_decode_attn_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv,
@@ -248,8 +251,9 @@ int sgd_decode_attn_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv
                            void *stream);
 
 /* Workspace bytes an operation needs for this cache shape (>= 256). For
- * SGD_OP_DECODE, `schedule` and `n_splits` as in sgd_decode_attn; for the
- * other ops they are ignored.  Returns 0 on invalid arguments. */
+ * SGD_OP_DECODE, `schedule` and `n_splits` as in sgd_decode_attn and G the columns per KV
+ * head (G * M of sgd_decode_attn_multi, up to 64); for the other ops they are ignored and
+ * 1 <= G <= 16.  Returns 0 on invalid arguments. */
 size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_splits);
 
 /* Number of CTAs sgd_decode_attn launches for these arguments (the partition's

@@ -85,7 +85,7 @@ Layout layout(int op, int B, int Hkv, int G, int D, int64_t T, int n_req) {
         L.row_info = take(off, (size_t)R * sizeof(RowInfo));
     }
     if (op == SGD_OP_DECODE) {
-        L.row_done = take(off, (size_t)R * 4);
+        L.row_done = take(off, (size_t)R * kMaxColGroups * 4);  // per row and column group
         const int64_t slots = (int64_t)n_req + R;
         L.o_part = take(off, (size_t)slots * G * D * 4);
         L.lse_part = take(off, (size_t)slots * G * 4);
@@ -112,6 +112,8 @@ PlanView plan_view(uint8_t *ws, const Layout &L) {
 }
 
 // CTAs requested from the partition for a decode / score launch.
+// G: columns per KV head (the decode's M * G); above 16 each planned range is run by one CTA per
+// group of 16 columns, so the automatic count is divided among the groups.
 int decode_n_req(const DevInfo &dev, const sgd_kv *kv, sgd_dtype q_dtype, int G, bool indexed, bool score,
                  int schedule, int n_splits, int *n_req) {
     if (schedule == 1 && !score) {
@@ -124,9 +126,10 @@ int decode_n_req(const DevInfo &dev, const sgd_kv *kv, sgd_dtype q_dtype, int G,
         return SGD_OK;
     }
     if (n_splits < 0) return SGD_ERR_ARG;
-    const int per = decode_ctas_per_sm(kv->dtype, q_dtype, kv->D, G, indexed, score);
+    const int per = decode_ctas_per_sm(kv->dtype, q_dtype, kv->D, std::min(G, 16), indexed, score);
     if (per < 1) return SGD_ERR_CUDA;
-    *n_req = dev.sms * per;
+    const int ncg = (G + 15) / 16;
+    *n_req = (dev.sms * per + ncg - 1) / ncg;
     return SGD_OK;
 }
 
@@ -153,8 +156,9 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !out || !lse || !workspace) return SGD_ERR_NULL;
-    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
+    if (G < 1 || G > 16 || M < 1 || G * M > 16 * kMaxColGroups) return SGD_ERR_SHAPE;
     const int NC = G * M;  // the kernels' columns per KV head: (query token, head) pairs
+    const int ncg = (NC + 15) / 16;  // CTAs per planned range, one per 16 columns
     // several query tokens, and kept blocks, run on the tensor-core kernel only
     if ((M > 1 || blocks) && decode_family(kv->dtype, q_dtype, kv->D, false) != kFamilyMma) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
@@ -191,7 +195,7 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     const int min_chunk = (n_splits > 0 || schedule == 1) ? granule : kAutoMinChunk;
     launch_plan(listed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
                 hdr, s, granule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
-                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M, blocks ? kPart : 1);
+                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M, blocks ? kPart : 1, ncg);
     DecodeArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q;
@@ -212,6 +216,7 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     a.T = kv->T;
     a.Kt = listed ? kept_total : 0;
     a.blk = blocks ? 1 : 0;
+    a.ncg = ncg;
     a.n_parts = kv->dtype == SGD_I8 && kv->scheme == SGD_SCHEME_A ? kv->n_parts : 0;
     a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
     a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
@@ -223,7 +228,7 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     a.status = &hdr->status;
     a.q_quant = q_quant;
     a.q_scale = &hdr->q_scale;
-    int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req, s);
+    int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req * ncg, s);
     if (e != 0) return SGD_ERR_CUDA;
     // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials
     if (decode_family(kv->dtype, q_dtype, kv->D, false) == kFamilyMma) return SGD_OK;
@@ -336,7 +341,8 @@ const char *sgd_error_string(int code) {
 size_t sgd_workspace_size(int op, const sgd_kv *kv, int G, int schedule, int n_splits) {
     if (check_kv(kv) != SGD_OK) return 0;
     if (op == SGD_OP_QUANTIZE) return layout(op, kv->B, kv->Hkv, 0, kv->D, kv->T, 0).total;
-    if (G < 1 || G > 16) return 0;
+    // G: query heads per KV head; for the decode, the columns M * G of sgd_decode_attn_multi
+    if (G < 1 || G > (op == SGD_OP_DECODE ? 16 * kMaxColGroups : 16)) return 0;
     DevInfo *dev;
     if (current_device(&dev) != SGD_OK) return 0;
     int n_req = 0;

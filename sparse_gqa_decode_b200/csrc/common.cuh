@@ -33,6 +33,7 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr int kGranule = 16;      // plan granularity (tokens)
+constexpr int kMaxColGroups = 4;  // decode columns per KV head up to 4 x 16 (M * G <= 64)
 constexpr int kPart = SGD_PARTITION;
 constexpr long long kWaitLimit = 1 << 22;  // bounded mbarrier polls before giving up
 

@@ -271,10 +271,10 @@ __device__ __forceinline__ int64_t col_row(const DecodeArgs &a, int b, int kvh, 
 // per-column logit factor (log2 units; INT8 also undoes the power-of-two Q pre-scale).
 template <class C>
 __device__ __forceinline__ void load_q_frags(const DecodeArgs &a, int b, int kvh, int g4, int t4,
-                                             uint32_t (&qf)[C::GT][C::KB][2], float (&colf)[C::GT][2]) {
+                                             uint32_t (&qf)[C::GT][C::KB][2], float (&colf)[C::GT][2], int col0 = 0) {
 #pragma unroll
     for (int gt = 0; gt < C::GT; ++gt) {
-        const int g = 8 * gt + g4;
+        const int g = col0 + 8 * gt + g4;  // column: this CTA's column group starts at col0
         const bool live = g < a.G * a.M;
         const __nv_bfloat16 *qrow = static_cast<const __nv_bfloat16 *>(a.q) + col_row(a, b, kvh, live ? g : 0) * C::D;
         if constexpr (!C::I8) {
@@ -685,26 +685,30 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
 // lse = ln sum_c exp(lse_c), out = sum_c exp(lse_c - lse) o_c, as merge_kernel computes it.
 // ------------------------------------------------------------------------------------------
 template <class C>
-__device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n, int b, int kvh, float *scratch) {
+__device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n, int b, int kvh, float *scratch,
+                                          int col0 = 0) {
     constexpr int NT = C::NW * 32;
-    const int G = a.G * a.M, tid = threadIdx.x;  // G here: the row's columns, (query token, head) pairs
+    // G here: this CTA's columns col0 .. col0 + G - 1 of the row's NCt (query token, head) pairs;
+    // a slot holds all NCt columns
+    const int NCt = a.G * a.M, G = min(C::NG, NCt - col0), tid = threadIdx.x;
     float *Ls = scratch;                       // [16] per head: running max, then the lse
     float *Ss = scratch + 16;                  // [16] running sum
     float *w = scratch + 32;                   // [chunk][G] lse, then weights
     const int chunk = (2 * C::TILE / 4 - 32) / G;
-    const float *lp = a.lse_part + (int64_t)slot0 * G;
-    const float *op = a.o_part + (int64_t)slot0 * G * C::D;
+    const float *lp = a.lse_part + (int64_t)slot0 * NCt + col0;  // lse of (slot c, column j): lp[c * NCt + j]
+    const float *op = a.o_part + ((int64_t)slot0 * NCt + col0) * C::D;
+    auto lse_at = [&](int c, int p) { return __ldcg(lp + (int64_t)(c + p / G) * NCt + p % G); };
     constexpr int kQ4 = C::NG * C::D / 4 / NT;  // float4 columns per thread at the most columns
-    const int Q = G * C::D / 4;
-    // float4 q of the row's [G][D] block -> its place in out (column n = 4q / D)
+    const int Q = G * C::D / 4, QSt = NCt * C::D / 4;  // float4s of this CTA's columns / of a slot
+    // float4 q of the CTA's [G][D] block -> its place in out (column col0 + 4q / D)
     auto dst4 = [&](int q) -> float4 & {
         const int n = (4 * q) / C::D;
-        return *reinterpret_cast<float4 *>(a.out + col_row(a, b, kvh, n) * C::D + (4 * q - n * C::D));
+        return *reinterpret_cast<float4 *>(a.out + col_row(a, b, kvh, col0 + n) * C::D + (4 * q - n * C::D));
     };
     if (n <= chunk) {
         // one round: every lse loaded once, the weights computed in place, then thread t reads
         // its float4 columns t, t + NT, ... of every slot, eight slots' loads in flight
-        for (int p = tid; p < n * G; p += NT) w[p] = __ldcg(lp + p);
+        for (int p = tid; p < n * G; p += NT) w[p] = lse_at(0, p);
         named_barrier_sync(1, NT);
         if (tid < G) {
             float M = -INFINITY, S = 0.f;
@@ -726,7 +730,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
             for (int j = 0; j < kQ4; ++j) {
                 const int q = tid + j * NT;
                 if (q < Q) {
-                    const float4 x = __ldcg(oc + (int64_t)c * Q + q);
+                    const float4 x = __ldcg(oc + (int64_t)c * QSt + q);
                     const float wc = w[c * G + (4 * q) / C::D];
                     acc[j].x += wc * x.x;
                     acc[j].y += wc * x.y;
@@ -740,7 +744,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
             const int q = tid + j * NT;
             if (q < Q) dst4(q) = acc[j];
         }
-        if (tid < G) a.lse[col_row(a, b, kvh, tid)] = Ls[tid];
+        if (tid < G) a.lse[col_row(a, b, kvh, col0 + tid)] = Ls[tid];
         named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
         return;
     }
@@ -753,7 +757,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
     for (int c0 = 0; c0 < n; c0 += chunk) {  // pass 1: max and sum of exp per head, online
         const int m = min(chunk, n - c0);
         named_barrier_sync(1, NT);
-        for (int p = tid; p < m * G; p += NT) w[p] = __ldcg(lp + (int64_t)c0 * G + p);
+        for (int p = tid; p < m * G; p += NT) w[p] = lse_at(c0, p);
         named_barrier_sync(1, NT);
         if (tid < G) {
             float M = Ls[tid], S = Ss[tid];
@@ -778,9 +782,9 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
         const int m = min(chunk, n - c0);
         named_barrier_sync(1, NT);
         for (int p = tid; p < m * G; p += NT)
-            w[p] = (Ls[p % G] > -INFINITY) ? expf(__ldcg(lp + (int64_t)c0 * G + p) - Ls[p % G]) : 0.f;
+            w[p] = (Ls[p % G] > -INFINITY) ? expf(lse_at(c0, p) - Ls[p % G]) : 0.f;
         named_barrier_sync(1, NT);
-        const float4 *oc = reinterpret_cast<const float4 *>(op + (int64_t)c0 * G * C::D);
+        const float4 *oc = reinterpret_cast<const float4 *>(op + (int64_t)c0 * NCt * C::D);
         float4 acc[kQ4];
 #pragma unroll
         for (int j = 0; j < kQ4; ++j) {
@@ -793,7 +797,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
             for (int j = 0; j < kQ4; ++j) {
                 const int q = tid + j * NT;
                 if (q < Q) {
-                    const float4 x = __ldcg(oc + (int64_t)c * Q + q);
+                    const float4 x = __ldcg(oc + (int64_t)c * QSt + q);
                     const float wc = w[c * G + (4 * q) / C::D];
                     acc[j].x += wc * x.x;
                     acc[j].y += wc * x.y;
@@ -808,7 +812,7 @@ __device__ __forceinline__ void merge_row(const DecodeArgs &a, int slot0, int n,
             if (q < Q) dst4(q) = acc[j];
         }
     }
-    if (tid < G) a.lse[col_row(a, b, kvh, tid)] = Ls[tid];
+    if (tid < G) a.lse[col_row(a, b, kvh, col0 + tid)] = Ls[tid];
     named_barrier_sync(1, NT);  // scratch is the stage's memory: free again
 }
 
@@ -840,7 +844,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         fence_barrier_init();
     }
     __syncthreads();
-    const int cta = blockIdx.x;
+    // decode with more than 16 columns: ncg CTAs share each planned range, one group of 16 each
+    const int ncg = (C::MODE == 0 && a.ncg > 1) ? a.ncg : 1;
+    const int cta = blockIdx.x / ncg, cg = blockIdx.x - cta * ncg;
+    const int col0 = cg * C::NG;
     if (a.plan.cta_begin[cta] >= a.plan.cta_begin[cta + 1]) return;
     if constexpr (C::MODE == 2) {
         // scheme-A scales are written at kvh * n_parts + (partition): the device count must agree
@@ -879,7 +886,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
         const int64_t tok_base = (int64_t)kvh * a.T + seq_start;  // cache row of token 0 of the sequence
         uint32_t qf[C::GT][C::KB][2];
         float colf[C::GT][2];
-        load_q_frags<C>(a, b, kvh, g4, t4, qf, colf);
+        load_q_frags<C>(a, b, kvh, g4, t4, qf, colf, col0);
         if constexpr (C::QS) {
             // each lane stores, and later reads, only its own slots; every consumer warp writes the
             // same values, and none still reads the previous segment's (the epilogue barriers)
@@ -983,7 +990,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                         for (int gt = 0; gt < C::GT; ++gt)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int32_t lim = lim0 + (8 * gt + 2 * t4 + (e & 1)) / a.G;
+                                const int32_t lim = lim0 + (col0 + 8 * gt + 2 * t4 + (e & 1)) / a.G;
                                 cm |= (uint32_t)((e < 2 ? pa : pb) <= lim) << (4 * gt + e);
                             }
                     }
@@ -1089,7 +1096,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
                 named_barrier_sync(1, C::NW * 32);
                 const int tid = threadIdx.x;
-                const int NC = a.G * a.M;  // columns: (query token, head) pairs
+                const int NCt = a.G * a.M;                 // columns of a row: (query token, head) pairs
+                const int NC = min(C::NG, NCt - col0);     // this CTA's: col0 .. col0 + NC - 1
                 if (tid < NC) {  // column n: the warps' weights replace their m in ml; the lse replaces warp 0's l
                     float M = -INFINITY, f[C::NW], L = 0.f;
 #pragma unroll
@@ -1107,30 +1115,30 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 named_barrier_sync(1, C::NW * 32);
                 // a row's only segment is its result; otherwise a partial in the segment's slot
                 const bool direct = cur.ri.nseg == 1;
-                float *part = a.o_part + (int64_t)slot * NC * C::D;
+                float *part = a.o_part + ((int64_t)slot * NCt + col0) * C::D;
                 for (int e = tid; e < NC * C::D; e += C::NW * 32) {
                     const int g = e / C::D, d = e - g * C::D;
                     float O = 0.f;
 #pragma unroll
                     for (int w = 0; w < C::NW; ++w) O += ml[(w * C::NG + g) * 2] * eo[(w * C::NG + g) * C::D + d];
-                    if (direct) a.out[col_row(a, b, kvh, g) * C::D + d] = O;
+                    if (direct) a.out[col_row(a, b, kvh, col0 + g) * C::D + d] = O;
                     else part[e] = O;
                 }
                 if (tid < NC) {
                     const float lv = ml[tid * 2 + 1];
-                    if (direct) a.lse[col_row(a, b, kvh, tid)] = lv;
-                    else a.lse_part[(int64_t)slot * NC + tid] = lv;
+                    if (direct) a.lse[col_row(a, b, kvh, col0 + tid)] = lv;
+                    else a.lse_part[(int64_t)slot * NCt + col0 + tid] = lv;
                 }
                 if (!direct) {
                     // the CTA that finishes the row's last outstanding segment merges the row
                     volatile int *merge_flag = reinterpret_cast<volatile int *>(kmxs);
                     __threadfence();
                     named_barrier_sync(1, C::NW * 32);
-                    if (tid == 0) *merge_flag = atomicAdd(a.plan.row_done + row, 1) == cur.ri.nseg - 1;
+                    if (tid == 0) *merge_flag = atomicAdd(a.plan.row_done + row * ncg + cg, 1) == cur.ri.nseg - 1;
                     named_barrier_sync(1, C::NW * 32);
                     if (*merge_flag) {
                         __threadfence();
-                        merge_row<C>(a, cur.ri.slot0, cur.ri.nseg, b, kvh, reinterpret_cast<float *>(sk));
+                        merge_row<C>(a, cur.ri.slot0, cur.ri.nseg, b, kvh, reinterpret_cast<float *>(sk), col0);
                     }
                 }
                 fence_proxy_async_shared();
@@ -1486,7 +1494,7 @@ int score_quantize_ctas_per_sm(int D, int G) {
 int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, bool score, int n_cta,
                   cudaStream_t s) {
     if (n_cta <= 0) return 0;
-    const bool g2 = a.G * a.M > 8;  // columns: (query token, head) pairs of a KV head
+    const bool g2 = std::min(a.G * a.M, 16) > 8;  // columns of one CTA: (query token, head) pairs
     if (decode_family(kv, q, a.D, score) == kFamilyMma) {
         if (score) {
             if (kv == SGD_I8) return g2 ? launch_mma_idx<128, 2, true, 1>(a, false, n_cta, s) : launch_mma_idx<128, 1, true, 1>(a, false, n_cta, s);

@@ -21,6 +21,7 @@ struct DecodeArgs {
     int M;                   // decode: query tokens per sequence (>= 1), causal over the cache's last M;
                              // the kernel's columns are the M * G (token, head) pairs of a KV head
     int blk;                 // decode: idx / cu_kept / Kt list kept 64-token blocks, not tokens
+    int ncg;                 // decode: CTAs per planned range, one per group of 16 columns (M * G > 16)
     int64_t T, Kt, n_parts;
     int q_f32;               // q is float32 (otherwise bf16)
     float sm_scale_log2;     // log2(e) / sqrt(D)
@@ -52,7 +53,7 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
                  float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0, const void *q_bf16 = nullptr,
-                 int64_t q_elems = 0, int M = 1, int len_unit = 1);
+                 int64_t q_elems = 0, int M = 1, int len_unit = 1, int ncg = 1);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 

@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
                                                     int n_req, int min_chunk, int mode, int granule,
                                                     PlanView pv, WsHeader *hdr, int staged, float *out,
                                                     float *lse, int G, int D, const __nv_bfloat16 *q,
-                                                    int64_t q_elems, int M, int len_unit) {
+                                                    int64_t q_elems, int M, int len_unit, int ncg) {
     __shared__ int32_t sm[33];
     extern __shared__ int32_t stage[];
     const int tid = threadIdx.x;
@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
             int4 *ri = reinterpret_cast<int4 *>(pv.row_info + r);
             ri[0] = make_int4(row_pos[r], len_of(b), seq_start_of(b), seq_len_of(b));
             ri[1] = make_int4(len_start_of(b), part0[b], carry + ex, v);
-            if (pv.row_done) pv.row_done[r] = 0;
+            if (pv.row_done)  // one finished-segment counter per row and column group
+                for (int j = 0; j < ncg; ++j) pv.row_done[r * ncg + j] = 0;
             if (out && v == 0) {  // a row with no tokens (reported above): zero output, lse -inf
                 for (int m = 0; m < M; ++m) {
                     const int64_t h0 = ((int64_t)b * M + m) * Hkv * G + (r / B) * G;
@@ -213,7 +214,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
-                 int G, int D, const void *q_bf16, int64_t q_elems, int M, int len_unit) {
+                 int G, int D, const void *q_bf16, int64_t q_elems, int M, int len_unit, int ncg) {
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
@@ -222,7 +223,7 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
     const int nt = std::min(1024, std::max(64, (want + 31) / 32 * 32));
     launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
              min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D,
-             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M, len_unit);
+             static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M, len_unit, ncg);
 }
 
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,

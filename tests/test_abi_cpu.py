@@ -107,7 +107,7 @@ def test_multi_token_decode_rejects_bad_args_on_host(sgd):
         return L.sgd_decode_attn_multi(p(0x3000), qdt, G, M, ctypes.byref(kv), None, None, 0, 0, 0, 0, p(0x4000),
                                        p(0x5000), p(0x6000), 1 << 20, None)
 
-    assert call(M=0) == -2 and call(M=3) == -2 and call(G=16, M=2) == -2  # G * M <= 16
+    assert call(M=0) == -2 and call(M=9) == -2 and call(G=16, M=5) == -2  # G * M <= 64
     assert call(cache=_kv(sgd, dtype=sgd.SGD_F32), qdt=sgd.SGD_F32) == -3  # tensor-core path only
     assert call(cache=_kv(sgd, dtype=sgd.SGD_I8, k_scale=0x30000, v_scale=0x40000, scheme=1, D=64)) == -3
 

@@ -510,9 +510,10 @@ def kept_with_tail(lengths, Hkv, M, seed):
 
 
 @pytest.mark.parametrize("kvdt", ["bf16", "int8A"])
-@pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (16, 1)])
+@pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (16, 1), (4, 8), (3, 16), (8, 8)])
 @pytest.mark.parametrize("indexed", [False, True])
 def test_multi_token_decode(sgd, kvdt, M, G, indexed):
+    # up to 16 columns (M * G) one CTA per range; 32, 48 and 64 columns: 2, 3 and 4 CTAs per range
     lengths = (1, 3, 70, 700, 3001)
     bt = make_multi(lengths, M, G, seed=31 + M)
     q, k, v, cu = dev(bt)

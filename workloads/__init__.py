@@ -102,11 +102,15 @@ CONFIGS = {
     9: Workload("oam_blocks_on_int8cache_A_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, select_on_codes=True,
                 blocks=True, seed=6),
+    # workload 4's cache with four query tokens (three draft tokens): 32 columns per KV head, two
+    # CTAs per split range
+    10: Workload("spec_M4_int8_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                 lengths=(131072,) * 8, scheme="A", M=4, seed=4),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..9), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..10), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
