@@ -953,49 +953,60 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
             uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
             const uint32_t kbase = smem_u32(sk), vbase = smem_u32(sv);
+            if constexpr (C::MODE >= 1) {
 #pragma unroll
-            for (int s = 0; s < C::SUB; ++s) {
-                const int rb = 16 * (s * C::NW + warp);
-                const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
-                if constexpr (C::MODE >= 1) {
+                for (int s = 0; s < C::SUB; ++s) {
+                    const int rb = 16 * (s * C::NW + warp);
+                    const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
                     if constexpr (C::I8)
                         score_subtile_i8<C>(a, kbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, colf, rf_pre[s],
                                             vn_cur[s]);
                     else
                         score_subtile<C>(a, kbase, vbase, rb, j0, t1, ready, tok_base, pA, t4, lane, qf, run_vmax);
-                    continue;
                 }
-                if (j0 >= t1 || !ready) continue;
-                float sacc[C::GT][4];
-                qk_subtile<C>(kbase, rb, pA, t4, qf, sacc, qsm);
-                bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
-                if constexpr (C::BLK) {  // the last block of a sequence is ragged
-                    vA = bpos[s] + pA < Lb;
-                    vB = bpos[s] + pA + 8 < Lb;
-                }
-                // several query tokens: token m sees sequence positions <= L_b - M + m; bit 4 gt + e
-                // keeps element e of column tile gt (only sub-tiles reaching the last M - 1
-                // positions mask anything)
-                uint32_t cm = ~0u;
-                if constexpr (C::CAUSAL) {
-                    int32_t pa = j0 + pA, pb = pa + 8;
-                    if constexpr (C::IDX) {
-                        pa = vA ? __ldg(ip + j0 + pA) : 0;
-                        pb = vB ? __ldg(ip + j0 + pA + 8) : 0;
-                    }
-                    const int32_t lim0 = Lb - a.M;
-                    if (__any_sync(0xffffffffu, max(pa, pb) > lim0)) {
-                        cm = 0u;
+            } else if (ready) {
+                // 1. logits of the warp's sub-tiles (log2 units, -inf where masked); 2. one running
+                // max update per column for all of them; 3. probabilities and O += V^T P^T per sub-tile.
+                // The sub-tiles' QK and PV chains are independent, so they overlap.
+                float z[C::SUB][C::GT][4];
+                bool live[C::SUB];
 #pragma unroll
-                        for (int gt = 0; gt < C::GT; ++gt)
+                for (int s = 0; s < C::SUB; ++s) {
+                    const int rb = 16 * (s * C::NW + warp);
+                    const int32_t j0 = t + rb;  // row-local position of sub-tile row 0
+                    live[s] = j0 < t1;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int32_t lim = lim0 + (col0 + 8 * gt + 2 * t4 + (e & 1)) / a.G;
-                                cm |= (uint32_t)((e < 2 ? pa : pb) <= lim) << (4 * gt + e);
-                            }
+                    for (int gt = 0; gt < C::GT; ++gt) z[s][gt][0] = z[s][gt][1] = z[s][gt][2] = z[s][gt][3] = -INFINITY;
+                    if (!live[s]) continue;
+                    float sacc[C::GT][4];
+                    qk_subtile<C>(kbase, rb, pA, t4, qf, sacc, qsm);
+                    bool vA = j0 + pA < t1, vB = j0 + pA + 8 < t1;
+                    if constexpr (C::BLK) {  // the last block of a sequence is ragged
+                        vA = bpos[s] + pA < Lb;
+                        vB = bpos[s] + pA + 8 < Lb;
                     }
-                }
-                {
+                    // several query tokens: token m sees sequence positions <= L_b - M + m; bit 4 gt + e
+                    // keeps element e of column tile gt (only sub-tiles reaching the last M - 1
+                    // positions mask anything)
+                    uint32_t cm = ~0u;
+                    if constexpr (C::CAUSAL) {
+                        int32_t pa = j0 + pA, pb = pa + 8;
+                        if constexpr (C::IDX) {
+                            pa = vA ? __ldg(ip + j0 + pA) : 0;
+                            pb = vB ? __ldg(ip + j0 + pA + 8) : 0;
+                        }
+                        const int32_t lim0 = Lb - a.M;
+                        if (__any_sync(0xffffffffu, max(pa, pb) > lim0)) {
+                            cm = 0u;
+#pragma unroll
+                            for (int gt = 0; gt < C::GT; ++gt)
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int32_t lim = lim0 + (col0 + 8 * gt + 2 * t4 + (e & 1)) / a.G;
+                                    cm |= (uint32_t)((e < 2 ? pa : pb) <= lim) << (4 * gt + e);
+                                }
+                        }
+                    }
                     // row (token) factors: scheme-A K scale of the token's 64-token partition
                     float rfA = rf_pre[s], rfB = rf_pre[s];
                     if constexpr (C::ROW_SCALE) {
@@ -1004,7 +1015,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                             rfB = row_scale[stage * C::ROWS + rb + pA + 8];
                         }
                     }
-                    uint32_t pb[C::GT][2];
 #pragma unroll
                     for (int gt = 0; gt < C::GT; ++gt) {
                         bool k0 = vA, k1 = vA, k2 = vB, k3 = vB;
@@ -1014,40 +1024,57 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                             k2 = k2 && (cm >> (4 * gt + 2) & 1u);
                             k3 = k3 && (cm >> (4 * gt + 3) & 1u);
                         }
-                        const float z0 = k0 ? sacc[gt][0] * rfA * colf[gt][0] : -INFINITY;
-                        const float z1 = k1 ? sacc[gt][1] * rfA * colf[gt][1] : -INFINITY;
-                        const float z2 = k2 ? sacc[gt][2] * rfB * colf[gt][0] : -INFINITY;
-                        const float z3 = k3 ? sacc[gt][3] * rfB * colf[gt][1] : -INFINITY;
-                        float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+                        if (k0) z[s][gt][0] = sacc[gt][0] * rfA * colf[gt][0];
+                        if (k1) z[s][gt][1] = sacc[gt][1] * rfA * colf[gt][1];
+                        if (k2) z[s][gt][2] = sacc[gt][2] * rfB * colf[gt][0];
+                        if (k3) z[s][gt][3] = sacc[gt][3] * rfB * colf[gt][1];
+                    }
+                }
+                float mu[C::GT][2];
 #pragma unroll
-                        for (int off = 4; off < 32; off <<= 1) {
-                            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                        }
-                        if (mx0 > m[gt][0]) {
-                            const float al = exp2f(m[gt][0] - mx0);
-                            m[gt][0] = mx0;
-                            l[gt][0] *= al;
+                for (int gt = 0; gt < C::GT; ++gt) {
+                    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                            for (int mt = 0; mt < C::KB; ++mt) {
-                                o[gt][mt][0] *= al;
-                                o[gt][mt][2] *= al;
-                            }
-                        }
-                        if (mx1 > m[gt][1]) {
-                            const float al = exp2f(m[gt][1] - mx1);
-                            m[gt][1] = mx1;
-                            l[gt][1] *= al;
+                    for (int s = 0; s < C::SUB; ++s) {
+                        mx0 = fmaxf(mx0, fmaxf(z[s][gt][0], z[s][gt][2]));
+                        mx1 = fmaxf(mx1, fmaxf(z[s][gt][1], z[s][gt][3]));
+                    }
 #pragma unroll
-                            for (int mt = 0; mt < C::KB; ++mt) {
-                                o[gt][mt][1] *= al;
-                                o[gt][mt][3] *= al;
-                            }
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    }
+                    if (mx0 > m[gt][0]) {
+                        const float al = exp2f(m[gt][0] - mx0);
+                        m[gt][0] = mx0;
+                        l[gt][0] *= al;
+#pragma unroll
+                        for (int mt = 0; mt < C::KB; ++mt) {
+                            o[gt][mt][0] *= al;
+                            o[gt][mt][2] *= al;
                         }
-                        const float mu0 = (m[gt][0] == -INFINITY) ? 0.f : m[gt][0];
-                        const float mu1 = (m[gt][1] == -INFINITY) ? 0.f : m[gt][1];
-                        const float p0 = exp2f(z0 - mu0), p2 = exp2f(z2 - mu0);
-                        const float p1 = exp2f(z1 - mu1), p3 = exp2f(z3 - mu1);
+                    }
+                    if (mx1 > m[gt][1]) {
+                        const float al = exp2f(m[gt][1] - mx1);
+                        m[gt][1] = mx1;
+                        l[gt][1] *= al;
+#pragma unroll
+                        for (int mt = 0; mt < C::KB; ++mt) {
+                            o[gt][mt][1] *= al;
+                            o[gt][mt][3] *= al;
+                        }
+                    }
+                    mu[gt][0] = (m[gt][0] == -INFINITY) ? 0.f : m[gt][0];
+                    mu[gt][1] = (m[gt][1] == -INFINITY) ? 0.f : m[gt][1];
+                }
+#pragma unroll
+                for (int s = 0; s < C::SUB; ++s) {
+                    if (!live[s]) continue;
+                    uint32_t pb[C::GT][2];
+#pragma unroll
+                    for (int gt = 0; gt < C::GT; ++gt) {
+                        const float p0 = exp2f(z[s][gt][0] - mu[gt][0]), p2 = exp2f(z[s][gt][2] - mu[gt][0]);
+                        const float p1 = exp2f(z[s][gt][1] - mu[gt][1]), p3 = exp2f(z[s][gt][3] - mu[gt][1]);
                         l[gt][0] += p0 + p2;
                         l[gt][1] += p1 + p3;
                         const uint32_t r0 = C::I8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
@@ -1055,7 +1082,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                         pb[gt][0] = movmatrix_trans(r0);
                         pb[gt][1] = movmatrix_trans(r1);
                     }
-                    pv_subtile<C>(vbase, rb, lane, pb, o);
+                    pv_subtile<C>(vbase, 16 * (s * C::NW + warp), lane, pb, o);
                 }
             }
             ++tile_no;
