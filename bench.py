@@ -18,6 +18,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -88,6 +89,52 @@ def algorithmic_bytes(wl, lengths):
     scales = (Hkv * P * 4 if wl.scheme == "A" else 8) if wl.scheme else 0
     st["decode"] = 2 * Hkv * n_att * D * eb + idx_bytes + scales + wl.M * (q + out)  # M query tokens
     return st
+
+
+def kernel_role(name):
+    """What a library kernel (demangled name) does in the step."""
+    if "decode_mma_kernel" in name:
+        m = re.search(r"MmaCfg<\d+, \d+, \w+, \w+, (\d+)", name)
+        return {"0": "decode", "1": "score", "2": "score_quantize"}.get(m.group(1) if m else "", "decode")
+    for key, role in (("quant_global_kernel", "v_codes"), ("topk_cluster_kernel", "topk"), ("plan_kernel", "plan"),
+                      ("block_max_kernel", "block_max"), ("quant_k_partition_kernel", "k_codes"),
+                      ("quant_amax_kernel", "amax"), ("quant_prep_kernel", "prep"), ("merge_kernel", "merge"),
+                      ("decode_generic_kernel", "decode")):
+        if key in name:
+            return role
+    return name
+
+
+def kernel_bytes(wl, lengths, role):
+    """Bytes the kernel of this role must move per launch (inputs read once, outputs written
+    once), or None where no figure is stated."""
+    Hkv, D, B = wl.Hkv, wl.D, wl.B
+    T = int(sum(lengths))
+    P = int(sum((int(L) + 63) // 64 for L in lengths))
+    q = B * wl.M * Hkv * wl.G * D * 2
+    scales = Hkv * P * 4 if wl.scheme == "A" else 4
+    if role == "score_quantize":  # K and V (bf16) in; K codes, scheme-A scales, scores out
+        return 2 * Hkv * T * D * 2 + Hkv * T * D + scales + Hkv * T * 4 + q
+    if role == "v_codes":  # V (bf16) in, V codes out
+        return Hkv * T * D * 2 + Hkv * T * D + 4
+    if role == "k_codes":  # K and V in (max|V| on the way), K codes and scales out
+        return 2 * Hkv * T * D * 2 + Hkv * T * D + scales
+    if role == "score":  # INT8 K codes, value norms and scales in; scores out
+        return Hkv * T * D + Hkv * T * 4 + scales + q + Hkv * T * 4
+    if role == "decode":
+        return algorithmic_bytes(wl, lengths)["decode"]
+    return None
+
+
+def demangle(names):
+    try:
+        r = subprocess.run(["c++filt"], input="\n".join(names), capture_output=True, text=True, timeout=30)
+        out = r.stdout.splitlines()
+        if r.returncode == 0 and len(out) == len(names):
+            return out
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return list(names)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -261,14 +308,15 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)"
 
 
-def load_traffic(stage, wl_name):
-    """DRAM bytes of the stage from a committed ncu summary, if its kernels are unchanged."""
+def load_traffic(key, wl_name, kind="kernels"):
+    """DRAM bytes per launch of a kernel role (kind "kernels") or per call of a stage ("stages")
+    from a committed ncu summary, if the sources it was taken from are unchanged."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         d = json.load(open(path))
     except (OSError, ValueError):
         return None
-    ent = d.get(wl_name, {}).get(stage)
+    ent = d.get(wl_name, {}).get(kind, {}).get(key)
     if not ent:
         return None
     srcs = [os.path.join(ROOT, p) for p in ent["sources"]]
@@ -418,6 +466,19 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
+    # per kernel: the same eager steps once more with every library launch bracketed by events
+    # on its stream (outside the timed region above)
+    per_kernel = {}
+    for i in range(K):
+        flush_l2(i)
+        sgd.kernel_timing_start(64)
+        pipe.run()
+        got = sgd.kernel_timing_stop()
+        for (name, ms), dn in zip(got, demangle([n for n, _ in got])):
+            ent = per_kernel.setdefault(kernel_role(dn), {"name": dn.split("(")[0], "ms": [], "per_step": 0})
+            ent["ms"].append(ms)
+    for ent in per_kernel.values():
+        ent["per_step"] = len(ent["ms"]) // K
     st = sgd.workspace_status(pipe.ws_d)
     if st:
         raise RuntimeError(f"device status {st:#x} after the timed steps")
@@ -461,11 +522,22 @@ def run_ours(args, rank, world, local_rank):
     med = {n: statistics.median(v) for n, v in stage_ms.items()}
     dom = max(med, key=lambda n: med[n])
     achieved = stages[dom] / (med[dom] / 1e3) / 1e9
+    # the dominant kernel: the largest time per step among the library's kernels
+    kern_report = {}
+    for role, ent in per_kernel.items():
+        kern_report[role] = {"kernel": ent["name"], "launches_per_step": ent["per_step"],
+                             "ms_per_launch": round(statistics.mean(ent["ms"]), 4),
+                             "ms_per_step": round(sum(ent["ms"]) / K, 4)}
+        kb = kernel_bytes(wl, pipe.lengths, role) if ent["per_step"] == 1 else None
+        if kb is not None:
+            gbs = kb / (statistics.mean(ent["ms"]) / 1e3) / 1e9
+            kern_report[role].update({"algorithmic_bytes": kb, "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4)})
+    dom_k = max(kern_report, key=lambda r: kern_report[r]["ms_per_step"]) if kern_report else None
     kernels = {"quantize_select": "sgd_quantize_select (plan + fused OAM score/K quantise + V codes + top-K)",
                "quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
                "select": "sgd_oam_select (plan + OAM score + top-K kernels)",
                "decode": "sgd_decode_attn (plan + split decode + merge kernels)"}
-    traffic = load_traffic(dom, wl.name)
+    traffic = load_traffic(dom, wl.name, "stages")
     stage_report = {}
     for n in names:
         gbs = stages[n] / (med[n] / 1e3) / 1e9
@@ -502,9 +574,19 @@ def run_ours(args, rank, world, local_rank):
         "pct_hbm_peak": round(100 * value / world / peak, 2),
         "seq_heads_per_s": round(world * wl.B * wl.Hq / (ms_per_step / 1e3), 1),
         "stages": stage_report,
-        "roofline": {"bound": "hbm", "kernel": kernels[dom], "achieved": round(achieved, 1), "peak": peak,
-                     "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "algorithmic_bytes": stages[dom]},
+        "kernels": kern_report,
+        "roofline": ({"bound": "hbm", "kernel": kern_report[dom_k]["kernel"], "role": dom_k,
+                      "achieved": kern_report[dom_k]["GB_s"], "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                      "frac": kern_report[dom_k]["frac_of_hbm"], "traffic": load_traffic(dom_k, wl.name),
+                      "algorithmic_bytes": kern_report[dom_k]["algorithmic_bytes"],
+                      "launch_ms": kern_report[dom_k]["ms_per_launch"],
+                      "timing": "CUDA events around each launch on its stream, eager steps, L2 flushed between steps"}
+                     if dom_k is not None and "GB_s" in kern_report[dom_k] else
+                     {"bound": "hbm", "kernel": kernels[dom], "achieved": round(achieved, 1), "peak": peak,
+                      "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                      "traffic": traffic, "algorithmic_bytes": stages[dom]}),
+        "stage_roofline": {"stage": dom, "calls": kernels[dom], "achieved": round(achieved, 1),
+                           "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": stages[dom]},
         "e2e": {"value": round(job_gbs(step_bytes, 1, e2e_ms, world), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": pipe.launches_per_step() * K,

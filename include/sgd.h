@@ -313,6 +313,21 @@ int sgd_workspace_status(const void *workspace, int32_t *status, void *stream);
 /* Static text for a status code. */
 const char *sgd_error_string(int code);
 
+/*
+ * Per-kernel timing, a measurement aid (not thread-safe; host state of the process).
+ * sgd_kernel_timing_start: creates 2 * max_launches CUDA events (1 <= max_launches <= 4096);
+ *   from then on every kernel the library launches, up to max_launches of them, is bracketed
+ *   by a cudaEventRecord of an event pair on the stream it is launched on.  Calls made while a
+ *   stream is captured into a graph add event-record nodes instead.
+ * sgd_kernel_timing_stop: turns it off, waits for the recorded events, writes the elapsed
+ *   milliseconds of launch k (in launch order) to ms[k] for k < max, the number of bracketed
+ *   launches to *count, and frees the events.  SGD_ERR_CUDA if an event failed.
+ * sgd_kernel_timing_name: the (mangled) name of launch k's kernel after _stop, or NULL.
+ */
+int sgd_kernel_timing_start(int max_launches);
+int sgd_kernel_timing_stop(float *ms, int max, int *count);
+const char *sgd_kernel_timing_name(int k);
+
 /* Library version, (major << 16) | minor. */
 int sgd_version(void);
 

@@ -72,6 +72,10 @@ lib.sgd_oam_select_blocks.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32,
                                       _vp]
 lib.sgd_decode_attn_blocks.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
                                        _vp]
+lib.sgd_kernel_timing_start.argtypes = [_i32]
+lib.sgd_kernel_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(ctypes.c_int32)]
+lib.sgd_kernel_timing_name.argtypes = [_i32]
+lib.sgd_kernel_timing_name.restype = ctypes.c_char_p
 lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
@@ -340,6 +344,20 @@ def decode_attn_noalloc(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tenso
                                        _ptr(status),
                                        _stream(stream)), "sgd_decode_attn_noalloc")
     return o, lse
+
+
+def kernel_timing_start(max_launches: int = 256) -> None:
+    """Bracket each kernel the library launches from now on with a CUDA event pair (a
+    measurement aid; see kernel_timing_stop)."""
+    _check(lib.sgd_kernel_timing_start(int(max_launches)), "sgd_kernel_timing_start")
+
+
+def kernel_timing_stop(max_launches: int = 4096):
+    """Stop bracketing; returns [(mangled kernel name, milliseconds), ...] in launch order."""
+    ms = (ctypes.c_float * max_launches)()
+    n = ctypes.c_int32(0)
+    _check(lib.sgd_kernel_timing_stop(ms, max_launches, ctypes.byref(n)), "sgd_kernel_timing_stop")
+    return [(lib.sgd_kernel_timing_name(k).decode(), float(ms[k])) for k in range(min(n.value, max_launches))]
 
 
 def decode_num_ctas(k, v, cu_seqlens, G: int, indexed: bool = False, schedule: int = 0, n_splits: int = 0) -> int:

@@ -9,6 +9,8 @@
 
 #include <algorithm>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "internal.h"
 
@@ -141,7 +143,35 @@ int fused_n_req(const DevInfo &dev, const sgd_kv *kv, int G) {
 
 cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
+// per-launch timing: event pairs around each launch while on (a measurement aid, one thread)
+struct KernelTiming {
+    bool on = false;
+    int n = 0;
+    std::vector<cudaEvent_t> ev;  // 2 per launch slot
+    std::vector<const void *> fn;
+    std::vector<std::string> names;
+    void release() {
+        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+        ev.clear();
+        fn.clear();
+    }
+};
+KernelTiming g_kt;
+
 }  // namespace
+
+int kt_begin(cudaStream_t s) {
+    if (!g_kt.on || g_kt.n >= (int)g_kt.fn.size()) return -1;
+    const int k = g_kt.n;
+    return cudaEventRecord(g_kt.ev[2 * k], s) == cudaSuccess ? k : -1;
+}
+
+void kt_end(cudaStream_t s, int k, const void *kern) {
+    if (cudaEventRecord(g_kt.ev[2 * k + 1], s) != cudaSuccess) return;
+    g_kt.fn[k] = kern;
+    g_kt.n = k + 1;
+}
+
 }  // namespace sgd
 
 using namespace sgd;
@@ -321,6 +351,51 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
 extern "C" {
 
 int sgd_version(void) { return (1 << 16) | 0; }
+
+int sgd_kernel_timing_start(int max_launches) {
+    if (max_launches < 1 || max_launches > 4096) return SGD_ERR_ARG;
+    g_kt.on = false;
+    g_kt.release();
+    g_kt.names.clear();
+    g_kt.n = 0;
+    g_kt.ev.assign(2 * (size_t)max_launches, nullptr);
+    for (auto &e : g_kt.ev) {
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            e = nullptr;
+            for (auto &x : g_kt.ev)
+                if (x) cudaEventDestroy(x);
+            g_kt.ev.clear();
+            return SGD_ERR_CUDA;
+        }
+    }
+    g_kt.fn.assign((size_t)max_launches, nullptr);
+    g_kt.on = true;
+    return SGD_OK;
+}
+
+int sgd_kernel_timing_stop(float *ms, int max, int *count) {
+    if (!ms || !count || max < 0) return SGD_ERR_NULL;
+    g_kt.on = false;
+    g_kt.names.clear();
+    int rc = SGD_OK;
+    for (int k = 0; k < g_kt.n; ++k) {
+        float t = 0.f;
+        if (cudaEventSynchronize(g_kt.ev[2 * k + 1]) != cudaSuccess ||
+            cudaEventElapsedTime(&t, g_kt.ev[2 * k], g_kt.ev[2 * k + 1]) != cudaSuccess)
+            rc = SGD_ERR_CUDA;
+        if (k < max) ms[k] = t;
+        const char *name = nullptr;
+        if (cudaFuncGetName(&name, g_kt.fn[k]) != cudaSuccess || !name) name = "?";
+        g_kt.names.emplace_back(name);
+    }
+    *count = g_kt.n;
+    g_kt.release();
+    return rc;
+}
+
+const char *sgd_kernel_timing_name(int k) {
+    return (k >= 0 && k < (int)g_kt.names.size()) ? g_kt.names[k].c_str() : nullptr;
+}
 
 const char *sgd_error_string(int code) {
     switch (code) {

@@ -39,13 +39,18 @@ constexpr long long kWaitLimit = 1 << 22;  // bounded mbarrier polls before givi
 
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
+// Per-launch timing (sgd_kernel_timing_start / _stop, api.cu): while it is on, every launch is
+// bracketed by a pair of events on its stream.  kt_begin returns the launch's slot or -1.
+int kt_begin(cudaStream_t s);
+void kt_end(cudaStream_t s, int slot, const void *kern);
+
 // ------------------------------------------------------------------------------------------
 // host: launch `kern` through cudaLaunchKernelEx, as clusters of `cluster` CTAs along x when
 // cluster > 1.  Returns the launch's cudaError_t.
 // ------------------------------------------------------------------------------------------
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                            unsigned cluster, Args &&...args) {
+inline cudaError_t launch_k_raw(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                unsigned cluster, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -63,6 +68,15 @@ inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_
     cfg.attrs = attr;
     cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            unsigned cluster, Args &&...args) {
+    const int slot = kt_begin(s);
+    const cudaError_t e = launch_k_raw(kern, grid, block, smem, s, cluster, std::forward<Args>(args)...);
+    if (slot >= 0) kt_end(s, slot, reinterpret_cast<const void *>(kern));
+    return e;
 }
 
 // ------------------------------------------------------------------------------------------

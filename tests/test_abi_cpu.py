@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sgd.h")
@@ -165,3 +166,12 @@ def test_block_entry_points_reject_bad_args_on_host(sgd):
     assert dec(blk=0) == -1
     assert dec(kept=4) == -2
     assert dec(cache=_kv(sgd, dtype=sgd.SGD_F32)) == -3  # tensor-core path only
+
+
+def test_kernel_timing_rejects_bad_args_and_needs_a_device(sgd):
+    L = sgd.lib
+    assert L.sgd_kernel_timing_start(0) == -8 and L.sgd_kernel_timing_start(5000) == -8
+    assert L.sgd_kernel_timing_stop(None, 0, None) == -1
+    assert L.sgd_kernel_timing_name(0) is None
+    if not torch.cuda.is_available():  # no device here: creating the events fails, nothing is left on
+        assert L.sgd_kernel_timing_start(4) == L.sgd_kernel_timing_start(4) != 0

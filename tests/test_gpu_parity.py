@@ -641,3 +641,21 @@ def test_decode_over_blocks_reports_a_block_number_out_of_range(sgd):
     out, lse, ws = sgd.decode_attn_blocks(q, 8, k, v, cu, blk, cu_kb)
     assert sgd.workspace_status(ws) & 0x8  # bad index
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+def test_kernel_timing_brackets_each_launch(sgd):
+    bt = make((700, 3000), G=8, D=128, Hkv=2, seed=2)
+    q, k, v, cu = dev(bt)
+    sgd.decode_attn(q, 8, k, v, cu)  # warm
+    torch.cuda.synchronize()
+    sgd.kernel_timing_start(8)
+    out, lse, _ = sgd.decode_attn(q, 8, k, v, cu)
+    got = sgd.kernel_timing_stop()
+    assert [("plan_kernel" in n, "decode_mma_kernel" in n) for n, _ in got] == [(True, False), (False, True)]
+    assert all(ms > 0 for _, ms in got)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    # off again: nothing more is recorded
+    sgd.decode_attn(q, 8, k, v, cu)
+    sgd.kernel_timing_start(1)
+    assert sgd.kernel_timing_stop() == []
