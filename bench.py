@@ -589,7 +589,8 @@ def run_ours(args, rank, world, local_rank):
                            "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": stages[dom]},
         "e2e": {"value": round(job_gbs(step_bytes, 1, e2e_ms, world), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": pipe.launches_per_step() * K,
+        # library launches per step as the per-launch timing counted them (the step's kernel list)
+        "gpu_launches": (sum(e["per_step"] for e in per_kernel.values()) or pipe.launches_per_step()) * K,
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
