@@ -227,6 +227,23 @@ def test_int8_decode_query_codes(sgd, mode, G, indexed):
         assert lerr < 0.25 * gap, f"lse error {lerr:.2e} vs quantisation effect {gap:.2e}"
 
 
+def test_query_codes_of_an_all_zero_query_row(sgd):
+    # scale 0 -> every code 0: the row's logits are all 0 and its output the mean of the dequantised V
+    bt = make((300, 45), G=8, D=128, Hkv=2, dist="outlier", seed=17)
+    bt.q[0, 3] = 0  # sequence 0, KV head 0, query head 3
+    bt.q[1, 8:16] = 0  # every query head of sequence 1, KV head 1
+    q, k, v, cu = dev(bt)
+    quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A"), "A")
+    ref = oracle.decode(oracle.dequant_q(*oracle.quantize_q(bt.q, "token")), bt.k, bt.v, bt.cu_seqlens, 8,
+                        quant=quant)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                   n_parts_=sgd.n_parts(bt.lengths), n_splits=5, q_quant="token")
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
+    assert abs(float(lse[0, 3]) - np.log(300)) < 1e-3 and abs(float(lse[1, 8]) - np.log(45)) < 1e-3
+
+
 def test_int8_d64_uses_cuda_core_path(sgd):
     bt = make((5, 300), G=8, D=64, Hkv=2, dist="outlier", seed=5)
     q, k, v, cu = dev(bt)
