@@ -298,6 +298,30 @@ def oam_select(q, k, v, cu_seqlens, G: int, beta: float, eps: float, keep_num: i
     return idx, cu_kept, scores
 
 
+def oam_select_multi(q, k, v, cu_seqlens, G: int, M: int, beta: float, eps: float, keep_num: int,
+                     keep_den: int, rows: Optional[Sequence] = None):
+    """oam_select for M query tokens per sequence (q [B, M, Hq, D]): one kept set per (sequence,
+    KV head) serves all M * G query rows, so the group maximum of the score runs over all of
+    them: s_t = max_{m,g} (q[b, m, kvh*G+g] . k_t) / sqrt(D) + beta * ln(||v_t|| + eps).
+    Same outputs as oam_select."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    B = cu.size - 1
+    Hkv = k.shape[0]
+    D = q.shape[-1]
+    kept = np.array([kept_count(int(cu[b + 1] - cu[b]), keep_num, keep_den) for b in range(B)], np.int64)
+    cu_kept = np.concatenate([[0], np.cumsum(kept)]).astype(np.int32)
+    idx = np.full((Hkv, int(cu_kept[-1])), -1, np.int32)
+    scores = {}
+    todo = rows if rows is not None else [(b, h) for h in range(Hkv) for b in range(B)]
+    for b, h in todo:
+        s0, e0 = int(cu[b]), int(cu[b + 1])
+        qg = _f64(q[b, :, h * G:(h + 1) * G]).reshape(M * G, D)
+        s = oam_scores(qg, k[h, s0:e0], v[h, s0:e0], beta, eps)
+        scores[(b, h)] = s
+        idx[h, cu_kept[b]:cu_kept[b + 1]] = topk(s, int(kept[b]))
+    return idx, cu_kept, scores
+
+
 def value_norms(v) -> np.ndarray:
     """||v_t||_2 of every row of v [..., T, D] in float64 (the norm the OAM score takes)."""
     x = _f64(v)

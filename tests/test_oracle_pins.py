@@ -581,3 +581,22 @@ def test_decode_over_blocks_is_attention_over_their_tokens():
     allb = np.array([[0, 1, 2, 0], [0, 1, 2, 0]], np.int32)
     o2, l2 = oracle.decode_blocks(bt.q, bt.k, bt.v, bt.cu_seqlens, 2, allb, np.array([0, 3, 4], np.int32))
     assert np.allclose(o2, dense[0], atol=1e-13) and np.allclose(l2, dense[1], atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# oam_select_multi: one kept set for the M query tokens of a speculative step
+# ---------------------------------------------------------------------------------------------
+def test_multi_token_scores_are_the_max_over_the_tokens_single_scores():
+    M, G = 3, 2
+    bt = _multi_batch(M, G=G, D=16, lengths=(40, 9), Hkv=2, seed=8)
+    idx, cu_kept, scores = oracle.oam_select_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, 1.0, 1e-6, 1, 4)
+    singles = [oracle.oam_select(bt.q[:, m], bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)[2] for m in range(M)]
+    for key, s in scores.items():
+        want = np.max(np.stack([sm[key] for sm in singles]), axis=0)  # beta * ln(|v| + eps) is common
+        assert np.allclose(s, want, rtol=0, atol=1e-12)
+        b, h = key
+        ref = sorted(sorted(range(s.size), key=lambda t: (-want[t], t))[:cu_kept[b + 1] - cu_kept[b]])
+        assert idx[h, cu_kept[b]:cu_kept[b + 1]].tolist() == ref
+    one = oracle.oam_select_multi(bt.q[:, :1], bt.k, bt.v, bt.cu_seqlens, G, 1, 1.0, 1e-6, 1, 4)
+    base = oracle.oam_select(bt.q[:, 0], bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)
+    assert np.array_equal(one[0], base[0]) and np.array_equal(one[1], base[1])
