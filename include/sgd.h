@@ -153,6 +153,21 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * sgd_oam_select_multi -- sgd_oam_select for M query tokens per sequence (the speculative step
+ * of sgd_decode_attn_multi): one kept set per (sequence, KV head) serves all M * G query rows,
+ * so the group maximum runs over all of them:
+ *   s_t = max_{m,g} (q[b, m, kvh*G+g] . k_t) / sqrt(D) + beta * ln(||v_t||_2 + eps).
+ * q        [B, M, Hq, D] BF16;  1 <= M, G * M <= 16;  the cache BF16 (D 64 or 128) or I8 (D 128,
+ *          with kv->v_norm) -- SGD_ERR_DTYPE otherwise
+ * workspace   sgd_workspace_size(SGD_OP_OAM_SELECT, kv, G * M, 0, 0) bytes
+ * Outputs and errors as in sgd_oam_select; M = 1 is sgd_oam_select.
+ */
+int sgd_oam_select_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv,
+                         float beta, float eps, int keep_num, int keep_den,
+                         int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * sgd_oam_select_blocks -- block-granular token dropping: whole 64-token blocks are kept
  * ([NSA] section 2.1 selects 64-token blocks so that the kept KV is read contiguously; here a
  * block is ranked by the best OAM score s_t of its tokens).  Block j of sequence b holds tokens

@@ -68,6 +68,7 @@ lib.sgd_oam_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _
 lib.sgd_decode_attn.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]
 lib.sgd_decode_attn_multi.argtypes = [_vp, _i32, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp,
                                       _sz, _vp]
+lib.sgd_oam_select_multi.argtypes = [_vp, _i32, _i32, _i32, _kvp, _f, _f, _i32, _i32, _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_oam_select_blocks.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i64, _vp, _vp, _i64, _vp, _sz,
                                       _vp]
 lib.sgd_decode_attn_blocks.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
@@ -202,6 +203,27 @@ def oam_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
     ws = _workspace(workspace_size(OP_OAM_SELECT, kv, G), k.device, workspace)
     _check(lib.sgd_oam_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, _ptr(idx),
                               _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)), "sgd_oam_select")
+    return idx, cu_kept, ws
+
+
+def oam_select_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                     beta: float, eps: float, keep_num: int, keep_den: int, lengths: Sequence[int],
+                     out=None, workspace=None, stream=None, k_scale=None, v_scale=None, scheme: str = "A",
+                     n_parts_: int = 0, v_norm=None):
+    """One kept set per (sequence, KV head) for the M query tokens of q [B, M, Hq, D] (the group
+    maximum over all M * G query rows).  Returns (idx [Hkv, Kt], cu_kept [B+1], ws)."""
+    Hkv, M = k.shape[0], q.shape[1]
+    Kt = kept_total(lengths, keep_num, keep_den)
+    kv = _kv(k, v, cu_seqlens, k_scale, v_scale, SCHEME_A if scheme == "A" else SCHEME_B, n_parts_, v_norm)
+    if out is None:
+        idx = torch.empty((Hkv, Kt), dtype=torch.int32, device=k.device)
+        cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
+    else:
+        idx, cu_kept = out
+    ws = _workspace(workspace_size(OP_OAM_SELECT, kv, G * M), k.device, workspace)
+    _check(lib.sgd_oam_select_multi(_ptr(q), _DT[q.dtype], G, M, ctypes.byref(kv), beta, eps, keep_num, keep_den,
+                                    _ptr(idx), _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)),
+           "sgd_oam_select_multi")
     return idx, cu_kept, ws
 
 

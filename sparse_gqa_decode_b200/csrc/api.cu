@@ -271,11 +271,13 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
 // blocks by their best token's score and keep whole blocks (n_blocks = sum_b ceil(L_b / 64)).
 int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps, int keep_num,
                 int keep_den, bool blocks, int64_t n_blocks, int32_t *idx, int32_t *cu_kept, int64_t kept_total,
-                void *workspace, size_t workspace_bytes, void *stream) {
+                void *workspace, size_t workspace_bytes, void *stream, int M = 1) {
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !idx || !cu_kept || !workspace) return SGD_ERR_NULL;
-    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
+    // several query tokens: the tensor-core score kernel, its columns the M * G query rows
+    if (M > 1 && decode_family(kv->dtype, q_dtype, kv->D, true) != kFamilyMma) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (kv->dtype == SGD_I8) {
         // scoring the INT8 cache: khat = code * scale, ||v|| from the norms stored at quantisation
@@ -297,8 +299,8 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
     DevInfo *dev;
     if ((rc = current_device(&dev)) != SGD_OK) return rc;
     int n_req = 0;
-    if ((rc = decode_n_req(*dev, kv, q_dtype, G, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
-    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    if ((rc = decode_n_req(*dev, kv, q_dtype, G * M, false, true, 0, 0, &n_req)) != SGD_OK) return rc;
+    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G * M, kv->D, kv->T, n_req);
     if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
@@ -315,7 +317,7 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
     a.B = kv->B;
     a.Hkv = kv->Hkv;
     a.G = G;
-    a.M = 1;
+    a.M = M;
     a.D = kv->D;
     a.T = kv->T;
     a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
@@ -480,6 +482,13 @@ int sgd_oam_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, fl
                    size_t workspace_bytes, void *stream) {
     return select_impl(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, false, 0, idx, cu_kept, kept_total, workspace,
                        workspace_bytes, stream);
+}
+
+int sgd_oam_select_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, float beta, float eps,
+                         int keep_num, int keep_den, int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                         void *workspace, size_t workspace_bytes, void *stream) {
+    return select_impl(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, false, 0, idx, cu_kept, kept_total, workspace,
+                       workspace_bytes, stream, M);
 }
 
 int sgd_oam_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,

@@ -485,11 +485,11 @@ __device__ __forceinline__ void score_subtile(const DecodeArgs &a, uint32_t kbas
 #pragma unroll
     for (int gt = 0; gt < C::GT; ++gt) {
         const int g0 = 8 * gt + 2 * t4;
-        if (g0 < a.G) {
+        if (g0 < a.G * a.M) {  // (query token, head) columns
             mA = fmaxf(mA, sacc[gt][0]);
             mB = fmaxf(mB, sacc[gt][2]);
         }
-        if (g0 + 1 < a.G) {
+        if (g0 + 1 < a.G * a.M) {
             mA = fmaxf(mA, sacc[gt][1]);
             mB = fmaxf(mB, sacc[gt][3]);
         }
@@ -568,11 +568,11 @@ __device__ __forceinline__ void score_subtile_i8(const DecodeArgs &a, uint32_t k
 #pragma unroll
     for (int gt = 0; gt < C::GT; ++gt) {
         const int g0 = 8 * gt + 2 * t4;
-        if (g0 < a.G) {
+        if (g0 < a.G * a.M) {  // (query token, head) columns
             mA = fmaxf(mA, sacc[gt][0] * colf[gt][0]);
             mB = fmaxf(mB, sacc[gt][2] * colf[gt][0]);
         }
-        if (g0 + 1 < a.G) {
+        if (g0 + 1 < a.G * a.M) {
             mA = fmaxf(mA, sacc[gt][1] * colf[gt][1]);
             mB = fmaxf(mB, sacc[gt][3] * colf[gt][1]);
         }

@@ -676,3 +676,34 @@ def test_kernel_timing_brackets_each_launch(sgd):
     sgd.decode_attn(q, 8, k, v, cu)
     sgd.kernel_timing_start(1)
     assert sgd.kernel_timing_stop() == []
+
+
+@pytest.mark.parametrize("cache", ["bf16", "int8A"])
+@pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (2, 4)])
+def test_multi_token_selection_then_decode(sgd, cache, M, G):
+    # one kept set for the M query tokens (group max over M * G rows), then the causal multi-token
+    # decode over it; the decode is checked on the oracle's own selection
+    lengths = (5, 300, 2500)
+    bt = make_multi(lengths, M, G, seed=61 + M)
+    q, k, v, cu = dev(bt)
+    kw, kk, vv, quant, vn = {}, k, v, None, None
+    if cache == "int8A":
+        vn = torch.empty((2, bt.T), dtype=torch.float32, device="cuda")
+        kk, vv, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths, v_norm=vn)
+        kw = dict(k_scale=ks, v_scale=vs, scheme="A", n_parts_=sgd.n_parts(bt.lengths))
+        quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A"), "A")
+    idx, cu_kept, ws = sgd.oam_select_multi(q, kk, vv, cu, G, 1.0, 1e-6, 1, 8, bt.lengths, v_norm=vn, **kw)
+    check_status(sgd, ws)
+    if cache == "bf16":
+        ref_idx, ref_cu, scores = oracle.oam_select_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, 1.0, 1e-6, 1, 8)
+    else:  # scored on code * scale: the oracle's dequantised keys, the unquantised value norms
+        khat = torch.from_numpy(np.stack([oracle.dequant_rows(quant[0][h], np.concatenate(
+            [oracle.k_scale_of_tokens(quant[2], "A", h, b, L, np.concatenate([[0], np.cumsum(oracle.n_parts(lengths))]))
+             for b, L in enumerate(lengths)])) for h in range(2)]))
+        ref_idx, ref_cu, scores = oracle.oam_select_multi(bt.q, khat, bt.v, bt.cu_seqlens, G, M, 1.0, 1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, len(lengths), 2)
+    ref = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, idx=ref_idx, cu_kept=ref_cu, quant=quant)
+    out, lse, ws = sgd.decode_attn_multi(q, G, kk, vv, cu, idx=torch.from_numpy(ref_idx).cuda(),
+                                         cu_kept=torch.from_numpy(ref_cu).cuda(), kept_total_=ref_idx.shape[1], **kw)
+    assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
