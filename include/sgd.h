@@ -40,7 +40,8 @@
  * at the start of the workspace (SGD_WS_STATUS_OFFSET), read it with
  * sgd_workspace_status after the stream completes.  No call aborts, traps or
  * throws.
- * Limits.  1 <= G <= 16; D in {64, 128}; Hkv * T < 2^31; B >= 1, Hkv >= 1.
+ * Limits.  1 <= G <= 16 (query heads per KV head); D in {64, 128}; Hkv * T < 2^31; B >= 1,
+ * Hkv >= 1; several query tokens: G * M <= 64 for the decode, <= 16 for the selection.
  */
 #ifndef SGD_H_
 #define SGD_H_

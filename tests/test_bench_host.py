@@ -1,0 +1,88 @@
+"""bench.py's host arithmetic without a GPU: the algorithmic bytes each stage and kernel must
+move (restated here from the data layout, independently of bench.py's formulas), the naming of
+the library's kernels in the per-launch timing, and the traffic record's staleness check."""
+import importlib.util
+import json
+import os
+
+import pytest
+
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_host", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_kernel_roles_from_demangled_names(bench):
+    r = bench.kernel_role
+    assert r("void sgd::decode_mma_kernel<sgd::MmaCfg<128, 1, false, false, 2, false, false, false> >") == \
+        "score_quantize"
+    assert r("void sgd::decode_mma_kernel<sgd::MmaCfg<128, 2, true, true, 0, true, false, false> >") == "decode"
+    assert r("void sgd::decode_mma_kernel<sgd::MmaCfg<128, 1, true, false, 1, false, false, false> >") == "score"
+    assert r("void sgd::quant_global_kernel<__nv_bfloat16, false>") == "v_codes"
+    assert r("void sgd::topk_cluster_kernel<512, 8, 2>") == "topk"
+    assert r("sgd::plan_kernel") == "plan" and r("sgd::block_max_kernel") == "block_max"
+    assert r("void sgd::decode_generic_kernel<128, float, true, 0>") == "decode"
+
+
+def test_demangle_reads_the_library_names(bench):
+    out = bench.demangle(["_ZN3sgd11plan_kernelEPKiS1_iiiiiiNS_8PlanViewEPNS_8WsHeaderEiPfS5_iiPK13__nv_bfloat16liii"])
+    assert out[0].startswith("sgd::plan_kernel(") or out[0].startswith("_ZN3sgd11plan_kernel")
+
+
+def test_fused_pass_and_decode_bytes_from_the_layout(bench):
+    # two sequences of 100 and 64 tokens, Hkv 2, G 4, D 128, scheme A, keep 1/8
+    wl = workloads.Workload("t", B=2, Hkv=2, G=4, D=128, kv_dtype="bf16", dist="normal", lengths=(100, 64),
+                            scheme="A", oam=True)
+    lengths = [100, 64]
+    T, Hkv, D = 164, 2, 128
+    parts = 2 + 1  # ceil(100/64) + ceil(64/64)
+    q = 2 * 8 * D * 2  # B * Hq * D bf16
+    fused = 2 * Hkv * T * D * 2 + Hkv * T * D + Hkv * parts * 4 + Hkv * T * 4 + q
+    assert bench.kernel_bytes(wl, lengths, "score_quantize") == fused
+    assert bench.kernel_bytes(wl, lengths, "v_codes") == Hkv * T * D * 2 + Hkv * T * D + 4
+    kept = 13 + 8  # ceil(100/8) + ceil(64/8)
+    out = 2 * 8 * (D + 1) * 4
+    decode = 2 * Hkv * kept * D + Hkv * kept * 4 + Hkv * parts * 4 + q + out
+    assert bench.algorithmic_bytes(wl, lengths)["decode"] == decode
+    assert bench.kernel_bytes(wl, lengths, "decode") == decode
+    assert bench.kernel_bytes(wl, lengths, "topk") is None
+
+
+def test_block_selection_counts_whole_blocks(bench):
+    wl = workloads.Workload("t", B=2, Hkv=1, G=8, D=128, kv_dtype="bf16", dist="normal", lengths=(130, 1000),
+                            scheme="A", oam=True, select_on_codes=True, blocks=True)
+    nb = [3, 16]
+    kept = 1 + 2  # ceil(3/8), ceil(16/8)
+    st = bench.algorithmic_bytes(wl, [130, 1000])
+    q, out = 2 * 8 * 128 * 2, 2 * 8 * 129 * 4
+    assert st["decode"] == 2 * 64 * kept * 128 + kept * 4 + sum(nb) * 4 + q + out
+
+
+def test_multi_token_decode_counts_every_query_token(bench):
+    wl = workloads.Workload("t", B=1, Hkv=1, G=8, D=128, kv_dtype="bf16", dist="normal", lengths=(640,),
+                            scheme="A", M=4)
+    st = bench.algorithmic_bytes(wl, [640])
+    assert st["decode"] == 2 * 640 * 128 + 10 * 4 + 4 * (8 * 128 * 2 + 8 * 129 * 4)
+
+
+def test_traffic_record_is_ignored_once_a_source_changes(bench, tmp_path, monkeypatch):
+    src = tmp_path / "k.cu"
+    src.write_text("one")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = {"w": {"kernels": {"decode": {"bytes_per_launch": 7, "sources": ["k.cu"],
+                                        "source_hash": bench.source_hash([str(src)])}}}}
+    (prof / "dram_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_traffic("decode", "w") == 7
+    src.write_text("two")
+    assert bench.load_traffic("decode", "w") is None
+    assert bench.load_traffic("decode", "other") is None
