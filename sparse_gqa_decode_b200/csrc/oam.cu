@@ -560,43 +560,58 @@ int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t 
 }
 
 // ------------------------------------------------------------------------------------------
-// block scores for block-granular selection ([NSA] section 2.1: 64-token selection blocks): one
-// warp per (KV head, block), two coalesced loads per lane, the block's best token score
+// block scores for block-granular selection ([NSA] section 2.1: 64-token selection blocks): each
+// warp takes kBlocksPerWarp consecutive blocks of one KV head, finds the first one's sequence
+// once, issues the loads of all its blocks together (two coalesced loads per lane and block) and
+// reduces each block to its best token score
 // ------------------------------------------------------------------------------------------
 constexpr int kBlockMaxWarps = 8;
+constexpr int kBlocksPerWarp = 4;
 
 __global__ void __launch_bounds__(kBlockMaxWarps * 32)
     block_max_kernel(const float *__restrict__ scores, const int32_t *__restrict__ cu_seq,
                      const int32_t *__restrict__ cu_blk, int B, int Hkv, int64_t T, int64_t Tb,
                      float *__restrict__ bscores, int32_t *status) {
+    const int64_t wpr = (Tb + kBlocksPerWarp - 1) / kBlocksPerWarp;  // warps per KV head
     const int64_t w = (int64_t)blockIdx.x * kBlockMaxWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (w >= (int64_t)Hkv * Tb) return;
-    const int h = (int)(w / Tb);
-    const int32_t j = (int32_t)(w - (int64_t)h * Tb);
-    const int b = upper_bound_i32(cu_blk, B + 1, j) - 1;  // sequence of block j
-    if (b < 0 || b >= B) {  // the caller's block count exceeds the lengths' (or the lengths are bad)
-        if (lane == 0) {
-            bscores[(int64_t)h * Tb + j] = -INFINITY;
-            atomicOr(status, SGD_STATUS_SIZE_MISMATCH);
-        }
-        return;
+    if (w >= (int64_t)Hkv * wpr) return;
+    const int h = (int)(w / wpr);
+    const int32_t j0 = (int32_t)((w - (int64_t)h * wpr) * kBlocksPerWarp);
+    if (j0 == 0 && h == 0 && lane == 0 && __ldg(cu_blk + B) != Tb) atomicOr(status, SGD_STATUS_SIZE_MISMATCH);
+    int b = upper_bound_i32(cu_blk, B + 1, j0) - 1;  // sequence of block j0
+    float v[kBlocksPerWarp][2];
+    int32_t n[kBlocksPerWarp];
+#pragma unroll
+    for (int i = 0; i < kBlocksPerWarp; ++i) {
+        const int32_t j = j0 + i;
+        v[i][0] = v[i][1] = -INFINITY;
+        n[i] = -1;  // no such block (past Tb, or past the lengths' blocks)
+        if (j >= Tb) continue;
+        while (b < B && __ldg(cu_blk + b + 1) <= j) ++b;  // blocks of empty sequences are skipped
+        if (b < 0 || b >= B) continue;
+        const int32_t s0 = __ldg(cu_seq + b), s1 = __ldg(cu_seq + b + 1);
+        const int32_t t0 = s0 + (j - __ldg(cu_blk + b)) * kPart;
+        n[i] = max(0, min(kPart, s1 - t0));
+        const float *row = scores + (int64_t)h * T + t0;
+        if (lane < n[i]) v[i][0] = __ldg(row + lane);
+        if (lane + 32 < n[i]) v[i][1] = __ldg(row + lane + 32);
     }
-    if (j == 0 && h == 0 && lane == 0 && __ldg(cu_blk + B) != Tb) atomicOr(status, SGD_STATUS_SIZE_MISMATCH);
-    const int32_t s0 = __ldg(cu_seq + b), s1 = __ldg(cu_seq + b + 1);
-    const int32_t t0 = s0 + (j - __ldg(cu_blk + b)) * kPart;
-    const int32_t n = min(kPart, s1 - t0);
-    const float *row = scores + (int64_t)h * T + t0;
-    float m = -INFINITY;
-    if (lane < n) m = __ldg(row + lane);
-    if (lane + 32 < n) m = fmaxf(m, __ldg(row + lane + 32));
-    m = warp_max(m);
-    if (lane == 0) bscores[(int64_t)h * Tb + j] = m;
+#pragma unroll
+    for (int i = 0; i < kBlocksPerWarp; ++i) {
+        const int32_t j = j0 + i;
+        if (j >= Tb) break;
+        const float m = warp_max(fmaxf(v[i][0], v[i][1]));
+        if (lane == 0) {
+            bscores[(int64_t)h * Tb + j] = m;
+            if (n[i] < 0) atomicOr(status, SGD_STATUS_SIZE_MISMATCH);  // the caller's count exceeds the lengths'
+        }
+    }
 }
 
 int launch_block_max(const float *scores, const int32_t *cu_seq, const int32_t *cu_blk, int B, int Hkv, int64_t T,
                      int64_t Tb, float *bscores, int32_t *status, cudaStream_t s) {
-    const int64_t warps = (int64_t)Hkv * Tb;
+    const int64_t warps = (int64_t)Hkv * ((Tb + kBlocksPerWarp - 1) / kBlocksPerWarp);
     if (warps <= 0) return 0;
     const unsigned grid = (unsigned)((warps + kBlockMaxWarps - 1) / kBlockMaxWarps);
     return (int)launch_k(block_max_kernel, dim3(grid), dim3(kBlockMaxWarps * 32), 0, s, 1, scores, cu_seq, cu_blk,
