@@ -42,7 +42,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9, 10])
+    p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -113,10 +113,14 @@ def kernel_bytes(wl, lengths, role):
     P = int(sum((int(L) + 63) // 64 for L in lengths))
     q = B * wl.M * Hkv * wl.G * D * 2
     scales = Hkv * P * 4 if wl.scheme == "A" else 4
-    if role == "score_quantize":  # K and V (bf16) in; K codes, scheme-A scales, scores out
-        return 2 * Hkv * T * D * 2 + Hkv * T * D + scales + Hkv * T * 4 + q
-    if role == "v_codes":  # V (bf16) in, V codes out
-        return Hkv * T * D * 2 + Hkv * T * D + 4
+    if role == "score_quantize":  # K and V (bf16) in; scores out; scheme A: K codes and scales out
+        codes = Hkv * T * D + scales if wl.scheme == "A" else 0
+        return 2 * Hkv * T * D * 2 + codes + Hkv * T * 4 + q
+    if role == "v_codes":  # V (bf16) in, V codes out; scheme B: K and V in one launch
+        n = 2 if wl.scheme == "B" else 1
+        return n * (Hkv * T * D * 2 + Hkv * T * D + 4)
+    if role == "amax":  # scheme B: K and V in (their maxima)
+        return 2 * Hkv * T * D * 2
     if role == "k_codes":  # K and V in (max|V| on the way), K codes and scales out
         return 2 * Hkv * T * D * 2 + Hkv * T * D + scales
     if role == "score":  # INT8 K codes, value norms and scales in; scores out

@@ -86,3 +86,13 @@ def test_traffic_record_is_ignored_once_a_source_changes(bench, tmp_path, monkey
     src.write_text("two")
     assert bench.load_traffic("decode", "w") is None
     assert bench.load_traffic("decode", "other") is None
+
+
+def test_scheme_b_codes_both_tensors_in_one_launch(bench):
+    wl = workloads.Workload("t", B=1, Hkv=2, G=4, D=128, kv_dtype="bf16", dist="normal", lengths=(100,),
+                            scheme="B")
+    T, Hkv, D = 100, 2, 128
+    assert bench.kernel_bytes(wl, [100], "v_codes") == 2 * (Hkv * T * D * 2 + Hkv * T * D + 4)
+    assert bench.kernel_bytes(wl, [100], "amax") == 2 * Hkv * T * D * 2
+    sel = wl.with_(oam=True)  # the fused pass of scheme B writes no K codes
+    assert bench.kernel_bytes(sel, [100], "score_quantize") == 2 * Hkv * T * D * 2 + Hkv * T * 4 + 1 * 8 * D * 2

@@ -106,11 +106,19 @@ CONFIGS = {
     # CTAs per split range
     10: Workload("spec_M4_int8_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
                  lengths=(131072,) * 8, scheme="A", M=4, seed=4),
+    # the INT8 scheme table on workload 4's batch: scheme B (per-tensor K), the per-tensor Q/K/V
+    # baseline (scheme B with one query scale) and scheme A with query codes per (sequence, head)
+    11: Workload("int8B_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                 lengths=(131072,) * 8, scheme="B", seed=4),
+    12: Workload("int8_qkv_per_tensor_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                 lengths=(131072,) * 8, scheme="B", q_quant="tensor", seed=4),
+    13: Workload("int8A_qcodes_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                 lengths=(131072,) * 8, scheme="A", q_quant="token", seed=4),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..10), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..13), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
