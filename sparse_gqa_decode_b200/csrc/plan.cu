@@ -36,8 +36,22 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
     }
     if (q) {  // per-tensor query scale for the decode: max|q| / 127 (IEEE division)
         __shared__ uint32_t qmax;  // float bits: non-negative floats order as integers
-        float m = 0.f;
-        for (int64_t i = tid; i < q_elems; i += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(q[i])));
+        // q is 16-byte aligned and D a multiple of 8: 16-byte loads, four in flight per thread
+        const uint4 *q4 = reinterpret_cast<const uint4 *>(q);
+        const int64_t nv = q_elems / 8;
+        uint32_t acc = 0u;  // |q| maxima as bf16x2 (exact)
+        for (int64_t i = tid; i < nv; i += 4 * (int64_t)blockDim.x) {
+            uint4 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t k = i + (int64_t)u * blockDim.x;
+                w[u] = (k < nv) ? __ldg(q4 + k) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                acc = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(acc, w[u].x), w[u].y), w[u].z), w[u].w);
+        }
+        float m = bf16x2_fold_max(acc);
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (tid == 0) qmax = 0u;
