@@ -707,3 +707,27 @@ def test_multi_token_selection_then_decode(sgd, cache, M, G):
                                          cu_kept=torch.from_numpy(ref_cu).cuda(), kept_total_=ref_idx.shape[1], **kw)
     assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
     check_status(sgd, ws)
+
+
+@pytest.mark.parametrize("mode", ["token", "tensor"])
+def test_decode_over_blocks_with_query_codes(sgd, mode):
+    lengths = (64, 130, 3001)
+    bt = make(lengths, G=8, D=128, Hkv=2, dist="outlier", seed=57)
+    q, k, v, cu = dev(bt)
+    nb = [-(-L // 64) for L in lengths]
+    keep = [1, 2, 12]
+    cu_kb = np.concatenate([[0], np.cumsum(keep)]).astype(np.int32)
+    rng = np.random.default_rng(9)
+    blk = np.zeros((2, int(cu_kb[-1])), np.int32)
+    for b, (n, K) in enumerate(zip(nb, keep)):
+        for h in range(2):
+            blk[h, cu_kb[b]:cu_kb[b + 1]] = np.sort(rng.choice(n, size=K, replace=False))
+    quant = (*oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A"), "A")
+    qd = oracle.dequant_q(*oracle.quantize_q(bt.q, mode))
+    ref = oracle.decode_blocks(qd, bt.k, bt.v, bt.cu_seqlens, 8, blk, cu_kb, quant=quant)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    out, lse, ws = sgd.decode_attn_blocks(q, 8, kc, vc, cu, torch.from_numpy(blk).cuda(), torch.from_numpy(cu_kb).cuda(),
+                                          k_scale=ks, v_scale=vs, scheme="A", n_parts_=sgd.n_parts(bt.lengths),
+                                          n_splits=11, q_quant=mode)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    check_status(sgd, ws)
