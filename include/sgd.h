@@ -15,7 +15,11 @@
  *   [CD] "共同设计 AI 模型注意力，实现快速的交互式长上下文推理" (Co-designing AI
  *        model attention for fast interactive long-context inference), NVIDIA
  *        developer blog -- decode equations 5-7 (decode streams the KV cache
- *        and is HBM-bound; arithmetic intensity about 2G).
+ *        and is HBM-bound; arithmetic intensity about 2G); speculative decoding
+ *        raises the decode's GEMM M from G to (1 + n_draft) * G.
+ *   [NSA] "硬件对齐的稀疏注意力机制：原理、优化与实践" (hardware-aligned sparse
+ *        attention, NSA) -- section 2.1: selection shared by a GQA group,
+ *        64-token selection blocks read contiguously.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -29,7 +33,8 @@
  * Pointers.  Every array argument is a DEVICE pointer of the current device
  * unless its comment says "host".  Arrays must start on a 16-byte boundary.
  * Ownership.  The caller allocates and frees every buffer, including the
- * workspace; the library never allocates, frees or synchronises, and never
+ * workspace; the library never allocates, frees or synchronises (except
+ * sgd_workspace_status and the measurement aid sgd_kernel_timing_*), and never
  * changes the current device.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
  * stream).  All work is enqueued on it; results are ready when it completes.
