@@ -175,3 +175,35 @@ def test_kernel_timing_rejects_bad_args_and_needs_a_device(sgd):
     assert L.sgd_kernel_timing_name(0) is None
     if not torch.cuda.is_available():  # no device here: creating the events fails, nothing is left on
         assert L.sgd_kernel_timing_start(4) == L.sgd_kernel_timing_start(4) != 0
+
+
+def test_multi_token_selection_and_plan_reject_bad_args_on_host(sgd):
+    L = sgd.lib
+    p = ctypes.c_void_p
+    kv = _kv(sgd)
+
+    def sel(G=8, M=2, cache=kv, qdt=sgd.SGD_BF16):
+        return L.sgd_oam_select_multi(p(0x3000), qdt, G, M, ctypes.byref(cache), 1.0, 1e-6, 1, 8, p(0x1000),
+                                      p(0x2000), 20, p(0x4000), 1 << 20, None)
+
+    assert sel(M=0) == -2 and sel(M=3) == -2 and sel(G=16, M=2) == -2  # G * M <= 16 for the selection
+    assert sel(cache=_kv(sgd, dtype=sgd.SGD_F32), qdt=sgd.SGD_F32) == -3  # tensor-core score kernel only
+
+    def plan(cu=0x1000, B=2, Hkv=2, n_req=8, min_chunk=16, mode=0, ws=0x6000, nbytes=1 << 20):
+        n = ctypes.c_int32(0)
+        return L.sgd_plan_segments(p(cu) if cu else None, B, Hkv, n_req, min_chunk, mode, p(0x7000), 64,
+                                   ctypes.byref(n), p(ws) if ws else None, nbytes, None)
+
+    assert plan(cu=0) == -1 and plan(ws=0) == -1
+    assert plan(B=0) == -2 and plan(mode=2) == -8
+    assert plan(min_chunk=8) == -8 and plan(min_chunk=24) == -8 and plan(n_req=0) == -8
+    assert plan(ws=0x6004) == -4 and plan(nbytes=64) == -5
+
+
+def test_workspace_size_limits(sgd):
+    kv = _kv(sgd)
+    L = sgd.lib
+    assert L.sgd_workspace_size(sgd.OP_QUANTIZE, ctypes.byref(kv), 1, 0, 0) >= 256  # no device needed
+    assert L.sgd_workspace_size(sgd.OP_DECODE, ctypes.byref(kv), 65, 0, 0) == 0  # decode columns <= 64
+    assert L.sgd_workspace_size(sgd.OP_OAM_SELECT, ctypes.byref(kv), 17, 0, 0) == 0  # selection G <= 16
+    assert L.sgd_workspace_size(sgd.OP_DECODE, ctypes.byref(kv), 0, 0, 0) == 0
