@@ -6,6 +6,18 @@ torch tensors into device pointers, allocates outputs and the workspace with tor
 passes the current CUDA stream.  Every step of the computation runs in the library's CUDA
 kernels; there is no CPU or PyTorch fallback, and importing fails loudly when the library
 has not been built (``python sparse_gqa_decode_b200/build.py``).
+
+A decode step, as the benchmark runs it::
+
+    kc, vc, ks, vs, idx, cu_kept, ws = quantize_select(q, k, v, cu, G, beta, eps, 1, 8, "A", lengths)
+    out, lse, ws = decode_attn(q, G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                               n_parts_=n_parts(lengths), idx=idx, cu_kept=cu_kept,
+                               kept_total_=idx.shape[1])
+
+Variants: ``oam_select`` on a bf16/f32 cache or on the INT8 cache with stored value norms;
+``decode_attn(..., q_quant="token"|"tensor")`` for INT8 query codes; ``oam_select_multi`` /
+``decode_attn_multi`` for several query tokens per sequence (speculative decoding);
+``oam_select_blocks`` / ``decode_attn_blocks`` for whole 64-token blocks.
 """
 from __future__ import annotations
 
@@ -16,9 +28,10 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "lib", "quantize_kv", "oam_select", "quantize_select", "decode_attn", "decode_attn_noalloc", "plan_segments", "workspace_status",
-    "workspace_size", "decode_num_ctas", "kept_total", "n_parts", "SGD_F32", "SGD_BF16", "SGD_I8",
-    "SCHEME_A", "SCHEME_B", "STATUS_BITS",
+    "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select", "decode_attn",
+    "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
+    "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
+    "kernel_timing_stop", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B", "STATUS_BITS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
