@@ -300,9 +300,10 @@ def oam_select(q, k, v, cu_seqlens, G: int, beta: float, eps: float, keep_num: i
 
 def oam_select_multi(q, k, v, cu_seqlens, G: int, M: int, beta: float, eps: float, keep_num: int,
                      keep_den: int, rows: Optional[Sequence] = None):
-    """oam_select for M query tokens per sequence (q [B, M, Hq, D]): one kept set per (sequence,
-    KV head) serves all M * G query rows, so the group maximum of the score runs over all of
-    them: s_t = max_{m,g} (q[b, m, kvh*G+g] . k_t) / sqrt(D) + beta * ln(||v_t|| + eps).
+    """oam_select for M query tokens per sequence (q [B, M, Hq, D]; the speculative step of
+    "共同设计 AI 模型注意力..." decode section, scored as "优化稀疏注意力中的令牌丢弃机制" section 3):
+    one kept set per (sequence, KV head) serves all M * G query rows, so the group maximum of
+    the score runs over all of them: s_t = max_{m,g} (q[b, m, kvh*G+g] . k_t) / sqrt(D) + beta * ln(||v_t|| + eps).
     Same outputs as oam_select."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     B = cu.size - 1
@@ -386,7 +387,10 @@ def select_blocks(scores, cu_seqlens, Hkv: int, keep_num: int, keep_den: int, bl
 
 def decode_blocks(q, k, v, cu_seqlens, G: int, blk, cu_kept_blocks, block: int = PART, quant=None, rows=None):
     """Decode attending, per (sequence, KV head), to every token of that row's kept blocks
-    (the last block of a sequence holds fewer than ``block`` tokens): out [B, Hq, D], lse [B, Hq]."""
+    ("硬件对齐的稀疏注意力机制" (NSA) section 2.1: selected attention keeps the original tokens of
+    the chosen 64-token blocks; the attention itself is "优化稀疏注意力中的令牌丢弃机制" section 2
+    over that subset).  The last block of a sequence holds fewer than ``block`` tokens.
+    -> out [B, Hq, D], lse [B, Hq]."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     ckb = np.asarray(cu_kept_blocks, dtype=np.int64)
     B = cu.size - 1
