@@ -12,6 +12,9 @@ pages state them.  Sources are cited by page title and section:
   [TD] "优化稀疏注意力中的令牌丢弃机制" (Optimizing token dropping in sparse attention):
        section 3 (OAM), section 5 (split-KV and its merge), section 6 (INT8 schemes A and B).
   [AO] "注意力优化（Attention Optimization）": GQA example (query head h uses KV head h // G).
+  [CD] "共同设计 AI 模型注意力，实现快速的交互式长上下文推理": decode section (speculative decoding
+       verifies several query tokens per step).
+  [NSA] "硬件对齐的稀疏注意力机制：原理、优化与实践": section 2.1 (64-token selection blocks).
 """
 from __future__ import annotations
 
