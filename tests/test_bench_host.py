@@ -96,3 +96,20 @@ def test_scheme_b_codes_both_tensors_in_one_launch(bench):
     assert bench.kernel_bytes(wl, [100], "amax") == 2 * Hkv * T * D * 2
     sel = wl.with_(oam=True)  # the fused pass of scheme B writes no K codes
     assert bench.kernel_bytes(sel, [100], "score_quantize") == 2 * Hkv * T * D * 2 + Hkv * T * 4 + 1 * 8 * D * 2
+
+
+@pytest.mark.parametrize("workload", [7, 9])
+def test_reference_arm_prints_the_contract_line(workload):
+    # the oracle arm runs on the host cores: one bounded step of the workload, one JSON line
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        str(workload), "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["config"]["workload"] == workloads.config(workload).name
