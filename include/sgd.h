@@ -86,7 +86,7 @@ typedef enum { SGD_SCHEME_A = 0, SGD_SCHEME_B = 1 } sgd_scheme;
 #define SGD_STATUS_EMPTY_SEQUENCE 0x1 /* a sequence has length < 1 */
 #define SGD_STATUS_WAIT_TIMEOUT 0x2   /* a bounded pipeline wait gave up */
 #define SGD_STATUS_SIZE_MISMATCH 0x4  /* device lengths disagree with host sizes */
-#define SGD_STATUS_BAD_INDEX 0x8      /* a kept index was outside its sequence */
+#define SGD_STATUS_BAD_INDEX 0x8      /* a kept index or block number was outside its sequence */
 
 #define SGD_WS_STATUS_OFFSET 0
 
