@@ -190,3 +190,39 @@ def test_config6_and_9_selection_over_the_int8_cache(sgd, n):
                             quant=(*quant, "A"), rows=rows)
     assert sgd.workspace_status(ws) == 0
     compare_rows(out, lse, *ref, rows, wl.G)
+
+
+def test_config10_four_query_tokens_int8_128k(sgd):
+    # 32 columns per KV head: two CTAs per split range, one per group of 16 columns
+    wl = workloads.config(10)
+    bt = workloads.generate(wl)
+    assert bt.q.shape == (wl.B, 4, wl.Hq, wl.D)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, wsq = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    del k, v
+    out, lse, ws = sgd.decode_attn_multi(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                         n_parts_=sgd.n_parts(bt.lengths))
+    assert sgd.workspace_status(wsq) == 0 and sgd.workspace_status(ws) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    rows = sample_rows(bt, n_extra=0)
+    ref_out, ref_lse = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, 4, quant=(*quant, "A"), rows=rows)
+    for m in range(4):
+        compare_rows(out[:, m], lse[:, m], ref_out[:, m], ref_lse[:, m], rows, wl.G)
+
+
+@pytest.mark.parametrize("n", [12, 13])
+def test_config12_13_query_codes_int8_128k(sgd, n):
+    # the scheme table: per-tensor Q/K/V (scheme B, one query scale) and scheme A with query codes
+    wl = workloads.config(n)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, wsq = sgd.quantize_kv(k, v, cu, wl.scheme, bt.lengths)
+    del k, v
+    out, lse, ws = sgd.decode_attn(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=wl.scheme,
+                                   n_parts_=sgd.n_parts(bt.lengths), q_quant=wl.q_quant)
+    assert sgd.workspace_status(wsq) == 0 and sgd.workspace_status(ws) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, wl.scheme)
+    qd = oracle.dequant_q(*oracle.quantize_q(bt.q, wl.q_quant))
+    rows = sample_rows(bt, n_extra=1)
+    ref = oracle.decode(qd, bt.k, bt.v, bt.cu_seqlens, wl.G, quant=(*quant, wl.scheme), rows=rows)
+    compare_rows(out, lse, *ref, rows, wl.G)
