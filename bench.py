@@ -95,7 +95,11 @@ def kernel_role(name):
     """What a library kernel (demangled name) does in the step."""
     if "decode_mma_kernel" in name:
         m = re.search(r"MmaCfg<\d+, \d+, \w+, \w+, (\d+)", name)
-        return {"0": "decode", "1": "score", "2": "score_quantize"}.get(m.group(1) if m else "", "decode")
+        mode = m.group(1) if m else ""
+        if not m and "MmaCfgI" in name:  # a mangled name: the fifth template argument is the mode
+            args = re.findall(r"L[ib](\d+)E", name.split("MmaCfgI", 1)[1])
+            mode = args[4] if len(args) > 4 else ""
+        return {"0": "decode", "1": "score", "2": "score_quantize"}.get(mode, "decode")
     for key, role in (("quant_global_kernel", "v_codes"), ("topk_cluster_kernel", "topk"), ("plan_kernel", "plan"),
                       ("block_max_kernel", "block_max"), ("quant_k_partition_kernel", "k_codes"),
                       ("quant_amax_kernel", "amax"), ("quant_prep_kernel", "prep"), ("merge_kernel", "merge"),

@@ -30,6 +30,11 @@ def test_kernel_roles_from_demangled_names(bench):
     assert r("void sgd::topk_cluster_kernel<512, 8, 2>") == "topk"
     assert r("sgd::plan_kernel") == "plan" and r("sgd::block_max_kernel") == "block_max"
     assert r("void sgd::decode_generic_kernel<128, float, true, 0>") == "decode"
+    # without a demangler the mangled names give the same roles
+    assert r("_ZN3sgd17decode_mma_kernelINS_6MmaCfgILi128ELi1ELb0ELb0ELi2ELb0ELb0ELb0EEEEEv14CUtensorMap_stS3_"
+             "NS_10DecodeArgsE") == "score_quantize"
+    assert r("_ZN3sgd17decode_mma_kernelINS_6MmaCfgILi128ELi1ELb1ELb1ELi0ELb0ELb0ELb0EEEEEv14CUtensorMap_stS3_"
+             "NS_10DecodeArgsE") == "decode"
 
 
 def test_demangle_reads_the_library_names(bench):
