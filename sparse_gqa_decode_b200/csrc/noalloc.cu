@@ -51,12 +51,14 @@ extern "C" int sgd_decode_attn_noalloc(const void *q, sgd_dtype q_dtype, int G, 
     if (rc != SGD_OK) return rc;
     const size_t need = sgd_workspace_size(SGD_OP_DECODE, kv, G, schedule, n_splits);
     if (need > SGD_NOALLOC_SCRATCH_BYTES) return SGD_ERR_SCRATCH_LIMIT;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return SGD_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the previous call's header is still there: start from a clear status word
-    if (cudaMemsetAsync(scratch, 0, sizeof(sgd::WsHeader), s) != cudaSuccess) return SGD_ERR_CUDA;
+    // The previous call's header is still in the array.  Nothing needs clearing here: the plan
+    // kernel, the first launch of the decode, zeroes the status word and the per-row counters
+    // before any other kernel of the call reads them, and a call rejected on the host launches
+    // nothing at all.
     rc = sgd_decode_attn(q, q_dtype, G, kv, idx, cu_kept, kept_total, schedule, n_splits, q_quant, out, lse,
-                         scratch,
-                         SGD_NOALLOC_SCRATCH_BYTES, stream);
+                         scratch, SGD_NOALLOC_SCRATCH_BYTES, stream);
     if (rc == SGD_OK && status) {
         if (cudaMemcpyAsync(status, static_cast<uint8_t *>(scratch) + SGD_WS_STATUS_OFFSET, sizeof(int32_t),
                             cudaMemcpyDeviceToDevice, s) != cudaSuccess)
