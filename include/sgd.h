@@ -349,6 +349,36 @@ int sgd_kernel_timing_start(int max_launches);
 int sgd_kernel_timing_stop(float *ms, int max, int *count);
 const char *sgd_kernel_timing_name(int k);
 
+/*
+ * sgd_stream_read -- measurement aid: the read-only HBM ceiling.  Reads the `bytes` bytes at
+ * `buf` (device, 16-byte aligned, bytes a positive multiple of 16) exactly once and XORs them,
+ * folded to 32-bit words, into *sink (device, 8-byte aligned); the decode kernels mostly read,
+ * so their bandwidth is compared with this rate as well as with a copy's.
+ * method   0: 16-byte loads from every thread, eight in flight each, grid-stride;
+ *          1: bulk asynchronous copies (cp.async.bulk) of 32 KB chunks into a six-stage
+ *             shared-memory ring per SM, each chunk folded by the CTA's warp
+ * status   device int32: SGD_STATUS_WAIT_TIMEOUT if a bounded wait of method 1 ran out
+ * Time it with events around the call on `stream`; the pages have no counterpart.
+ */
+int sgd_stream_read(const void *buf, size_t bytes, int method, unsigned long long *sink, int32_t *status,
+                    void *stream);
+
+/*
+ * sgd_test_pipeline_timeout -- test aid for the bounded pipeline waits (failure detection).
+ * Every wait of the decode and score kernels on their shared-memory pipeline is bounded: when
+ * it runs out, the kernel sets SGD_STATUS_WAIT_TIMEOUT in the workspace status word, each CTA
+ * lets its copies already in flight land and the launch ends promptly with the context usable
+ * (no trap, no fault); the outputs of that call are then undefined.
+ * polls        > 0: from the next call on, a wait gives up after `polls` polls instead of the
+ *              built-in limit (about 4 million); 0 restores the built-in limit
+ * idle_producer != 0: the producer warps issue no copies at all, so every consumer wait runs out
+ *              with nothing in flight -- how a test makes the timeout path run without a fault;
+ *              0 restores normal operation
+ * Host state of the process, not thread-safe; affects calls enqueued after it.  SGD_ERR_ARG for
+ * polls < 0.  The pages have no counterpart: this serves testing only.
+ */
+int sgd_test_pipeline_timeout(int64_t polls, int idle_producer);
+
 /* Library version, (major << 16) | minor. */
 int sgd_version(void);
 

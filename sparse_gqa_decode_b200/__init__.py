@@ -31,7 +31,7 @@ __all__ = [
     "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select", "decode_attn",
     "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
-    "kernel_timing_stop", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B", "STATUS_BITS",
+    "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B", "STATUS_BITS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,8 @@ lib.sgd_oam_select_blocks.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32,
                                       _vp]
 lib.sgd_decode_attn_blocks.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _sz,
                                        _vp]
+lib.sgd_test_pipeline_timeout.argtypes = [_i64, _i32]
+lib.sgd_stream_read.argtypes = [_vp, _sz, _i32, _vp, _vp, _vp]
 lib.sgd_kernel_timing_start.argtypes = [_i32]
 lib.sgd_kernel_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(ctypes.c_int32)]
 lib.sgd_kernel_timing_name.argtypes = [_i32]
@@ -379,6 +381,26 @@ def decode_attn_noalloc(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tenso
                                        _ptr(status),
                                        _stream(stream)), "sgd_decode_attn_noalloc")
     return o, lse
+
+
+def stream_read(buf: torch.Tensor, method: int = 0, sink=None, status=None, stream=None):
+    """Measurement aid: read every byte of ``buf`` once (method 0: 16-byte loads, 1: bulk copies
+    into shared memory), XOR-folded into ``sink`` ([1] int64).  Returns (sink, status)."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int64, device=buf.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size() // 16 * 16
+    _check(lib.sgd_stream_read(_ptr(buf), nbytes, int(method), _ptr(sink), _ptr(status), _stream(stream)),
+           "sgd_stream_read")
+    return sink, status
+
+
+def test_pipeline_timeout(polls: int, idle_producer: bool) -> None:
+    """Test aid: lower the bounded pipeline-wait limit to ``polls`` polls (0 = the built-in limit)
+    and, with ``idle_producer``, keep the kernels' producer warps from issuing copies, so that the
+    waits run out and report SGD_STATUS_WAIT_TIMEOUT.  Affects calls made afterwards."""
+    _check(lib.sgd_test_pipeline_timeout(int(polls), 1 if idle_producer else 0), "sgd_test_pipeline_timeout")
 
 
 def kernel_timing_start(max_launches: int = 256) -> None:

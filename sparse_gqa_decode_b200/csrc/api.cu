@@ -158,7 +158,19 @@ struct KernelTiming {
 };
 KernelTiming g_kt;
 
+// sgd_test_pipeline_timeout: a lowered wait limit and idle producers (host state of the process)
+struct TestHooks {
+    long long wait_limit = 0;  // 0: kWaitLimit
+    int idle_producer = 0;
+};
+TestHooks g_hooks;
+
 }  // namespace
+
+void apply_test_hooks(DecodeArgs &a) {
+    a.wait_limit = g_hooks.wait_limit > 0 ? g_hooks.wait_limit : kWaitLimit;
+    a.idle_producer = g_hooks.idle_producer;
+}
 
 int kt_begin(cudaStream_t s) {
     if (!g_kt.on || g_kt.n >= (int)g_kt.fn.size()) return -1;
@@ -258,6 +270,7 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     a.status = &hdr->status;
     a.q_quant = q_quant;
     a.q_scale = &hdr->q_scale;
+    apply_test_hooks(a);
     int e = launch_decode(a, kv->dtype, q_dtype, indexed, false, n_req * ncg, s);
     if (e != 0) return SGD_ERR_CUDA;
     // the tensor-core kernel merges each row itself (its last CTA); the CUDA-core one leaves partials
@@ -333,6 +346,7 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
     a.scores = reinterpret_cast<float *>(ws + L.scores);
     a.plan = pv;
     a.status = &hdr->status;
+    apply_test_hooks(a);
     int e = launch_decode(a, kv->dtype, q_dtype, false, true, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
     if (blocks) {  // block scores, then the top blocks of each row (the plan's partition offsets = block offsets)
@@ -353,6 +367,27 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
 extern "C" {
 
 int sgd_version(void) { return (1 << 16) | 0; }
+
+int sgd_stream_read(const void *buf, size_t bytes, int method, unsigned long long *sink, int32_t *status,
+                    void *stream) {
+    if (!buf || !sink || !status) return SGD_ERR_NULL;
+    if (bytes == 0 || bytes % 16 != 0) return SGD_ERR_SHAPE;
+    if (method != 0 && method != 1) return SGD_ERR_ARG;
+    if (!aligned16(buf) || (reinterpret_cast<uintptr_t>(sink) & 7u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+        return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    int rc = current_device(&dev);
+    if (rc != SGD_OK) return rc;
+    return launch_stream_read(buf, bytes, method, sink, status, dev->sms, as_stream(stream)) == 0 ? SGD_OK
+                                                                                                  : SGD_ERR_CUDA;
+}
+
+int sgd_test_pipeline_timeout(int64_t polls, int idle_producer) {
+    if (polls < 0) return SGD_ERR_ARG;
+    g_hooks.wait_limit = (long long)polls;
+    g_hooks.idle_producer = idle_producer != 0;
+    return SGD_OK;
+}
 
 int sgd_kernel_timing_start(int max_launches) {
     if (max_launches < 1 || max_launches > 4096) return SGD_ERR_ARG;
@@ -563,6 +598,7 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     a.amax_bits = hdr->amax_bits;
     a.plan = pv;
     a.status = &hdr->status;
+    apply_test_hooks(a);
     int e = launch_score_quantize(a, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
     e = launch_quantize_global(kv->k, kv->v, kv->dtype, kv->Hkv, kv->D, kv->T, scheme, k_codes, v_codes, k_scale,

@@ -115,20 +115,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity.  Every wait is bounded: after kWaitLimit polls
-// the wait records SGD_STATUS_WAIT_TIMEOUT, raises the CTA's abort flag and returns false.
-// Once the flag is up every later wait of the CTA returns false at once, so all warps still
-// run through the same (named) barriers and the kernel ends promptly instead of hanging.
+// Waits for the phase with the given parity.  Every wait is bounded: after `limit` polls
+// (kWaitLimit unless a test lowers it) the wait records SGD_STATUS_WAIT_TIMEOUT, raises the
+// CTA's abort flag and returns false.  Once the flag is up every later wait of the CTA returns
+// false at once, so all warps still run through the same (named) barriers and the kernel ends
+// promptly instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
-                                          volatile int32_t *abort_flag) {
+                                          volatile int32_t *abort_flag, long long limit) {
     if (*abort_flag) return false;
-    for (long long i = 0; i < kWaitLimit; ++i) {
+    for (long long i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 1023) == 1023 && *abort_flag) return false;
     }
     *abort_flag = 1;
     atomicOr(status, SGD_STATUS_WAIT_TIMEOUT);
     return false;
+}
+
+// Bounded wait for a phase that a copy this thread issued completes, regardless of the abort
+// flag: a producer calls it before it exits so that no copy is still writing into the CTA's
+// shared memory when the CTA ends.  False if the limit ran out.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, long long limit) {
+    for (long long i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// Orders this thread's generic-proxy shared-memory accesses before later async-proxy ones (a
+// stage read by the threads, then refilled by TMA or a bulk copy).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 2-D tiled TMA load of one box into shared memory, completing on `bar` (tx bytes).
@@ -159,6 +175,9 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
 __device__ __forceinline__ void cp_async_4(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+
+// Waits until every cp.async this thread issued has landed in shared memory.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");

@@ -46,10 +46,6 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_shared() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
 
 template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false, bool CAUSAL_ = false,
@@ -107,6 +103,7 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                                              volatile int32_t *abort_flag, float *row_scale,
                                              int cta, int lane) {
     if (!C::IDX && lane != 0) return;
+    if (a.idle_producer) return;  // test aid: nothing is issued, so every consumer wait runs out
     uint64_t pol = 0;
     if constexpr (!C::IDX) {
         prefetch_tensormap(tmK);
@@ -117,9 +114,11 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
     cur.init(a.plan, a.B * a.Hkv, cta);
     int stage = 0;
     uint32_t phase = 0;
+    uint32_t filled = 0, fill_par = 0;  // per stage: filled at least once; parity of its last fill
+    bool stop = false;
     int row, slot;
     int32_t t0, t1;
-    while (cur.next(row, t0, t1, slot)) {
+    while (!stop && cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
         const int64_t seq0 = (int64_t)kvh * a.T + cur.ri.seq_start;
         const int32_t Lb = cur.ri.seq_len;
@@ -171,7 +170,16 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
             load_tile_blk(t0 + C::ROWS);
         }
         for (int32_t t = t0; t < t1; t += C::ROWS) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag)) return;
+            // a consumer that gave up still releases its stages: after any wait, the abort flag
+            // (raised before that release) says whether the stage was really consumed
+            bool ok = mbar_wait(&empty[stage], phase ^ 1, a.status, abort_flag, a.wait_limit) && !*abort_flag;
+            if constexpr (C::IDX) ok = __all_sync(0xffffffffu, ok);  // the gathers need the whole warp
+            if (!ok) {
+                stop = true;
+                break;
+            }
+            filled |= 1u << stage;
+            fill_par = (fill_par & ~(1u << stage)) | (phase << stage);
             uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
             if constexpr (C::BLK) {
@@ -254,6 +262,15 @@ __device__ __forceinline__ void mma_producer(const CUtensorMap *tmK, const CUten
                 phase ^= 1;
             }
         }
+    }
+    // Before the producer (and with it, eventually, the CTA) ends, every copy it issued has
+    // landed: the consumers may have given up on a stage whose copy is still in flight.
+    if constexpr (C::IDX) {
+        cp_async_wait_all();
+    } else {
+#pragma unroll
+        for (int st = 0; st < C::STAGES; ++st)
+            if ((filled >> st) & 1u) mbar_drain(&full[st], (fill_par >> st) & 1u, a.wait_limit);
     }
 }
 
@@ -616,7 +633,7 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
         int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + cur.ri.seq_start) * C::D + half * (C::D / LPR);
         float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + cur.ri.part0;
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
-            const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
+            const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag, a.wait_limit);
             const uint32_t kbase = smem_u32(smem + stage * C::STAGE_BYTES);
             const int32_t j = t + vr;
             const bool vrow = ready && j < t1;
@@ -949,7 +966,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MINB)
                 }
             }
             if constexpr (C::KONLY) load_norms(vn_nxt, t + C::ROWS);
-            const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag);
+            // warp-uniform: the MMAs and shuffles below need every lane
+            const bool ready = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase, a.status, abort_flag, a.wait_limit));
             uint8_t *sk = smem + stage * C::STAGE_BYTES;
             uint8_t *sv = sk + C::TILE;
             const uint32_t kbase = smem_u32(sk), vbase = smem_u32(sv);

@@ -40,7 +40,12 @@ struct DecodeArgs {
     float *out;              // decode: [B, M, Hq, D] result (written by the kernel itself on the MMA path)
     float *lse;              // decode: [B, M, Hq]
     int32_t *status;
+    long long wait_limit;    // polls before a pipeline wait gives up (kWaitLimit unless a test lowers it)
+    int idle_producer;       // test aid: the producer warps issue no copies (every consumer wait runs out)
 };
+
+// The test hooks of sgd_test_pipeline_timeout (api.cu) applied to a launch's arguments.
+void apply_test_hooks(DecodeArgs &a);
 
 // kernel families
 enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
@@ -89,5 +94,11 @@ int launch_topk(const float *scores, const int32_t *cu, int B, int Hkv, int64_t 
 // (sequence b's blocks are cu_blk[b] .. cu_blk[b+1]; its last block may be ragged).
 int launch_block_max(const float *scores, const int32_t *cu_seq, const int32_t *cu_blk, int B, int Hkv, int64_t T,
                      int64_t Tb, float *bscores, int32_t *status, cudaStream_t s);
+
+// stream.cu
+// Read-only streaming of `bytes` bytes (method 0: 16-byte loads; 1: bulk copies into shared
+// memory), every byte XOR-folded into *sink.
+int launch_stream_read(const void *buf, size_t bytes, int method, unsigned long long *sink, int32_t *status,
+                       int sm_count, cudaStream_t s);
 
 }  // namespace sgd

@@ -207,3 +207,10 @@ def test_workspace_size_limits(sgd):
     assert L.sgd_workspace_size(sgd.OP_DECODE, ctypes.byref(kv), 65, 0, 0) == 0  # decode columns <= 64
     assert L.sgd_workspace_size(sgd.OP_OAM_SELECT, ctypes.byref(kv), 17, 0, 0) == 0  # selection G <= 16
     assert L.sgd_workspace_size(sgd.OP_DECODE, ctypes.byref(kv), 0, 0, 0) == 0
+
+
+def test_pipeline_timeout_hook_is_host_state_only(sgd):
+    # the test aid of the bounded waits: a negative limit is rejected, 0 restores the built-in one
+    assert sgd.lib.sgd_test_pipeline_timeout(-1, 0) == -8
+    assert sgd.lib.sgd_test_pipeline_timeout(4096, 1) == 0
+    assert sgd.lib.sgd_test_pipeline_timeout(0, 0) == 0
