@@ -118,3 +118,22 @@ def test_reference_arm_prints_the_contract_line(workload):
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["config"]["workload"] == workloads.config(workload).name
+
+
+def test_rates_against_the_three_denominators(bench):
+    f = bench.fractions(4000.0, 6400.0, 7000.0)
+    assert f["frac_of_hbm"] == pytest.approx(0.625) and f["frac_of_nominal"] == pytest.approx(0.5)
+    assert f["frac_of_read_only"] == pytest.approx(4000 / 7000, abs=1e-4)
+    assert "frac_of_read_only" not in bench.fractions(1.0, 2.0, None)
+
+
+def test_cpu_baseline_counts_the_same_rows_on_one_or_several_threads(bench):
+    # a small copy of the default workload: every row fits the budget, so both runs cover all rows
+    wl = workloads.config(5, B=2, Hkv=2, length_range=(200, 900))
+    bt = workloads.generate(wl, 5)
+    _, s1, _, t1 = bench.cpu_baseline_sample(bt, wl, budget_s=60.0, threads=1)
+    _, s4, _, t4 = bench.cpu_baseline_sample(bt, wl, budget_s=60.0, threads=4)
+    assert t1 == 1 and t4 == 4
+    tokens = int(bt.lengths.sum()) * wl.Hkv
+    for s in (s1, s4):
+        assert s.startswith(f"4 (sequence, KV head) rows of the workload, shortest first, {tokens} tokens")

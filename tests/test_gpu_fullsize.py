@@ -226,3 +226,82 @@ def test_config12_13_query_codes_int8_128k(sgd, n):
     rows = sample_rows(bt, n_extra=1)
     ref = oracle.decode(qd, bt.k, bt.v, bt.cu_seqlens, wl.G, quant=(*quant, wl.scheme), rows=rows)
     compare_rows(out, lse, *ref, rows, wl.G)
+
+
+def check_kept_sets(idx, cu_kept, ref_idx, ref_cu, scores, max_diff):
+    """Every row's kept set against the oracle's top-K: identical except tokens whose oracle score
+    lies within 1e-4 of the row's K-th score; positions ascending."""
+    assert cu_kept.cpu().tolist() == ref_cu.tolist()
+    got = idx.cpu().numpy()
+    n_diff = 0
+    for (b, h), s in scores.items():
+        a, e = int(ref_cu[b]), int(ref_cu[b + 1])
+        kth = np.sort(s)[::-1][e - a - 1]
+        g, w = set(got[h, a:e].tolist()), set(ref_idx[h, a:e].tolist())
+        assert (np.diff(got[h, a:e]) > 0).all(), (b, h)
+        for t in g ^ w:
+            assert abs(s[t] - kth) <= 1e-4, (b, h, t)
+        n_diff += len(g ^ w)
+    assert n_diff <= max_diff
+
+
+@pytest.mark.parametrize("n,scheme", [(5, "A"), (4, "A"), (4, "B")])
+def test_fused_quantize_select_full_size(sgd, n, scheme):
+    """The call the benchmark times, sgd_quantize_select, at full size: workload 5 (4 sequences of
+    32K-128K tokens) and workload 4's 8 x 128K cache, where a bf16 tensor is 2 GiB and byte offsets
+    pass 2^31.  Every K and V code and every scale bit-exact, the stored value norms, every row's
+    kept set, then the decode over the kept tokens on sampled rows, all against the oracle."""
+    wl = workloads.config(n)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    vn = torch.empty(k.shape[:2], dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, idx, cu_kept, wsq = sgd.quantize_select(q, k, v, cu, wl.G, wl.beta, wl.eps, wl.keep_num,
+                                                            wl.keep_den, scheme, bt.lengths, v_norm=vn)
+    del k, v
+    assert sgd.workspace_status(wsq) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    assert np.array_equal(ks.cpu().numpy().reshape(quant[2].shape), quant[2])
+    assert np.array_equal(vs.cpu().numpy(), quant[3])
+    for h in range(wl.Hkv):  # every code and value norm, one head at a time
+        assert np.array_equal(kc[h].cpu().numpy(), quant[0][h]), h
+        assert np.array_equal(vc[h].cpu().numpy(), quant[1][h]), h
+        ref_vn = oracle.value_norms(bt.v[h])
+        assert np.allclose(vn[h].double().cpu().numpy(), ref_vn, rtol=1e-5, atol=0), h
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, wl.beta, wl.eps,
+                                                wl.keep_num, wl.keep_den)
+    check_kept_sets(idx, cu_kept, ref_idx, ref_cu, scores, max_diff=4 * wl.B * wl.Hkv)
+    out, lse, ws = sgd.decode_attn(q, wl.G, kc, vc, cu, k_scale=ks, v_scale=vs, scheme=scheme,
+                                   n_parts_=sgd.n_parts(bt.lengths), idx=idx, cu_kept=cu_kept,
+                                   kept_total_=idx.shape[1])
+    assert sgd.workspace_status(ws) == 0
+    rows = sample_rows(bt, n_extra=2)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, idx=ref_idx, cu_kept=ref_cu,
+                        quant=(*quant, scheme), rows=rows)
+    compare_rows(out, lse, *ref, rows, wl.G)
+
+
+def test_config14_ragged_int8_decode(sgd):
+    """The ragged INT8 batch (16 log-uniform lengths in [512, 128K] over the scheme-A cache) in the
+    bench's launch configuration: every code and scale bit-exact, sampled rows (shortest and longest
+    included) of the equal-work split decode against the oracle, and the one-CTA-per-row schedule
+    agreeing with it on every row."""
+    wl = workloads.config(14)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    kc, vc, ks, vs, wsq = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    del k, v
+    kw = dict(k_scale=ks, v_scale=vs, scheme="A", n_parts_=sgd.n_parts(bt.lengths))
+    o0, l0, ws0 = sgd.decode_attn(q, wl.G, kc, vc, cu, schedule=0, **kw)
+    o1, l1, ws1 = sgd.decode_attn(q, wl.G, kc, vc, cu, schedule=1, **kw)
+    assert sgd.workspace_status(wsq) == 0 and sgd.workspace_status(ws0) == 0 and sgd.workspace_status(ws1) == 0
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    assert np.array_equal(ks.cpu().numpy().reshape(quant[2].shape), quant[2])
+    assert np.array_equal(vs.cpu().numpy(), quant[3])
+    assert np.array_equal(kc.cpu().numpy(), quant[0]) and np.array_equal(vc.cpu().numpy(), quant[1])
+    rows = sample_rows(bt, n_extra=4)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, wl.G, quant=(*quant, "A"), rows=rows)
+    compare_rows(o0, l0, *ref, rows, wl.G)
+    compare_rows(o1, l1, *ref, rows, wl.G)
+    scale = o1.abs().max().item()
+    assert (o0 - o1).abs().max().item() <= OUT_TOL * scale
+    assert (l0 - l1).abs().max().item() <= LSE_TOL

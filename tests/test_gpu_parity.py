@@ -591,10 +591,17 @@ BLOCK_LENGTHS = (1, 64, 65, 130, 700, 4099)
 @pytest.mark.parametrize("cache", ["bf16", "int8A", "int8B"])
 @pytest.mark.parametrize("G,D", [(8, 128), (4, 64)])
 def test_block_selection_matches_oracle(sgd, cache, G, D):
-    if cache != "bf16" and D != 128:
-        pytest.skip("the INT8 cache is scored at D = 128")
     bt = make(BLOCK_LENGTHS, G=G, D=D, Hkv=2, dist="outlier", seed=41 + G)
     q, k, v, cu = dev(bt)
+    if cache != "bf16" and D != 128:
+        # the INT8 cache is scored at D = 128 only: the call is rejected on the host
+        scheme = cache[-1]
+        vn = torch.empty((2, bt.T), dtype=torch.float32, device="cuda")
+        kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn)
+        with pytest.raises(sgd.SgdError, match=r"\(-3\)"):
+            sgd.oam_select_blocks(q, kc, vc, cu, G, 1.0, 1e-6, 1, 4, bt.lengths, k_scale=ks, v_scale=vs,
+                                  scheme=scheme, n_parts_=sgd.n_parts(bt.lengths), v_norm=vn)
+        return
     if cache == "bf16":
         blk, cu_kb, ws = sgd.oam_select_blocks(q, k, v, cu, G, 1.0, 1e-6, 1, 4, bt.lengths)
         _, _, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)
@@ -615,10 +622,18 @@ def test_block_selection_matches_oracle(sgd, cache, G, D):
 @pytest.mark.parametrize("cache", ["bf16", "int8A", "int8B"])
 @pytest.mark.parametrize("G,D", [(8, 128), (16, 128), (4, 64)])
 def test_decode_over_blocks_matches_oracle(sgd, cache, G, D):
-    if cache != "bf16" and D != 128:
-        pytest.skip("the INT8 cache decodes on tensor cores at D = 128")
     bt = make(BLOCK_LENGTHS, G=G, D=D, Hkv=2, dist="outlier", seed=43 + G)
     q, k, v, cu = dev(bt)
+    if cache != "bf16" and D != 128:
+        # kept blocks of an INT8 cache decode on the tensor cores at D = 128 only: rejected on the host
+        scheme = cache[-1]
+        kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths)
+        tb = torch.zeros((2, bt.wl.B), dtype=torch.int32, device="cuda")
+        tcu = torch.arange(bt.wl.B + 1, dtype=torch.int32, device="cuda")
+        with pytest.raises(sgd.SgdError, match=r"\(-3\)"):
+            sgd.decode_attn_blocks(q, G, kc, vc, cu, tb, tcu, k_scale=ks, v_scale=vs, scheme=scheme,
+                                   n_parts_=sgd.n_parts(bt.lengths))
+        return
     # a seeded kept-block set: a quarter of each row's blocks, always with its ragged last block
     rng = np.random.default_rng(5)
     nb = [-(-int(L) // 64) for L in BLOCK_LENGTHS]

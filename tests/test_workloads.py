@@ -58,3 +58,13 @@ def test_named_configurations_and_their_seeds():
     assert workloads.config(5).scheme == "A" and workloads.config(5).oam
     assert workloads.config(7).seed == 5 and workloads.config(9).seed == 6  # shared batches
     assert workloads.config(4, lengths=(64,) * 8).lengths == (64,) * 8
+
+
+def test_ragged_int8_workload_shares_the_ragged_lengths():
+    # workload 14 is workload 3's ragged batch (same seed, lengths drawn first) over workload 4's
+    # INT8 cache distribution; one KV head is enough to see the lengths
+    a = workloads.generate(workloads.config(3).with_(Hkv=1))
+    b = workloads.generate(workloads.config(14).with_(Hkv=1))
+    assert a.lengths.tolist() == b.lengths.tolist()
+    assert b.outlier_channels is not None and workloads.config(14).scheme == "A"
+    assert (512 <= b.lengths).all() and (b.lengths <= 131072).all()

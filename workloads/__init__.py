@@ -114,11 +114,15 @@ CONFIGS = {
                  lengths=(131072,) * 8, scheme="B", q_quant="tensor", seed=4),
     13: Workload("int8A_qcodes_B8_L128K", B=8, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
                  lengths=(131072,) * 8, scheme="A", q_quant="token", seed=4),
+    # the ragged batch of workload 3 (its seed, so the same 16 log-uniform lengths in [512, 128K]:
+    # the lengths are the first draw) over workload 4's INT8 scheme-A cache distribution
+    14: Workload("ragged_int8A_B16_L512-128K", B=16, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
+                 length_range=(512, 131072), scheme="A", seed=3),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..13), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..14), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
