@@ -472,6 +472,87 @@ def test_quantize_select_equals_separate_calls(sgd, scheme, G, D, dtype):
 
 
 # ---------------------------------------------------------------------------------------------
+# batches of many short sequences: hundreds of rows per CTA range, both schedules, the whole path
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("B", [256, 257, 300])
+def test_batches_of_many_short_sequences(sgd, B):
+    rng = np.random.default_rng(B)
+    lengths = [int(x) for x in rng.integers(1, 260, size=B)]
+    lengths[3] = 64  # a row of whole granules
+    bt = make(lengths, G=8, D=128, Hkv=2, dist="outlier", seed=70 + B)
+    q, k, v, cu = dev(bt)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8)
+    for schedule, n_splits in ((0, 0), (0, 37), (1, 0)):
+        out, lse, ws = sgd.decode_attn(q, 8, k, v, cu, schedule=schedule, n_splits=n_splits)
+        assert_close(out, lse, *ref, OUT_TOL["bf16"])
+        check_status(sgd, ws)
+    idx, cu_kept, wss = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 4, bt.lengths)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 1.0, 1e-6, 1, 4)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, B, 2)
+    check_status(sgd, wss)
+    kc, vc, ks, vs, idx2, cu2, wsq = sgd.quantize_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 4, "A", bt.lengths)
+    check_status(sgd, wsq)
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    assert np.array_equal(kc.cpu().numpy(), quant[0]) and np.array_equal(ks.cpu().numpy(), quant[2])
+    check_selection(idx2, cu2.cpu(), ref_idx, ref_cu, scores, B, 2)
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                   n_parts_=sgd.n_parts(bt.lengths), idx=idx2, cu_kept=cu2, kept_total_=idx2.shape[1])
+    check_status(sgd, ws)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=idx2.cpu().numpy(), cu_kept=cu2.cpu().numpy(),
+                        quant=(*quant, "A"))
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------------------------
+# a mid-size batch: 32 rows of 700-31000 tokens over every SM, so rows span many CTA ranges and the
+# row merges, the fused pass and the selection all run in the automatic split the bench uses
+# ---------------------------------------------------------------------------------------------
+MID_LENGTHS = (20000, 9001, 31000, 700)
+
+
+def test_mid_size_decode_selection_and_fused_pass(sgd):
+    bt = make(MID_LENGTHS, G=8, D=128, Hkv=8, dist="outlier", seed=404)
+    q, k, v, cu = dev(bt)
+    out, lse, ws = sgd.decode_attn(q, 8, k, v, cu)
+    check_status(sgd, ws)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8)
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+    kc, vc, ks, vs, idx, cu_kept, wsq = sgd.quantize_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, "A", bt.lengths)
+    check_status(sgd, wsq)
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    for h in range(8):
+        assert np.array_equal(kc[h].cpu().numpy(), quant[0][h]) and np.array_equal(vc[h].cpu().numpy(), quant[1][h])
+    assert np.array_equal(ks.cpu().numpy(), quant[2]) and np.array_equal(vs.cpu().numpy(), quant[3])
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 1.0, 1e-6, 1, 8)
+    check_selection(idx, cu_kept.cpu(), ref_idx, ref_cu, scores, bt.wl.B, 8)
+    sidx, scu, wss = sgd.oam_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, bt.lengths)
+    check_status(sgd, wss)
+    check_selection(sidx, scu.cpu(), ref_idx, ref_cu, scores, bt.wl.B, 8)
+    kw = dict(k_scale=ks, v_scale=vs, scheme="A", n_parts_=sgd.n_parts(bt.lengths))
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, **kw)  # dense INT8
+    check_status(sgd, ws)
+    assert_close(out, lse, *oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, quant=(*quant, "A")), OUT_TOL["bf16"])
+    out, lse, ws = sgd.decode_attn(q, 8, kc, vc, cu, idx=idx, cu_kept=cu_kept, kept_total_=idx.shape[1], **kw)
+    check_status(sgd, ws)
+    ref = oracle.decode(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, idx=idx.cpu().numpy(), cu_kept=cu_kept.cpu().numpy(),
+                        quant=(*quant, "A"))
+    assert_close(out, lse, *ref, OUT_TOL["bf16"])
+
+
+def test_mid_size_with_column_groups(sgd):
+    # four query tokens of G = 8: two CTAs per range, one per group of 16 (query token, head) columns
+    bt = make_multi(MID_LENGTHS, M=4, G=8, Hkv=8, seed=405)
+    q, k, v, cu = dev(bt)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, "A", bt.lengths)
+    out, lse, ws = sgd.decode_attn_multi(q, 8, kc, vc, cu, k_scale=ks, v_scale=vs, scheme="A",
+                                         n_parts_=sgd.n_parts(bt.lengths))
+    check_status(sgd, ws)
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    ref = oracle.decode_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, 8, 4, quant=(*quant, "A"))
+    assert_close_multi(out, lse, *ref, OUT_TOL["bf16"])
+
+
+# ---------------------------------------------------------------------------------------------
 # device status reporting
 # ---------------------------------------------------------------------------------------------
 def test_empty_sequence_is_reported(sgd):
