@@ -52,7 +52,19 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-north-star", action="store_true",
                    help="skip the workload 4 / 14 decode stages and the read-only ceiling")
+    p.add_argument("--scale", type=float, default=1.0,
+                   help="sequence lengths times this factor (a smaller case of the same shapes, for profiling)")
     return p.parse_args()
+
+
+def scaled(wl, scale):
+    """The workload with every sequence length times `scale` (at least one token)."""
+    if scale == 1.0:
+        return wl
+    if wl.lengths is not None:
+        return wl.with_(lengths=tuple(max(1, int(round(L * scale))) for L in wl.lengths))
+    lo, hi = wl.length_range
+    return wl.with_(length_range=(max(1, int(round(lo * scale))), max(1, int(round(hi * scale)))))
 
 
 # ------------------------------------------------------------------------------------------------
@@ -518,6 +530,8 @@ def decode_stage_record(sgd, n, dev, K, W, flush_l2, peak, read_only, world):
            "algorithmic_bytes": nbytes,
            "kernel": dk["name"], "kernel_ms": round(k_ms, 4), "kernel_GB_s": round(k_gbs, 1),
            **fractions(k_gbs, peak, read_only),
+           # DRAM bytes per launch from the committed ncu record (None once the kernel's sources change)
+           "traffic": load_traffic("decode", wl.name),
            "call_ms": round(call_ms, 4), "call_GB_s": round(c_gbs, 1),
            "call_frac_of_hbm": round(c_gbs / peak, 4),
            "other_kernels_ms": {r: round(statistics.mean(e["ms"]), 4) for r, e in kern.items() if r != "decode"},
@@ -532,7 +546,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = workloads.config(args.workload)
+    wl = scaled(workloads.config(args.workload), args.scale)
     bt = workloads.generate(wl, seed=wl.seed if wl.seed is not None else args.workload)  # the same batch on every rank
     pipe = Pipeline(sgd, wl, bt, dev)
     stages = algorithmic_bytes(wl, pipe.lengths)
@@ -712,6 +726,7 @@ def run_ours(args, rank, world, local_rank):
             "l2": "flushed between steps (untimed 256 MiB write then 256 MiB read: L2 left clean); inputs > L2",
             "parallelism": f"dp{world} (independent copies, no collective)",
             "launch": launch,
+            **({"length_scale": args.scale} if args.scale != 1.0 else {}),
         },
         "eager_ms_per_step": round(eager_ms, 4),
         "pct_hbm_peak": round(100 * value / world / peak, 2),
@@ -767,7 +782,7 @@ def run_reference(args, rank, world):
     batch)."""
     if rank != 0:
         return None
-    wl = workloads.config(args.workload)
+    wl = scaled(workloads.config(args.workload), args.scale)
     bt = workloads.generate(wl, seed=wl.seed if wl.seed is not None else args.workload)
     cu = bt.cu_seqlens.numpy()
     rows = sorted(((b, h) for h in range(wl.Hkv) for b in range(wl.B)), key=lambda r: int(cu[r[0] + 1] - cu[r[0]]))
