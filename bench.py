@@ -120,6 +120,7 @@ def kernel_role(name):
             mode = args[4] if len(args) > 4 else ""
         return {"0": "decode", "1": "score", "2": "score_quantize"}.get(mode, "decode")
     for key, role in (("quant_global_kernel", "v_codes"), ("topk_cluster_kernel", "topk"), ("plan_kernel", "plan"),
+                      ("plan_fast_kernel", "plan"),
                       ("block_max_kernel", "block_max"), ("quant_k_partition_kernel", "k_codes"),
                       ("quant_amax_kernel", "amax"), ("quant_prep_kernel", "prep"), ("merge_kernel", "merge"),
                       ("decode_generic_kernel", "decode")):

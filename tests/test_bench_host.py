@@ -29,6 +29,7 @@ def test_kernel_roles_from_demangled_names(bench):
     assert r("void sgd::quant_global_kernel<__nv_bfloat16, false>") == "v_codes"
     assert r("void sgd::topk_cluster_kernel<512, 8, 2>") == "topk"
     assert r("sgd::plan_kernel") == "plan" and r("sgd::block_max_kernel") == "block_max"
+    assert r("sgd::plan_fast_kernel(const int *, const int *, int, int)") == "plan"
     assert r("void sgd::decode_generic_kernel<128, float, true, 0>") == "decode"
     # without a demangler the mangled names give the same roles
     assert r("_ZN3sgd17decode_mma_kernelINS_6MmaCfgILi128ELi1ELb0ELb0ELi2ELb0ELb0ELb0EEEEEv14CUtensorMap_stS3_"
