@@ -198,6 +198,13 @@ def test_multi_token_selection_and_plan_reject_bad_args_on_host(sgd):
     assert plan(B=0) == -2 and plan(mode=2) == -8
     assert plan(min_chunk=8) == -8 and plan(min_chunk=24) == -8 and plan(n_req=0) == -8
     assert plan(ws=0x6004) == -4 and plan(nbytes=64) == -5
+    # the workspace bound include/sgd.h states passes the size check for any shape (no device here,
+    # so the call then fails on the device query); a few hundred bytes less does not
+    for B, Hkv, n_req, mode in ((1, 1, 1, 0), (2, 2, 8, 0), (37, 8, 296, 0), (5000, 3, 148, 0), (9, 8, 0, 1)):
+        n = B * Hkv if mode == 1 else n_req
+        bound = 2048 + 4 * (B + 2 * B * Hkv + 3 * n + 6) + 32 * B * Hkv
+        assert plan(B=B, Hkv=Hkv, n_req=max(n_req, 1), mode=mode, nbytes=bound) != -5
+        assert plan(B=B, Hkv=Hkv, n_req=max(n_req, 1), mode=mode, nbytes=bound - 2048) == -5
 
 
 def test_workspace_size_limits(sgd):
