@@ -180,13 +180,17 @@ def n_parts(lengths: Sequence[int], part: int = PART) -> np.ndarray:
     return np.array([(int(L) + part - 1) // part for L in lengths], dtype=np.int64)
 
 
-def quantize_kv(k, v, cu_seqlens, scheme: str, part: int = PART):
+def quantize_kv(k, v, cu_seqlens, scheme: str, part: int = PART, k_scale=None, v_scale=None):
     """Quantise a packed cache k, v [Hkv, T, D] (torch or numpy, bf16/f32 values).
 
     Scheme A: K gets one scale per (KV head, sequence, ``part``-token partition), laid out as
     k_scale [Hkv, sum_b ceil(L_b / part)] with sequence b's partitions starting at
     sum_{b'<b} ceil(L_b' / part); V gets one scale over the whole tensor.
     Scheme B: K and V each get one scale over the whole tensor (k_scale has shape [1]).
+    Calibrated scales ([TD] section 6 names per-tensor static quantisation and credits INT8's
+    small error to calibrated scales): a given ``v_scale`` (and, scheme B, ``k_scale``) replaces
+    that tensor's max|x| / 127; the codes follow the same rule, so values beyond the scale's
+    range saturate at +-127.  Scheme A's K partition scales are computed as always.
     Returns (k_codes int8 [Hkv,T,D], v_codes, k_scale float32, v_scale float32 [1]).
     """
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -197,13 +201,17 @@ def quantize_kv(k, v, cu_seqlens, scheme: str, part: int = PART):
     vc = np.empty((Hkv, T, D), np.int8)
     L = lib()
     # V: one scale over every element of the tensor (both schemes)
-    v_amax = np.float32(0)
-    for h in range(Hkv):
-        v_amax = max(v_amax, amax(v[h]))
-    v_scale = scale_from_amax(v_amax)
+    if v_scale is None:
+        v_amax = np.float32(0)
+        for h in range(Hkv):
+            v_amax = max(v_amax, amax(v[h]))
+        v_scale = scale_from_amax(v_amax)
+    v_scale = np.float32(v_scale)
     for h in range(Hkv):
         vc[h] = quantize(v[h], v_scale)
     if scheme == "A":
+        if k_scale is not None:
+            raise ValueError("scheme A computes its K partition scales")
         parts = n_parts(lengths, part)
         cu_parts = np.concatenate([[0], np.cumsum(parts)])
         k_scale = np.empty((Hkv, int(cu_parts[-1])), np.float32)
@@ -218,10 +226,13 @@ def quantize_kv(k, v, cu_seqlens, scheme: str, part: int = PART):
                 k_scale[h, cu_parts[b]:cu_parts[b + 1]] = sc
                 kc[h, s:e] = codes
     elif scheme == "B":
-        k_amax = np.float32(0)
-        for h in range(Hkv):
-            k_amax = max(k_amax, amax(k[h]))
-        ks = scale_from_amax(k_amax)
+        if k_scale is None:
+            k_amax = np.float32(0)
+            for h in range(Hkv):
+                k_amax = max(k_amax, amax(k[h]))
+            ks = scale_from_amax(k_amax)
+        else:
+            ks = np.float32(k_scale)
         for h in range(Hkv):
             kc[h] = quantize(k[h], ks)
         k_scale = np.array([ks], np.float32)

@@ -16,6 +16,10 @@ import test_oracle_pins as pins
 
 ORACLE_PY = oracle.__file__
 
+
+def pins_golden_dir():
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
 # (name, original text, mutated text)
 MUTANTS = [
     ("query codes: per-row scale taken from the whole tensor",
@@ -38,12 +42,18 @@ MUTANTS = [
     ("block selection: ties prefer the higher block",
      "blk[h, cu_kept[b]:cu_kept[b + 1]] = topk(bs[(b, h)], int(kept[b]))",
      "blk[h, cu_kept[b]:cu_kept[b + 1]] = np.sort(bs[(b, h)].size - 1 - topk(bs[(b, h)][::-1], int(kept[b])))"),
+    ("calibrated quantisation: the given V scale ignored", "    if v_scale is None:\n        v_amax",
+     "    if True:\n        v_amax"),
+    ("calibrated quantisation: scheme B codes K with the V scale", "ks = np.float32(k_scale)",
+     "ks = np.float32(v_scale)"),
     ("block decode: ragged last block not cut at the sequence end",
      "toks = np.concatenate([np.arange(j * block, min((j + 1) * block, L))",
      "toks = np.concatenate([np.arange(j * block, (j + 1) * block)"),
 ]
 
 PIN_CALLS = [
+    lambda: pins.test_calibrated_scales_hand_example(pins_golden_dir()),
+    lambda: pins.test_calibrated_with_the_computed_scales_is_the_dynamic_quantisation(),
     lambda: pins.test_query_quantisation_per_row_and_per_tensor(),
     lambda: pins.test_value_norms_closed_form_and_library(),
     lambda: pins.test_int8_selection_with_exact_codes_is_the_plain_selection(),

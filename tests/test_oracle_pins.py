@@ -285,6 +285,40 @@ def test_scheme_b_equals_scheme_a_with_one_partition():
     assert ks_a.ravel()[0] == ks_b[0] and vs_a[0] == vs_b[0]
 
 
+def test_calibrated_scales_hand_example(golden_dir):
+    c = _load(golden_dir, "quantize_worked_cases.json")["calibrated"]
+    k = np.array(c["k"], np.float32).reshape(1, 1, 8)
+    v = np.array(c["v"], np.float32).reshape(1, 1, 8)
+    cu = np.array([0, 1], np.int64)
+    kc, vc, ks, vs = oracle.quantize_kv(k, v, cu, "A", v_scale=c["A"]["v_scale"])
+    assert vc[0, 0].tolist() == c["A"]["v_codes"] and vs.tolist() == [c["A"]["v_scale"]]
+    # the K partition scales and codes are scheme A's own (one 1-token partition: scale max|k|/127)
+    assert ks.shape == (1, 1) and ks[0, 0] == np.float32(40.0) / np.float32(127.0)
+    assert kc[0, 0, 2] == 127 and kc[0, 0, 5] == 0
+    kc, vc, ks, vs = oracle.quantize_kv(k, v, cu, "B", k_scale=c["B"]["k_scale"], v_scale=c["B"]["v_scale"])
+    assert kc[0, 0].tolist() == c["B"]["k_codes"] and vc[0, 0].tolist() == c["B"]["v_codes"]
+    assert ks.tolist() == [c["B"]["k_scale"]] and vs.tolist() == [c["B"]["v_scale"]]
+
+
+def test_calibrated_with_the_computed_scales_is_the_dynamic_quantisation():
+    bt = _tiny_batch(G=2, D=8, lengths=(70, 64, 3, 129), Hkv=2, dtype="bf16")
+    for scheme in ("A", "B"):
+        kc, vc, ks, vs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+        kw = {"k_scale": ks[0]} if scheme == "B" else {}
+        got = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme, v_scale=vs[0], **kw)
+        for a, b in zip(got, (kc, vc, ks, vs)):
+            assert np.array_equal(a, b)
+    # a calibrated V scale of a quarter of the computed one: codes are 4x (within the rounding) and
+    # saturate where 4x leaves the range
+    kc, vc, ks, vs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A")
+    _, vc4, _, _ = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, "A", v_scale=vs[0] / 4)
+    x = bt.v.float().numpy().astype(np.float64) / np.float64(np.float32(vs[0] / 4))
+    inside = np.abs(x) < 126.5
+    assert np.all(np.abs(vc4[inside].astype(np.int64) - np.rint(x[inside])) <= 1)
+    assert np.all(vc4[x >= 127.5] == 127) and np.all(vc4[x <= -127.5] == -127)
+    assert (np.abs(x) >= 127.5).any()
+
+
 # ---------------------------------------------------------------------------------------------
 # OAM scores and top-K
 # ---------------------------------------------------------------------------------------------
