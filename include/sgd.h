@@ -65,8 +65,20 @@ typedef enum { SGD_F32 = 0, SGD_BF16 = 1, SGD_I8 = 2 } sgd_dtype;
  *   A: one K scale per (KV head, sequence, 64-token partition counted from
  *      the sequence's first token; the last partition takes the remainder),
  *      one V scale for the whole tensor;
- *   B: one K scale and one V scale, each for the whole tensor. */
-typedef enum { SGD_SCHEME_A = 0, SGD_SCHEME_B = 1 } sgd_scheme;
+ *   B: one K scale and one V scale, each for the whole tensor.
+ * The _CALIBRATED forms, for sgd_quantize_kv and sgd_quantize_select only, take
+ * every per-tensor scale as an input instead of computing it: [TD] section 6 names
+ * per-tensor static quantisation and credits INT8's small error to calibrated
+ * scales.  A_CALIBRATED reads the V scale from v_scale (the K partition scales are
+ * still computed); B_CALIBRATED reads k_scale[0] and v_scale[0].  Values beyond
+ * 127.5 * scale saturate to +-127.  The codes they give are scheme A or B codes:
+ * an sgd_kv describing them names SGD_SCHEME_A or SGD_SCHEME_B. */
+typedef enum {
+    SGD_SCHEME_A = 0,
+    SGD_SCHEME_B = 1,
+    SGD_SCHEME_A_CALIBRATED = 2,
+    SGD_SCHEME_B_CALIBRATED = 3
+} sgd_scheme;
 
 #define SGD_PARTITION 64 /* scheme-A partition length in tokens */
 
@@ -87,6 +99,7 @@ typedef enum { SGD_SCHEME_A = 0, SGD_SCHEME_B = 1 } sgd_scheme;
 #define SGD_STATUS_WAIT_TIMEOUT 0x2   /* a bounded pipeline wait gave up */
 #define SGD_STATUS_SIZE_MISMATCH 0x4  /* device lengths disagree with host sizes */
 #define SGD_STATUS_BAD_INDEX 0x8      /* a kept index or block number was outside its sequence */
+#define SGD_STATUS_BAD_SCALE 0x10     /* a calibrated scale was negative or not finite: its codes are 0 */
 
 #define SGD_WS_STATUS_OFFSET 0
 
@@ -126,11 +139,14 @@ typedef struct {
  *   group.  Scheme B: K is one group and V is one group.
  * in       cache to quantise: dtype BF16 or F32 (k_scale/v_scale/scheme ignored)
  * k_codes, v_codes   [Hkv, T, D] int8 outputs
- * k_scale  A: [Hkv, n_parts] (n_parts = sum_b ceil(L_b/64), passed below), B: [1]
- * v_scale  [1]
+ * k_scale  A: [Hkv, n_parts] (n_parts = sum_b ceil(L_b/64), passed below), B: [1]; output,
+ *          except with B_CALIBRATED: input, the calibrated K scale
+ * v_scale  [1]: output, except with A_CALIBRATED / B_CALIBRATED: input, the calibrated V scale
+ *          (a zero scale gives zero codes; a negative or non-finite one sets
+ *          SGD_STATUS_BAD_SCALE in the workspace status and gives zero codes)
  * v_norm   optional [Hkv, T] float32 output (NULL: not written): ||v_t||_2 of every value row,
  *          so that sgd_oam_select can later score the INT8 cache without the original values
- * Codes and scales are bit-exact functions of the input.
+ * Codes and scales are bit-exact functions of the input (and of the calibrated scales).
  */
 int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts,
                     int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm,
@@ -199,7 +215,10 @@ int sgd_oam_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv 
  * cache).  With a BF16 cache and BF16 q (D in {64, 128}) the K and V of every token are read
  * from HBM once for both: the OAM score pass also writes the scheme-A K codes and scales (or
  * takes max|K| for scheme B) and max|V|; a second pass writes the V codes (and the scheme-B K
- * codes), then the top-K runs.  Other dtypes run the two calls one after the other.
+ * codes), then the top-K runs.  With calibrated scales (SGD_SCHEME_A_CALIBRATED /
+ * B_CALIBRATED) no scale waits for a maximum over the tensor, so the score pass writes every
+ * code (and v_norm) itself and the second pass does not run: K and V are read once in all.
+ * Other dtypes run the two calls one after the other.
  * Arguments as in sgd_quantize_kv and sgd_oam_select; kv must be BF16 or F32.
  * Workspace: sgd_workspace_size(SGD_OP_QUANTIZE_SELECT, ...).
  */

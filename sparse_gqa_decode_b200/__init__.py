@@ -31,17 +31,19 @@ __all__ = [
     "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select", "decode_attn",
     "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
-    "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B", "STATUS_BITS",
+    "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B",
+    "SCHEME_A_CALIBRATED", "SCHEME_B_CALIBRATED", "STATUS_BITS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsgd.so")
 
 SGD_F32, SGD_BF16, SGD_I8 = 0, 1, 2
-SCHEME_A, SCHEME_B = 0, 1
+SCHEME_A, SCHEME_B, SCHEME_A_CALIBRATED, SCHEME_B_CALIBRATED = 0, 1, 2, 3
 OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE, OP_QUANTIZE_SELECT = 0, 1, 2, 3
 PARTITION = 64
-STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index"}
+STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index",
+               0x10: "bad calibrated scale"}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python sparse_gqa_decode_b200/build.py` "
@@ -175,22 +177,50 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     return int(st.value)
 
 
+def _quant_scheme(scheme: str, k_scale_in, v_scale_in) -> int:
+    """The C scheme value: A / B, or their calibrated forms when per-tensor scales are given."""
+    if scheme not in ("A", "B"):
+        raise ValueError("scheme must be 'A' or 'B'")
+    if v_scale_in is None:
+        if k_scale_in is not None:
+            raise ValueError("a calibrated K scale goes with a calibrated V scale")
+        return SCHEME_A if scheme == "A" else SCHEME_B
+    if scheme == "A" and k_scale_in is not None:
+        raise ValueError("scheme A computes its K partition scales: no k_scale_in")
+    if scheme == "B" and k_scale_in is None:
+        raise ValueError("scheme B with calibrated scales takes k_scale_in too")
+    return SCHEME_A_CALIBRATED if scheme == "A" else SCHEME_B_CALIBRATED
+
+
+def _scale_buffers(k, sch: int, parts: int, k_scale_in, v_scale_in):
+    """k_scale / v_scale of a quantisation: the calibrated inputs where given, else new outputs."""
+    Hkv = k.shape[0]
+    if sch in (SCHEME_A, SCHEME_A_CALIBRATED):
+        ks = torch.empty((Hkv, parts), dtype=torch.float32, device=k.device)
+    else:
+        ks = k_scale_in if k_scale_in is not None else torch.empty(1, dtype=torch.float32, device=k.device)
+    vs = v_scale_in if v_scale_in is not None else torch.empty(1, dtype=torch.float32, device=k.device)
+    return ks, vs
+
+
 def quantize_kv(k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, scheme: str,
-                lengths: Sequence[int], out=None, workspace=None, stream=None, v_norm=None):
+                lengths: Sequence[int], out=None, workspace=None, stream=None, v_norm=None,
+                k_scale_in=None, v_scale_in=None):
     """INT8 codes and scales of a bf16/f32 cache.  Returns (k_codes, v_codes, k_scale, v_scale, ws).
 
     ``lengths`` are the host copies of the sequence lengths (buffer sizes only).  ``v_norm``: an
     optional float32 [Hkv, T] tensor that receives ||v_t|| (for oam_select over the INT8 cache).
+    ``v_scale_in`` (and, scheme B, ``k_scale_in``): calibrated per-tensor scales, float32 [1] device
+    tensors, used instead of max|x| / 127; they are returned as the scales.
     """
-    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    sch = _quant_scheme(scheme, k_scale_in, v_scale_in)
     Hkv, T, D = k.shape
-    parts = n_parts(lengths) if sch == SCHEME_A else 0
+    parts = n_parts(lengths) if sch in (SCHEME_A, SCHEME_A_CALIBRATED) else 0
     kv = _kv(k, v, cu_seqlens)
     if out is None:
         kc = torch.empty((Hkv, T, D), dtype=torch.int8, device=k.device)
         vc = torch.empty_like(kc)
-        ks = torch.empty((Hkv, parts) if sch == SCHEME_A else (1,), dtype=torch.float32, device=k.device)
-        vs = torch.empty(1, dtype=torch.float32, device=k.device)
+        ks, vs = _scale_buffers(k, sch, parts, k_scale_in, v_scale_in)
     else:
         kc, vc, ks, vs = out
     ws = _workspace(workspace_size(OP_QUANTIZE, kv), k.device, workspace)
@@ -265,19 +295,19 @@ def oam_select_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seql
 
 def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
                     beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
-                    out=None, workspace=None, stream=None, v_norm=None):
+                    out=None, workspace=None, stream=None, v_norm=None, k_scale_in=None, v_scale_in=None):
     """quantize_kv and oam_select of one cache in one call (K and V read once for both).
-    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws); ``v_norm`` as in quantize_kv."""
-    sch = SCHEME_A if scheme == "A" else SCHEME_B
+    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws); ``v_norm``, ``k_scale_in`` and
+    ``v_scale_in`` as in quantize_kv (with calibrated scales one pass writes every code)."""
+    sch = _quant_scheme(scheme, k_scale_in, v_scale_in)
     Hkv, T, D = k.shape
-    parts = n_parts(lengths) if sch == SCHEME_A else 0
+    parts = n_parts(lengths) if sch in (SCHEME_A, SCHEME_A_CALIBRATED) else 0
     Kt = kept_total(lengths, keep_num, keep_den)
     kv = _kv(k, v, cu_seqlens)
     if out is None:
         kc = torch.empty((Hkv, T, D), dtype=torch.int8, device=k.device)
         vc = torch.empty_like(kc)
-        ks = torch.empty((Hkv, parts) if sch == SCHEME_A else (1,), dtype=torch.float32, device=k.device)
-        vs = torch.empty(1, dtype=torch.float32, device=k.device)
+        ks, vs = _scale_buffers(k, sch, parts, k_scale_in, v_scale_in)
         idx = torch.empty((Hkv, Kt), dtype=torch.int32, device=k.device)
         cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
     else:

@@ -362,6 +362,12 @@ int select_impl(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float
                     &hdr->status, s);
     return e == 0 ? SGD_OK : SGD_ERR_CUDA;
 }
+bool quant_scheme_ok(sgd_scheme s) {
+    return s == SGD_SCHEME_A || s == SGD_SCHEME_B || s == SGD_SCHEME_A_CALIBRATED || s == SGD_SCHEME_B_CALIBRATED;
+}
+// the scheme-A forms: K scales per 64-token partition
+bool has_partitions(sgd_scheme s) { return s == SGD_SCHEME_A || s == SGD_SCHEME_A_CALIBRATED; }
+
 }  // namespace
 
 extern "C" {
@@ -495,8 +501,8 @@ int sgd_quantize_kv(const sgd_kv *in, sgd_scheme scheme, int64_t n_parts, int8_t
     if (rc != SGD_OK) return rc;
     if (!k_codes || !v_codes || !k_scale || !v_scale || !workspace) return SGD_ERR_NULL;
     if (in->dtype != SGD_BF16 && in->dtype != SGD_F32) return SGD_ERR_DTYPE;
-    if (scheme != SGD_SCHEME_A && scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
-    if (scheme == SGD_SCHEME_A && (n_parts < in->B || n_parts > in->T / SGD_PARTITION + in->B)) return SGD_ERR_SHAPE;
+    if (!quant_scheme_ok(scheme)) return SGD_ERR_DTYPE;
+    if (has_partitions(scheme) && (n_parts < in->B || n_parts > in->T / SGD_PARTITION + in->B)) return SGD_ERR_SHAPE;
     if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace)) return SGD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
         (reinterpret_cast<uintptr_t>(v_norm) & 3u))
@@ -544,8 +550,8 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     if (G < 1 || G > 16) return SGD_ERR_SHAPE;
     if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
-    if (scheme != SGD_SCHEME_A && scheme != SGD_SCHEME_B) return SGD_ERR_DTYPE;
-    if (scheme == SGD_SCHEME_A && (n_parts < kv->B || n_parts > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
+    if (!quant_scheme_ok(scheme)) return SGD_ERR_DTYPE;
+    if (has_partitions(scheme) && (n_parts < kv->B || n_parts > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
     if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
     if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
     if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
@@ -586,24 +592,34 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     a.M = 1;
     a.D = kv->D;
     a.T = kv->T;
-    a.n_parts = scheme == SGD_SCHEME_A ? n_parts : 0;
+    const bool cal = scheme == SGD_SCHEME_A_CALIBRATED || scheme == SGD_SCHEME_B_CALIBRATED;
+    const sgd_scheme base = has_partitions(scheme) ? SGD_SCHEME_A : SGD_SCHEME_B;
+    a.n_parts = base == SGD_SCHEME_A ? n_parts : 0;
     a.sm_scale = (float)(1.0 / sqrt((double)kv->D));
     a.sm_scale_log2 = (float)(1.4426950408889634 / sqrt((double)kv->D));
     a.beta = beta;
     a.eps = eps;
     a.scores = reinterpret_cast<float *>(ws + L.scores);
-    a.qscheme = scheme;
+    a.qscheme = base;
     a.k_codes = k_codes;
     a.k_scale_out = k_scale;
     a.amax_bits = hdr->amax_bits;
+    if (cal) {  // every code (and norm) in the score pass: no second pass
+        a.cal_v_scale = v_scale;
+        a.cal_k_scale = base == SGD_SCHEME_B ? k_scale : nullptr;
+        a.v_codes_out = v_codes;
+        a.v_norm_out = v_norm;
+    }
     a.plan = pv;
     a.status = &hdr->status;
     apply_test_hooks(a);
     int e = launch_score_quantize(a, n_req, s);
     if (e != 0) return SGD_ERR_CUDA;
-    e = launch_quantize_global(kv->k, kv->v, kv->dtype, kv->Hkv, kv->D, kv->T, scheme, k_codes, v_codes, k_scale,
-                               v_scale, v_norm, hdr, dev->sms, s);
-    if (e != 0) return SGD_ERR_CUDA;
+    if (!cal) {
+        e = launch_quantize_global(kv->k, kv->v, kv->dtype, kv->Hkv, kv->D, kv->T, base, k_codes, v_codes, k_scale,
+                                   v_scale, v_norm, hdr, dev->sms, s);
+        if (e != 0) return SGD_ERR_CUDA;
+    }
     e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
                     &hdr->status, s);
     return e == 0 ? SGD_OK : SGD_ERR_CUDA;

@@ -49,7 +49,7 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
 constexpr int kQuantWarps = 8;  // K-quantising warps of the fused score + quantise pass
 
 template <int D_, int GT_, bool I8_, bool IDX_, int MODE_, bool QI8_ = false, bool CAUSAL_ = false,
-          bool BLK_ = false>
+          bool BLK_ = false, bool CAL_ = false>
 struct MmaCfg {
     static constexpr int D = D_, GT = GT_, NG = 8 * GT_;
     static constexpr bool I8 = I8_, IDX = IDX_;
@@ -57,6 +57,7 @@ struct MmaCfg {
     static constexpr bool CAUSAL = CAUSAL_;  // several query tokens: causal limit per column
     static constexpr bool BLK = BLK_;  // kept 64-token blocks: one TMA box per block, at its start
     static constexpr int MODE = MODE_;  // 0 = decode, 1 = OAM score, 2 = OAM score + K quantise + max|V|
+    static constexpr bool CAL = CAL_;   // mode 2 with calibrated per-tensor scales: every code in the pass
     static constexpr bool KONLY = I8 && MODE == 1;  // scores of an INT8 cache: K tiles only
     static constexpr int NW = 4;        // consumer warps
     static constexpr int SUB = I8 ? 2 : 1;  // 16-token sub-tiles per consumer warp per stage
@@ -92,6 +93,7 @@ struct MmaCfg {
     static_assert(!CAUSAL || MODE == 0, "several query tokens: decode only");
     static_assert(!BLK || (MODE == 0 && !IDX && !CAUSAL && ROWS % kPart == 0), "a tile is whole blocks");
     static_assert(MODE != 2 || ROWS == kPart, "a fused tile is one scheme-A partition");
+    static_assert(!CAL || MODE == 2, "calibrated scales: the fused pass");
 };
 
 // ------------------------------------------------------------------------------------------
@@ -608,10 +610,40 @@ __device__ __forceinline__ void score_subtile_i8(const DecodeArgs &a, uint32_t k
     }
 }
 
+// Codes of NH 16-byte bf16 chunks (8 values each) to NH / 2 16-byte stores at dst (SAT: under a
+// calibrated scale, codes4_sat); s == 0 gives zero codes.
+template <int NH, bool SAT>
+__device__ __forceinline__ void store_code_chunks(int8_t *dst, const uint4 (&cw)[NH], float s, float r, float c) {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < NH; i += 2) {  // 16 codes per 16-byte store
+        float x[8], y[8];
+        Vec<__nv_bfloat16>::unpack(cw[i], x);
+        Vec<__nv_bfloat16>::unpack(cw[i + 1], y);
+        uint4 w;
+        if constexpr (SAT) {
+            w.x = (s != 0.f) ? codes4_sat<true>(x, s, r, c) : 0u;
+            w.y = (s != 0.f) ? codes4_sat<true>(x + 4, s, r, c) : 0u;
+            w.z = (s != 0.f) ? codes4_sat<true>(y, s, r, c) : 0u;
+            w.w = (s != 0.f) ? codes4_sat<true>(y + 4, s, r, c) : 0u;
+        } else {
+            w.x = (s != 0.f) ? codes4<true>(x, s, r) : 0u;
+            w.y = (s != 0.f) ? codes4<true>(x + 4, s, r) : 0u;
+            w.z = (s != 0.f) ? codes4<true>(y, s, r) : 0u;
+            w.w = (s != 0.f) ? codes4<true>(y + 4, s, r) : 0u;
+        }
+        d[i / 2] = w;
+    }
+}
+
 // Mode 2, K-quantising warp qw: rows RW*qw .. RW*qw + RW-1 of every tile (a tile is one scheme-A
 // partition, RW = 64 / NQ).  Scheme A: the tile's max|K| is met across the NQ warps through shared memory,
 // then each warp writes the codes of its rows and warp 0 the partition scale.  Scheme B: only
 // the running max|K|.  Every quantising warp takes every tile.
+// With calibrated per-tensor scales the warps also write the codes of their V rows (and, scheme
+// B, of their K rows) and, if asked, each V row's norm, summed in the order the V-codes pass
+// sums it (per 16-byte chunk in element order, then chunk c with c ^ 8, ^ 4, ^ 2, ^ 1), so the
+// norms are the same bits whichever call writes them.
 template <class C>
 __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *smem, uint64_t *full, uint64_t *empty,
                                                volatile int32_t *abort_flag, float *kmxs,
@@ -628,9 +660,25 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
     static_assert(NH % 2 == 0 && RW * LPR == 32, "quantising lane map");
     const int rho = lane % RW, half = lane / RW;  // lane: row rho of the warp, part `half` of it
     const int vr = RW * qw + rho;
+    auto chunk_at = [&](uint32_t base, int i) {  // chunk half * NH + i of tile row vr (128B swizzle)
+        const int c = half * NH + i, bx = c >> 3, cc = c & 7;
+        return lds128(base + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
+    };
+    constexpr bool cal = C::CAL;
+    float vs = 0.f, ks = 0.f;
+    if constexpr (cal) {
+        const bool report = cta == 0 && qw == 0 && lane == 0;
+        vs = calibrated_scale(a.cal_v_scale, a.status, report);
+        if (a.qscheme == SGD_SCHEME_B) ks = calibrated_scale(a.cal_k_scale, a.status, report);
+    }
+    const float vrc = (vs != 0.f) ? __frcp_rn(vs) : 0.f, vcl = 127.f * vs;
+    const float krc = (ks != 0.f) ? __frcp_rn(ks) : 0.f, kcl = 127.f * ks;
     while (cur.next(row, t0, t1, slot)) {
         const int b = row % a.B, kvh = row / a.B;
-        int8_t *codes_row0 = a.k_codes + ((int64_t)kvh * a.T + cur.ri.seq_start) * C::D + half * (C::D / LPR);
+        const int64_t row0 = (int64_t)kvh * a.T + cur.ri.seq_start;  // cache row of the sequence's token 0
+        int8_t *codes_row0 = a.k_codes + row0 * C::D + half * (C::D / LPR);
+        int8_t *vcodes_row0 = nullptr;
+        if constexpr (cal) vcodes_row0 = a.v_codes_out + row0 * C::D + half * (C::D / LPR);
         float *scale_row0 = a.k_scale_out + (int64_t)kvh * a.n_parts + cur.ri.part0;
         for (int32_t t = t0; t < t1; t += C::ROWS, ++tile_no) {
             const bool ready = mbar_wait(&full[stage], phase, a.status, abort_flag, a.wait_limit);
@@ -641,8 +689,7 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
             uint32_t km2[4] = {0u, 0u, 0u, 0u};  // four independent running maxima
 #pragma unroll
             for (int i = 0; i < NH; ++i) {
-                const int c = half * NH + i, bx = c >> 3, cc = c & 7;
-                kw[i] = lds128(kbase + bx * C::ROWS * 128 + vr * 128 + ((cc ^ (vr & 7)) << 4));
+                kw[i] = chunk_at(kbase, i);
                 km2[0] = bf16x2_absmax(km2[0], kw[i].x);
                 km2[1] = bf16x2_absmax(km2[1], kw[i].y);
                 km2[2] = bf16x2_absmax(km2[2], kw[i].z);
@@ -652,7 +699,11 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
                               fmaxf(bf16x2_fold_max(km2[2]), bf16x2_fold_max(km2[3])));
             if (!vrow) kmx = 0.f;
             if (a.qscheme == SGD_SCHEME_B) {
-                run_kmax = fmaxf(run_kmax, kmx);
+                if constexpr (!cal) {
+                    run_kmax = fmaxf(run_kmax, kmx);
+                } else if (vrow) {  // K codes under the calibrated K scale
+                    store_code_chunks<NH, true>(codes_row0 + (int64_t)j * C::D, kw, ks, krc, kcl);
+                }
             } else {
                 kmx = warp_max(kmx);
                 const int parity = tile_no & 1;
@@ -663,24 +714,38 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
                 for (int w = 0; w < C::NQ; ++w) tm = fmaxf(tm, kmxs[parity * C::NQ + w]);
                 const float sc = __fdiv_rn(tm, 127.f);
                 const float r = (sc != 0.f) ? __frcp_rn(sc) : 0.f;
-                if (vrow) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(codes_row0 + (int64_t)j * C::D);
-#pragma unroll
-#pragma unroll
-                    for (int i = 0; i < NH; i += 2) {  // 16 codes per 16-byte store
-                        float x[8], y[8];
-                        Vec<__nv_bfloat16>::unpack(kw[i], x);
-                        Vec<__nv_bfloat16>::unpack(kw[i + 1], y);
-                        uint4 w;
-                        w.x = (sc != 0.f) ? codes4<true>(x, sc, r) : 0u;
-                        w.y = (sc != 0.f) ? codes4<true>(x + 4, sc, r) : 0u;
-                        w.z = (sc != 0.f) ? codes4<true>(y, sc, r) : 0u;
-                        w.w = (sc != 0.f) ? codes4<true>(y + 4, sc, r) : 0u;
-                        dst[i / 2] = w;
-                    }
-                }
+                if (vrow) store_code_chunks<NH, false>(codes_row0 + (int64_t)j * C::D, kw, sc, r, 0.f);
                 // (the partition count was checked against the host's n_parts before any write)
                 if (qw == 0 && lane == 0 && ready) scale_row0[t / kPart] = sc;
+            }
+            if constexpr (cal) {  // V codes under the calibrated V scale, and the row norms
+                uint4 vw[NH];
+#pragma unroll
+                for (int i = 0; i < NH; ++i) vw[i] = chunk_at(kbase + C::TILE, i);
+                if (vrow) store_code_chunks<NH, true>(vcodes_row0 + (int64_t)j * C::D, vw, vs, vrc, vcl);
+                if (a.v_norm_out) {
+                    float p[NH];  // per-chunk sums of squares, in element order
+#pragma unroll
+                    for (int i = 0; i < NH; ++i) {
+                        float x[8];
+                        Vec<__nv_bfloat16>::unpack(vw[i], x);
+                        float px = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) px = fmaf(x[e], x[e], px);
+                        p[i] = px;
+                    }
+                    // chunk c pairs with c ^ o: on the lane of half ^ (o / NH) for o >= NH, in
+                    // this lane below
+#pragma unroll
+                    for (int o = CPR / 2; o >= NH; o >>= 1)
+#pragma unroll
+                        for (int i = 0; i < NH; ++i) p[i] += __shfl_xor_sync(0xffffffffu, p[i], RW * (o / NH));
+#pragma unroll
+                    for (int o = NH / 2; o; o >>= 1)
+#pragma unroll
+                        for (int i = 0; i < o; ++i) p[i] = p[i] + p[i + o];
+                    if (vrow && half == 0) a.v_norm_out[row0 + j] = sqrtf(p[0]);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
@@ -690,7 +755,7 @@ __device__ __forceinline__ void quant_consumer(const DecodeArgs &a, uint8_t *sme
             }
         }
     }
-    if (a.qscheme == SGD_SCHEME_B) {
+    if (a.qscheme == SGD_SCHEME_B && !cal) {  // (calibrated: no maximum wanted)
         run_kmax = warp_max(run_kmax);
         if (lane == 0) atomicMax(&a.amax_bits[0], __float_as_uint(run_kmax));
     }
@@ -1568,12 +1633,19 @@ int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, 
     }
 }
 
-int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s) {
-    if (n_cta <= 0) return 0;
+template <bool CAL>
+static int launch_score_quantize_cfg(const DecodeArgs &a, int n_cta, cudaStream_t s) {
     const bool g2 = a.G > 8;
     if (a.D == 128)
-        return g2 ? launch_mma<MmaCfg<128, 2, false, false, 2>>(a, n_cta, s) : launch_mma<MmaCfg<128, 1, false, false, 2>>(a, n_cta, s);
-    return g2 ? launch_mma<MmaCfg<64, 2, false, false, 2>>(a, n_cta, s) : launch_mma<MmaCfg<64, 1, false, false, 2>>(a, n_cta, s);
+        return g2 ? launch_mma<MmaCfg<128, 2, false, false, 2, false, false, false, CAL>>(a, n_cta, s)
+                  : launch_mma<MmaCfg<128, 1, false, false, 2, false, false, false, CAL>>(a, n_cta, s);
+    return g2 ? launch_mma<MmaCfg<64, 2, false, false, 2, false, false, false, CAL>>(a, n_cta, s)
+              : launch_mma<MmaCfg<64, 1, false, false, 2, false, false, false, CAL>>(a, n_cta, s);
+}
+
+int launch_score_quantize(const DecodeArgs &a, int n_cta, cudaStream_t s) {
+    if (n_cta <= 0) return 0;
+    return a.cal_v_scale ? launch_score_quantize_cfg<true>(a, n_cta, s) : launch_score_quantize_cfg<false>(a, n_cta, s);
 }
 
 int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s) {

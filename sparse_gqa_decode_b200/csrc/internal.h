@@ -34,6 +34,12 @@ struct DecodeArgs {
     int8_t *k_codes;         // [Hkv, T, D]
     float *k_scale_out;      // [Hkv, n_parts]
     uint32_t *amax_bits;     // [2]: max|K| (scheme B), max|V| as float bits
+    // mode 2 with calibrated per-tensor scales (cal_v_scale non-NULL): the pass also writes the V
+    // codes (and, scheme B, the K codes with cal_k_scale) and, if v_norm_out, every ||v_t||
+    const float *cal_k_scale;
+    const float *cal_v_scale;
+    int8_t *v_codes_out;     // [Hkv, T, D]
+    float *v_norm_out;       // [Hkv, T] or NULL
     PlanView plan;
     float *o_part;           // [slots, M * G, D]
     float *lse_part;         // [slots, M * G]
@@ -82,7 +88,7 @@ int launch_merge(const DecodeArgs &a, float *out, float *lse, cudaStream_t s);
 // vnorm (NULL: not wanted): [Hkv, T] L2 norm of every V row, written by the V-codes pass.
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
                            sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
-                           float *vnorm, const WsHeader *hdr, int sm_count, cudaStream_t s);
+                           float *vnorm, WsHeader *hdr, int sm_count, cudaStream_t s);
 int launch_quantize(const void *k, const void *v, sgd_dtype dt, const int32_t *cu, int B, int Hkv, int D,
                     int64_t T, sgd_scheme scheme, int64_t n_parts, int8_t *kc, int8_t *vc, float *k_scale,
                     float *v_scale, float *vnorm, WsHeader *hdr, int32_t *seq_part0, int sm_count, cudaStream_t s);

@@ -69,10 +69,8 @@ __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
     return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
 }
 
-// OUTLINE: take the rare exact path through an out-of-line call (keeps a large unrolled caller
-// compact; a small grid-stride loop is faster with it inline).
-template <bool OUTLINE = false>
-__device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
+// The fast result of codes4 and whether it stands (no branch).
+__device__ __forceinline__ uint32_t codes4_fast(const float *x, float r, bool &fast) {
     const uint64_t rr = f32x2(r, r), mm = f32x2(12582912.f, 12582912.f);
     uint64_t t01, t23, n01, n23, e01, e23;
     const uint64_t x01 = f32x2(x[0], x[1]), x23 = f32x2(x[2], x[3]);
@@ -84,10 +82,17 @@ __device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e23) : "l"(x23), "l"(rr), "l"(n23));
     const float e[4] = {__uint_as_float((uint32_t)e01), __uint_as_float((uint32_t)(e01 >> 32)),
                         __uint_as_float((uint32_t)e23), __uint_as_float((uint32_t)(e23 >> 32))};
-    uint32_t w = __byte_perm(__byte_perm((uint32_t)t01, (uint32_t)(t01 >> 32), 0x0040),
-                             __byte_perm((uint32_t)t23, (uint32_t)(t23 >> 32), 0x0040), 0x5410);
-    const bool fast = fabsf(e[0]) < 0.4999f && fabsf(e[1]) < 0.4999f && fabsf(e[2]) < 0.4999f &&
-                      fabsf(e[3]) < 0.4999f;
+    fast = fabsf(e[0]) < 0.4999f && fabsf(e[1]) < 0.4999f && fabsf(e[2]) < 0.4999f && fabsf(e[3]) < 0.4999f;
+    return __byte_perm(__byte_perm((uint32_t)t01, (uint32_t)(t01 >> 32), 0x0040),
+                       __byte_perm((uint32_t)t23, (uint32_t)(t23 >> 32), 0x0040), 0x5410);
+}
+
+// OUTLINE: take the rare exact path through an out-of-line call (keeps a large unrolled caller
+// compact; a small grid-stride loop is faster with it inline).
+template <bool OUTLINE = false>
+__device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
+    bool fast;
+    uint32_t w = codes4_fast(x, r, fast);
     if (!fast) {
         if constexpr (OUTLINE) {
             w = codes4_exact(x[0], x[1], x[2], x[3], s, r);
@@ -100,11 +105,37 @@ __device__ __forceinline__ uint32_t codes4(const float *x, float s, float r) {
     return w;
 }
 
-template <int VE>
-__device__ __forceinline__ void store_codes(int8_t *dst, const float (&x)[VE], float s, float r) {
+// Codes of four values under a calibrated scale s, which need not cover them: each value is first
+// clamped to +-c, c = RN(127 * s).  A value inside is unchanged; one at or beyond c has a
+// quotient of at least 127 * (1 - 2^-24), so its code is +-127 before and after the clamp; and
+// |clamped * r| <= 127 * (1 + 2^-24)^2 stays in codes4's range.
+template <bool OUTLINE = false>
+__device__ __forceinline__ uint32_t codes4_sat(const float *x, float s, float r, float c) {
+    float y[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = fminf(fmaxf(x[j], -c), c);
+    return codes4<OUTLINE>(y, s, r);
+}
+
+// A calibrated per-tensor scale as read by every thread: a negative or non-finite value counts as
+// zero (zero codes) and, where `report`, sets SGD_STATUS_BAD_SCALE.
+__device__ __forceinline__ float calibrated_scale(const float *p, int32_t *status, bool report) {
+    const float s = __ldg(p);
+    if (s >= 0.f && s <= 3.402823466e38f) return s;
+    if (report) atomicOr(status, SGD_STATUS_BAD_SCALE);
+    return 0.f;
+}
+
+template <int VE, bool SAT = false>
+__device__ __forceinline__ void store_codes(int8_t *dst, const float (&x)[VE], float s, float r, float c = 0.f) {
     uint32_t w[VE / 4];
 #pragma unroll
-    for (int i = 0; i < VE / 4; ++i) w[i] = (s != 0.f) ? codes4(x + 4 * i, s, r) : 0u;
+    for (int i = 0; i < VE / 4; ++i) {
+        if constexpr (SAT)
+            w[i] = (s != 0.f) ? codes4_sat(x + 4 * i, s, r, c) : 0u;
+        else
+            w[i] = (s != 0.f) ? codes4(x + 4 * i, s, r) : 0u;
+    }
     if constexpr (VE == 8)
         *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
     else

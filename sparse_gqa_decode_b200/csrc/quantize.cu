@@ -165,24 +165,30 @@ constexpr int kGlobalUnroll = 4;  // independent 16-byte loads per thread and te
 // a row's vpr 16-byte vectors sit on vpr consecutive lanes of one warp (vpr divides 32; the
 // grid-stride index keeps warps aligned), so the row's sum of squares is a shuffle tree over
 // them.  Loop bounds are taken per warp so that every lane reaches every shuffle.
-template <typename T, bool NORMS>
+// SAT (calibrated scales): scale0 and scale1 are inputs, read instead of written, and the codes
+// saturate (codes4_sat); otherwise each scale is max|x| / 127 from the header and is written out.
+template <typename T, bool NORMS, bool SAT>
 __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__ x0, int8_t *__restrict__ c0,
                                                            float *scale0, int which0, const T *__restrict__ x1,
                                                            int8_t *__restrict__ c1, float *scale1, int which1,
-                                                           int64_t nvec, const WsHeader *hdr,
+                                                           int64_t nvec, WsHeader *hdr,
                                                            float *__restrict__ vnorm, int vnorm_of, int vpr) {
     constexpr int VE = Vec<T>::VE;
-    const float s0 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which0]), 127.f);
-    const float r0 = (s0 != 0.f) ? __frcp_rn(s0) : 0.f;
-    float s1 = 0.f, r1 = 0.f;
-    if (x1) {
-        s1 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which1]), 127.f);
-        r1 = (s1 != 0.f) ? __frcp_rn(s1) : 0.f;
+    const bool report = blockIdx.x == 0 && threadIdx.x == 0;
+    float s0, s1 = 0.f;
+    if constexpr (SAT) {
+        s0 = calibrated_scale(scale0, &hdr->status, report);
+        if (x1) s1 = calibrated_scale(scale1, &hdr->status, report);
+    } else {
+        s0 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which0]), 127.f);
+        if (x1) s1 = __fdiv_rn(__uint_as_float(hdr->amax_bits[which1]), 127.f);
+        if (report) {
+            *scale0 = s0;
+            if (x1) *scale1 = s1;
+        }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        *scale0 = s0;
-        if (x1) *scale1 = s1;
-    }
+    const float r0 = (s0 != 0.f) ? __frcp_rn(s0) : 0.f, r1 = (s1 != 0.f) ? __frcp_rn(s1) : 0.f;
+    const float cl0 = 127.f * s0, cl1 = 127.f * s1;  // saturation bounds (SAT)
     const int lane = NORMS ? (threadIdx.x & 31) : 0;  // without norms no loop bound is taken per warp
     auto row_norm = [&](const float (&x)[VE], int64_t iv, bool in) {
         float ss = 0.f;
@@ -208,11 +214,11 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
         for (int u = 0; u < kGlobalUnroll; ++u) {
             float x[VE];
             Vec<T>::unpack(w0[u], x);
-            store_codes<VE>(c0 + (i + u * stride) * VE, x, s0, r0);
+            store_codes<VE, SAT>(c0 + (i + u * stride) * VE, x, s0, r0, cl0);
             if (NORMS && vnorm_of == 0) row_norm(x, i + u * stride, true);
             if (x1) {
                 Vec<T>::unpack(w1[u], x);
-                store_codes<VE>(c1 + (i + u * stride) * VE, x, s1, r1);
+                store_codes<VE, SAT>(c1 + (i + u * stride) * VE, x, s1, r1, cl1);
                 if (NORMS && vnorm_of == 1) row_norm(x, i + u * stride, true);
             }
         }
@@ -221,29 +227,43 @@ __global__ void __launch_bounds__(256) quant_global_kernel(const T *__restrict__
         const bool in = i < nvec;
         float x[VE];
         Vec<T>::unpack(in ? __ldcs(p0 + i) : make_uint4(0, 0, 0, 0), x);
-        if (in) store_codes<VE>(c0 + i * VE, x, s0, r0);
+        if (in) store_codes<VE, SAT>(c0 + i * VE, x, s0, r0, cl0);
         if (NORMS && vnorm_of == 0) row_norm(x, i, in);
         if (x1) {
             Vec<T>::unpack(in ? __ldcs(p1 + i) : make_uint4(0, 0, 0, 0), x);
-            if (in) store_codes<VE>(c1 + i * VE, x, s1, r1);
+            if (in) store_codes<VE, SAT>(c1 + i * VE, x, s1, r1, cl1);
             if (NORMS && vnorm_of == 1) row_norm(x, i, in);
         }
     }
 }
 
-// Resident CTAs per SM of quant_global_kernel<T> on the current device (cached per device).
-template <typename T>
-static int global_ctas_per_sm() {
-    static int cache[64] = {0};
+// Resident CTAs per SM of one quant_global_kernel instantiation on the current device (cached
+// per device and instantiation: the variant with norms holds more registers).
+template <typename K>
+static int ctas_per_sm(K kern, int slot) {
+    static int cache[64][8] = {};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 4;
-    if (cache[dev] == 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot >= 8) return 3;
+    if (cache[dev][slot] == 0) {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_global_kernel<T, false>, 256, 0) != cudaSuccess || n < 1)
-            n = 4;
-        cache[dev] = n;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 256, 0) != cudaSuccess || n < 1) n = 3;
+        cache[dev][slot] = n;
     }
-    return cache[dev];
+    return cache[dev][slot];
+}
+
+// One launch of quant_global_kernel over all of x0 (and x1): codes with per-tensor scales, the
+// calibrated (`sat`) or the computed ones, and optionally the norms of one tensor's rows.  One
+// CTA per resident slot: the grid-stride loop then ends in one wave.
+template <typename T>
+static cudaError_t launch_global(bool sat, const T *x0, int8_t *c0, float *scale0, int which0, const T *x1,
+                                 int8_t *c1, float *scale1, int which1, int64_t nvec, WsHeader *hdr, float *vnorm,
+                                 int vnorm_of, int vpr, int sm_count, cudaStream_t s) {
+    auto kern = sat ? (vnorm ? quant_global_kernel<T, true, true> : quant_global_kernel<T, false, true>)
+                    : (vnorm ? quant_global_kernel<T, true, false> : quant_global_kernel<T, false, false>);
+    const int slot = (sizeof(T) == 2 ? 4 : 0) + (sat ? 2 : 0) + (vnorm ? 1 : 0);
+    return launch_k(kern, dim3(sm_count * ctas_per_sm(kern, slot)), dim3(256), 0, s, 1, x0, c0, scale0, which0, x1,
+                    c1, scale1, which1, nvec, hdr, vnorm, vnorm_of, vpr);
 }
 
 template <typename T, int D>
@@ -252,15 +272,17 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
                          float *v_scale, float *vnorm, WsHeader *hdr, int32_t *seq_part0, int sm_count,
                          cudaStream_t s) {
     constexpr int VE = Vec<T>::VE;
+    const bool cal = scheme == SGD_SCHEME_A_CALIBRATED || scheme == SGD_SCHEME_B_CALIBRATED;
+    const bool partitions = scheme == SGD_SCHEME_A || scheme == SGD_SCHEME_A_CALIBRATED;
     const int64_t nvec = (int64_t)Hkv * Ttot * D / VE;
-    cudaError_t e = launch_k(quant_prep_kernel, dim3(1), dim3(1024), 0, s, 1, cu, B, n_parts,
-                               (int)(scheme == SGD_SCHEME_A), seq_part0, hdr);
+    cudaError_t e = launch_k(quant_prep_kernel, dim3(1), dim3(1024), 0, s, 1, cu, B, n_parts, (int)partitions,
+                             seq_part0, hdr);
     if (e != cudaSuccess) return (int)e;
     const int grid_stream = sm_count * 8;
     const T *none = nullptr;
     int8_t *no_codes = nullptr;
     float *no_scale = nullptr;
-    if (scheme == SGD_SCHEME_A) {
+    if (partitions) {
         const int64_t total = (int64_t)Hkv * n_parts;
         const int grid = (int)std::min<int64_t>(total, (int64_t)sm_count * 8);
         if (grid > 0) {
@@ -268,35 +290,35 @@ static int quantize_impl(const T *k, const T *v, const int32_t *cu, int B, int H
                            (const int32_t *)seq_part0, B, Hkv, Ttot, n_parts, kc, k_scale, hdr);
             if (e != cudaSuccess) return (int)e;
         }
-        e = launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v, vc,
-                     v_scale, 1, none, no_codes, no_scale, 0, nvec, (const WsHeader *)hdr, vnorm, 0, D / VE);
+        e = launch_global(cal, v, vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr, vnorm, 0, D / VE, sm_count,
+                          s);
     } else {
-        e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
-        if (e != cudaSuccess) return (int)e;
-        e = launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k, kc,
-                     k_scale, 0, v, vc, v_scale, 1, nvec, (const WsHeader *)hdr, vnorm, 1, D / VE);
+        if (!cal) {  // calibrated scales need no maxima
+            e = launch_k(quant_amax_kernel<T>, dim3(grid_stream), dim3(256), 0, s, 1, k, v, nvec, hdr);
+            if (e != cudaSuccess) return (int)e;
+        }
+        e = launch_global(cal, k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr, vnorm, 1, D / VE, sm_count, s);
     }
     return (int)e;
 }
 
+// The second pass of the fused quantise-and-select (dynamic scales only): the V codes (scheme
+// A) or the K and V codes (scheme B) with the maxima the score pass took.
 template <typename T>
 static int quantize_global_impl(const T *k, const T *v, int Hkv, int D, int64_t Ttot, sgd_scheme scheme, int8_t *kc,
-                                int8_t *vc, float *k_scale, float *v_scale, float *vnorm, const WsHeader *hdr,
+                                int8_t *vc, float *k_scale, float *v_scale, float *vnorm, WsHeader *hdr,
                                 int sm_count, cudaStream_t s) {
     const int64_t nvec = (int64_t)Hkv * Ttot * D / Vec<T>::VE;
-    const T *none = nullptr;
-    int8_t *no_codes = nullptr;
-    float *no_scale = nullptr;
+    const int vpr = D / Vec<T>::VE;
     if (scheme == SGD_SCHEME_A)
-        return (int)launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, v,
-                             vc, v_scale, 1, none, no_codes, no_scale, 0, nvec, hdr, vnorm, 0, D / Vec<T>::VE);
-    return (int)launch_k(vnorm ? quant_global_kernel<T, true> : quant_global_kernel<T, false>, dim3(sm_count * global_ctas_per_sm<T>()), dim3(256), 0, s, 1, k,
-                         kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr, vnorm, 1, D / Vec<T>::VE);
+        return (int)launch_global<T>(false, v, vc, v_scale, 1, nullptr, nullptr, nullptr, 0, nvec, hdr, vnorm, 0,
+                                     vpr, sm_count, s);
+    return (int)launch_global<T>(false, k, kc, k_scale, 0, v, vc, v_scale, 1, nvec, hdr, vnorm, 1, vpr, sm_count, s);
 }
 
 int launch_quantize_global(const void *k, const void *v, sgd_dtype dt, int Hkv, int D, int64_t T,
                            sgd_scheme scheme, int8_t *kc, int8_t *vc, float *k_scale, float *v_scale,
-                           float *vnorm, const WsHeader *hdr, int sm_count, cudaStream_t s) {
+                           float *vnorm, WsHeader *hdr, int sm_count, cudaStream_t s) {
     if (dt == SGD_BF16)
         return quantize_global_impl(static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v),
                                     Hkv, D, T, scheme, kc, vc, k_scale, v_scale, vnorm, hdr, sm_count, s);

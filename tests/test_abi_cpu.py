@@ -127,6 +127,13 @@ def test_quantize_and_select_reject_bad_args_on_host(sgd):
                              None) == -2  # fewer partitions than sequences
     assert L.sgd_quantize_kv(ctypes.byref(kv), 0, 3, p(0x1000), p(0x1000), p(0x2000), p(0x3000), None, p(0x4000), 16,
                              None) == -5  # workspace too small
+    # the calibrated schemes: A_CALIBRATED checks the partitions like A, B_CALIBRATED takes none;
+    # both pass the host checks (no device here: the call then fails on the device query)
+    quant = lambda sch, parts: L.sgd_quantize_kv(ctypes.byref(kv), sch, parts, p(0x1000), p(0x1000), p(0x2000),
+                                                 p(0x3000), None, p(0x4000), 4096, None)
+    assert sgd.SCHEME_A_CALIBRATED == 2 and sgd.SCHEME_B_CALIBRATED == 3
+    assert quant(2, 1) == -2 and quant(4, 3) == -3 and quant(-1, 3) == -3
+    assert quant(2, 3) not in (-1, -2, -3, -4, -5, -8) and quant(3, 0) not in (-1, -2, -3, -4, -5, -8)
     sel = lambda **kw: L.sgd_oam_select(p(0x3000), kw.get("qdt", sgd.SGD_BF16), kw.get("G", 8), ctypes.byref(kv),
                                         kw.get("beta", 1.0), 1e-6, kw.get("num", 1), kw.get("den", 8), p(0x1000),
                                         p(0x2000), kw.get("kt", 20), p(0x4000), 1 << 20, None)
@@ -221,3 +228,13 @@ def test_pipeline_timeout_hook_is_host_state_only(sgd):
     assert sgd.lib.sgd_test_pipeline_timeout(-1, 0) == -8
     assert sgd.lib.sgd_test_pipeline_timeout(4096, 1) == 0
     assert sgd.lib.sgd_test_pipeline_timeout(0, 0) == 0
+
+
+def test_binding_picks_the_calibrated_scheme(sgd):
+    qs = sgd._quant_scheme
+    one = object()  # stands for a device scale tensor (only its presence matters here)
+    assert qs("A", None, None) == sgd.SCHEME_A and qs("B", None, None) == sgd.SCHEME_B
+    assert qs("A", None, one) == sgd.SCHEME_A_CALIBRATED and qs("B", one, one) == sgd.SCHEME_B_CALIBRATED
+    for bad in (("A", one, one), ("B", None, one), ("A", one, None), ("C", None, None)):
+        with pytest.raises(ValueError):
+            qs(*bad)

@@ -280,6 +280,42 @@ def test_fused_quantize_select_full_size(sgd, n, scheme):
     compare_rows(out, lse, *ref, rows, wl.G)
 
 
+@pytest.mark.parametrize("n,scheme", [(5, "A"), (4, "B")])
+def test_fused_quantize_select_calibrated_full_size(sgd, n, scheme):
+    """sgd_quantize_select with calibrated per-tensor scales at full size, where one pass writes
+    every code: the scales are 1/4 of the computed ones (the largest values saturate).  Every code
+    and scale bit-exact against the oracle with the same scales; the value norms and every kept
+    set the same bits as the call with computed scales."""
+    wl = workloads.config(n)
+    bt = workloads.generate(wl)
+    q, k, v, cu = (t.cuda() for t in (bt.q, bt.k, bt.v, bt.cu_seqlens))
+    dyn_quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    k_cal = np.float32(dyn_quant[2].ravel()[0] * np.float32(0.25)) if scheme == "B" else None
+    v_cal = np.float32(dyn_quant[3][0] * np.float32(0.25))
+    del dyn_quant
+    cal = dict(v_scale_in=torch.tensor([float(v_cal)], dtype=torch.float32, device="cuda"))
+    if scheme == "B":
+        cal["k_scale_in"] = torch.tensor([float(k_cal)], dtype=torch.float32, device="cuda")
+    vn = torch.empty(k.shape[:2], dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, idx, cu_kept, wsq = sgd.quantize_select(q, k, v, cu, wl.G, wl.beta, wl.eps, wl.keep_num,
+                                                            wl.keep_den, scheme, bt.lengths, v_norm=vn, **cal)
+    assert sgd.workspace_status(wsq) == 0
+    vn_dyn = torch.empty_like(vn)
+    dyn = sgd.quantize_select(q, k, v, cu, wl.G, wl.beta, wl.eps, wl.keep_num, wl.keep_den, scheme, bt.lengths,
+                              v_norm=vn_dyn)
+    assert torch.equal(idx, dyn[4]) and torch.equal(cu_kept, dyn[5]) and torch.equal(vn, vn_dyn)
+    del dyn, k, v
+    quant = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme, k_scale=k_cal, v_scale=v_cal)
+    assert np.array_equal(ks.cpu().numpy().reshape(quant[2].shape), quant[2])
+    assert np.array_equal(vs.cpu().numpy(), quant[3])
+    saturated = 0
+    for h in range(wl.Hkv):
+        assert np.array_equal(kc[h].cpu().numpy(), quant[0][h]), h
+        assert np.array_equal(vc[h].cpu().numpy(), quant[1][h]), h
+        saturated += int((np.abs(quant[1][h].astype(np.int32)) == 127).sum())
+    assert saturated > 0
+
+
 def test_config14_ragged_int8_decode(sgd):
     """The ragged INT8 batch (16 log-uniform lengths in [512, 128K] over the scheme-A cache) in the
     bench's launch configuration: every code and scale bit-exact, sampled rows (shortest and longest

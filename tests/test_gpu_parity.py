@@ -489,6 +489,89 @@ def test_quantize_select_equals_separate_calls(sgd, scheme, G, D, dtype):
 
 
 # ---------------------------------------------------------------------------------------------
+# calibrated per-tensor scales ([TD] section 6, static quantisation): the given scale replaces
+# max|x| / 127 and values beyond its range saturate; scales are fractions of the oracle's own
+# computed ones, so frac < 1 makes the largest values saturate
+# ---------------------------------------------------------------------------------------------
+def _calibrated(bt, scheme, frac):
+    _, _, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    k_cal = np.float32(rks[0] * np.float32(frac)) if scheme == "B" else None
+    return k_cal, np.float32(rvs[0] * np.float32(frac))
+
+
+def _on_device(x):
+    return None if x is None else torch.tensor([float(x)], dtype=torch.float32, device="cuda")
+
+
+@pytest.mark.parametrize("frac", [1.0, 0.375])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("bf16", 64), ("f32", 128)])
+@pytest.mark.parametrize("scheme", ["A", "B"])
+def test_quantize_calibrated_bit_exact(sgd, scheme, dtype, D, frac):
+    bt = make((1, 63, 64, 65, 700, 4099), G=8, D=D, Hkv=3, dtype=dtype, dist="outlier", seed=131 + D)
+    q, k, v, cu = dev(bt)
+    T = int(bt.cu_seqlens[-1])
+    k_cal, v_cal = _calibrated(bt, scheme, frac)
+    vn = torch.empty((3, T), dtype=torch.float32, device="cuda")
+    kc, vc, ks, vs, ws = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn, k_scale_in=_on_device(k_cal),
+                                         v_scale_in=_on_device(v_cal))
+    check_status(sgd, ws)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme, k_scale=k_cal, v_scale=v_cal)
+    assert np.array_equal(kc.cpu().numpy(), rkc) and np.array_equal(vc.cpu().numpy(), rvc)
+    assert np.array_equal(ks.cpu().numpy().reshape(rks.shape), rks) and vs.cpu().numpy()[0] == rvs[0]
+    if frac < 1:
+        assert (np.abs(rvc.astype(np.int32)) == 127).sum() > 10  # saturation exercised
+    vn_dyn = torch.empty_like(vn)
+    sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn_dyn)
+    assert torch.equal(vn, vn_dyn)
+
+
+@pytest.mark.parametrize("G,D,dtype", [(8, 128, "bf16"), (16, 128, "bf16"), (4, 64, "bf16"), (8, 128, "f32")])
+@pytest.mark.parametrize("scheme", ["A", "B"])
+def test_quantize_select_calibrated(sgd, scheme, G, D, dtype):
+    bt = make((1, 63, 64, 65, 700, 4099), G=G, D=D, Hkv=3, dtype=dtype, dist="outlier", seed=141 + G + D)
+    s0 = int(bt.cu_seqlens[5])  # scheme A: exact rounding ties in one K partition (scale 1)
+    bt.k[2, s0 + 64:s0 + 128] = 0
+    bt.k[2, s0 + 64:s0 + 80, :6] = torch.tensor([2.5, 3.5, -2.5, 126.5, 127.0, -0.5]).to(bt.k.dtype)
+    q, k, v, cu = dev(bt)
+    if dtype == "f32":
+        q = q.float()
+    T = int(bt.cu_seqlens[-1])
+    k_cal, v_cal = _calibrated(bt, scheme, 0.5)
+    cal = dict(k_scale_in=_on_device(k_cal), v_scale_in=_on_device(v_cal))
+    vn = torch.empty((3, T), dtype=torch.float32, device="cuda")
+    fused = sgd.quantize_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths, v_norm=vn, **cal)
+    check_status(sgd, fused[6])
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme, k_scale=k_cal, v_scale=v_cal)
+    assert np.array_equal(fused[0].cpu().numpy(), rkc) and np.array_equal(fused[1].cpu().numpy(), rvc)
+    assert np.array_equal(fused[2].cpu().numpy().reshape(rks.shape), rks)
+    assert fused[3].cpu().numpy()[0] == rvs[0]
+    if scheme == "A":
+        assert fused[0][2, s0 + 64, :6].tolist() == [2, 4, -2, 126, 127, 0]
+    # the separate calibrated call gives the same bits; the kept sets and norms are the dynamic call's
+    sep = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, **cal)
+    assert torch.equal(fused[0], sep[0]) and torch.equal(fused[1], sep[1]) and torch.equal(fused[2], sep[2])
+    vn_dyn = torch.empty_like(vn)
+    dyn = sgd.quantize_select(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths, v_norm=vn_dyn)
+    assert torch.equal(fused[4], dyn[4]) and torch.equal(fused[5], dyn[5]) and torch.equal(vn, vn_dyn)
+    ref_idx, ref_cu, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 8)
+    check_selection(fused[4], fused[5].cpu(), ref_idx, ref_cu, scores, bt.wl.B, 3)
+
+
+@pytest.mark.parametrize("call", ["quantize_kv", "quantize_select"])
+def test_calibrated_scale_that_is_not_a_scale(sgd, call):
+    bt = make((65, 700), G=8, D=128, Hkv=2, dist="outlier", seed=151)
+    q, k, v, cu = dev(bt)
+    for bad, status in ((-1.0, 0x10), (float("nan"), 0x10), (float("inf"), 0x10), (0.0, 0)):
+        if call == "quantize_kv":
+            kc, vc, ks, vs, ws = sgd.quantize_kv(k, v, cu, "A", bt.lengths, v_scale_in=_on_device(bad))
+        else:
+            kc, vc, ks, vs, _, _, ws = sgd.quantize_select(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, "A", bt.lengths,
+                                                           v_scale_in=_on_device(bad))
+        assert sgd.workspace_status(ws) == status, bad
+        assert not vc.any() and kc.any()  # V codes zero, K codes (own partition scales) written
+
+
+# ---------------------------------------------------------------------------------------------
 # batches of many short sequences: hundreds of rows per CTA range, both schedules, the whole path
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("B", [256, 257, 300, 7000])

@@ -68,6 +68,7 @@ class Workload:
     seed: Optional[int] = None  # the draw's seed when it is not the workload's number
     M: int = 1  # query tokens per sequence and step (speculative decode: 1 + draft tokens)
     blocks: bool = False  # OAM keeps whole 64-token blocks (ranked by their best token)
+    calibrated: bool = False  # the per-tensor scales are given (calibrated once) instead of computed
 
     @property
     def Hq(self) -> int:
@@ -118,11 +119,14 @@ CONFIGS = {
     # the lengths are the first draw) over workload 4's INT8 scheme-A cache distribution
     14: Workload("ragged_int8A_B16_L512-128K", B=16, Hkv=8, G=8, D=128, kv_dtype="bf16", dist="outlier",
                  length_range=(512, 131072), scheme="A", seed=3),
+    # workload 5 (its seed: the same batch) with the V scale calibrated: one pass writes every code
+    15: Workload("oam_int8A_calibrated_B4_L32K-128K", B=4, Hkv=8, G=8, D=128, kv_dtype="bf16",
+                 dist="outlier", length_range=(32768, 131072), scheme="A", oam=True, calibrated=True, seed=5),
 }
 
 
 def config(n: int, **overrides) -> Workload:
-    """Workload ``n`` (1..14), optionally with fields replaced (e.g. shorter lengths for tests)."""
+    """Workload ``n`` (1..15), optionally with fields replaced (e.g. shorter lengths for tests)."""
     return CONFIGS[n].with_(**overrides) if overrides else CONFIGS[n]
 
 
