@@ -616,7 +616,8 @@ def calibrated_record(sgd, dev, K, W, flush_l2, peak, read_only, world, ref=None
         kb = kernel_bytes(wl, pipe.lengths, role) if len(e["ms"]) == K else None
         if kb is not None:
             gbs = kb / (statistics.mean(e["ms"]) / 1e3) / 1e9
-            kernels[role].update({"algorithmic_bytes": kb, "GB_s": round(gbs, 1), **fractions(gbs, peak, read_only)})
+            kernels[role].update({"algorithmic_bytes": kb, "GB_s": round(gbs, 1), **fractions(gbs, peak, read_only),
+                                  "traffic": load_traffic(role, wl.name)})
     gbs = world * step_bytes / (ms / 1e3) / 1e9
     rec = {"workload": wl.name, "scheme": wl.scheme + " with the V scale calibrated",
            "step": "sgd_quantize_select with a calibrated V scale (one pass: score, K codes and scales, V codes) "
