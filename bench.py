@@ -574,6 +574,66 @@ def capture_step(pipe, dev):
     return graph, launch
 
 
+def kept_rows(idx, cu_kept, cu_seqlens, T):
+    """Cache row numbers (kvh * T + token) of every kept token: the rows a kept-set decode reads
+    from the K codes and from the V codes.  idx [Hkv, Kt] (positions within their sequence),
+    cu_kept / cu_seqlens [B+1]."""
+    Hkv, Kt = idx.shape
+    col = torch.arange(Kt, device=idx.device, dtype=torch.int64)
+    seq = torch.searchsorted(cu_kept.to(torch.int64), col, right=True) - 1  # sequence of each kept column
+    start = cu_seqlens.to(torch.int64)[seq]
+    head = torch.arange(Hkv, device=idx.device, dtype=torch.int64)[:, None] * T
+    return (head + start[None, :] + idx.to(torch.int64)).to(torch.int32).reshape(-1)
+
+
+def gather_ceiling(sgd, pipe, flush_l2, reps=10):
+    """The scattered-row read ceiling for the step's kept-set decode: sgd_gather_read over the same
+    K and V code rows, L2 flushed before each call, best of `reps` (CUDA events)."""
+    wl = pipe.wl
+    if wl.select_on_codes:
+        kc, vc, (idx, cu_kept) = pipe.kc, pipe.vc, pipe.sel_out
+    else:
+        kc, vc, idx, cu_kept = pipe.qout[0], pipe.qout[1], pipe.qout[4], pipe.qout[5]
+    rows = kept_rows(idx, cu_kept, pipe.cu, kc.shape[1])
+    dense = torch.arange(rows.numel(), dtype=torch.int32, device=rows.device)  # control: the same count, contiguous
+    row_bytes = kc.shape[2] * kc.element_size()
+
+    def best_ms(r):
+        sgd.gather_read(kc, r, row_bytes, b=vc)  # checked once, untimed
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i, (a, b) in enumerate(ev):
+            flush_l2(i)
+            a.record()
+            sgd.gather_read(kc, r, row_bytes, b=vc, check=False)
+            b.record()
+        torch.cuda.synchronize()
+        return min(a.elapsed_time(b) for a, b in ev)
+
+    ms, ms_dense = best_ms(rows), best_ms(dense)
+    nbytes = 2 * rows.numel() * row_bytes
+    # second control: the vector stream (sgd_stream_read, no indices) over as many bytes of the codes
+    flat = kc.reshape(-1)[: nbytes // 16 * 16]
+    sink = torch.zeros(1, dtype=torch.int64, device=kc.device)
+    status = torch.zeros(1, dtype=torch.int32, device=kc.device)
+    sgd.stream_read(flat, 0, sink, status)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for i, (a, b) in enumerate(ev):
+        flush_l2(i)
+        a.record()
+        sgd.stream_read(flat, 0, sink, status)
+        b.record()
+    torch.cuda.synchronize()
+    ms_stream = min(a.elapsed_time(b) for a, b in ev)
+    return {"GB_s": round(nbytes / (ms / 1e3) / 1e9, 1), "bytes": nbytes, "rows": 2 * rows.numel(),
+            "row_bytes": row_bytes, "ms": round(ms, 4),
+            "dense_control_GB_s": round(nbytes / (ms_dense / 1e3) / 1e9, 1), "dense_control_ms": round(ms_dense, 4),
+            "stream_control_GB_s": round(flat.numel() / (ms_stream / 1e3) / 1e9, 1),
+            "stream_control_ms": round(ms_stream, 4),
+            "how": "sgd_gather_read over the kept tokens' K and V code rows (16-byte loads, indices of each batch "
+                   "first); controls: as many rows from the start of each tensor, contiguous, and the vector stream "
+                   f"of sgd_stream_read over as many bytes; L2 flushed before each call, best of {reps}"}
+
+
 def calibrated_record(sgd, dev, K, W, flush_l2, peak, read_only, world, ref=None):
     """The headline step with calibrated per-tensor scales (workload 15: workload 5's batch, its V
     scale calibrated once, untimed, from the same cache, so every code equals the computed-scale
@@ -750,6 +810,11 @@ def run_ours(args, rank, world, local_rank):
         if args.scale == 1.0 and not wl.calibrated:
             calibrated = calibrated_record(sgd, dev, K, args.warmup, flush_l2, peak, ro["GB_s"], world, ref=pipe)
     ro_gbs = ro["GB_s"] if ro else None
+    # the scattered-row ceiling of the kept-set decode (INT8 codes of kept tokens)
+    gather = None
+    if wl.oam and wl.scheme and not wl.blocks and wl.M == 1 and args.scale == 1.0:
+        gather = gather_ceiling(sgd, pipe, flush_l2)
+        gather["GB_s"] = round(-reduce_max(-gather["GB_s"], dev, world), 1)  # the slowest rank's
 
     if rank != 0:
         return None
@@ -766,6 +831,8 @@ def run_ours(args, rank, world, local_rank):
         if kb is not None:
             gbs = kb / (statistics.mean(ent["ms"]) / 1e3) / 1e9
             kern_report[role].update({"algorithmic_bytes": kb, "GB_s": round(gbs, 1), **fractions(gbs, peak, ro_gbs)})
+    if gather and "GB_s" in kern_report.get("decode", {}):
+        kern_report["decode"]["frac_of_gather_ceiling"] = round(kern_report["decode"]["GB_s"] / gather["GB_s"], 4)
     dom_k = max(kern_report, key=lambda r: kern_report[r]["ms_per_step"]) if kern_report else None
     kernels = {"quantize_select": "sgd_quantize_select (plan + fused OAM score/K quantise + V codes + top-K)",
                "quantize": "sgd_quantize_kv (prep + K-partition + V kernels)",
@@ -835,6 +902,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": (sum(e["per_step"] for e in per_kernel.values()) or pipe.launches_per_step()) * K,
         "clocks": clk,
         "read_only": ro,
+        "gather_ceiling": gather,
         "nominal_hbm_GB_s": NOMINAL_HBM_GBS,
         # spec bar: the 128K INT8 split-KV decode at >= 0.70 of measured HBM, dense and ragged
         "north_star": north or None,

@@ -383,6 +383,22 @@ int sgd_stream_read(const void *buf, size_t bytes, int method, unsigned long lon
                     void *stream);
 
 /*
+ * sgd_gather_read -- measurement aid: the ceiling of reading scattered rows, as a decode over a
+ * kept set does (one K row and one V row of codes per kept token).  For every i < n_rows reads
+ * the row_bytes bytes at a + rows[i] * row_bytes and, if b is not NULL, at b + rows[i] *
+ * row_bytes, each exactly once, and XORs them, folded to 32-bit words, into *sink (device,
+ * 8-byte aligned).  16-byte loads from every thread; the indices of a batch of eight loads
+ * are read before its rows.
+ * a, b      device, 16-byte aligned (b may be NULL)
+ * row_bytes a power of two in [16, 4096]
+ * rows      device int32 [n_rows], row numbers (any order, repeats allowed; the caller keeps them
+ *           inside the buffers: they are not checked)
+ * Time it with events around the call on `stream`; the pages have no counterpart.
+ */
+int sgd_gather_read(const void *a, const void *b, int64_t row_bytes, const int32_t *rows, int64_t n_rows,
+                    unsigned long long *sink, void *stream);
+
+/*
  * sgd_test_pipeline_timeout -- test aid for the bounded pipeline waits (failure detection).
  * Every wait of the decode and score kernels on their shared-memory pipeline is bounded: when
  * it runs out, the kernel sets SGD_STATUS_WAIT_TIMEOUT in the workspace status word, each CTA

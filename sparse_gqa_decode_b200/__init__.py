@@ -31,7 +31,7 @@ __all__ = [
     "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select", "decode_attn",
     "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
-    "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B",
+    "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "gather_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B",
     "SCHEME_A_CALIBRATED", "SCHEME_B_CALIBRATED", "STATUS_BITS",
 ]
 
@@ -90,6 +90,7 @@ lib.sgd_decode_attn_blocks.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i
                                        _vp]
 lib.sgd_test_pipeline_timeout.argtypes = [_i64, _i32]
 lib.sgd_stream_read.argtypes = [_vp, _sz, _i32, _vp, _vp, _vp]
+lib.sgd_gather_read.argtypes = [_vp, _vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, _vp]
 lib.sgd_kernel_timing_start.argtypes = [_i32]
 lib.sgd_kernel_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(ctypes.c_int32)]
 lib.sgd_kernel_timing_name.argtypes = [_i32]
@@ -424,6 +425,24 @@ def stream_read(buf: torch.Tensor, method: int = 0, sink=None, status=None, stre
     _check(lib.sgd_stream_read(_ptr(buf), nbytes, int(method), _ptr(sink), _ptr(status), _stream(stream)),
            "sgd_stream_read")
     return sink, status
+
+
+def gather_read(a: torch.Tensor, rows: torch.Tensor, row_bytes: int, b=None, sink=None, stream=None,
+                check: bool = True):
+    """Measurement aid: read rows ``rows`` (int32 row numbers) of ``row_bytes`` bytes from ``a``
+    (and ``b``) once, XOR-folded into ``sink`` ([1] int64).  ``check`` first verifies on the host
+    that every row lies inside the tensors (a synchronising reduction: leave it to an untimed
+    first call).  Returns sink."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int64, device=a.device)
+    if check and rows.numel():
+        lo, hi = int(rows.min()), int(rows.max())
+        for t in (a, b):
+            if t is not None and (lo < 0 or (hi + 1) * row_bytes > t.numel() * t.element_size()):
+                raise ValueError("a row lies outside the tensor")
+    _check(lib.sgd_gather_read(_ptr(a), _ptr(b), int(row_bytes), _ptr(rows), rows.numel(), _ptr(sink),
+                               _stream(stream)), "sgd_gather_read")
+    return sink
 
 
 def test_pipeline_timeout(polls: int, idle_producer: bool) -> None:

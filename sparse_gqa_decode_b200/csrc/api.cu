@@ -388,6 +388,22 @@ int sgd_stream_read(const void *buf, size_t bytes, int method, unsigned long lon
                                                                                                   : SGD_ERR_CUDA;
 }
 
+int sgd_gather_read(const void *a, const void *b, int64_t row_bytes, const int32_t *rows, int64_t n_rows,
+                    unsigned long long *sink, void *stream) {
+    if (!a || !rows || !sink) return SGD_ERR_NULL;
+    if (row_bytes < 16 || row_bytes > 4096 || (row_bytes & (row_bytes - 1)) != 0 || n_rows < 1 ||
+        n_rows >= (int64_t(1) << 40))
+        return SGD_ERR_SHAPE;
+    if (!aligned16(a) || (b && !aligned16(b)) || (reinterpret_cast<uintptr_t>(rows) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sink) & 7u))
+        return SGD_ERR_ALIGN;
+    DevInfo *dev;
+    int rc = current_device(&dev);
+    if (rc != SGD_OK) return rc;
+    return launch_gather_read(a, b, row_bytes, rows, n_rows, sink, dev->sms, as_stream(stream)) == 0 ? SGD_OK
+                                                                                                     : SGD_ERR_CUDA;
+}
+
 int sgd_test_pipeline_timeout(int64_t polls, int idle_producer) {
     if (polls < 0) return SGD_ERR_ARG;
     g_hooks.wait_limit = (long long)polls;

@@ -106,5 +106,8 @@ int launch_block_max(const float *scores, const int32_t *cu_seq, const int32_t *
 // memory), every byte XOR-folded into *sink.
 int launch_stream_read(const void *buf, size_t bytes, int method, unsigned long long *sink, int32_t *status,
                        int sm_count, cudaStream_t s);
+// Scattered-row read (sgd_gather_read): n_rows rows of row_bytes at a (and b) by row index.
+int launch_gather_read(const void *a, const void *b, int64_t row_bytes, const int32_t *rows, int64_t n_rows,
+                       unsigned long long *sink, int sm_count, cudaStream_t s);
 
 }  // namespace sgd

@@ -10,6 +10,10 @@
 //             (cp.async.bulk) into a ring of shared-memory stages; each landed chunk is folded
 //             into the word by the CTA's warp before the stage is refilled.
 // Each CTA XORs its word into sink[0].
+//
+// sgd_gather_read, the same measurement for scattered rows: the rows a kept-token decode reads
+// (one K row and one V row of codes per kept token), by a row index, 16-byte loads from every
+// thread with the indices of a batch loaded before its rows.
 #include "internal.h"
 
 namespace sgd {
@@ -107,6 +111,64 @@ __global__ void __launch_bounds__(32) stream_bulk_kernel(const uint8_t *__restri
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0 && acc) atomicXor(sink, (unsigned long long)acc);
+}
+
+constexpr int kGatherUnroll = 8;
+
+// Item i of the gather: chunk c (16 bytes) of tensor t (0: a, 1: b) of listed row j, with
+// i = (j * nt + t) * C + c, so consecutive threads read consecutive chunks of one row.  C = 2^lc
+// chunks per row and nt = 2^lt tensors, so the split is shifts and masks.
+__global__ void __launch_bounds__(512) gather_read_kernel(const uint8_t *__restrict__ a, const uint8_t *__restrict__ b,
+                                                          int64_t row_bytes, const int32_t *__restrict__ rows,
+                                                          int64_t n_items, int lc, int lt, unsigned long long *sink) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    uint32_t acc = 0u;
+    for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < n_items; i0 += kGatherUnroll * stride) {
+        int32_t r[kGatherUnroll];
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u) {  // every index of the batch first
+            const int64_t i = i0 + u * stride;
+            r[u] = (i < n_items) ? __ldg(rows + (i >> (lc + lt))) : 0;
+        }
+        uint4 w[kGatherUnroll];
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u) {
+            const int64_t i = i0 + u * stride;
+            w[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < n_items) {
+                const int c = (int)(i & ((1 << lc) - 1)), t = (int)((i >> lc) & ((1 << lt) - 1));
+                const uint8_t *base = t ? b : a;
+                w[u] = __ldcs(reinterpret_cast<const uint4 *>(base + (int64_t)r[u] * row_bytes) + c);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u) acc ^= w[u].x ^ w[u].y ^ w[u].z ^ w[u].w;
+    }
+    // one atomic per CTA (a small read must not wait on thousands of same-address atomics)
+    __shared__ uint32_t part[16];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t x = 0u;
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) x ^= part[k];
+        if (x) atomicXor(sink, (unsigned long long)x);
+    }
+}
+
+int launch_gather_read(const void *a, const void *b, int64_t row_bytes, const int32_t *rows, int64_t n_rows,
+                       unsigned long long *sink, int sm_count, cudaStream_t s) {
+    int per = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, gather_read_kernel, 512, 0) != cudaSuccess || per < 1)
+        per = 2;
+    const int lt = b ? 1 : 0;
+    int lc = 0;
+    while ((int64_t(16) << lc) < row_bytes) ++lc;  // row_bytes = 16 * 2^lc (checked by the caller)
+    const int64_t n_items = n_rows << (lc + lt);
+    return (int)launch_k(gather_read_kernel, dim3(sm_count * per), dim3(512), 0, s, 1,
+                         static_cast<const uint8_t *>(a), static_cast<const uint8_t *>(b), row_bytes, rows, n_items,
+                         lc, lt, sink);
 }
 
 int launch_stream_read(const void *buf, size_t bytes, int method, unsigned long long *sink, int32_t *status,

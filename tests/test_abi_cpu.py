@@ -238,3 +238,14 @@ def test_binding_picks_the_calibrated_scheme(sgd):
     for bad in (("A", one, one), ("B", None, one), ("A", one, None), ("C", None, None)):
         with pytest.raises(ValueError):
             qs(*bad)
+
+
+def test_gather_read_rejects_bad_args_on_host(sgd):
+    L = sgd.lib
+    p = ctypes.c_void_p
+    g = lambda a=0x1000, b=0x2000, rb=128, rows=0x3000, n=10, sink=0x4000: L.sgd_gather_read(
+        p(a) if a else None, p(b) if b else None, rb, p(rows) if rows else None, n, p(sink) if sink else None, None)
+    assert g(a=0) == -1 and g(rows=0) == -1 and g(sink=0) == -1
+    assert g(rb=0) == -2 and g(rb=24) == -2 and g(rb=48) == -2 and g(rb=8192) == -2 and g(n=0) == -2
+    assert g(a=0x1008) == -4 and g(b=0x2008) == -4 and g(rows=0x3002) == -4 and g(sink=0x4004) == -4
+    assert g(b=0) not in (-1, -2, -4)  # b is optional; no device here, so the call fails later

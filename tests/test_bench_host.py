@@ -138,3 +138,24 @@ def test_cpu_baseline_counts_the_same_rows_on_one_or_several_threads(bench):
     tokens = int(bt.lengths.sum()) * wl.Hkv
     for s in (s1, s4):
         assert s.startswith(f"4 (sequence, KV head) rows of the workload, shortest first, {tokens} tokens")
+
+
+def test_kept_rows_are_the_cache_rows_of_the_kept_tokens(bench):
+    # the rows the gather ceiling reads: kvh * T + cu_seqlens[b] + idx, against a plain loop
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(7)
+    lengths = [5, 1, 17, 9]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    kept = [max(1, (L + 3) // 4) for L in lengths]
+    cu_kept = np.concatenate([[0], np.cumsum(kept)]).astype(np.int32)
+    Hkv, T, Kt = 3, int(cu[-1]), int(cu_kept[-1])
+    idx = np.zeros((Hkv, Kt), np.int32)
+    for h in range(Hkv):
+        for b, L in enumerate(lengths):
+            idx[h, cu_kept[b]:cu_kept[b + 1]] = np.sort(rng.choice(L, kept[b], replace=False))
+    rows = bench.kept_rows(torch.from_numpy(idx), torch.from_numpy(cu_kept), torch.from_numpy(cu), T).numpy()
+    ref = [h * T + cu[b] + idx[h, j] for h in range(Hkv) for b in range(len(lengths))
+           for j in range(cu_kept[b], cu_kept[b + 1])]
+    assert rows.dtype == np.int32 and rows.tolist() == ref
+    assert rows.min() >= 0 and rows.max() < Hkv * T

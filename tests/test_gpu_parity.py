@@ -927,3 +927,37 @@ def test_decode_over_blocks_with_query_codes(sgd, mode):
                                           n_splits=11, q_quant=mode)
     assert_close(out, lse, *ref, OUT_TOL["bf16"])
     check_status(sgd, ws)
+
+
+# ---------------------------------------------------------------------------------------------
+# measurement aids: the read-only stream and the scattered-row read fold every byte they read
+# ---------------------------------------------------------------------------------------------
+def _xor_words(x: np.ndarray) -> int:
+    return int(np.bitwise_xor.reduce(x.view(np.uint32).ravel())) if x.size else 0
+
+
+@pytest.mark.parametrize("method", [0, 1])
+def test_stream_read_folds_every_byte(sgd, method):
+    rng = np.random.default_rng(3 + method)
+    host = rng.integers(0, 256, size=(3 << 20) + 4096, dtype=np.uint8)  # not a whole number of chunks
+    buf = torch.from_numpy(host).cuda()
+    sink, status = sgd.stream_read(buf, method)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert (int(sink.item()) & 0xffffffff) == _xor_words(host)
+
+
+def test_gather_read_folds_the_listed_rows(sgd):
+    rng = np.random.default_rng(11)
+    a = rng.integers(0, 256, size=(5000, 128), dtype=np.uint8)
+    b = rng.integers(0, 256, size=(5000, 128), dtype=np.uint8)
+    rows = rng.integers(0, 5000, size=9999).astype(np.int32)  # repeats allowed; a ragged last batch
+    da, db, dr = (torch.from_numpy(x).cuda() for x in (a, b, rows))
+    sink = sgd.gather_read(da, dr, 128, b=db)
+    torch.cuda.synchronize()
+    assert (int(sink.item()) & 0xffffffff) == _xor_words(np.concatenate([a[rows], b[rows]]))
+    sink1 = sgd.gather_read(da, dr[:7], 128)
+    torch.cuda.synchronize()
+    assert (int(sink1.item()) & 0xffffffff) == _xor_words(a[rows[:7]])
+    with pytest.raises(ValueError):
+        sgd.gather_read(da, torch.tensor([5000], dtype=torch.int32, device="cuda"), 128)
