@@ -37,9 +37,9 @@ FLUSH_BYTES = 256 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, "about 8 TB/s"
 READ_ONLY_BYTES = 4 << 30  # the read-only ceiling streams 4 GiB (far above L2)
-# the spec decode stages timed beside the default workload: workload 4 (8 x 128K, INT8
-# scheme A, dense) and workload 14 (the ragged 512-128K batch over the same INT8 cache)
-NORTH_STAR_WORKLOADS = (4, 14)
+# the 128K INT8 split-KV decode stages timed beside the default workload: workload 4 (8 x 128K,
+# INT8 scheme A, dense) and workload 14 (the ragged 512-128K batch over the same INT8 cache)
+INT8_DECODE_WORKLOADS = (4, 14)
 CALIBRATED_WORKLOAD = 15  # workload 5 with a calibrated V scale
 
 
@@ -51,8 +51,9 @@ def parse():
     p.add_argument("--workload", type=int, default=5, choices=[2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-north-star", action="store_true",
-                   help="skip the workload 4 / 14 decode stages and the read-only ceiling")
+    p.add_argument("--no-extra-records", action="store_true",
+                   help="skip the records beside the step: the read-only ceiling, the workload 4 / 14 INT8 decode "
+                        "stages, the calibrated-scale step and the gather ceiling")
     p.add_argument("--scale", type=float, default=1.0,
                    help="sequence lengths times this factor (a smaller case of the same shapes, for profiling)")
     return p.parse_args()
@@ -799,12 +800,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, dev, world)
 
-    # the read-only ceiling and the spec decode stages (every rank takes the same steps)
+    # the read-only ceiling and the INT8 decode stages (every rank takes the same steps)
     peak, peak_src = load_peaks()
     ro, north, calibrated = None, {}, None
-    if not args.no_north_star:
+    if not args.no_extra_records:
         ro = read_only_ceiling(sgd, dev)
-        for n in NORTH_STAR_WORKLOADS:
+        for n in INT8_DECODE_WORKLOADS:
             rec = decode_stage_record(sgd, n, dev, K, args.warmup, flush_l2, peak, ro["GB_s"], world)
             north[rec["workload"]] = rec
         if args.scale == 1.0 and not wl.calibrated:
@@ -904,8 +905,8 @@ def run_ours(args, rank, world, local_rank):
         "read_only": ro,
         "gather_ceiling": gather,
         "nominal_hbm_GB_s": NOMINAL_HBM_GBS,
-        # spec bar: the 128K INT8 split-KV decode at >= 0.70 of measured HBM, dense and ragged
-        "north_star": north or None,
+        # the 128K INT8 split-KV decode stages, dense (workload 4) and ragged (workload 14)
+        "int8_decode_stages": north or None,
         "calibrated_scales": calibrated,
     }
     if world == 1 and not args.no_cpu_baseline:
