@@ -230,6 +230,34 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * sgd_quantize_select_multi -- sgd_quantize_select with the selection of sgd_oam_select_multi:
+ * one kept set per (sequence, KV head) for M query tokens, s_t = max over the M * G query rows
+ * (q [B, M, Hq, D] BF16 for the fused pass; 1 <= M, G * M <= 16).  The codes, scales and norms
+ * are those of sgd_quantize_kv (they do not depend on q).
+ * workspace   sgd_workspace_size(SGD_OP_QUANTIZE_SELECT, kv, G * M, 0, 0) bytes
+ * Other arguments, outputs and errors as in sgd_quantize_select; M = 1 is sgd_quantize_select.
+ */
+int sgd_quantize_select_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv,
+                              float beta, float eps, int keep_num, int keep_den, sgd_scheme scheme,
+                              int64_t n_parts, int8_t *k_codes, int8_t *v_codes, float *k_scale,
+                              float *v_scale, float *v_norm, int32_t *idx, int32_t *cu_kept,
+                              int64_t kept_total, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * sgd_quantize_select_blocks -- sgd_quantize_select with the selection of sgd_oam_select_blocks:
+ * whole 64-token blocks ranked by their best token's OAM score ([NSA] section 2.1), the token
+ * scores taken in the same pass over K and V that quantises them.
+ * n_blocks, blk, cu_kept_blocks, kept_blocks_total   as in sgd_oam_select_blocks
+ * Other arguments, outputs and errors as in sgd_quantize_select.
+ */
+int sgd_quantize_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv,
+                               float beta, float eps, int keep_num, int keep_den, sgd_scheme scheme,
+                               int64_t n_parts, int8_t *k_codes, int8_t *v_codes, float *k_scale,
+                               float *v_scale, float *v_norm, int64_t n_blocks, int32_t *blk,
+                               int32_t *cu_kept_blocks, int64_t kept_blocks_total, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/*
  * sgd_decode_attn -- split-KV flash-decoding ([TD] section 5, [CD] eq. 5-7).
  *   out[b, h] = sum_t softmax_t(z_t) vhat_t, z_t = q[b, h] . khat_t / sqrt(D),
  *   over every token of sequence b (idx == NULL) or over the kept tokens

@@ -28,7 +28,8 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select", "decode_attn",
+    "lib", "quantize_kv", "oam_select", "oam_select_multi", "oam_select_blocks", "quantize_select",
+    "quantize_select_multi", "quantize_select_blocks", "decode_attn",
     "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
     "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "gather_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B",
@@ -99,6 +100,10 @@ lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, 
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _vp, _sz, _vp]
+lib.sgd_quantize_select_multi.argtypes = [_vp, _i32, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp]
+lib.sgd_quantize_select_blocks.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp,
+                                           _vp, _vp, _i64, _vp, _vp, _i64, _vp, _sz, _vp]
 lib.sgd_decode_attn_noalloc.argtypes = [_vp, _i32, _i32, _kvp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp,
                                         _vp]
 
@@ -294,16 +299,13 @@ def oam_select_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seql
     return blk, cu_kb, ws
 
 
-def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
-                    beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
-                    out=None, workspace=None, stream=None, v_norm=None, k_scale_in=None, v_scale_in=None):
-    """quantize_kv and oam_select of one cache in one call (K and V read once for both).
-    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws); ``v_norm``, ``k_scale_in`` and
-    ``v_scale_in`` as in quantize_kv (with calibrated scales one pass writes every code)."""
+def _quantize_select(q, k, v, cu_seqlens, G, M, beta, eps, keep_num, keep_den, scheme, lengths, out, workspace,
+                     stream, v_norm, k_scale_in, v_scale_in, blocks):
     sch = _quant_scheme(scheme, k_scale_in, v_scale_in)
     Hkv, T, D = k.shape
-    parts = n_parts(lengths) if sch in (SCHEME_A, SCHEME_A_CALIBRATED) else 0
-    Kt = kept_total(lengths, keep_num, keep_den)
+    nb = n_parts(lengths)
+    parts = nb if sch in (SCHEME_A, SCHEME_A_CALIBRATED) else 0
+    Kt = kept_blocks_total(lengths, keep_num, keep_den) if blocks else kept_total(lengths, keep_num, keep_den)
     kv = _kv(k, v, cu_seqlens)
     if out is None:
         kc = torch.empty((Hkv, T, D), dtype=torch.int8, device=k.device)
@@ -313,11 +315,48 @@ def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
         cu_kept = torch.empty(cu_seqlens.numel(), dtype=torch.int32, device=k.device)
     else:
         kc, vc, ks, vs, idx, cu_kept = out
-    ws = _workspace(workspace_size(OP_QUANTIZE_SELECT, kv, G), k.device, workspace)
-    _check(lib.sgd_quantize_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), beta, eps, keep_num, keep_den, sch,
-                                   parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(v_norm), _ptr(idx),
-                                   _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream)), "sgd_quantize_select")
+    ws = _workspace(workspace_size(OP_QUANTIZE_SELECT, kv, G * M), k.device, workspace)
+    common = (beta, eps, keep_num, keep_den, sch, parts, _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(v_norm))
+    tail = (_ptr(idx), _ptr(cu_kept), Kt, _ptr(ws), ws.numel(), _stream(stream))
+    if blocks:
+        rc = lib.sgd_quantize_select_blocks(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), *common, nb, *tail)
+        name = "sgd_quantize_select_blocks"
+    elif M > 1:
+        rc = lib.sgd_quantize_select_multi(_ptr(q), _DT[q.dtype], G, M, ctypes.byref(kv), *common, *tail)
+        name = "sgd_quantize_select_multi"
+    else:
+        rc = lib.sgd_quantize_select(_ptr(q), _DT[q.dtype], G, ctypes.byref(kv), *common, *tail)
+        name = "sgd_quantize_select"
+    _check(rc, name)
     return kc, vc, ks, vs, idx, cu_kept, ws
+
+
+def quantize_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                    beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
+                    out=None, workspace=None, stream=None, v_norm=None, k_scale_in=None, v_scale_in=None):
+    """quantize_kv and oam_select of one cache in one call (K and V read once for both).
+    Returns (k_codes, v_codes, k_scale, v_scale, idx, cu_kept, ws); ``v_norm``, ``k_scale_in`` and
+    ``v_scale_in`` as in quantize_kv (with calibrated scales one pass writes every code)."""
+    return _quantize_select(q, k, v, cu_seqlens, G, 1, beta, eps, keep_num, keep_den, scheme, lengths, out,
+                            workspace, stream, v_norm, k_scale_in, v_scale_in, False)
+
+
+def quantize_select_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                          beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
+                          out=None, workspace=None, stream=None, v_norm=None, k_scale_in=None, v_scale_in=None):
+    """quantize_select for the M query tokens of q [B, M, Hq, D]: one kept set per (sequence, KV
+    head) from the group maximum over all M * G query rows, as oam_select_multi."""
+    return _quantize_select(q, k, v, cu_seqlens, G, q.shape[1], beta, eps, keep_num, keep_den, scheme, lengths, out,
+                            workspace, stream, v_norm, k_scale_in, v_scale_in, False)
+
+
+def quantize_select_blocks(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor, G: int,
+                           beta: float, eps: float, keep_num: int, keep_den: int, scheme: str, lengths: Sequence[int],
+                           out=None, workspace=None, stream=None, v_norm=None, k_scale_in=None, v_scale_in=None):
+    """quantize_select keeping whole 64-token blocks, as oam_select_blocks.  Returns (k_codes,
+    v_codes, k_scale, v_scale, blk [Hkv, NBt], cu_kept_blocks [B+1], ws)."""
+    return _quantize_select(q, k, v, cu_seqlens, G, 1, beta, eps, keep_num, keep_den, scheme, lengths, out,
+                            workspace, stream, v_norm, k_scale_in, v_scale_in, True)
 
 
 def decode_attn(q: torch.Tensor, G: int, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,

@@ -555,21 +555,24 @@ int sgd_oam_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv 
                        kept_blocks_total, workspace, workspace_bytes, stream);
 }
 
-int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
-                        int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
-                        int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm, int32_t *idx,
-                        int32_t *cu_kept, int64_t kept_total, void *workspace, size_t workspace_bytes,
-                        void *stream) {
+// The quantisation and selection behind sgd_quantize_select, _multi (M query tokens, G * M <= 16
+// columns) and _blocks (whole 64-token blocks ranked by their best token, n_blocks of them).
+static int quantize_select_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, float beta,
+                                float eps, int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts,
+                                int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm,
+                                bool blocks, int64_t n_blocks, int32_t *idx, int32_t *cu_kept, int64_t kept_total,
+                                void *workspace, size_t workspace_bytes, void *stream) {
     int rc = check_kv(kv);
     if (rc != SGD_OK) return rc;
     if (!q || !idx || !cu_kept || !workspace || !k_codes || !v_codes || !k_scale || !v_scale) return SGD_ERR_NULL;
-    if (G < 1 || G > 16) return SGD_ERR_SHAPE;
+    if (G < 1 || G > 16 || M < 1 || G * M > 16) return SGD_ERR_SHAPE;
     if (kv->dtype != SGD_BF16 && kv->dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (q_dtype != SGD_BF16 && q_dtype != SGD_F32) return SGD_ERR_DTYPE;
     if (!quant_scheme_ok(scheme)) return SGD_ERR_DTYPE;
     if (has_partitions(scheme) && (n_parts < kv->B || n_parts > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
     if (keep_num < 0 || keep_den < 1 || keep_num > keep_den) return SGD_ERR_ARG;
-    if (kept_total < kv->B || kept_total > kv->T) return SGD_ERR_SHAPE;
+    if (blocks && (n_blocks < kv->B || n_blocks > kv->T / SGD_PARTITION + kv->B)) return SGD_ERR_SHAPE;
+    if (kept_total < kv->B || kept_total > (blocks ? n_blocks : kv->T)) return SGD_ERR_SHAPE;
     if (!isfinite(beta) || !isfinite(eps) || eps < 0.f) return SGD_ERR_ARG;
     if (!aligned16(q) || !aligned16(workspace) || !aligned16(k_codes) || !aligned16(v_codes)) return SGD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(cu_kept) & 3u) ||
@@ -581,14 +584,14 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
         rc = sgd_quantize_kv(kv, scheme, n_parts, k_codes, v_codes, k_scale, v_scale, v_norm, workspace,
                              workspace_bytes, stream);
         if (rc != SGD_OK) return rc;
-        return sgd_oam_select(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, idx, cu_kept, kept_total, workspace,
-                              workspace_bytes, stream);
+        return select_impl(q, q_dtype, G, kv, beta, eps, keep_num, keep_den, blocks, n_blocks, idx, cu_kept,
+                           kept_total, workspace, workspace_bytes, stream, M);
     }
     DevInfo *dev;
     if ((rc = current_device(&dev)) != SGD_OK) return rc;
-    const int n_req = fused_n_req(*dev, kv, G);
+    const int n_req = fused_n_req(*dev, kv, G * M);
     if (n_req < 1) return SGD_ERR_CUDA;
-    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G, kv->D, kv->T, n_req);
+    const Layout L = layout(SGD_OP_OAM_SELECT, kv->B, kv->Hkv, G * M, kv->D, kv->T, n_req);
     if (workspace_bytes < L.total) return SGD_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
@@ -605,7 +608,7 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
     a.B = kv->B;
     a.Hkv = kv->Hkv;
     a.G = G;
-    a.M = 1;
+    a.M = M;
     a.D = kv->D;
     a.T = kv->T;
     const bool cal = scheme == SGD_SCHEME_A_CALIBRATED || scheme == SGD_SCHEME_B_CALIBRATED;
@@ -636,9 +639,48 @@ int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *k
                                    v_scale, v_norm, hdr, dev->sms, s);
         if (e != 0) return SGD_ERR_CUDA;
     }
+    if (blocks) {  // block scores, then the top blocks of each row (the plan's partition offsets = block offsets)
+        float *bs = reinterpret_cast<float *>(ws + L.bscores);
+        e = launch_block_max(a.scores, kv->cu_seqlens, pv.seq_part0, kv->B, kv->Hkv, kv->T, n_blocks, bs,
+                             &hdr->status, s);
+        if (e != 0) return SGD_ERR_CUDA;
+        e = launch_topk(bs, pv.seq_part0, kv->B, kv->Hkv, n_blocks, keep_num, keep_den, idx, cu_kept, kept_total,
+                        &hdr->status, s);
+        return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+    }
     e = launch_topk(a.scores, kv->cu_seqlens, kv->B, kv->Hkv, kv->T, keep_num, keep_den, idx, cu_kept, kept_total,
                     &hdr->status, s);
     return e == 0 ? SGD_OK : SGD_ERR_CUDA;
+}
+
+int sgd_quantize_select(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
+                        int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
+                        int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm, int32_t *idx,
+                        int32_t *cu_kept, int64_t kept_total, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    return quantize_select_impl(q, q_dtype, G, 1, kv, beta, eps, keep_num, keep_den, scheme, n_parts, k_codes, v_codes,
+                                k_scale, v_scale, v_norm, false, 0, idx, cu_kept, kept_total, workspace,
+                                workspace_bytes, stream);
+}
+
+int sgd_quantize_select_multi(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv, float beta, float eps,
+                              int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
+                              int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm, int32_t *idx,
+                              int32_t *cu_kept, int64_t kept_total, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    return quantize_select_impl(q, q_dtype, G, M, kv, beta, eps, keep_num, keep_den, scheme, n_parts, k_codes, v_codes,
+                                k_scale, v_scale, v_norm, false, 0, idx, cu_kept, kept_total, workspace,
+                                workspace_bytes, stream);
+}
+
+int sgd_quantize_select_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, float beta, float eps,
+                               int keep_num, int keep_den, sgd_scheme scheme, int64_t n_parts, int8_t *k_codes,
+                               int8_t *v_codes, float *k_scale, float *v_scale, float *v_norm, int64_t n_blocks,
+                               int32_t *blk, int32_t *cu_kept_blocks, int64_t kept_blocks_total, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    return quantize_select_impl(q, q_dtype, G, 1, kv, beta, eps, keep_num, keep_den, scheme, n_parts, k_codes, v_codes,
+                                k_scale, v_scale, v_norm, true, n_blocks, blk, cu_kept_blocks, kept_blocks_total,
+                                workspace, workspace_bytes, stream);
 }
 
 int sgd_decode_attn(const void *q, sgd_dtype q_dtype, int G, const sgd_kv *kv, const int32_t *idx,

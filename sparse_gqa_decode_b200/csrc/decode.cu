@@ -1635,7 +1635,7 @@ int launch_decode(const DecodeArgs &a, sgd_dtype kv, sgd_dtype q, bool indexed, 
 
 template <bool CAL>
 static int launch_score_quantize_cfg(const DecodeArgs &a, int n_cta, cudaStream_t s) {
-    const bool g2 = a.G > 8;
+    const bool g2 = a.G * a.M > 8;  // columns: the (query token, head) pairs
     if (a.D == 128)
         return g2 ? launch_mma<MmaCfg<128, 2, false, false, 2, false, false, false, CAL>>(a, n_cta, s)
                   : launch_mma<MmaCfg<128, 1, false, false, 2, false, false, false, CAL>>(a, n_cta, s);

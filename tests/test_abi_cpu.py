@@ -249,3 +249,24 @@ def test_gather_read_rejects_bad_args_on_host(sgd):
     assert g(rb=0) == -2 and g(rb=24) == -2 and g(rb=48) == -2 and g(rb=8192) == -2 and g(n=0) == -2
     assert g(a=0x1008) == -4 and g(b=0x2008) == -4 and g(rows=0x3002) == -4 and g(sink=0x4004) == -4
     assert g(b=0) not in (-1, -2, -4)  # b is optional; no device here, so the call fails later
+
+
+def test_quantize_select_multi_and_blocks_reject_bad_args_on_host(sgd):
+    L = sgd.lib
+    p = ctypes.c_void_p
+    kv = _kv(sgd)
+    outs = (p(0x1000), p(0x1000), p(0x2000), p(0x3000), None)
+
+    def multi(G=8, M=2, kt=20):
+        return L.sgd_quantize_select_multi(p(0x3000), sgd.SGD_BF16, G, M, ctypes.byref(kv), 1.0, 1e-6, 1, 8, 0, 3,
+                                           *outs, p(0x5000), p(0x6000), kt, p(0x4000), 1 << 20, None)
+
+    def blocks(nb=3, kt=3):
+        return L.sgd_quantize_select_blocks(p(0x3000), sgd.SGD_BF16, 8, ctypes.byref(kv), 1.0, 1e-6, 1, 4, 0, 3,
+                                            *outs, nb, p(0x5000), p(0x6000), kt, p(0x4000), 1 << 20, None)
+
+    assert multi(M=0) == -2 and multi(G=8, M=3) == -2 and multi(G=16, M=2) == -2
+    assert multi(G=4, M=4) not in (-1, -2, -3, -4, -8)  # 16 columns pass the host checks
+    assert blocks(nb=1) == -2  # fewer blocks than sequences
+    assert blocks(kt=4) == -2  # more kept blocks than blocks
+    assert blocks() not in (-1, -2, -3, -4, -8)

@@ -961,3 +961,56 @@ def test_gather_read_folds_the_listed_rows(sgd):
     assert (int(sink1.item()) & 0xffffffff) == _xor_words(a[rows[:7]])
     with pytest.raises(ValueError):
         sgd.gather_read(da, torch.tensor([5000], dtype=torch.int32, device="cuda"), 128)
+
+
+# ---------------------------------------------------------------------------------------------
+# quantise and select in one call for several query tokens, or by 64-token blocks: the same codes,
+# scales and norms as sgd_quantize_kv and the same kept sets as oam_select_multi / _blocks, which
+# are checked against the oracle
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (2, 4), (16, 1)])
+def test_quantize_select_multi_equals_separate_calls(sgd, scheme, M, G):
+    lengths = (5, 64, 300, 2500)
+    bt = make_multi(lengths, M, G, seed=71 + M + G)
+    q, k, v, cu = dev(bt)
+    vn = torch.empty((2, bt.T), dtype=torch.float32, device="cuda")
+    fused = sgd.quantize_select_multi(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths, v_norm=vn)
+    check_status(sgd, fused[6])
+    vn2 = torch.empty_like(vn)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn2)
+    idx, cu_kept, _ = sgd.oam_select_multi(q, k, v, cu, G, 1.0, 1e-6, 1, 8, bt.lengths)
+    for a, b in zip(fused[:6], (kc, vc, ks, vs, idx, cu_kept)):
+        assert torch.equal(a, b)
+    assert torch.equal(vn, vn2)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    assert np.array_equal(fused[0].cpu().numpy(), rkc) and np.array_equal(fused[1].cpu().numpy(), rvc)
+    ref_idx, ref_cu, scores = oracle.oam_select_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, 1.0, 1e-6, 1, 8)
+    check_selection(fused[4], fused[5].cpu(), ref_idx, ref_cu, scores, len(lengths), 2)
+
+
+@pytest.mark.parametrize("scheme", ["A", "B", "A-calibrated"])
+@pytest.mark.parametrize("G,D", [(8, 128), (4, 64), (16, 128)])
+def test_quantize_select_blocks_equals_separate_calls(sgd, scheme, G, D):
+    bt = make(BLOCK_LENGTHS, G=G, D=D, Hkv=2, dist="outlier", seed=81 + G + D)
+    q, k, v, cu = dev(bt)
+    base = scheme[0]
+    cal = {}
+    if scheme.endswith("calibrated"):
+        cal = dict(v_scale_in=_on_device(_calibrated(bt, base, 0.5)[1]))
+    fused = sgd.quantize_select_blocks(q, k, v, cu, G, 1.0, 1e-6, 1, 4, base, bt.lengths, **cal)
+    check_status(sgd, fused[6])
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, base, bt.lengths, **cal)
+    blk, cu_kb, _ = sgd.oam_select_blocks(q, k, v, cu, G, 1.0, 1e-6, 1, 4, bt.lengths)
+    for a, b in zip(fused[:6], (kc, vc, ks, vs, blk, cu_kb)):
+        assert torch.equal(a, b)
+    _, _, scores = oracle.oam_select(bt.q, bt.k, bt.v, bt.cu_seqlens, G, 1.0, 1e-6, 1, 4)
+    ref_blk, ref_cu, bscores = oracle.select_blocks(scores, bt.cu_seqlens, 2, 1, 4)
+    check_selection(fused[4], fused[5].cpu(), ref_blk, ref_cu, bscores, bt.wl.B, 2)
+
+
+def test_quantize_select_multi_rejects_too_many_columns(sgd):
+    bt = make_multi((64, 300), 4, 8, seed=5)  # M * G = 32 > 16
+    q, k, v, cu = dev(bt)
+    with pytest.raises(sgd.SgdError):  # the workspace query already refuses 32 columns
+        sgd.quantize_select_multi(q, k, v, cu, 8, 1.0, 1e-6, 1, 8, "A", bt.lengths)
