@@ -27,6 +27,10 @@
 //     swizzled shared-memory reads of both K and V are bank-conflict free.
 //   * at the end of each (row, token range) segment the four warps' (m, l, O) are
 //     combined through shared memory into one partial (o_c, lse_c).
+// The same pipeline scores tokens (OAM, mode 1) and, with eight more warps that quantise
+// each 64-token K tile (one scheme-A partition) while the consumer warps score it, runs the
+// one-pass quantise-and-select (mode 2); with calibrated per-tensor scales those warps also
+// write the V codes and the value norms.
 // CUDA-core kernel: every other dtype/shape (F32 cache, INT8 with D = 64, ...).
 #include <math.h>
 
