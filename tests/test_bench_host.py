@@ -159,3 +159,19 @@ def test_kept_rows_are_the_cache_rows_of_the_kept_tokens(bench):
            for j in range(cu_kept[b], cu_kept[b + 1])]
     assert rows.dtype == np.int32 and rows.tolist() == ref
     assert rows.min() >= 0 and rows.max() < Hkv * T
+
+
+def test_calibrated_fused_pass_counts_every_code(bench):
+    # with calibrated scales the fused pass also writes the V codes (scheme B: the K codes too);
+    # the step's algorithmic bytes are those of the computed-scale step
+    lengths = [100, 64]
+    T, Hkv, D, parts = 164, 2, 128, 3
+    q = 2 * 8 * D * 2
+    for scheme in ("A", "B"):
+        wl = workloads.Workload("t", B=2, Hkv=2, G=4, D=128, kv_dtype="bf16", dist="normal", lengths=(100, 64),
+                                scheme=scheme, oam=True)
+        cal = wl.with_(calibrated=True)
+        scales = Hkv * parts * 4 if scheme == "A" else 0
+        want = 2 * Hkv * T * D * 2 + 2 * Hkv * T * D + scales + Hkv * T * 4 + q
+        assert bench.kernel_bytes(cal, lengths, "score_quantize") == want
+        assert bench.algorithmic_bytes(cal, lengths) == bench.algorithmic_bytes(wl, lengths)

@@ -68,3 +68,16 @@ def test_ragged_int8_workload_shares_the_ragged_lengths():
     assert a.lengths.tolist() == b.lengths.tolist()
     assert b.outlier_channels is not None and workloads.config(14).scheme == "A"
     assert (512 <= b.lengths).all() and (b.lengths <= 131072).all()
+
+
+def test_calibrated_workload_is_the_default_batch():
+    # workload 15 draws workload 5's batch (its seed): the calibrated step quantises the same cache
+    w5, w15 = workloads.config(5), workloads.config(15)
+    assert w15.calibrated and not w5.calibrated
+    assert w15.with_(name=w5.name, calibrated=False, seed=None) == w5
+    small5 = w5.with_(length_range=(300, 900))
+    small15 = w15.with_(length_range=(300, 900))
+    a = workloads.generate(small5, seed=5)
+    b = workloads.generate(small15, seed=small15.seed)
+    for x, y in ((a.q, b.q), (a.k, b.k), (a.v, b.v), (a.cu_seqlens, b.cu_seqlens)):
+        assert torch.equal(x, y)
