@@ -959,6 +959,12 @@ def test_gather_read_folds_the_listed_rows(sgd):
     sink1 = sgd.gather_read(da, dr[:7], 128)
     torch.cuda.synchronize()
     assert (int(sink1.item()) & 0xffffffff) == _xor_words(a[rows[:7]])
+    for row_bytes in (16, 4096):  # the smallest and the largest rows
+        flat = rng.integers(0, 256, size=row_bytes * 300, dtype=np.uint8)
+        rr = rng.integers(0, 300, size=517).astype(np.int32)
+        s2 = sgd.gather_read(torch.from_numpy(flat).cuda(), torch.from_numpy(rr).cuda(), row_bytes)
+        torch.cuda.synchronize()
+        assert (int(s2.item()) & 0xffffffff) == _xor_words(flat.reshape(300, row_bytes)[rr]), row_bytes
     with pytest.raises(ValueError):
         sgd.gather_read(da, torch.tensor([5000], dtype=torch.int32, device="cuda"), 128)
 
@@ -968,22 +974,28 @@ def test_gather_read_folds_the_listed_rows(sgd):
 # scales and norms as sgd_quantize_kv and the same kept sets as oam_select_multi / _blocks, which
 # are checked against the oracle
 # ---------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("scheme", ["A", "B"])
+@pytest.mark.parametrize("scheme", ["A", "B", "B-calibrated"])
 @pytest.mark.parametrize("M,G", [(2, 8), (4, 4), (2, 4), (16, 1)])
 def test_quantize_select_multi_equals_separate_calls(sgd, scheme, M, G):
     lengths = (5, 64, 300, 2500)
     bt = make_multi(lengths, M, G, seed=71 + M + G)
     q, k, v, cu = dev(bt)
+    base, cal = scheme[0], {}
+    if scheme.endswith("calibrated"):
+        k_cal, v_cal = _calibrated(bt, base, 0.5)
+        cal = dict(k_scale_in=_on_device(k_cal), v_scale_in=_on_device(v_cal))
+    scheme = base
     vn = torch.empty((2, bt.T), dtype=torch.float32, device="cuda")
-    fused = sgd.quantize_select_multi(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths, v_norm=vn)
+    fused = sgd.quantize_select_multi(q, k, v, cu, G, 1.0, 1e-6, 1, 8, scheme, bt.lengths, v_norm=vn, **cal)
     check_status(sgd, fused[6])
     vn2 = torch.empty_like(vn)
-    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn2)
+    kc, vc, ks, vs, _ = sgd.quantize_kv(k, v, cu, scheme, bt.lengths, v_norm=vn2, **cal)
     idx, cu_kept, _ = sgd.oam_select_multi(q, k, v, cu, G, 1.0, 1e-6, 1, 8, bt.lengths)
     for a, b in zip(fused[:6], (kc, vc, ks, vs, idx, cu_kept)):
         assert torch.equal(a, b)
     assert torch.equal(vn, vn2)
-    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme)
+    okw = {} if not cal else dict(k_scale=k_cal, v_scale=v_cal)
+    rkc, rvc, rks, rvs = oracle.quantize_kv(bt.k, bt.v, bt.cu_seqlens, scheme, **okw)
     assert np.array_equal(fused[0].cpu().numpy(), rkc) and np.array_equal(fused[1].cpu().numpy(), rvc)
     ref_idx, ref_cu, scores = oracle.oam_select_multi(bt.q, bt.k, bt.v, bt.cu_seqlens, G, M, 1.0, 1e-6, 1, 8)
     check_selection(fused[4], fused[5].cpu(), ref_idx, ref_cu, scores, len(lengths), 2)
