@@ -66,7 +66,7 @@ def load(path: str):
                                  ctypes.c_double, ctypes.c_double, _dp]
     L.orc_topk.argtypes = [ctypes.c_int64, _dp, ctypes.c_int64, _i32p]
     L.orc_plan.argtypes = [ctypes.c_int, _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                           ctypes.c_int64, _i32p, _i32p, _i64p, _i64p, _i32p]
+                           ctypes.c_int, ctypes.c_int64, _i32p, _i32p, _i64p, _i64p, _i32p]
     L.orc_plan.restype = ctypes.c_int64
     return L
 
@@ -510,8 +510,9 @@ def decode_multi(q, k, v, cu_seqlens, G: int, M: int, idx=None, cu_kept=None, qu
 
 
 # ----------------------------------------------------------------------------------------------
-def plan(row_lengths, n_req: int, granule: int, min_chunk: int, mode: int):
-    """Segments (cta, row, start, length) of the split-KV partition, and the CTA count."""
+def plan(row_lengths, n_req: int, granule: int, min_chunk: int, mode: int, row_cost: int = 0):
+    """Segments (cta, row, start, length) of the split-KV partition, and the CTA count.  Each row
+    occupies its length rounded up to ``granule`` plus ``row_cost`` positions of the stream."""
     lens = np.ascontiguousarray(row_lengths, dtype=np.int64)
     R = lens.size
     cap = int(max(1, n_req) + R + 8) if mode == 0 else R
@@ -520,7 +521,7 @@ def plan(row_lengths, n_req: int, granule: int, min_chunk: int, mode: int):
     start = np.empty(cap, np.int64)
     length = np.empty(cap, np.int64)
     ncta = ctypes.c_int32(0)
-    n = lib().orc_plan(R, _ptr(lens, _i64p), int(n_req), int(granule), int(min_chunk), int(mode), cap,
+    n = lib().orc_plan(R, _ptr(lens, _i64p), int(n_req), int(granule), int(min_chunk), int(mode), int(row_cost), cap,
                        _ptr(cta, _i32p), _ptr(row, _i32p), _ptr(start, _i64p), _ptr(length, _i64p),
                        ctypes.byref(ncta))
     if n < 0:

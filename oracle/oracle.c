@@ -261,7 +261,9 @@ int orc_topk(int64_t n, const double *s, int64_t K, int32_t *idx)
 /* chunks handled by separate CTAs so that a 128K row and a 512 row do not   */
 /* leave CTAs idle).  The rule, written out:                                 */
 /*   - the rows (one per (KV head, sequence), in stream order) are laid end  */
-/*     to end, each padded to a multiple of `granule` tokens;                */
+/*     to end, each padded to a multiple of `granule` tokens and followed by */
+/*     `row_cost` more positions (a fixed work charge per row: its segment   */
+/*     setup and merge; 0 gives the plain token split);                      */
 /*   - mode 0 (equal work): the padded stream of W tokens is cut into CTA    */
 /*     ranges of S = max(min_chunk, round_up(ceil(W / n_req), granule))      */
 /*     tokens, the last one shorter; mode 1: one CTA per row;                */
@@ -272,10 +274,10 @@ int orc_topk(int64_t n, const double *s, int64_t K, int32_t *idx)
 /* returns their number, the number of CTAs through *n_cta, or -1.           */
 /* ------------------------------------------------------------------------ */
 int64_t orc_plan(int R, const int64_t *len, int n_req, int granule, int min_chunk,
-                 int mode, int64_t max_segs, int32_t *seg_cta, int32_t *seg_row,
+                 int mode, int row_cost, int64_t max_segs, int32_t *seg_cta, int32_t *seg_row,
                  int64_t *seg_start, int64_t *seg_len, int32_t *n_cta)
 {
-    if (R < 1 || granule < 1 || (mode == 0 && n_req < 1))
+    if (R < 1 || granule < 1 || row_cost < 0 || (mode == 0 && n_req < 1))
         return -1;
     int64_t *pos = (int64_t *)malloc(((size_t)R + 1) * sizeof(int64_t));
     if (!pos)
@@ -286,7 +288,7 @@ int64_t orc_plan(int R, const int64_t *len, int n_req, int granule, int min_chun
             free(pos);
             return -1;
         }
-        pos[r + 1] = pos[r] + (len[r] + granule - 1) / granule * granule;
+        pos[r + 1] = pos[r] + (len[r] + granule - 1) / granule * granule + row_cost;
     }
     const int64_t W = pos[R];
     int64_t count = 0;

@@ -44,6 +44,7 @@ MUTANTS = [
      "if (si > sj)\n        return 1;\n    if (si < sj)\n        return -1;"),
     ("plan: chunk size not rounded to the granule", "S = (S + granule - 1) / granule * granule;", ""),
     ("plan: segment start in stream coordinates", "seg_start[count] = lo - pos[r];", "seg_start[count] = lo;"),
+    ("plan: the per-row charge dropped", "/ granule * granule + row_cost;", "/ granule * granule;"),
 ]
 
 # pins re-run against each mutant (call -> raises on a caught mistake)

@@ -464,16 +464,21 @@ def test_plan_hand_example(golden_dir):
     p = oracle.plan(g["row_lengths"], g["n_req"], g["granule"], g["min_chunk"], 0)
     segs = [list(map(int, t)) for t in zip(p["cta"], p["row"], p["start"], p["len"])]
     assert segs == g["segments"] and p["n_cta"] == g["n_cta"]
+    c = g["row_cost_case"]
+    p = oracle.plan(c["row_lengths"], c["n_req"], c["granule"], c["min_chunk"], 0, c["row_cost"])
+    segs = [list(map(int, t)) for t in zip(p["cta"], p["row"], p["start"], p["len"])]
+    assert segs == c["segments"] and p["n_cta"] == c["n_cta"]
 
 
+@pytest.mark.parametrize("row_cost", [0, 256])
 @pytest.mark.parametrize("seed", range(12))
-def test_plan_covers_every_token_once_with_equal_work(seed):
+def test_plan_covers_every_token_once_with_equal_work(seed, row_cost):
     rng = np.random.default_rng(seed)
     R = int(rng.integers(1, 40))
     lens = np.rint(np.exp(rng.uniform(0, 10, R))).astype(np.int64)
     n_req = int(rng.integers(1, 300))
     gran = 16
-    p = oracle.plan(lens, n_req, gran, gran, 0)
+    p = oracle.plan(lens, n_req, gran, gran, 0, row_cost)
     assert p["n_cta"] <= n_req
     covered = [np.zeros(L, np.int32) for L in lens]
     for c, r, s, l in zip(p["cta"], p["row"], p["start"], p["len"]):
@@ -483,12 +488,19 @@ def test_plan_covers_every_token_once_with_equal_work(seed):
     # segments come in stream order; a CTA's padded work is at most S
     order = list(zip(p["cta"], p["row"]))
     assert order == sorted(order)
-    W = int(sum((L + gran - 1) // gran * gran for L in lens))
+    W = int(sum((L + gran - 1) // gran * gran + row_cost for L in lens))
     S = max(gran, -(-(-(-W // n_req)) // gran) * gran)
     work = np.zeros(p["n_cta"], np.int64)
     for c, l in zip(p["cta"], p["len"]):
         work[c] += (l + gran - 1) // gran * gran
     assert work.max() <= S
+    # with a row charge, a CTA's tokens plus the charges of the rows starting in it stay within
+    # S plus one charge (a row's charge follows its tokens and may spill into the next range)
+    if row_cost:
+        starts = np.zeros(p["n_cta"], np.int64)
+        for c, s in zip(p["cta"], p["start"]):
+            starts[c] += row_cost if s == 0 else 0
+        assert (work + starts).max() <= S + row_cost
     one = oracle.plan(lens, 0, gran, gran, 1)
     assert one["n_cta"] == R and one["len"].tolist() == lens.tolist()
 
