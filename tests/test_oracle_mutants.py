@@ -68,8 +68,8 @@ PIN_CALLS = [
     lambda g: pins.test_topk_all_equal_keeps_lowest_indices_and_keep_all(),
     lambda g: pins.test_beta_zero_is_classic_qk_ranking_and_q_zero_is_norm_ranking(),
     lambda g: pins.test_plan_hand_example(g),
-    lambda g: pins.test_plan_covers_every_token_once_with_equal_work(3),
-    lambda g: pins.test_plan_covers_every_token_once_with_equal_work(5, 256),
+    lambda g: pins.plan_coverage(3),
+    lambda g: pins.plan_coverage(5, 256),
 ]
 
 

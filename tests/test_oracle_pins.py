@@ -472,7 +472,11 @@ def test_plan_hand_example(golden_dir):
 
 @pytest.mark.parametrize("row_cost", [0, 256])
 @pytest.mark.parametrize("seed", range(12))
-def test_plan_covers_every_token_once_with_equal_work(seed, row_cost=0):
+def test_plan_covers_every_token_once_with_equal_work(seed, row_cost):
+    plan_coverage(seed, row_cost)
+
+
+def plan_coverage(seed, row_cost=0):
     rng = np.random.default_rng(seed)
     R = int(rng.integers(1, 40))
     lens = np.rint(np.exp(rng.uniform(0, 10, R))).astype(np.int64)
