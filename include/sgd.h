@@ -81,6 +81,9 @@ typedef enum {
 } sgd_scheme;
 
 #define SGD_PARTITION 64 /* scheme-A partition length in tokens */
+/* tokens of work the automatic split-KV partition charges each row beside its tokens (its
+ * segment setup, epilogue and merge), so that CTAs covering many short rows take fewer tokens */
+#define SGD_ROW_COST 256
 
 /* status codes */
 #define SGD_OK 0
@@ -333,11 +336,16 @@ int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedul
  * sgd_plan_segments -- the split-KV partition used by sgd_decode_attn, for
  * inspection.  Rows are (KV head, sequence) pairs in memory order
  * (row = kvh * B + b) with lengths cu[b+1] - cu[b]; each row is padded to a
- * multiple of 16 tokens and the rows are laid end to end; mode 0 cuts this
- * stream into CTA ranges of S = max(min_chunk, round_up(ceil(W / n_req), 16))
- * tokens, mode 1 gives each row its own CTA.  A segment is the intersection of
- * one CTA range with the real tokens of one row.
+ * multiple of 16 tokens, followed by row_cost more positions (a fixed work
+ * charge; rows of no tokens take none), and the rows are laid end to end;
+ * mode 0 cuts this stream of W positions into CTA ranges of
+ * S = max(min_chunk, round_up(ceil(W / n_req), 16)), mode 1 gives each row its
+ * own CTA.  A segment is the intersection of one CTA range with the real
+ * tokens of one row.  sgd_decode_attn's automatic split (schedule 0, no
+ * n_splits, tokens rather than blocks) uses row_cost = SGD_ROW_COST and
+ * min_chunk 256; a forced split uses row_cost 0.
  * cu        [B+1] device int32 (cu_seqlens, or cu_kept for a kept set)
+ * row_cost  a multiple of 16 in [0, 65536]
  * segs      [max_segs, 4] device int32 output: (cta, row, row-local start, length)
  *           in stream order
  * n_segs    [2] device int32 output: number of segments, number of CTAs used
@@ -345,7 +353,7 @@ int sgd_decode_num_ctas(const sgd_kv *kv, int G, const int32_t *idx, int schedul
  *           2048 + 4 * (B + 2 * B * Hkv + 3 * n_req + 6) + 32 * B * Hkv bytes
  *           (mode 1: n_req = B * Hkv); SGD_ERR_WORKSPACE when smaller
  */
-int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode,
+int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode, int row_cost,
                       int32_t *segs, int64_t max_segs, int32_t *n_segs,
                       void *workspace, size_t workspace_bytes, void *stream);
 

@@ -33,7 +33,7 @@ __all__ = [
     "decode_attn_multi", "decode_attn_blocks", "decode_attn_noalloc", "plan_segments", "workspace_status",
     "workspace_size", "decode_num_ctas", "kept_total", "kept_blocks_total", "n_parts", "kernel_timing_start",
     "kernel_timing_stop", "test_pipeline_timeout", "stream_read", "gather_read", "SGD_F32", "SGD_BF16", "SGD_I8", "SCHEME_A", "SCHEME_B",
-    "SCHEME_A_CALIBRATED", "SCHEME_B_CALIBRATED", "STATUS_BITS",
+    "SCHEME_A_CALIBRATED", "SCHEME_B_CALIBRATED", "STATUS_BITS", "ROW_COST",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -41,6 +41,7 @@ LIB_PATH = os.path.join(_HERE, "libsgd.so")
 
 SGD_F32, SGD_BF16, SGD_I8 = 0, 1, 2
 SCHEME_A, SCHEME_B, SCHEME_A_CALIBRATED, SCHEME_B_CALIBRATED = 0, 1, 2, 3
+ROW_COST = 256  # SGD_ROW_COST: the automatic split's work charge per row, in tokens
 OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE, OP_QUANTIZE_SELECT = 0, 1, 2, 3
 PARTITION = 64
 STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index",
@@ -96,7 +97,7 @@ lib.sgd_kernel_timing_start.argtypes = [_i32]
 lib.sgd_kernel_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(ctypes.c_int32)]
 lib.sgd_kernel_timing_name.argtypes = [_i32]
 lib.sgd_kernel_timing_name.restype = ctypes.c_char_p
-lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
+lib.sgd_plan_segments.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp]
 lib.sgd_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32), _vp]
 lib.sgd_quantize_select.argtypes = [_vp, _i32, _i32, _kvp, _f, _f, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _i64, _vp, _sz, _vp]
@@ -512,8 +513,11 @@ def decode_num_ctas(k, v, cu_seqlens, G: int, indexed: bool = False, schedule: i
     return int(n)
 
 
-def plan_segments(cu: torch.Tensor, B: int, Hkv: int, n_req: int, min_chunk: int, mode: int, stream=None):
-    """The split-KV partition: int32 [n_segs, 4] rows (cta, row, start, length), and the CTA count."""
+def plan_segments(cu: torch.Tensor, B: int, Hkv: int, n_req: int, min_chunk: int, mode: int, row_cost: int = 0,
+                  stream=None):
+    """The split-KV partition: int32 [n_segs, 4] rows (cta, row, start, length), and the CTA count.
+    ``row_cost``: positions charged to each row beside its tokens (the decode's automatic split
+    uses ROW_COST)."""
     R = B * Hkv
     cap = n_req + R + 8
     segs = torch.full((cap, 4), -1, dtype=torch.int32, device=cu.device)
@@ -521,7 +525,7 @@ def plan_segments(cu: torch.Tensor, B: int, Hkv: int, n_req: int, min_chunk: int
     n = R if mode == 1 else n_req
     nbytes = 2048 + 4 * (B + 2 * R + 3 * n + 6) + 32 * R  # the bound sgd.h states
     ws = torch.empty(nbytes, dtype=torch.uint8, device=cu.device)
-    _check(lib.sgd_plan_segments(_ptr(cu), B, Hkv, n_req, min_chunk, mode, _ptr(segs), cap, _ptr(nseg), _ptr(ws),
-                                 ws.numel(), _stream(stream)), "sgd_plan_segments")
+    _check(lib.sgd_plan_segments(_ptr(cu), B, Hkv, n_req, min_chunk, mode, int(row_cost), _ptr(segs), cap, _ptr(nseg),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "sgd_plan_segments")
     n, ncta = (int(x) for x in nseg.tolist())
     return segs[:n].cpu(), ncta

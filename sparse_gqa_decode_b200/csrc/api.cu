@@ -235,9 +235,14 @@ int decode_impl(const void *q, sgd_dtype q_dtype, int G, int M, const sgd_kv *kv
     // blocks: segments start and end on block boundaries (granule 64), lengths counted in blocks
     const int granule = blocks ? kPart : kGranule;
     const int min_chunk = (n_splits > 0 || schedule == 1) ? granule : kAutoMinChunk;
+    // the automatic token split charges every row SGD_ROW_COST tokens of work (its segment setup,
+    // epilogue and merge), while the stream positions stay below 2^31
+    const int64_t R = (int64_t)kv->B * kv->Hkv;
+    const bool charge = !blocks && schedule == 0 && n_splits == 0 &&
+                        (int64_t)kv->Hkv * kv->T + R * (kGranule + SGD_ROW_COST) < (int64_t(1) << 31);
     launch_plan(listed ? cu_kept : kv->cu_seqlens, kv->cu_seqlens, kv->B, kv->Hkv, n_req, min_chunk, schedule, pv,
                 hdr, s, granule, out, lse, G, kv->D, q_quant == 2 ? static_cast<const __nv_bfloat16 *>(q) : nullptr,
-                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M, blocks ? kPart : 1, ncg);
+                (int64_t)kv->B * M * kv->Hkv * G * kv->D, M, blocks ? kPart : 1, ncg, charge ? SGD_ROW_COST : 0);
     DecodeArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q;
@@ -706,13 +711,15 @@ int sgd_decode_attn_blocks(const void *q, sgd_dtype q_dtype, int G, const sgd_kv
                        q_quant, out, lse, workspace, workspace_bytes, stream);
 }
 
-int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode, int32_t *segs,
-                      int64_t max_segs, int32_t *n_segs, void *workspace, size_t workspace_bytes, void *stream) {
+int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chunk, int mode, int row_cost,
+                      int32_t *segs, int64_t max_segs, int32_t *n_segs, void *workspace, size_t workspace_bytes,
+                      void *stream) {
     if (!cu || !segs || !n_segs || !workspace) return SGD_ERR_NULL;
     if (B < 1 || Hkv < 1 || (int64_t)B * Hkv >= (int64_t(1) << 24)) return SGD_ERR_SHAPE;
     if (mode != 0 && mode != 1) return SGD_ERR_ARG;
     if (mode == 1) n_req = B * Hkv;
     if (n_req < 1 || min_chunk < kGranule || min_chunk % kGranule != 0 || max_segs < 0) return SGD_ERR_ARG;
+    if (row_cost < 0 || row_cost > (1 << 16) || row_cost % kGranule != 0) return SGD_ERR_ARG;
     if (!aligned16(workspace)) return SGD_ERR_ALIGN;
     const Layout L = layout(SGD_OP_DECODE, B, Hkv, 1, 64, 1, n_req);
     if (workspace_bytes < L.row_done) return SGD_ERR_WORKSPACE;  // the plan arrays only
@@ -724,7 +731,8 @@ int sgd_plan_segments(const int32_t *cu, int B, int Hkv, int n_req, int min_chun
     PlanView pv = plan_view(ws, L);
     pv.row_done = nullptr;  // no decode follows
     cudaStream_t s = as_stream(stream);
-    launch_plan(cu, cu, B, Hkv, n_req, min_chunk, mode, pv, hdr, s);
+    launch_plan(cu, cu, B, Hkv, n_req, min_chunk, mode, pv, hdr, s, kGranule, nullptr, nullptr, 0, 0, nullptr, 0, 1, 1,
+                1, row_cost);
     launch_plan_dump(pv, cu, B, Hkv, n_req, segs, max_segs, n_segs, hdr, s);
     return cudaGetLastError() == cudaSuccess ? SGD_OK : SGD_ERR_CUDA;
 }

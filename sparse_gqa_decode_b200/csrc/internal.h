@@ -64,7 +64,7 @@ enum Family { kFamilyMma = 0, kFamilyGeneric = 1 };
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule = kGranule,
                  float *out = nullptr, float *lse = nullptr, int G = 0, int D = 0, const void *q_bf16 = nullptr,
-                 int64_t q_elems = 0, int M = 1, int len_unit = 1, int ncg = 1);
+                 int64_t q_elems = 0, int M = 1, int len_unit = 1, int ncg = 1, int row_cost = 0);
 void launch_plan_dump(const PlanView &pv, const int32_t *cu, int B, int Hkv, int n_req, int32_t *segs,
                       int64_t max_segs, int32_t *n_segs, const WsHeader *hdr, cudaStream_t s);
 

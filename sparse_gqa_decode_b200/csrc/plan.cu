@@ -21,7 +21,7 @@ constexpr size_t kPlanFastBytes = 160 * 1024;
 // at the end, so no step waits on a global-memory round trip after the first loads.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu_len,
                                                     const int32_t *__restrict__ cu_seq, int B, int Hkv,
-                                                    int n_req, int min_chunk, int mode, int granule,
+                                                    int n_req, int min_chunk, int mode, int granule, int row_cost,
                                                     PlanView pv, WsHeader *hdr, int staged, float *out,
                                                     float *lse, int G, int D, const __nv_bfloat16 *q,
                                                     int64_t q_elems, int M, int len_unit, int ncg) {
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         if (r < R) {
             const int32_t L = len_of(r % B);
             if (L < 1) atomicOr(&hdr->status, SGD_STATUS_EMPTY_SEQUENCE);
-            v = (int32_t)align_up(max(L, 0), granule);
+            v = (L > 0) ? (int32_t)align_up(L, granule) + row_cost : 0;
         }
         int32_t total;
         const int32_t ex = block_exclusive_scan(v, total, sm);
@@ -128,7 +128,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
             int r0 = R;
             if (a < e) {
                 r0 = upper_bound_i32(row_pos, R + 1, a) - 1;
-                for (int r = r0; r < R && row_pos[r] < e; ++r) v += (row_pos[r + 1] > row_pos[r]) ? 1 : 0;
+                for (int r = r0; r < R && row_pos[r] < e; ++r) {  // rows whose tokens meet [a, e)
+                    const int32_t Lr = len_of(r % B);
+                    v += (Lr > 0 && row_pos[r] + Lr > a) ? 1 : 0;
+                }
             }
             pv.cta_row0[i] = r0;
         }
@@ -213,6 +216,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
 __global__ void __launch_bounds__(1024) plan_fast_kernel(const int32_t *__restrict__ cu_len,
                                                          const int32_t *__restrict__ cu_seq, int B, int Hkv,
                                                          int n_req, int min_chunk, int mode, int granule,
+                                                         int row_cost,
                                                          PlanView pv, WsHeader *hdr, float *out, float *lse, int G,
                                                          int D, const __nv_bfloat16 *q, int64_t q_elems, int M,
                                                          int len_unit, int ncg) {
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(1024) plan_fast_kernel(const int32_t *__restri
         const int b = base + tid;
         int32_t pad = 0, np = 0;
         if (b < B) {
-            pad = (int32_t)align_up(max(len[b], 0), granule);
+            pad = (len[b] > 0) ? (int32_t)align_up(len[b], granule) + row_cost : 0;
             np = (max(slen[b], 0) + kPart - 1) / kPart;
         }
         int2 tot;
@@ -297,7 +301,6 @@ __global__ void __launch_bounds__(1024) plan_fast_kernel(const int32_t *__restri
     }
     __syncthreads();  // P complete
     auto row_pos = [&](int r) -> int32_t { return r >= R ? W : (r / B) * Wh + P[r % B]; };
-    auto row_pad = [&](int r) -> int32_t { const int b = r % B; return P[b + 1] - P[b]; };
     auto cta_begin = [&](int i) -> int32_t {
         if (mode == 0) return (int32_t)min((int64_t)i * S, (int64_t)W);
         return row_pos(min(i, R));
@@ -314,7 +317,10 @@ __global__ void __launch_bounds__(1024) plan_fast_kernel(const int32_t *__restri
             if (a < e) {
                 const int kvh = a / Wh;
                 r0 = kvh * B + upper_bound_i32(P, B + 1, a - kvh * Wh) - 1;
-                for (int r = r0; r < R && row_pos(r) < e; ++r) vc += row_pad(r) > 0 ? 1 : 0;
+                for (int r = r0; r < R && row_pos(r) < e; ++r) {  // rows whose tokens meet [a, e)
+                    const int32_t Lr = len[r % B];
+                    vc += (Lr > 0 && row_pos(r) + Lr > a) ? 1 : 0;
+                }
             }
             pv.cta_row0[i] = r0;
             pv.cta_begin[i] = a;
@@ -388,7 +394,7 @@ __global__ void plan_dump_kernel(PlanView pv, const int32_t *cu, int B, int Hkv,
 
 void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, int n_req, int min_chunk,
                  int mode, const PlanView &pv, WsHeader *hdr, cudaStream_t s, int granule, float *out, float *lse,
-                 int G, int D, const void *q_bf16, int64_t q_elems, int M, int len_unit, int ncg) {
+                 int G, int D, const void *q_bf16, int64_t q_elems, int M, int len_unit, int ncg, int row_cost) {
     // one thread per row / CTA / sequence where they fit: fewer warps make each of the kernel's
     // block barriers cheaper (the loops stride over anything larger)
     const int want = std::max(std::max(B * Hkv, n_req), B) + 1;
@@ -398,14 +404,14 @@ void launch_plan(const int32_t *cu_len, const int32_t *cu_seq, int B, int Hkv, i
         cudaFuncSetAttribute(plan_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPlanFastBytes) ==
             cudaSuccess) {
         launch_k(plan_fast_kernel, dim3(1), dim3(nt), seq_bytes, s, 1, cu_len, cu_seq, B, Hkv, n_req, min_chunk, mode,
-                 granule, pv, hdr, out, lse, G, D, static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M, len_unit,
-                 ncg);
+                 granule, row_cost, pv, hdr, out, lse, G, D, static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M,
+                 len_unit, ncg);
         return;
     }
     const size_t stage_bytes = (size_t)(B * Hkv + n_req + 2 + 5 * B) * sizeof(int32_t);
     const int staged = stage_bytes <= kPlanStageBytes;
     launch_k(plan_kernel, dim3(1), dim3(nt), staged ? stage_bytes : 0, s, 1, cu_len, cu_seq, B, Hkv, n_req,
-             min_chunk, mode, granule, pv, hdr, staged, out, lse, G, D,
+             min_chunk, mode, granule, row_cost, pv, hdr, staged, out, lse, G, D,
              static_cast<const __nv_bfloat16 *>(q_bf16), q_elems, M, len_unit, ncg);
 }
 

@@ -196,14 +196,16 @@ def test_multi_token_selection_and_plan_reject_bad_args_on_host(sgd):
     assert sel(M=0) == -2 and sel(M=3) == -2 and sel(G=16, M=2) == -2  # G * M <= 16 for the selection
     assert sel(cache=_kv(sgd, dtype=sgd.SGD_F32), qdt=sgd.SGD_F32) == -3  # tensor-core score kernel only
 
-    def plan(cu=0x1000, B=2, Hkv=2, n_req=8, min_chunk=16, mode=0, ws=0x6000, nbytes=1 << 20):
+    def plan(cu=0x1000, B=2, Hkv=2, n_req=8, min_chunk=16, mode=0, ws=0x6000, nbytes=1 << 20, row_cost=0):
         n = ctypes.c_int32(0)
-        return L.sgd_plan_segments(p(cu) if cu else None, B, Hkv, n_req, min_chunk, mode, p(0x7000), 64,
+        return L.sgd_plan_segments(p(cu) if cu else None, B, Hkv, n_req, min_chunk, mode, row_cost, p(0x7000), 64,
                                    ctypes.byref(n), p(ws) if ws else None, nbytes, None)
 
     assert plan(cu=0) == -1 and plan(ws=0) == -1
     assert plan(B=0) == -2 and plan(mode=2) == -8
     assert plan(min_chunk=8) == -8 and plan(min_chunk=24) == -8 and plan(n_req=0) == -8
+    assert plan(row_cost=-16) == -8 and plan(row_cost=24) == -8 and plan(row_cost=1 << 17) == -8
+    assert plan(row_cost=sgd.ROW_COST) not in (-1, -2, -4, -5, -8)
     assert plan(ws=0x6004) == -4 and plan(nbytes=64) == -5
     # the workspace bound include/sgd.h states passes the size check for any shape (no device here,
     # so the call then fails on the device query); a few hundred bytes less does not

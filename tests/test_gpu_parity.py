@@ -132,18 +132,19 @@ def test_identical_keys_give_mean_of_v(sgd):
 # ---------------------------------------------------------------------------------------------
 # partition
 # ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("row_cost", [0, 256, 48])
 @pytest.mark.parametrize("seed", range(6))
 @pytest.mark.parametrize("mode", [0, 1])
-def test_plan_matches_oracle_bit_exact(sgd, seed, mode):
+def test_plan_matches_oracle_bit_exact(sgd, seed, mode, row_cost):
     rng = np.random.default_rng(seed)
     B, Hkv = int(rng.integers(1, 20)), int(rng.integers(1, 9))
     lens = np.rint(np.exp(rng.uniform(0, 11, B))).astype(np.int64)
     cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).cuda()
     n_req = int(rng.integers(1, 400))
     min_chunk = 16 * int(rng.integers(1, 20))
-    segs, ncta = sgd.plan_segments(cu, B, Hkv, n_req, min_chunk, mode)
+    segs, ncta = sgd.plan_segments(cu, B, Hkv, n_req, min_chunk, mode, row_cost)
     row_len = np.tile(lens, Hkv)  # row = kvh * B + b
-    ref = oracle.plan(row_len, n_req, 16, min_chunk, mode)
+    ref = oracle.plan(row_len, n_req, 16, min_chunk, mode, row_cost)
     got = segs.numpy()
     assert ncta == ref["n_cta"]
     assert got[:, 0].tolist() == ref["cta"].tolist()
@@ -160,13 +161,13 @@ def test_plan_of_large_batches_matches_oracle(sgd, B, Hkv, n_req):
     rng = np.random.default_rng(B + Hkv)
     lens = rng.integers(1, 300, B).astype(np.int64)
     cu = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)).cuda()
-    for mode in (0, 1):
-        segs, ncta = sgd.plan_segments(cu, B, Hkv, n_req, 64, mode)
-        ref = oracle.plan(np.tile(lens, Hkv), n_req, 16, 64, mode)
+    for mode, row_cost in ((0, 0), (1, 0), (0, sgd.ROW_COST)):
+        segs, ncta = sgd.plan_segments(cu, B, Hkv, n_req, 64, mode, row_cost)
+        ref = oracle.plan(np.tile(lens, Hkv), n_req, 16, 64, mode, row_cost)
         got = segs.numpy()
         assert ncta == ref["n_cta"]
         for j, key in enumerate(("cta", "row", "start", "len")):
-            assert got[:, j].tolist() == ref[key].tolist(), key
+            assert got[:, j].tolist() == ref[key].tolist(), (key, mode, row_cost)
 
 
 # ---------------------------------------------------------------------------------------------
