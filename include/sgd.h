@@ -83,7 +83,7 @@ typedef enum {
 #define SGD_PARTITION 64 /* scheme-A partition length in tokens */
 /* tokens of work the automatic split-KV partition charges each row beside its tokens (its
  * segment setup, epilogue and merge), so that CTAs covering many short rows take fewer tokens */
-#define SGD_ROW_COST 256
+#define SGD_ROW_COST 512
 
 /* status codes */
 #define SGD_OK 0

@@ -41,7 +41,7 @@ LIB_PATH = os.path.join(_HERE, "libsgd.so")
 
 SGD_F32, SGD_BF16, SGD_I8 = 0, 1, 2
 SCHEME_A, SCHEME_B, SCHEME_A_CALIBRATED, SCHEME_B_CALIBRATED = 0, 1, 2, 3
-ROW_COST = 256  # SGD_ROW_COST: the automatic split's work charge per row, in tokens
+ROW_COST = 512  # SGD_ROW_COST: the automatic split's work charge per row, in tokens
 OP_QUANTIZE, OP_OAM_SELECT, OP_DECODE, OP_QUANTIZE_SELECT = 0, 1, 2, 3
 PARTITION = 64
 STATUS_BITS = {0x1: "empty sequence", 0x2: "wait timeout", 0x4: "size mismatch", 0x8: "bad index",
