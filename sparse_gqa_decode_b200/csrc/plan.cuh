@@ -5,15 +5,17 @@
 // idle when each CTA owns a whole sequence; splitting the KV of every row
 // across CTAs and reducing afterwards balances the work.  The reading used here:
 //   rows = (KV head, sequence) pairs in memory order, row = kvh * B + b;
-//   each row is padded to a multiple of kGranule tokens and the rows are laid
-//   end to end into one stream of W tokens;
+//   each row is padded to a multiple of kGranule tokens, followed by row_cost
+//   more positions (a fixed work charge for its segment setup and merge; 0 for
+//   a forced split and the score passes), and the rows are laid end to end
+//   into one stream of W positions;
 //   mode 0 cuts the stream into CTA ranges of S = max(min_chunk,
-//   round_up(ceil(W / n_req), kGranule)) tokens, mode 1 gives each row a CTA;
+//   round_up(ceil(W / n_req), kGranule)) positions, mode 1 gives each row a CTA;
 //   a segment = one CTA range intersected with the real tokens of one row;
 //   segments are numbered in stream order and each yields one partial result.
-// Because CTA boundaries are multiples of kGranule and a row's padding is
-// shorter than kGranule, no CTA starts inside padding and every segment holds
-// at least one real token.
+// Every segment holds at least one real token; a CTA range that falls wholly
+// in charged positions has no segment (the plan counts only rows whose real
+// tokens meet the range).
 #pragma once
 
 #include "common.cuh"
