@@ -272,3 +272,22 @@ def test_quantize_select_multi_and_blocks_reject_bad_args_on_host(sgd):
     assert blocks(nb=1) == -2  # fewer blocks than sequences
     assert blocks(kt=4) == -2  # more kept blocks than blocks
     assert blocks() not in (-1, -2, -3, -4, -8)
+
+
+def test_binding_constants_match_the_header(sgd):
+    text = open(HEADER).read()
+
+    def define(name):
+        m = re.search(r"#define\s+" + name + r"\s+\(?(\w+)", text)
+        return int(m.group(1).rstrip("u"), 0)
+
+    assert define("SGD_ROW_COST") == sgd.ROW_COST
+    assert define("SGD_PARTITION") == 64
+    for bit, name in ((0x1, "SGD_STATUS_EMPTY_SEQUENCE"), (0x2, "SGD_STATUS_WAIT_TIMEOUT"),
+                      (0x4, "SGD_STATUS_SIZE_MISMATCH"), (0x8, "SGD_STATUS_BAD_INDEX"), (0x10, "SGD_STATUS_BAD_SCALE")):
+        assert define(name) == bit and bit in sgd.STATUS_BITS
+    enum = re.search(r"typedef enum \{(.*?)\} sgd_scheme;", text, re.S).group(1)
+    values = dict(re.findall(r"(SGD_SCHEME_\w+)\s*=\s*(\d+)", enum))
+    assert {k: int(v) for k, v in values.items()} == {
+        "SGD_SCHEME_A": sgd.SCHEME_A, "SGD_SCHEME_B": sgd.SCHEME_B,
+        "SGD_SCHEME_A_CALIBRATED": sgd.SCHEME_A_CALIBRATED, "SGD_SCHEME_B_CALIBRATED": sgd.SCHEME_B_CALIBRATED}
